@@ -1,0 +1,41 @@
+"""Oracle package — TEST INFRASTRUCTURE ONLY.
+
+A plain float64 CPU statement of the block discrete-diffusion denoising step
+(see `oracle.model`) and of the Philox4x32-10 generator its sampler draws from
+(see `oracle.philox`).  Only `tests/`, `__graft_entry__.smoke()` and the
+`cpu_baseline` / `--impl reference` legs of `bench.py` may import this package.
+It shares no code with the CUDA library; the only thing both sides use is the
+seeded input generator module `synth_inputs`.
+
+Parity status of each function is recorded beside its pin in tests/.
+"""
+from .model import (Oracle, Shape, StepResult, apply_rope, attention, lm_head_stats, moe,
+                    renoise_tokens, rms_norm, rope_angles, route_top_k, sample, silu,
+                    swiglu_ffn, tokens_per_forward, tokens_per_second)
+from .philox import philox4x32_10, uniform_token
+
+
+def shape_of(w) -> Shape:
+    """Oracle shape record from a synth_inputs.Workload."""
+    s = w.shape
+    return Shape(n_layers=s.n_layers, d_model=s.d_model, n_q_heads=s.n_q_heads,
+                 n_kv_heads=s.n_kv_heads, head_dim=s.head_dim, n_experts=s.n_experts,
+                 top_k=s.top_k, expert_hidden=s.expert_hidden, shared_hidden=s.shared_hidden,
+                 vocab=s.vocab, rope_base=s.rope_base, rms_eps=s.rms_eps)
+
+
+def for_workload(w, keep_layers: bool = True, layer_override=None) -> Oracle:
+    """Oracle over the seeded weights of workload `w` (generated on the CPU).
+
+    layer_override(l, tensors) may edit a layer's tensors (planted cases)."""
+    import synth_inputs as si
+
+    def layer_fn(l):
+        t = si.layer_weights(w, l, "cpu")
+        if layer_override is not None:
+            t = layer_override(l, t)
+        return t
+
+    g = si.global_weights(w, "cpu")
+    return Oracle(shape_of(w), layer_fn, g["embed"], g["final_norm"], g["router_bias"],
+                  batch=w.batch, keep_layers=keep_layers)

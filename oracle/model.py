@@ -1,0 +1,395 @@
+"""Oracle for the block discrete-diffusion denoising step (TEST INFRASTRUCTURE ONLY).
+
+A plain, slow, float64 CPU statement of what one denoising step, the causal
+prefill and the block commit compute.  Only `tests/`, the `smoke()` entry of
+`__graft_entry__` and the CPU-baseline leg of `bench.py` may import it; the
+product path never does.  It shares no code with the CUDA library.
+
+Sources ("DiffusionGemma Technical Report" as restated on five web pages):
+  * codemajin.net "DiffusionGemma architecture", section 3.2: one weight-shared
+    transformer used two ways: a causal encoder that turns the prompt and the
+    committed blocks into a KV cache, and a bidirectional decoder that updates
+    the whole 256-token block while attending to that cache; blocks are
+    committed to the cache one after the other and never rewritten.
+  * same page, section 3.1 (forward-process formula): at full noise every
+    position is a uniformly random vocabulary token.
+  * same page, section 3.3, and aibars.net "Uniform State Diffusion":
+    confident predictions are accepted, the other positions are reset to
+    uniformly random tokens; tokens of the current block may change again at
+    later steps (section 3.2, multinomial diffusion).
+  * same page, section 2.1: MoE, 128 experts of which 8 plus one shared expert
+    are active per token, vocabulary ~262k.
+  * aiboss88.com "hybrid attention architecture": prefill uses causal attention
+    and writes the KV cache, denoising switches to bidirectional attention in
+    which every canvas token sees every other one.
+The pages leave the transformer's internals open; the readings taken here are
+plain ones: pre-norm RMSNorm (gain initialised to one), rotate-half RoPE at
+absolute positions, attention scale 1/sqrt(head_dim), GQA, top-k routing by
+(logit desc, index asc) with a softmax over the k selected logits, an ungated
+shared expert, SwiGLU experts, no embedding scaling, the LM head tied to the
+embedding, confidence = maximum softmax probability.
+
+Every function is written for clarity, not speed: each step below follows the
+definition directly, with library matmuls as the only building block.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import numpy as np
+
+from .philox import philox4x32_10, uniform_token
+
+
+# ---------------------------------------------------------------------------
+# primitives
+# ---------------------------------------------------------------------------
+def rms_norm(h: np.ndarray, gain: np.ndarray, eps: float) -> np.ndarray:
+    """u = h / sqrt(mean(h^2) + eps) * gain, per row."""
+    ms = np.mean(h * h, axis=-1, keepdims=True)
+    return h / np.sqrt(ms + eps) * gain
+
+
+def silu(x: np.ndarray) -> np.ndarray:
+    return x / (1.0 + np.exp(-x))
+
+
+def rope_angles(positions: np.ndarray, head_dim: int, base: float):
+    """cos/sin of angle pos * base^(-2j/D) for j < D/2 (rotate-half pairs j, j+D/2)."""
+    half = head_dim // 2
+    j = np.arange(half, dtype=np.float64)
+    inv = base ** (-2.0 * j / head_dim)
+    ang = np.asarray(positions, dtype=np.float64)[:, None] * inv[None, :]
+    return np.cos(ang), np.sin(ang)
+
+
+def apply_rope(x: np.ndarray, cos: np.ndarray, sin: np.ndarray) -> np.ndarray:
+    """Rotate pairs (j, j+D/2) of x[..., n, D] by the angles of row n."""
+    half = x.shape[-1] // 2
+    x1, x2 = x[..., :half], x[..., half:]
+    return np.concatenate([x1 * cos - x2 * sin, x2 * cos + x1 * sin], axis=-1)
+
+
+def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, key_limit: np.ndarray) -> np.ndarray:
+    """Grouped-query attention.
+
+    q [Hq, n, D]; k, v [Hkv, S, D]; query row i sees keys j < key_limit[i].
+    Returns o [n, Hq*D] (heads concatenated).
+    """
+    Hq, n, D = q.shape
+    Hkv, S, _ = k.shape
+    group = Hq // Hkv
+    visible = np.arange(S)[None, :] < np.asarray(key_limit)[:, None]
+    out = np.empty((n, Hq, D))
+    for h in range(Hq):
+        g = h // group
+        s = q[h] @ k[g].T / np.sqrt(D)
+        s = np.where(visible, s, -np.inf)
+        s = s - s.max(axis=1, keepdims=True)
+        p = np.exp(s)
+        p = p / p.sum(axis=1, keepdims=True)
+        out[:, h, :] = p @ v[g]
+    return out.reshape(n, Hq * D)
+
+
+def route_top_k(logits: np.ndarray, k: int):
+    """Top-k experts per row ordered by (logit desc, index asc); gates are the
+    softmax of the k selected logits.  Returns idx int64 [n,k], gates [n,k]."""
+    n, E = logits.shape
+    idx = np.empty((n, k), dtype=np.int64)
+    for i in range(n):
+        order = sorted(range(E), key=lambda e: (-logits[i, e], e))
+        idx[i] = order[:k]
+    sel = np.take_along_axis(logits.astype(np.float64), idx, axis=1)
+    sel = sel - sel.max(axis=1, keepdims=True)
+    g = np.exp(sel)
+    return idx, g / g.sum(axis=1, keepdims=True)
+
+
+def swiglu_ffn(x: np.ndarray, wg: np.ndarray, wu: np.ndarray, wd: np.ndarray) -> np.ndarray:
+    """(SiLU(x Wg^T) * (x Wu^T)) Wd^T with weights stored [out, in]."""
+    return (silu(x @ wg.T) * (x @ wu.T)) @ wd.T
+
+
+def moe(u: np.ndarray, lw, idx: np.ndarray, gates: np.ndarray) -> np.ndarray:
+    """Shared expert (weight 1) plus the gate-weighted routed experts."""
+    out = swiglu_ffn(u, lw["ws_gate"], lw["ws_up"], lw["ws_down"])
+    for e in np.unique(idx):
+        rows, slots = np.nonzero(idx == e)
+        y = swiglu_ffn(u[rows], lw.expert(e, "w_gate"), lw.expert(e, "w_up"),
+                       lw.expert(e, "w_down"))
+        out[rows] += gates[rows, slots][:, None] * y
+    return out
+
+
+def lm_head_stats(z: np.ndarray, embed, temperature: float, row_chunk: int = 64,
+                  vocab_chunk: int = 32768):
+    """Per row of logits s = z E^T / T: max m, lowest argmax a, log-sum-exp,
+    confidence exp(m - lse), log-probability m - lse and the top-1/top-2
+    probability margin.  `embed` is the [V, d] tied embedding (any array or
+    bf16 tensor); whole logit rows are formed before any statistic is taken."""
+    n = z.shape[0]
+    V = embed.shape[0]
+    res = {k: np.empty(n) for k in ("max", "lse", "conf", "logp", "margin")}
+    res["argmax"] = np.empty(n, dtype=np.int64)
+    logits = np.empty((min(n, row_chunk), V))
+    for r0 in range(0, n, row_chunk):
+        zr = z[r0:r0 + row_chunk]
+        s = logits[:zr.shape[0]]
+        for v0 in range(0, V, vocab_chunk):
+            s[:, v0:v0 + vocab_chunk] = zr @ _f64(embed[v0:v0 + vocab_chunk]).T
+        s /= temperature
+        rows = np.arange(s.shape[0])
+        a = np.argmax(s, axis=1)                      # first (lowest) index of the max
+        m = s[rows, a]
+        lse = m + np.log(np.exp(s - m[:, None]).sum(axis=1))
+        s[rows, a] = -np.inf
+        m2 = s.max(axis=1)
+        sl = slice(r0, r0 + s.shape[0])
+        res["argmax"][sl] = a
+        res["max"][sl] = m
+        res["lse"][sl] = lse
+        res["conf"][sl] = np.exp(m - lse)
+        res["logp"][sl] = m - lse
+        res["margin"][sl] = np.exp(m - lse) - np.exp(m2 - lse)
+    return res
+
+
+def renoise_tokens(positions, step: int, seq_ids, seed: int, vocab: int) -> np.ndarray:
+    """Uniform replacement tokens: Philox4x32-10 with counter (absolute
+    position, step, sequence, 0) and key (seed low word, seed high word)."""
+    positions = np.asarray(positions, dtype=np.uint64)
+    seq_ids = np.broadcast_to(np.asarray(seq_ids, dtype=np.uint64), positions.shape)
+    w0, _, _, _ = philox4x32_10(positions, np.full(positions.shape, step, np.uint64),
+                                seq_ids, np.zeros(positions.shape, np.uint64),
+                                seed & 0xFFFFFFFF, (seed >> 32) & 0xFFFFFFFF)
+    return uniform_token(w0, vocab)
+
+
+def sample(argmax: np.ndarray, conf: np.ndarray, tau: float, noise: np.ndarray) -> np.ndarray:
+    """Keep the argmax where conf >= tau, else take the uniform draw (a NaN
+    confidence re-noises)."""
+    keep = np.asarray(conf) >= tau
+    return np.where(keep, argmax, noise)
+
+
+def tokens_per_forward(total_tokens: int, total_steps: int, n_blocks: int) -> float:
+    """TPF: generated tokens over (denoising steps + K - 1), the K - 1 being the
+    extra forward that commits each finished block (codemajin.net section 5.1)."""
+    return total_tokens / (total_steps + n_blocks - 1)
+
+
+def tokens_per_second(tpf: float, t_fwd_s: float) -> float:
+    """TPS = TPF / t_fwd (codemajin.net section 5.1)."""
+    return tpf / t_fwd_s
+
+
+# ---------------------------------------------------------------------------
+# weights
+# ---------------------------------------------------------------------------
+class LayerWeights:
+    """fp64 view of one layer's bf16 weights; routed experts are converted on
+    demand so a 128-expert layer never sits in memory as fp64 all at once."""
+
+    def __init__(self, tensors: dict):
+        self._t = tensors
+        self._cache = {}
+
+    def __getitem__(self, name):
+        if name not in self._cache:
+            self._cache[name] = _f64(self._t[name])
+        return self._cache[name]
+
+    def expert(self, e: int, name: str) -> np.ndarray:
+        return _f64(self._t[name][int(e)])
+
+    def raw(self, name):
+        return self._t[name]
+
+
+def _index(tokens):
+    try:
+        import torch
+        return torch.as_tensor(np.asarray(tokens, dtype=np.int64))
+    except ImportError:  # pragma: no cover
+        return np.asarray(tokens, dtype=np.int64)
+
+
+def _f64(t) -> np.ndarray:
+    try:
+        import torch
+        if isinstance(t, torch.Tensor):
+            return t.detach().to("cpu").to(torch.float64).numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.asarray(t, dtype=np.float64)
+
+
+@dataclass
+class Shape:
+    n_layers: int
+    d_model: int
+    n_q_heads: int
+    n_kv_heads: int
+    head_dim: int
+    n_experts: int
+    top_k: int
+    expert_hidden: int
+    shared_hidden: int
+    vocab: int
+    rope_base: float = 10000.0
+    rms_eps: float = 1e-6
+
+
+# ---------------------------------------------------------------------------
+# the model
+# ---------------------------------------------------------------------------
+@dataclass
+class StepResult:
+    canvas_out: np.ndarray
+    conf: np.ndarray
+    argmax: np.ndarray
+    lse: np.ndarray
+    logp: np.ndarray
+    margin: np.ndarray
+    hidden: list = field(default_factory=list)      # per layer boundary, [B, C, d]
+    experts: list = field(default_factory=list)     # per layer, [B, C, k]
+    router_logits: list = field(default_factory=list)
+    router_margin: list = field(default_factory=list)  # k-th minus (k+1)-th logit
+
+
+class Oracle:
+    """Block discrete-diffusion decoder, fp64.
+
+    layer_fn(l) -> dict of bf16 tensors for layer l (names as in the C ABI);
+    embed: [V, d] bf16; router_bias: [E] fp32 or None.
+    """
+
+    def __init__(self, shape: Shape, layer_fn, embed, final_norm, router_bias=None,
+                 batch: int = 1, keep_layers: bool = True):
+        self.s = shape
+        self.layer_fn = layer_fn
+        self.embed = embed            # kept in storage precision; rows converted on use
+        self.final_norm = _f64(final_norm)
+        self.router_bias = None if router_bias is None else _f64(router_bias)
+        self.B = batch
+        self.keep_layers = keep_layers
+        self._layers = {}
+        # KV cache per layer: list over sequences of (K [Hkv, P, D], V [Hkv, P, D])
+        self.k_cache = [[np.zeros((shape.n_kv_heads, 0, shape.head_dim)) for _ in range(batch)]
+                        for _ in range(shape.n_layers)]
+        self.v_cache = [[np.zeros((shape.n_kv_heads, 0, shape.head_dim)) for _ in range(batch)]
+                        for _ in range(shape.n_layers)]
+        self.P = 0
+
+    # -- weights --
+    def layer(self, l: int) -> LayerWeights:
+        if l in self._layers:
+            return self._layers[l]
+        lw = LayerWeights(self.layer_fn(l))
+        if self.keep_layers:
+            self._layers[l] = lw
+        return lw
+
+    # -- one transformer layer over new rows of one sequence --
+    def _layer_forward(self, l: int, h: np.ndarray, b: int, pos0: int, causal: bool,
+                       need_ffn: bool = True, dbg: dict | None = None):
+        s = self.s
+        lw = self.layer(l)
+        n = h.shape[0]
+        D, Hq, Hkv = s.head_dim, s.n_q_heads, s.n_kv_heads
+        u = rms_norm(h, lw["attn_norm"], s.rms_eps)
+        qkv = u @ lw["wqkv"].T
+        q = qkv[:, :Hq * D].reshape(n, Hq, D).transpose(1, 0, 2)
+        k = qkv[:, Hq * D:(Hq + Hkv) * D].reshape(n, Hkv, D).transpose(1, 0, 2)
+        v = qkv[:, (Hq + Hkv) * D:].reshape(n, Hkv, D).transpose(1, 0, 2)
+        cos, sin = rope_angles(np.arange(pos0, pos0 + n), D, s.rope_base)
+        q = apply_rope(q, cos, sin)
+        k = apply_rope(k, cos, sin)
+        keys = np.concatenate([self.k_cache[l][b][:, :pos0], k], axis=1)
+        vals = np.concatenate([self.v_cache[l][b][:, :pos0], v], axis=1)
+        if causal:
+            limit = pos0 + 1 + np.arange(n)
+        else:
+            limit = np.full(n, pos0 + n)
+        o = attention(q, keys, vals, limit)
+        h = h + o @ lw["wo"].T
+        if need_ffn:
+            u2 = rms_norm(h, lw["ffn_norm"], s.rms_eps)
+            r = u2 @ lw["w_router"].T
+            if self.router_bias is not None:
+                r = r + self.router_bias
+            idx, gates = route_top_k(r, s.top_k)
+            h = h + moe(u2, lw, idx, gates)
+            if dbg is not None:
+                dbg["idx"], dbg["logits"] = idx, r
+                srt = -np.sort(-r, axis=1)
+                dbg["margin"] = (srt[:, s.top_k - 1] - srt[:, s.top_k]
+                                 if s.top_k < s.n_experts else np.full(n, np.inf))
+        return h, k, v
+
+    # -- causal encoder --
+    def _causal_append(self, tokens: np.ndarray):
+        """Causal forward of new rows at positions [P, P+n) for every sequence,
+        appending their keys/values to the cache (the last layer's MoE does not
+        feed the cache and is skipped)."""
+        tokens = np.asarray(tokens)
+        B, n = tokens.shape
+        s = self.s
+        for b in range(B):
+            h = _f64(self.embed[_index(tokens[b])])
+            for l in range(s.n_layers):
+                last = l == s.n_layers - 1
+                h, k, v = self._layer_forward(l, h, b, self.P, causal=True, need_ffn=not last)
+                self.k_cache[l][b] = np.concatenate([self.k_cache[l][b][:, :self.P], k], axis=1)
+                self.v_cache[l][b] = np.concatenate([self.v_cache[l][b][:, :self.P], v], axis=1)
+        self.P += n
+
+    def prefill(self, tokens: np.ndarray):
+        """Reset the cache and encode the prompt causally."""
+        s = self.s
+        for l in range(s.n_layers):
+            for b in range(self.B):
+                self.k_cache[l][b] = np.zeros((s.n_kv_heads, 0, s.head_dim))
+                self.v_cache[l][b] = np.zeros((s.n_kv_heads, 0, s.head_dim))
+        self.P = 0
+        self._causal_append(tokens)
+
+    def commit_block(self, block: np.ndarray):
+        """Append a finished block to the cache (one causal forward)."""
+        self._causal_append(block)
+
+    # -- bidirectional decoder + sampler --
+    def denoise_step(self, canvas: np.ndarray, step: int, seed: int, tau: float,
+                     temperature: float = 1.0, record: bool = True) -> StepResult:
+        canvas = np.asarray(canvas)
+        B, C = canvas.shape
+        s = self.s
+        hidden = [np.empty((B, C, s.d_model)) for _ in range(s.n_layers + 1)] if record else []
+        experts = [np.empty((B, C, s.top_k), dtype=np.int64) for _ in range(s.n_layers)] if record else []
+        rlog = [np.empty((B, C, s.n_experts)) for _ in range(s.n_layers)] if record else []
+        rmar = [np.empty((B, C)) for _ in range(s.n_layers)] if record else []
+        z = np.empty((B, C, s.d_model))
+        for b in range(B):
+            h = _f64(self.embed[_index(canvas[b])])
+            if record:
+                hidden[0][b] = h
+            for l in range(s.n_layers):
+                dbg = {}
+                h, _, _ = self._layer_forward(l, h, b, self.P, causal=False, dbg=dbg)
+                if record:
+                    hidden[l + 1][b] = h
+                    experts[l][b] = dbg["idx"]
+                    rlog[l][b] = dbg["logits"]
+                    rmar[l][b] = dbg["margin"]
+            z[b] = rms_norm(h, self.final_norm, s.rms_eps)
+        st = lm_head_stats(z.reshape(B * C, s.d_model), self.embed, temperature)
+        pos = np.tile(np.arange(self.P, self.P + C), B)
+        seq = np.repeat(np.arange(B), C)
+        noise = renoise_tokens(pos, step, seq, seed, s.vocab)
+        out = sample(st["argmax"], st["conf"], tau, noise)
+        rs = lambda a: a.reshape(B, C)
+        return StepResult(canvas_out=rs(out), conf=rs(st["conf"]), argmax=rs(st["argmax"]),
+                          lse=rs(st["lse"]), logp=rs(st["logp"]), margin=rs(st["margin"]),
+                          hidden=hidden, experts=experts, router_logits=rlog,
+                          router_margin=rmar)
