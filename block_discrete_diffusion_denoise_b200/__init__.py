@@ -1,0 +1,213 @@
+"""Python binding of libdg.so, the C ABI declared in include/dg.h.
+
+Argument marshalling only: every step of the denoising path runs in the CUDA
+kernels of the library.  Importing works without a GPU (the tests check the
+exported symbols on CPU); creating a context needs the built library and a
+CUDA device and fails loudly otherwise — there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libdg.so")
+
+DG_OK = 0
+STATUS = {0: "DG_OK", 1: "DG_ERR_INVALID_ARG", 2: "DG_ERR_OOM", 3: "DG_ERR_CAPACITY", 4: "DG_ERR_CUDA",
+          5: "DG_ERR_DEVICE_TIMEOUT", 6: "DG_ERR_STATE", 7: "DG_ERR_UNSUPPORTED"}
+
+# every function declared in include/dg.h
+EXPORTS = ["dg_create", "dg_destroy", "dg_prefill", "dg_denoise_step", "dg_denoise_step_host",
+           "dg_commit_block", "dg_sync", "dg_cached_len", "dg_last_error", "dg_debug_capture",
+           "dg_debug_hidden", "dg_debug_experts", "dg_debug_lmhead", "dg_debug_router",
+           "dg_debug_sample", "dg_debug_wait_timeout", "dg_debug_gemm", "dg_debug_launch_count"]
+
+
+class dg_config(ctypes.Structure):
+    _fields_ = [("n_layers", ctypes.c_int32), ("d_model", ctypes.c_int32),
+                ("n_q_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("n_experts", ctypes.c_int32),
+                ("top_k", ctypes.c_int32), ("expert_hidden", ctypes.c_int32),
+                ("shared_hidden", ctypes.c_int32), ("vocab", ctypes.c_int32),
+                ("rope_base", ctypes.c_float), ("rms_eps", ctypes.c_float),
+                ("temperature", ctypes.c_float), ("canvas", ctypes.c_int32),
+                ("max_batch", ctypes.c_int32), ("max_seq", ctypes.c_int32),
+                ("prefill_rows", ctypes.c_int32)]
+
+
+LAYER_FIELDS = ["attn_norm", "wqkv", "wo", "ffn_norm", "w_router", "w_gate", "w_up", "w_down",
+                "ws_gate", "ws_up", "ws_down"]
+
+
+class dg_layer_weights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in LAYER_FIELDS]
+
+
+class dg_weights(ctypes.Structure):
+    _fields_ = [("embed", ctypes.c_void_p), ("final_norm", ctypes.c_void_p),
+                ("router_bias", ctypes.c_void_p), ("layers", ctypes.POINTER(dg_layer_weights))]
+
+
+class DGError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libdg.so and declare its signatures (raises if it is missing)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is not built; run python -m block_discrete_diffusion_denoise_b200.build")
+    lib = ctypes.CDLL(path)
+    P, I32, I64, U64, F32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64, ctypes.c_float
+    sig = {
+        "dg_create": ([ctypes.POINTER(dg_config), ctypes.POINTER(dg_weights), P, ctypes.POINTER(P)], I32),
+        "dg_destroy": ([P], I32),
+        "dg_prefill": ([P, P, I32, I32], I32),
+        "dg_denoise_step": ([P, P, I32, U64, F32, P, P, P], I32),
+        "dg_denoise_step_host": ([P, P, I32, U64, F32, P, P, P], I32),
+        "dg_commit_block": ([P, P], I32),
+        "dg_sync": ([P], I32),
+        "dg_cached_len": ([P], I32),
+        "dg_last_error": ([P], ctypes.c_char_p),
+        "dg_debug_capture": ([P, I32], I32),
+        "dg_debug_hidden": ([P, I32, P], I32),
+        "dg_debug_experts": ([P, I32, P], I32),
+        "dg_debug_lmhead": ([P, P, P, P, P], I32),
+        "dg_debug_router": ([P, P, I32, P, P], I32),
+        "dg_debug_sample": ([P, P, P, I32, I32, U64, F32, P], I32),
+        "dg_debug_wait_timeout": ([P, U64], I32),
+        "dg_debug_gemm": ([P, P, I32, I32, P, I32, I32, P], I32),
+        "dg_debug_launch_count": ([P], I64),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = res
+    _lib = lib
+    return lib
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    return t.data_ptr()
+
+
+class Context:
+    """One dg_ctx.  `weights` holds torch CUDA tensors (bf16) named as in
+    dg.h: embed, final_norm, router_bias (fp32 or None) and layers (list of
+    dicts with the LAYER_FIELDS keys).  The tensors are referenced for the
+    lifetime of the context."""
+
+    def __init__(self, cfg: dict, weights: dict, stream=None):
+        self.lib = load_library()
+        self._weights = weights
+        c = dg_config()
+        for name, _ in dg_config._fields_:
+            setattr(c, name, cfg[name])
+        self.cfg = dict(cfg)
+        layers = (dg_layer_weights * cfg["n_layers"])()
+        for i, lw in enumerate(weights["layers"]):
+            for f in LAYER_FIELDS:
+                setattr(layers[i], f, _ptr(lw[f]))
+        w = dg_weights(embed=_ptr(weights["embed"]), final_norm=_ptr(weights["final_norm"]),
+                       router_bias=_ptr(weights.get("router_bias")),
+                       layers=ctypes.cast(layers, ctypes.POINTER(dg_layer_weights)))
+        self._layers_c = layers
+        handle = ctypes.c_void_p()
+        st = self.lib.dg_create(ctypes.byref(c), ctypes.byref(w), stream, ctypes.byref(handle))
+        if st != DG_OK:
+            raise DGError(st, "dg_create failed (check shape and weight alignment)")
+        self.ctx = handle
+
+    def _check(self, st):
+        if st != DG_OK:
+            raise DGError(st, self.lib.dg_last_error(self.ctx).decode())
+
+    def close(self):
+        if getattr(self, "ctx", None):
+            self.lib.dg_destroy(self.ctx)
+            self.ctx = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # --- the path ---
+    def prefill(self, tokens):
+        B, P = tokens.shape
+        self._check(self.lib.dg_prefill(self.ctx, _ptr(tokens), B, P))
+
+    def denoise_step(self, canvas_in, step, seed, tau, canvas_out, conf, settled=None):
+        self._check(self.lib.dg_denoise_step(self.ctx, _ptr(canvas_in), int(step), int(seed), float(tau),
+                                             _ptr(canvas_out), _ptr(conf), _ptr(settled)))
+
+    def denoise_step_host(self, canvas_in, step, seed, tau, canvas_out, conf=None, settled=None):
+        """Host-buffer variant: numpy int32/float32 arrays (or pinned CPU tensors)."""
+        def hp(a):
+            if a is None:
+                return None
+            return a.ctypes.data if hasattr(a, "ctypes") else a.data_ptr()
+        self._check(self.lib.dg_denoise_step_host(self.ctx, hp(canvas_in), int(step), int(seed), float(tau),
+                                                  hp(canvas_out), hp(conf), hp(settled)))
+
+    def commit_block(self, block):
+        self._check(self.lib.dg_commit_block(self.ctx, _ptr(block)))
+
+    def sync(self):
+        self._check(self.lib.dg_sync(self.ctx))
+
+    @property
+    def cached_len(self) -> int:
+        return self.lib.dg_cached_len(self.ctx)
+
+    # --- test hooks ---
+    def debug_capture(self, enable: bool):
+        self._check(self.lib.dg_debug_capture(self.ctx, 1 if enable else 0))
+
+    def debug_hidden(self, layer, out):
+        self._check(self.lib.dg_debug_hidden(self.ctx, layer, _ptr(out)))
+
+    def debug_experts(self, layer, out):
+        self._check(self.lib.dg_debug_experts(self.ctx, layer, _ptr(out)))
+
+    def debug_lmhead(self, argmax=None, lse=None, conf=None, margin=None):
+        self._check(self.lib.dg_debug_lmhead(self.ctx, _ptr(argmax), _ptr(lse), _ptr(conf), _ptr(margin)))
+
+    def debug_router(self, logits, idx, gates):
+        self._check(self.lib.dg_debug_router(self.ctx, _ptr(logits), logits.shape[0], _ptr(idx), _ptr(gates)))
+
+    def debug_sample(self, argmax, conf, batch, step, seed, tau, out):
+        self._check(self.lib.dg_debug_sample(self.ctx, _ptr(argmax), _ptr(conf), batch, int(step), int(seed),
+                                             float(tau), _ptr(out)))
+
+    def debug_wait_timeout(self, limit_ns: int):
+        self._check(self.lib.dg_debug_wait_timeout(self.ctx, int(limit_ns)))
+
+    def debug_gemm(self, w, x, splits, out):
+        M, K = w.shape
+        self._check(self.lib.dg_debug_gemm(self.ctx, _ptr(w), M, K, _ptr(x), x.shape[0], int(splits), _ptr(out)))
+
+    @property
+    def launch_count(self) -> int:
+        return self.lib.dg_debug_launch_count(self.ctx)
+
+
+def config_from_shape(shape, max_batch=1, max_seq=4096, canvas=256, temperature=1.0, prefill_rows=0) -> dict:
+    """dg_config fields for a model shape (anything with the dg_config names)."""
+    return dict(n_layers=shape.n_layers, d_model=shape.d_model, n_q_heads=shape.n_q_heads,
+                n_kv_heads=shape.n_kv_heads, head_dim=shape.head_dim, n_experts=shape.n_experts,
+                top_k=shape.top_k, expert_hidden=shape.expert_hidden, shared_hidden=shape.shared_hidden,
+                vocab=shape.vocab, rope_base=shape.rope_base, rms_eps=shape.rms_eps,
+                temperature=temperature, canvas=canvas, max_batch=max_batch, max_seq=max_seq,
+                prefill_rows=prefill_rows)

@@ -1,0 +1,818 @@
+// C ABI of the denoising step (include/dg.h): context, workspace plan, TMA
+// descriptors, the layer loop shared by the causal encoder (prefill, block
+// commit) and the bidirectional decoder (denoising step), and test hooks.
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "../../include/dg.h"
+#include "attention.cuh"
+#include "common.cuh"
+#include "gemm.cuh"
+#include "kernels.cuh"
+
+using namespace dg;
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+struct LayerMaps {
+  CUtensorMap wqkv, wo, wr, wg, wu, wd, wsg, wsu, wsd;
+};
+
+}  // namespace
+
+struct dg_ctx {
+  dg_config cfg{};
+  int dev = 0;
+  int sms = 148;
+  cudaStream_t stream = nullptr;
+  std::vector<dg_layer_weights> layers;
+  const uint16_t* embed = nullptr;
+  const uint16_t* final_norm = nullptr;
+  const float* router_bias = nullptr;
+  // sizes
+  int d = 0, D = 0, Hq = 0, Hkv = 0, E = 0, k = 0, F = 0, Fs = 0, V = 0, L = 0, QKV = 0, HD = 0;
+  int R = 0;        // workspace rows (max of step rows and prefill rows)
+  int R_step = 0;   // max_batch * canvas
+  size_t part_cap = 0, opart_rows_cap = 0;
+  // device buffers
+  void* ws = nullptr;
+  uint16_t* kcache = nullptr;
+  uint16_t* vcache = nullptr;
+  float* h = nullptr;
+  uint16_t* u = nullptr;
+  float* part = nullptr;
+  uint16_t* q = nullptr;
+  uint16_t* o = nullptr;
+  float* opart = nullptr;
+  float2* ml = nullptr;
+  int32_t* idx = nullptr;
+  float* gates = nullptr;
+  int32_t* perm_tok = nullptr;
+  int32_t* inv_slot = nullptr;
+  int4* gu_tiles = nullptr;
+  int4* dn_tiles = nullptr;
+  int32_t* counters = nullptr;
+  uint16_t* xp = nullptr;
+  uint16_t* hbuf = nullptr;
+  uint16_t* hsbuf = nullptr;
+  float* yp = nullptr;
+  float4* lm_part = nullptr;
+  float2* rope = nullptr;
+  int* err_word = nullptr;
+  int32_t* dbg_argmax = nullptr;
+  float* dbg_lse = nullptr;
+  float* dbg_conf = nullptr;
+  float* dbg_margin = nullptr;
+  int32_t* io_canvas_in = nullptr;
+  int32_t* io_canvas_out = nullptr;
+  float* io_conf = nullptr;
+  int32_t* io_settled = nullptr;
+  size_t max_gu_tiles = 0, max_dn_tiles = 0;
+  // capture (test hook)
+  bool capture = false;
+  float* cap_h = nullptr;
+  int32_t* cap_idx = nullptr;
+  // tensor maps
+  std::vector<LayerMaps> lmaps;
+  CUtensorMap m_u16{}, m_u128{}, m_o16{}, m_xp16{}, m_h16{}, m_hs16{}, m_embed{};
+  // state
+  int B = 0;
+  int P = 0;
+  bool prefilled = false;
+  uint64_t wait_limit_ns = 1000000000ull;
+  int64_t launches = 0;
+  std::string last_error;
+};
+
+namespace {
+
+dg_status fail(dg_ctx* c, dg_status s, const char* fmt, ...) {
+  if (c) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    c->last_error = buf;
+  }
+  return s;
+}
+
+#define DG_CUDA(c, call)                                                                     \
+  do {                                                                                       \
+    cudaError_t e_ = (call);                                                                 \
+    if (e_ != cudaSuccess) return fail((c), DG_ERR_CUDA, "%s: %s", #call, cudaGetErrorString(e_)); \
+  } while (0)
+
+#define DG_LAUNCHED(c)                                                                              \
+  do {                                                                                              \
+    (c)->launches++;                                                                                \
+    cudaError_t e_ = cudaGetLastError();                                                            \
+    if (e_ != cudaSuccess) return fail((c), DG_ERR_CUDA, "launch failed at %s:%d: %s", __FILE__, __LINE__, \
+                                       cudaGetErrorString(e_));                                     \
+  } while (0)
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// bf16 matrix [rows, cols] row-major; box = 64 columns x box_rows rows, 128-byte swizzle
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc || base == nullptr) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+DevErr dev_err(const dg_ctx* c) { return DevErr{c->err_word, c->wait_limit_ns}; }
+
+int choose_splits(int tiles, int k_steps, int sms, size_t max_splits_by_cap) {
+  int best = 1;
+  double best_cost = 1e30;
+  for (int s = 1; s <= 8; ++s) {
+    if (k_steps / s < 4 || static_cast<size_t>(s) > max_splits_by_cap) break;
+    const double rounds = std::ceil(static_cast<double>(tiles) * s / sms);
+    const double cost = rounds / s + 0.03 * s;
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best = s;
+    }
+  }
+  return best;
+}
+
+// out[s][t][m] = partial sums over split s of W[m, :] . X[t, :]
+dg_status gemm_dense(dg_ctx* c, const CUtensorMap& w, const CUtensorMap& x, int M, int T, int K, int* splits_out) {
+  GemmParams p;
+  memset(&p, 0, sizeof(p));
+  p.a_map[0] = w;
+  p.b_map = x;
+  p.b_box_rows = 16;
+  p.M = M;
+  p.T = T;
+  p.k_steps = K / 64;
+  p.bn = std::min(GEMM_BN, (T + 15) / 16 * 16);
+  p.n_tiles_n = (T + p.bn - 1) / p.bn;
+  const int m_tiles = (M + GEMM_BM - 1) / GEMM_BM;
+  const size_t cap_s = c->part_cap / (static_cast<size_t>(T) * M);
+  p.splits = choose_splits(m_tiles * p.n_tiles_n, p.k_steps, c->sms, cap_s);
+  p.tiles_static = m_tiles * p.n_tiles_n * p.splits;
+  p.out_f32 = c->part;
+  p.err = dev_err(c);
+  const int grid = std::min(c->sms, p.tiles_static);
+  gemm_kernel<GEMM_DENSE><<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, c->stream>>>(p);
+  DG_LAUNCHED(c);
+  *splits_out = p.splits;
+  return DG_OK;
+}
+
+dg_status attention(dg_ctx* c, int l, int B, int n, int pos0, bool causal) {
+  const size_t layer_off = static_cast<size_t>(l) * c->cfg.max_batch * c->Hkv * c->cfg.max_seq * c->D;
+  AttnParams p;
+  p.q = c->q;
+  p.kc = c->kcache + layer_off;
+  p.vc = c->vcache + layer_off;
+  p.o = c->o;
+  p.opart = c->opart;
+  p.ml = c->ml;
+  p.n = n;
+  p.B = B;
+  p.Hq = c->Hq;
+  p.Hkv = c->Hkv;
+  p.S_max = c->cfg.max_seq;
+  p.pos0 = pos0;
+  p.causal = causal ? 1 : 0;
+  p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c->D)));
+  const int G = c->Hq / c->Hkv;
+  const int qblocks = (n * G + ATT_QROWS - 1) / ATT_QROWS;
+  const int ctas = qblocks * B * c->Hkv;
+  const int keys = pos0 + n;
+  const size_t rows = static_cast<size_t>(B) * n * c->Hq;
+  int n_chunks = std::max(1, (2 * c->sms + ctas - 1) / ctas);
+  n_chunks = std::min(n_chunks, std::max(1, (keys + 255) / 256));
+  n_chunks = std::min<int>(n_chunks, static_cast<int>(c->opart_rows_cap / rows));
+  n_chunks = std::max(n_chunks, 1);
+  int chunk_len = ((keys + n_chunks - 1) / n_chunks + ATT_KB - 1) / ATT_KB * ATT_KB;
+  n_chunks = (keys + chunk_len - 1) / chunk_len;
+  p.chunk_len = chunk_len;
+  p.n_chunks = n_chunks;
+  dim3 grid(qblocks, B * c->Hkv, n_chunks);
+  switch (c->D) {
+    case 64:
+      attn_kernel<64><<<grid, 128, att_smem_bytes<64>(), c->stream>>>(p);
+      break;
+    case 128:
+      attn_kernel<128><<<grid, 128, att_smem_bytes<128>(), c->stream>>>(p);
+      break;
+    case 176:
+      attn_kernel<176><<<grid, 128, att_smem_bytes<176>(), c->stream>>>(p);
+      break;
+    default:
+      return fail(c, DG_ERR_UNSUPPORTED, "head_dim %d", c->D);
+  }
+  DG_LAUNCHED(c);
+  if (n_chunks > 1) {
+    attn_merge_kernel<<<static_cast<unsigned>(rows), 64, 0, c->stream>>>(c->opart, c->ml, n_chunks,
+                                                                         static_cast<int>(rows), c->D, c->o);
+    DG_LAUNCHED(c);
+  }
+  return DG_OK;
+}
+
+dg_status moe(dg_ctx* c, int l, int T) {
+  const LayerMaps& lm = c->lmaps[l];
+  const dg_layer_weights& lw = c->layers[l];
+  int s3 = 1;
+  dg_status st = gemm_dense(c, lm.wr, c->m_u16, c->E, T, c->d, &s3);
+  if (st != DG_OK) return st;
+  int32_t* cap = c->capture ? c->cap_idx + static_cast<size_t>(l) * c->R_step * c->k : nullptr;
+  router_topk_kernel<<<(T * 32 + 255) / 256, 256, 0, c->stream>>>(c->part, s3, T, c->E, c->k, c->router_bias,
+                                                                   c->idx, c->gates, cap);
+  DG_LAUNCHED(c);
+  permute_kernel<<<1, PERM_THREADS, 0, c->stream>>>(c->idx, T, c->k, c->E, c->F, c->Fs, c->d, c->perm_tok,
+                                                     c->inv_slot, c->gu_tiles, c->dn_tiles, c->counters);
+  DG_LAUNCHED(c);
+  const int rows = T * c->k;
+  gather_rows_kernel<<<std::min(4 * c->sms, (rows * (c->d / 8) + 255) / 256), 256, 0, c->stream>>>(
+      c->u, c->perm_tok, rows, c->d, c->xp);
+  DG_LAUNCHED(c);
+  (void)lw;
+
+  GemmParams p;
+  memset(&p, 0, sizeof(p));
+  p.a_map[0] = lm.wg;
+  p.a_map[1] = lm.wu;
+  p.as_map[0] = lm.wsg;
+  p.as_map[1] = lm.wsu;
+  p.b_map = c->m_xp16;
+  p.bs_map = c->m_u16;
+  p.b_box_rows = 16;
+  p.k_steps = c->d / 64;
+  p.tile_count = c->counters + 0;
+  p.tiles = c->gu_tiles;
+  p.n_groups_routed = c->E;
+  p.a_rows_per_group = c->F;
+  p.h_out = c->hbuf;
+  p.h_ld = c->F;
+  p.hs_out = c->hsbuf;
+  p.hs_ld = c->Fs;
+  p.err = dev_err(c);
+  gemm_kernel<GEMM_GATEUP><<<c->sms, GEMM_THREADS, GEMM_SMEM_BYTES, c->stream>>>(p);
+  DG_LAUNCHED(c);
+
+  memset(&p, 0, sizeof(p));
+  p.a_map[0] = lm.wd;
+  p.as_map[0] = lm.wsd;
+  p.b_map = c->m_h16;
+  p.bs_map = c->m_hs16;
+  p.b_box_rows = 16;
+  p.k_steps = c->F / 64;
+  p.k_steps_shared = c->Fs / 64;
+  p.tile_count = c->counters + 1;
+  p.tiles = c->dn_tiles;
+  p.n_groups_routed = c->E;
+  p.a_rows_per_group = c->d;
+  p.out_f32 = c->yp;
+  p.out_ld = c->d;
+  p.shared_row_base = rows;
+  p.err = dev_err(c);
+  gemm_kernel<GEMM_DOWN><<<c->sms, GEMM_THREADS, GEMM_SMEM_BYTES, c->stream>>>(p);
+  DG_LAUNCHED(c);
+  return DG_OK;
+}
+
+// Forward of B x n new rows at positions [pos0, pos0 + n).
+//   causal = true : encoder (prefill chunk / block commit); K/V are written
+//                   to the cache; the last layer stops after its K/V.
+//   causal = false: denoising step; canvas K/V go to cache rows [P, P+C)
+//                   (beyond the committed length), then the LM head runs.
+dg_status forward(dg_ctx* c, const int32_t* tokens, int tok_stride, int tok_off, int B, int n, int pos0,
+                  bool causal, int32_t* settled) {
+  const int T = B * n;
+  const float eps = c->cfg.rms_eps;
+  float* cap0 = (c->capture && !causal) ? c->cap_h : nullptr;
+  embed_norm_kernel<<<T, 256, 0, c->stream>>>(tokens, tok_stride, tok_off, n, c->embed,
+                                               static_cast<const uint16_t*>(c->layers[0].attn_norm), eps, c->d,
+                                               c->h, c->u, cap0, settled, B);
+  DG_LAUNCHED(c);
+  for (int l = 0; l < c->L; ++l) {
+    const LayerMaps& lm = c->lmaps[l];
+    const dg_layer_weights& lw = c->layers[l];
+    int s1 = 1;
+    dg_status st = gemm_dense(c, lm.wqkv, c->m_u16, c->QKV, T, c->d, &s1);
+    if (st != DG_OK) return st;
+    const size_t layer_off = static_cast<size_t>(l) * c->cfg.max_batch * c->Hkv * c->cfg.max_seq * c->D;
+    rope_qkv_kernel<<<T, 256, 0, c->stream>>>(c->part, s1, T, n, pos0, c->Hq, c->Hkv, c->D, c->rope, c->q,
+                                               c->kcache + layer_off, c->vcache + layer_off, c->cfg.max_seq);
+    DG_LAUNCHED(c);
+    if (causal && l == c->L - 1) break;  // only this layer's keys/values feed the cache
+    st = attention(c, l, B, n, pos0, causal);
+    if (st != DG_OK) return st;
+    int s2 = 1;
+    st = gemm_dense(c, lm.wo, c->m_o16, c->d, T, c->HD, &s2);
+    if (st != DG_OK) return st;
+    residual_norm_kernel<<<T, 256, 0, c->stream>>>(c->h, c->part, s2, T, c->d,
+                                                    static_cast<const uint16_t*>(lw.ffn_norm), eps, c->u);
+    DG_LAUNCHED(c);
+    st = moe(c, l, T);
+    if (st != DG_OK) return st;
+    const uint16_t* next_gain = l + 1 < c->L ? static_cast<const uint16_t*>(c->layers[l + 1].attn_norm)
+                                             : c->final_norm;
+    float* cap = (c->capture && !causal) ? c->cap_h + static_cast<size_t>(l + 1) * c->R_step * c->d : nullptr;
+    combine_norm_kernel<<<T, 256, 0, c->stream>>>(c->h, c->yp, c->inv_slot, c->gates, c->k, T * c->k, c->d,
+                                                   next_gain, eps, c->u, cap);
+    DG_LAUNCHED(c);
+  }
+  return DG_OK;
+}
+
+dg_status lm_head_and_sample(dg_ctx* c, int B, int step, uint64_t seed, float tau, int32_t* canvas_out,
+                             float* conf_out, int32_t* settled) {
+  const int T = B * c->cfg.canvas;
+  GemmParams p;
+  memset(&p, 0, sizeof(p));
+  p.a_map[0] = c->m_u128;
+  p.b_map = c->m_embed;
+  p.b_box_rows = 128;
+  p.M = T;
+  p.k_steps = c->d / 64;
+  p.n_mtiles = (T + GEMM_BM - 1) / GEMM_BM;
+  const int n_vtiles = c->V / GEMM_BN;
+  p.tiles_static = n_vtiles * p.n_mtiles;
+  p.lm_part = c->lm_part;
+  p.logit_scale_log2 = static_cast<float>(1.4426950408889634 / static_cast<double>(c->cfg.temperature));
+  p.err = dev_err(c);
+  gemm_kernel<GEMM_LMHEAD><<<std::min(c->sms, p.tiles_static), GEMM_THREADS, GEMM_SMEM_BYTES, c->stream>>>(p);
+  DG_LAUNCHED(c);
+  SampleArgs a;
+  a.n_vtiles = n_vtiles;
+  a.T = T;
+  a.C = c->cfg.canvas;
+  a.P = c->P;
+  a.step = step;
+  a.vocab = c->V;
+  a.seed_lo = static_cast<uint32_t>(seed & 0xFFFFFFFFull);
+  a.seed_hi = static_cast<uint32_t>(seed >> 32);
+  a.tau = tau;
+  a.canvas_out = canvas_out;
+  a.conf_out = conf_out;
+  a.settled = settled;
+  a.dbg_argmax = c->dbg_argmax;
+  a.dbg_lse = c->dbg_lse;
+  a.dbg_conf = c->dbg_conf;
+  a.dbg_margin = c->dbg_margin;
+  lmhead_merge_sample_kernel<<<T, 256, 0, c->stream>>>(c->lm_part, a);
+  DG_LAUNCHED(c);
+  return DG_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+template <typename T>
+T* carve(char*& cur, size_t count) {
+  T* p = reinterpret_cast<T*>(cur);
+  cur += (count * sizeof(T) + 255) / 256 * 256;
+  return p;
+}
+
+dg_status set_smem_attrs(dg_ctx* c) {
+  DG_CUDA(c, cudaFuncSetAttribute(gemm_kernel<GEMM_DENSE>, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES));
+  DG_CUDA(c, cudaFuncSetAttribute(gemm_kernel<GEMM_GATEUP>, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES));
+  DG_CUDA(c, cudaFuncSetAttribute(gemm_kernel<GEMM_DOWN>, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES));
+  DG_CUDA(c, cudaFuncSetAttribute(gemm_kernel<GEMM_LMHEAD>, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES));
+  DG_CUDA(c, cudaFuncSetAttribute(attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, att_smem_bytes<64>()));
+  DG_CUDA(c, cudaFuncSetAttribute(attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, att_smem_bytes<128>()));
+  DG_CUDA(c, cudaFuncSetAttribute(attn_kernel<176>, cudaFuncAttributeMaxDynamicSharedMemorySize, att_smem_bytes<176>()));
+  return DG_OK;
+}
+
+void free_all(dg_ctx* c) {
+  if (c->ws) cudaFree(c->ws);
+  if (c->kcache) cudaFree(c->kcache);
+  if (c->vcache) cudaFree(c->vcache);
+  if (c->cap_h) cudaFree(c->cap_h);
+  if (c->cap_idx) cudaFree(c->cap_idx);
+  c->ws = nullptr;
+  c->kcache = c->vcache = nullptr;
+  c->cap_h = nullptr;
+  c->cap_idx = nullptr;
+}
+
+}  // namespace
+
+// =============================================================================
+// C ABI
+// =============================================================================
+extern "C" {
+
+dg_status dg_create(const dg_config* cfg, const dg_weights* w, void* cuda_stream, dg_ctx** out) {
+  if (!cfg || !w || !out) return DG_ERR_INVALID_ARG;
+  *out = nullptr;
+  dg_ctx* c = new dg_ctx();
+  c->cfg = *cfg;
+  dg_config& g = c->cfg;
+  if (g.prefill_rows <= 0) g.prefill_rows = 2048;
+  auto reject = [&](dg_status s, const char* why) {
+    static thread_local std::string msg;
+    msg = why;
+    delete c;
+    return s;
+  };
+  if (g.n_layers <= 0 || g.d_model <= 0 || g.n_q_heads <= 0 || g.n_kv_heads <= 0 || g.n_experts <= 0 ||
+      g.top_k <= 0 || g.expert_hidden <= 0 || g.shared_hidden <= 0 || g.vocab <= 0 || g.canvas <= 0 ||
+      g.max_batch <= 0 || g.max_seq <= 0 || !(g.rms_eps >= 0.f) || !(g.temperature > 0.f) ||
+      !(g.rope_base > 0.f))
+    return reject(DG_ERR_INVALID_ARG, "non-positive dimension");
+  if (g.d_model % 128 || g.expert_hidden % 64 || g.shared_hidden % 64 || g.vocab % 128 ||
+      (g.head_dim != 64 && g.head_dim != 128 && g.head_dim != 176) || g.n_q_heads % g.n_kv_heads ||
+      (g.n_q_heads * g.head_dim) % 64 || g.n_experts > PERM_MAXE || g.top_k > 16 || g.top_k > g.n_experts ||
+      g.canvas % 16 || g.canvas > 256 || g.max_seq < g.canvas)
+    return reject(DG_ERR_UNSUPPORTED, "unsupported shape");
+  if (!w->embed || !w->final_norm || !w->layers) return reject(DG_ERR_INVALID_ARG, "null weights");
+  c->layers.assign(w->layers, w->layers + g.n_layers);
+  for (const auto& lw : c->layers) {
+    const void* ptrs[] = {lw.attn_norm, lw.wqkv, lw.wo, lw.ffn_norm, lw.w_router, lw.w_gate,
+                          lw.w_up, lw.w_down, lw.ws_gate, lw.ws_up, lw.ws_down};
+    for (const void* pp : ptrs)
+      if (!pp || !aligned16(pp)) return reject(DG_ERR_INVALID_ARG, "layer weight null or not 16-byte aligned");
+  }
+  if (!aligned16(w->embed)) return reject(DG_ERR_INVALID_ARG, "embed not 16-byte aligned");
+  c->embed = static_cast<const uint16_t*>(w->embed);
+  c->final_norm = static_cast<const uint16_t*>(w->final_norm);
+  c->router_bias = w->router_bias;
+  c->stream = static_cast<cudaStream_t>(cuda_stream);
+  c->d = g.d_model;
+  c->D = g.head_dim;
+  c->Hq = g.n_q_heads;
+  c->Hkv = g.n_kv_heads;
+  c->E = g.n_experts;
+  c->k = g.top_k;
+  c->F = g.expert_hidden;
+  c->Fs = g.shared_hidden;
+  c->V = g.vocab;
+  c->L = g.n_layers;
+  c->QKV = (c->Hq + 2 * c->Hkv) * c->D;
+  c->HD = c->Hq * c->D;
+  c->R_step = g.max_batch * g.canvas;
+  c->R = std::max(c->R_step, g.prefill_rows);
+  if (const char* s = getenv("DG_WAIT_LIMIT_NS")) c->wait_limit_ns = strtoull(s, nullptr, 10);
+
+  cudaError_t e = cudaGetDevice(&c->dev);
+  if (e != cudaSuccess) {
+    dg_status st = fail(c, DG_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    delete c;
+    return st;
+  }
+  cudaDeviceGetAttribute(&c->sms, cudaDevAttrMultiProcessorCount, c->dev);
+  if (set_smem_attrs(c) != DG_OK) {
+    delete c;
+    return DG_ERR_CUDA;
+  }
+
+  // ---- workspace plan ----
+  const size_t R = c->R, d = c->d, k = c->k;
+  const size_t mmax = std::max<size_t>({static_cast<size_t>(c->QKV), d, static_cast<size_t>(c->E)});
+  c->part_cap = std::max<size_t>(R, 5 * 256) * mmax;
+  c->opart_rows_cap = std::max<size_t>(16 * 256, 2 * R) * c->Hq;
+  const size_t chunks_max = (R * k + 127) / 128 + c->E;
+  c->max_gu_tiles = chunks_max * (c->F / 64) + ((R + 127) / 128) * (c->Fs / 64);
+  c->max_dn_tiles = (chunks_max + (R + 127) / 128) * (d / 128);
+  size_t bytes = 0;
+  auto add = [&](size_t n, size_t sz) { bytes += (n * sz + 255) / 256 * 256; };
+  add(R * d, 4);                                  // h
+  add(R * d, 2);                                  // u
+  add(c->part_cap, 4);                            // part
+  add(R * c->HD, 2);                              // q
+  add(R * c->HD, 2);                              // o
+  add(c->opart_rows_cap * c->D, 4);               // opart
+  add(c->opart_rows_cap, 8);                      // ml
+  add(R * k, 4);                                  // idx
+  add(R * k, 4);                                  // gates
+  add(R * k, 4);                                  // perm_tok
+  add(R * k, 4);                                  // inv_slot
+  add(c->max_gu_tiles, 16);                       // gu_tiles
+  add(c->max_dn_tiles, 16);                       // dn_tiles
+  add(16, 4);                                     // counters
+  add(R * k * d, 2);                              // xp
+  add(R * k * c->F, 2);                           // hbuf
+  add(R * c->Fs, 2);                              // hsbuf
+  add((R * k + R) * d, 4);                        // yp
+  add(static_cast<size_t>(c->V / GEMM_BN) * c->R_step, 16);  // lm_part
+  add(static_cast<size_t>(g.max_seq) * (c->D / 2), 8);        // rope
+  add(4, 4);                                      // err word
+  add(c->R_step, 4);                              // dbg_argmax
+  add(c->R_step, 4);
+  add(c->R_step, 4);
+  add(c->R_step, 4);
+  add(c->R_step, 4);                              // io canvas in
+  add(c->R_step, 4);                              // io canvas out
+  add(c->R_step, 4);                              // io conf
+  add(g.max_batch, 4);                            // io settled
+  e = cudaMalloc(&c->ws, bytes);
+  if (e != cudaSuccess) {
+    dg_status st = fail(c, DG_ERR_OOM, "workspace %zu bytes: %s", bytes, cudaGetErrorString(e));
+    delete c;
+    return st;
+  }
+  char* cur = static_cast<char*>(c->ws);
+  c->h = carve<float>(cur, R * d);
+  c->u = carve<uint16_t>(cur, R * d);
+  c->part = carve<float>(cur, c->part_cap);
+  c->q = carve<uint16_t>(cur, R * c->HD);
+  c->o = carve<uint16_t>(cur, R * c->HD);
+  c->opart = carve<float>(cur, c->opart_rows_cap * c->D);
+  c->ml = carve<float2>(cur, c->opart_rows_cap);
+  c->idx = carve<int32_t>(cur, R * k);
+  c->gates = carve<float>(cur, R * k);
+  c->perm_tok = carve<int32_t>(cur, R * k);
+  c->inv_slot = carve<int32_t>(cur, R * k);
+  c->gu_tiles = carve<int4>(cur, c->max_gu_tiles);
+  c->dn_tiles = carve<int4>(cur, c->max_dn_tiles);
+  c->counters = carve<int32_t>(cur, 16);
+  c->xp = carve<uint16_t>(cur, R * k * d);
+  c->hbuf = carve<uint16_t>(cur, R * k * c->F);
+  c->hsbuf = carve<uint16_t>(cur, R * c->Fs);
+  c->yp = carve<float>(cur, (R * k + R) * d);
+  c->lm_part = carve<float4>(cur, static_cast<size_t>(c->V / GEMM_BN) * c->R_step);
+  c->rope = carve<float2>(cur, static_cast<size_t>(g.max_seq) * (c->D / 2));
+  c->err_word = carve<int>(cur, 4);
+  c->dbg_argmax = carve<int32_t>(cur, c->R_step);
+  c->dbg_lse = carve<float>(cur, c->R_step);
+  c->dbg_conf = carve<float>(cur, c->R_step);
+  c->dbg_margin = carve<float>(cur, c->R_step);
+  c->io_canvas_in = carve<int32_t>(cur, c->R_step);
+  c->io_canvas_out = carve<int32_t>(cur, c->R_step);
+  c->io_conf = carve<float>(cur, c->R_step);
+  c->io_settled = carve<int32_t>(cur, g.max_batch);
+
+  const size_t cache_elems = static_cast<size_t>(c->L) * g.max_batch * c->Hkv * g.max_seq * c->D;
+  e = cudaMalloc(&c->kcache, cache_elems * 2);
+  if (e == cudaSuccess) e = cudaMalloc(&c->vcache, cache_elems * 2);
+  if (e != cudaSuccess) {
+    dg_status st = fail(c, DG_ERR_OOM, "KV cache 2 x %zu bytes: %s", cache_elems * 2, cudaGetErrorString(e));
+    free_all(c);
+    delete c;
+    return st;
+  }
+  // zero everything once: stale rows of token-side operands then hold finite values
+  cudaMemsetAsync(c->ws, 0, bytes, c->stream);
+  cudaMemsetAsync(c->kcache, 0, cache_elems * 2, c->stream);
+  cudaMemsetAsync(c->vcache, 0, cache_elems * 2, c->stream);
+
+  // RoPE table: angle pos * base^(-2j/D) in double precision, stored fp32
+  {
+    const int half = c->D / 2;
+    std::vector<float2> tab(static_cast<size_t>(g.max_seq) * half);
+    for (int pos = 0; pos < g.max_seq; ++pos)
+      for (int j = 0; j < half; ++j) {
+        const double inv = std::pow(static_cast<double>(g.rope_base), -2.0 * j / c->D);
+        const double a = pos * inv;
+        tab[static_cast<size_t>(pos) * half + j] = make_float2(static_cast<float>(std::cos(a)),
+                                                               static_cast<float>(std::sin(a)));
+      }
+    e = cudaMemcpyAsync(c->rope, tab.data(), tab.size() * sizeof(float2), cudaMemcpyHostToDevice, c->stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(c->stream);
+    if (e != cudaSuccess) {
+      dg_status st = fail(c, DG_ERR_CUDA, "rope upload: %s", cudaGetErrorString(e));
+      free_all(c);
+      delete c;
+      return st;
+    }
+  }
+
+  // ---- TMA descriptors ----
+  bool ok = true;
+  c->lmaps.resize(c->L);
+  for (int l = 0; l < c->L; ++l) {
+    const dg_layer_weights& lw = c->layers[l];
+    LayerMaps& m = c->lmaps[l];
+    ok &= make_map(&m.wqkv, lw.wqkv, c->QKV, d, 128);
+    ok &= make_map(&m.wo, lw.wo, d, c->HD, 128);
+    ok &= make_map(&m.wr, lw.w_router, c->E, d, 128);
+    ok &= make_map(&m.wg, lw.w_gate, static_cast<uint64_t>(c->E) * c->F, d, 64);
+    ok &= make_map(&m.wu, lw.w_up, static_cast<uint64_t>(c->E) * c->F, d, 64);
+    ok &= make_map(&m.wd, lw.w_down, static_cast<uint64_t>(c->E) * d, c->F, 128);
+    ok &= make_map(&m.wsg, lw.ws_gate, c->Fs, d, 64);
+    ok &= make_map(&m.wsu, lw.ws_up, c->Fs, d, 64);
+    ok &= make_map(&m.wsd, lw.ws_down, d, c->Fs, 128);
+  }
+  ok &= make_map(&c->m_u16, c->u, R, d, 16);
+  ok &= make_map(&c->m_u128, c->u, R, d, 128);
+  ok &= make_map(&c->m_o16, c->o, R, c->HD, 16);
+  ok &= make_map(&c->m_xp16, c->xp, R * k, d, 16);
+  ok &= make_map(&c->m_h16, c->hbuf, R * k, c->F, 16);
+  ok &= make_map(&c->m_hs16, c->hsbuf, R, c->Fs, 16);
+  ok &= make_map(&c->m_embed, c->embed, c->V, d, 128);
+  if (!ok) {
+    dg_status st = fail(c, DG_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+    free_all(c);
+    delete c;
+    return st;
+  }
+  *out = c;
+  return DG_OK;
+}
+
+dg_status dg_destroy(dg_ctx* c) {
+  if (!c) return DG_ERR_INVALID_ARG;
+  cudaStreamSynchronize(c->stream);
+  free_all(c);
+  delete c;
+  return DG_OK;
+}
+
+dg_status dg_prefill(dg_ctx* c, const int32_t* tokens, int32_t B, int32_t P) {
+  if (!c) return DG_ERR_INVALID_ARG;
+  if (!tokens || B <= 0 || P <= 0) return fail(c, DG_ERR_INVALID_ARG, "prefill: bad arguments");
+  if (B > c->cfg.max_batch || P + c->cfg.canvas > c->cfg.max_seq)
+    return fail(c, DG_ERR_CAPACITY, "prefill: batch %d / length %d beyond capacity", B, P);
+  c->B = B;
+  c->P = 0;
+  c->prefilled = false;
+  const int chunk = std::max(1, c->R / B);
+  for (int p0 = 0; p0 < P; p0 += chunk) {
+    const int n = std::min(chunk, P - p0);
+    dg_status st = forward(c, tokens, P, p0, B, n, p0, true, nullptr);
+    if (st != DG_OK) return st;
+  }
+  c->P = P;
+  c->prefilled = true;
+  return DG_OK;
+}
+
+dg_status dg_denoise_step(dg_ctx* c, const int32_t* canvas_in, int32_t step, uint64_t seed, float tau,
+                          int32_t* canvas_out, float* conf, int32_t* settled) {
+  if (!c) return DG_ERR_INVALID_ARG;
+  if (!canvas_in || !canvas_out || !conf) return fail(c, DG_ERR_INVALID_ARG, "step: null buffer");
+  if (!c->prefilled) return fail(c, DG_ERR_STATE, "step before prefill");
+  if (c->P + c->cfg.canvas > c->cfg.max_seq) return fail(c, DG_ERR_CAPACITY, "step: cache full");
+  dg_status st = forward(c, canvas_in, c->cfg.canvas, 0, c->B, c->cfg.canvas, c->P, false, settled);
+  if (st != DG_OK) return st;
+  return lm_head_and_sample(c, c->B, step, seed, tau, canvas_out, conf, settled);
+}
+
+dg_status dg_denoise_step_host(dg_ctx* c, const int32_t* canvas_in_host, int32_t step, uint64_t seed, float tau,
+                               int32_t* canvas_out_host, float* conf_host, int32_t* settled_host) {
+  if (!c) return DG_ERR_INVALID_ARG;
+  if (!canvas_in_host || !canvas_out_host) return fail(c, DG_ERR_INVALID_ARG, "step_host: null buffer");
+  if (!c->prefilled) return fail(c, DG_ERR_STATE, "step before prefill");
+  const size_t T = static_cast<size_t>(c->B) * c->cfg.canvas;
+  DG_CUDA(c, cudaMemcpyAsync(c->io_canvas_in, canvas_in_host, T * 4, cudaMemcpyHostToDevice, c->stream));
+  dg_status st = dg_denoise_step(c, c->io_canvas_in, step, seed, tau, c->io_canvas_out, c->io_conf,
+                                 settled_host ? c->io_settled : nullptr);
+  if (st != DG_OK) return st;
+  DG_CUDA(c, cudaMemcpyAsync(canvas_out_host, c->io_canvas_out, T * 4, cudaMemcpyDeviceToHost, c->stream));
+  if (conf_host) DG_CUDA(c, cudaMemcpyAsync(conf_host, c->io_conf, T * 4, cudaMemcpyDeviceToHost, c->stream));
+  if (settled_host)
+    DG_CUDA(c, cudaMemcpyAsync(settled_host, c->io_settled, c->B * 4, cudaMemcpyDeviceToHost, c->stream));
+  return dg_sync(c);
+}
+
+dg_status dg_commit_block(dg_ctx* c, const int32_t* block) {
+  if (!c) return DG_ERR_INVALID_ARG;
+  if (!block) return fail(c, DG_ERR_INVALID_ARG, "commit: null block");
+  if (!c->prefilled) return fail(c, DG_ERR_STATE, "commit before prefill");
+  if (c->P + 2 * c->cfg.canvas > c->cfg.max_seq)
+    return fail(c, DG_ERR_CAPACITY, "commit: no room for another block");
+  dg_status st = forward(c, block, c->cfg.canvas, 0, c->B, c->cfg.canvas, c->P, true, nullptr);
+  if (st != DG_OK) return st;
+  c->P += c->cfg.canvas;
+  return DG_OK;
+}
+
+dg_status dg_sync(dg_ctx* c) {
+  if (!c) return DG_ERR_INVALID_ARG;
+  DG_CUDA(c, cudaStreamSynchronize(c->stream));
+  int word = 0;
+  DG_CUDA(c, cudaMemcpy(&word, c->err_word, 4, cudaMemcpyDeviceToHost));
+  if (word != 0) {
+    DG_CUDA(c, cudaMemset(c->err_word, 0, 4));
+    return fail(c, DG_ERR_DEVICE_TIMEOUT, "a device wait exceeded %llu ns (code %d)",
+                static_cast<unsigned long long>(c->wait_limit_ns), word);
+  }
+  return DG_OK;
+}
+
+int32_t dg_cached_len(const dg_ctx* c) { return c ? c->P : -1; }
+
+const char* dg_last_error(const dg_ctx* c) { return c ? c->last_error.c_str() : "null context"; }
+
+dg_status dg_debug_capture(dg_ctx* c, int32_t enable) {
+  if (!c) return DG_ERR_INVALID_ARG;
+  if (enable && !c->cap_h) {
+    DG_CUDA(c, cudaMalloc(&c->cap_h, static_cast<size_t>(c->L + 1) * c->R_step * c->d * 4));
+    DG_CUDA(c, cudaMalloc(&c->cap_idx, static_cast<size_t>(c->L) * c->R_step * c->k * 4));
+  }
+  if (!enable && c->cap_h) {
+    cudaStreamSynchronize(c->stream);
+    cudaFree(c->cap_h);
+    cudaFree(c->cap_idx);
+    c->cap_h = nullptr;
+    c->cap_idx = nullptr;
+  }
+  c->capture = enable != 0;
+  return DG_OK;
+}
+
+dg_status dg_debug_hidden(dg_ctx* c, int32_t layer, float* out) {
+  if (!c || !out || !c->cap_h || layer < 0 || layer > c->L) return fail(c, DG_ERR_INVALID_ARG, "debug_hidden");
+  const size_t n = static_cast<size_t>(c->B) * c->cfg.canvas * c->d;
+  DG_CUDA(c, cudaMemcpyAsync(out, c->cap_h + static_cast<size_t>(layer) * c->R_step * c->d, n * 4,
+                             cudaMemcpyDeviceToDevice, c->stream));
+  return DG_OK;
+}
+
+dg_status dg_debug_experts(dg_ctx* c, int32_t layer, int32_t* out) {
+  if (!c || !out || !c->cap_idx || layer < 0 || layer >= c->L) return fail(c, DG_ERR_INVALID_ARG, "debug_experts");
+  const size_t n = static_cast<size_t>(c->B) * c->cfg.canvas * c->k;
+  DG_CUDA(c, cudaMemcpyAsync(out, c->cap_idx + static_cast<size_t>(layer) * c->R_step * c->k, n * 4,
+                             cudaMemcpyDeviceToDevice, c->stream));
+  return DG_OK;
+}
+
+dg_status dg_debug_lmhead(dg_ctx* c, int32_t* argmax, float* lse, float* conf, float* margin) {
+  if (!c) return DG_ERR_INVALID_ARG;
+  const size_t n = static_cast<size_t>(c->B) * c->cfg.canvas;
+  if (argmax) DG_CUDA(c, cudaMemcpyAsync(argmax, c->dbg_argmax, n * 4, cudaMemcpyDeviceToDevice, c->stream));
+  if (lse) DG_CUDA(c, cudaMemcpyAsync(lse, c->dbg_lse, n * 4, cudaMemcpyDeviceToDevice, c->stream));
+  if (conf) DG_CUDA(c, cudaMemcpyAsync(conf, c->dbg_conf, n * 4, cudaMemcpyDeviceToDevice, c->stream));
+  if (margin) DG_CUDA(c, cudaMemcpyAsync(margin, c->dbg_margin, n * 4, cudaMemcpyDeviceToDevice, c->stream));
+  return DG_OK;
+}
+
+dg_status dg_debug_router(dg_ctx* c, const float* logits, int32_t n_rows, int32_t* idx, float* gates) {
+  if (!c || !logits || !idx || !gates || n_rows <= 0) return fail(c, DG_ERR_INVALID_ARG, "debug_router");
+  router_topk_kernel<<<(n_rows * 32 + 255) / 256, 256, 0, c->stream>>>(logits, 1, n_rows, c->E, c->k, nullptr, idx,
+                                                                        gates, nullptr);
+  DG_LAUNCHED(c);
+  return DG_OK;
+}
+
+dg_status dg_debug_sample(dg_ctx* c, const int32_t* argmax, const float* conf, int32_t B, int32_t step,
+                          uint64_t seed, float tau, int32_t* out) {
+  if (!c || !argmax || !conf || !out || B <= 0) return fail(c, DG_ERR_INVALID_ARG, "debug_sample");
+  const int T = B * c->cfg.canvas;
+  sample_only_kernel<<<(T + 255) / 256, 256, 0, c->stream>>>(argmax, conf, T, c->cfg.canvas, c->P, step,
+                                                              static_cast<uint32_t>(seed & 0xFFFFFFFFull),
+                                                              static_cast<uint32_t>(seed >> 32), tau, c->V, out);
+  DG_LAUNCHED(c);
+  return DG_OK;
+}
+
+dg_status dg_debug_wait_timeout(dg_ctx* c, uint64_t limit_ns) {
+  if (!c || limit_ns == 0 || limit_ns > 10000000000ull) return fail(c, DG_ERR_INVALID_ARG, "wait_timeout");
+  wait_timeout_kernel<<<1, 32, 0, c->stream>>>(DevErr{c->err_word, limit_ns});
+  DG_LAUNCHED(c);
+  return DG_OK;
+}
+
+dg_status dg_debug_gemm(dg_ctx* c, const void* w, int32_t M, int32_t K, const void* x, int32_t T, int32_t splits,
+                        float* out) {
+  if (!c || !w || !x || !out || M <= 0 || T <= 0 || K <= 0 || K % 64 || splits < 1 || splits > K / 64 ||
+      !aligned16(w) || !aligned16(x))
+    return fail(c, DG_ERR_INVALID_ARG, "debug_gemm");
+  GemmParams p;
+  memset(&p, 0, sizeof(p));
+  if (!make_map(&p.a_map[0], w, M, K, 128) || !make_map(&p.b_map, x, T, K, 16))
+    return fail(c, DG_ERR_CUDA, "debug_gemm: tensor map");
+  p.b_box_rows = 16;
+  p.M = M;
+  p.T = T;
+  p.k_steps = K / 64;
+  p.bn = std::min(GEMM_BN, (T + 15) / 16 * 16);
+  p.n_tiles_n = (T + p.bn - 1) / p.bn;
+  p.splits = splits;
+  p.tiles_static = ((M + GEMM_BM - 1) / GEMM_BM) * p.n_tiles_n * splits;
+  p.out_f32 = out;
+  p.err = dev_err(c);
+  gemm_kernel<GEMM_DENSE><<<std::min(c->sms, p.tiles_static), GEMM_THREADS, GEMM_SMEM_BYTES, c->stream>>>(p);
+  DG_LAUNCHED(c);
+  return DG_OK;
+}
+
+int64_t dg_debug_launch_count(const dg_ctx* c) { return c ? c->launches : -1; }
+
+}  // extern "C"

@@ -1,0 +1,451 @@
+// Memory-bound kernels of the step: embedding gather + RMSNorm, split-K
+// reduction + residual + RMSNorm, QKV reduction + RoPE + KV write, router
+// top-k, token permutation and expert tile lists, row gather, gate-weighted
+// combine + residual + RMSNorm, LM-head partial merge + Philox sampler.
+#pragma once
+
+#include "common.cuh"
+
+namespace dg {
+
+// ---------------------------------------------------------------------------
+// Philox4x32-10 (Salmon et al., SC'11): 4-word counter, 2-word key, ten rounds
+// of two 32x32->64 multiplies with the key bumped by the Weyl constants.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint2 k) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    if (r > 0) {
+      k.x += 0x9E3779B9u;
+      k.y += 0xBB67AE85u;
+    }
+    const uint32_t lo0 = 0xD2511F53u * c.x, hi0 = __umulhi(0xD2511F53u, c.x);
+    const uint32_t lo1 = 0xCD9E8D57u * c.z, hi1 = __umulhi(0xCD9E8D57u, c.z);
+    c = make_uint4(hi1 ^ c.y ^ k.x, lo1, hi0 ^ c.w ^ k.y, lo0);
+  }
+  return c;
+}
+
+__device__ __forceinline__ int uniform_token(uint32_t w, int vocab) {
+  if ((vocab & (vocab - 1)) == 0) return static_cast<int>(w & static_cast<uint32_t>(vocab - 1));
+  return static_cast<int>((static_cast<uint64_t>(w) * static_cast<uint64_t>(vocab)) >> 32);
+}
+
+// ---------------------------------------------------------------------------
+// embedding gather (bf16 -> fp32 residual) + RMSNorm -> bf16
+// tokens[b * tok_stride + tok_off + i], row = b * n + i
+// ---------------------------------------------------------------------------
+__global__ void embed_norm_kernel(const int32_t* __restrict__ tokens, int tok_stride, int tok_off, int n,
+                                  const uint16_t* __restrict__ embed, const uint16_t* __restrict__ gain,
+                                  float eps, int d, float* __restrict__ h, uint16_t* __restrict__ u,
+                                  float* __restrict__ capture, int32_t* settled, int n_settled) {
+  __shared__ float red[32];
+  const int row = blockIdx.x;
+  const int b = row / n, i = row % n;
+  if (settled != nullptr && row == 0 && threadIdx.x < n_settled) settled[threadIdx.x] = 1;
+  const int tok = tokens[static_cast<size_t>(b) * tok_stride + tok_off + i];
+  const uint16_t* e = embed + static_cast<size_t>(tok) * d;
+  float ss = 0.f;
+  for (int j = threadIdx.x; j < d; j += blockDim.x) {
+    const float x = bf16_to_f32(e[j]);
+    h[static_cast<size_t>(row) * d + j] = x;
+    if (capture) capture[static_cast<size_t>(row) * d + j] = x;
+    ss += x * x;
+  }
+  ss = block_sum(ss, red);
+  const float r = rsqrtf(ss / d + eps);
+  for (int j = threadIdx.x; j < d; j += blockDim.x) {
+    const float x = h[static_cast<size_t>(row) * d + j];
+    u[static_cast<size_t>(row) * d + j] = f32_to_bf16(x * r * bf16_to_f32(gain[j]));
+  }
+}
+
+// h[row] += sum_s part[s][row]; u[row] = RMSNorm(h[row]) * gain
+__global__ void residual_norm_kernel(float* __restrict__ h, const float* __restrict__ part, int splits,
+                                     int T, int d, const uint16_t* __restrict__ gain, float eps,
+                                     uint16_t* __restrict__ u) {
+  __shared__ float red[32];
+  const int row = blockIdx.x;
+  float ss = 0.f;
+  for (int j = threadIdx.x; j < d; j += blockDim.x) {
+    float x = h[static_cast<size_t>(row) * d + j];
+    for (int s = 0; s < splits; ++s) x += part[(static_cast<size_t>(s) * T + row) * d + j];
+    h[static_cast<size_t>(row) * d + j] = x;
+    ss += x * x;
+  }
+  ss = block_sum(ss, red);
+  const float r = rsqrtf(ss / d + eps);
+  for (int j = threadIdx.x; j < d; j += blockDim.x)
+    u[static_cast<size_t>(row) * d + j] = f32_to_bf16(h[static_cast<size_t>(row) * d + j] * r * bf16_to_f32(gain[j]));
+}
+
+// Reduce QKV split-K partials, rotate q and k (pairs j, j + D/2) at absolute
+// position pos0 + i, write q [row][Hq][D] bf16 and k, v into the cache rows.
+// cache layout: [B][Hkv][S_max][D] (this layer's base pointers).
+__global__ void rope_qkv_kernel(const float* __restrict__ part, int splits, int T, int n, int pos0, int Hq,
+                                int Hkv, int D, const float2* __restrict__ rope_tab,
+                                uint16_t* __restrict__ q, uint16_t* __restrict__ kc, uint16_t* __restrict__ vc,
+                                int S_max) {
+  const int row = blockIdx.x;
+  const int b = row / n, i = row % n;
+  const int pos = pos0 + i;
+  const int QKV = (Hq + 2 * Hkv) * D;
+  const int half = D / 2;
+  const float* base = part + static_cast<size_t>(row) * QKV;
+  const size_t sstride = static_cast<size_t>(T) * QKV;
+  // rotated heads: Hq query + Hkv key heads, half pairs each
+  for (int idx = threadIdx.x; idx < (Hq + Hkv) * half; idx += blockDim.x) {
+    const int hh = idx / half, j = idx % half;
+    const int c = hh * D + j;
+    float x1 = 0.f, x2 = 0.f;
+    for (int s = 0; s < splits; ++s) {
+      x1 += base[s * sstride + c];
+      x2 += base[s * sstride + c + half];
+    }
+    const float2 cs = rope_tab[static_cast<size_t>(pos) * half + j];
+    const float y1 = x1 * cs.x - x2 * cs.y;
+    const float y2 = x2 * cs.x + x1 * cs.y;
+    if (hh < Hq) {
+      uint16_t* dst = q + (static_cast<size_t>(row) * Hq + hh) * D;
+      dst[j] = f32_to_bf16(y1);
+      dst[j + half] = f32_to_bf16(y2);
+    } else {
+      const int g = hh - Hq;
+      uint16_t* dst = kc + ((static_cast<size_t>(b) * Hkv + g) * S_max + pos) * D;
+      dst[j] = f32_to_bf16(y1);
+      dst[j + half] = f32_to_bf16(y2);
+    }
+  }
+  for (int idx = threadIdx.x; idx < Hkv * D; idx += blockDim.x) {
+    const int g = idx / D, j = idx % D;
+    const int c = (Hq + Hkv) * D + idx;
+    float x = 0.f;
+    for (int s = 0; s < splits; ++s) x += base[s * sstride + c];
+    vc[((static_cast<size_t>(b) * Hkv + g) * S_max + pos) * D + j] = f32_to_bf16(x);
+  }
+}
+
+// Router: logits = sum_s part[s][row][e] (+ bias[e]); top-k by (logit desc,
+// index asc); gates = softmax over the k selected.  One warp per row.
+__global__ void router_topk_kernel(const float* __restrict__ part, int splits, int T, int E, int k,
+                                   const float* __restrict__ bias, int32_t* __restrict__ idx_out,
+                                   float* __restrict__ gates_out, int32_t* __restrict__ capture) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= T) return;
+  constexpr int MAXPER = 8;  // E <= 256
+  float v[MAXPER];
+  uint32_t taken = 0;
+#pragma unroll
+  for (int c = 0; c < MAXPER; ++c) {
+    const int e = c * 32 + lane;
+    float x = -INFINITY;
+    if (e < E) {
+      x = 0.f;
+      for (int s = 0; s < splits; ++s) x += part[(static_cast<size_t>(s) * T + warp) * E + e];
+      if (bias) x += bias[e];
+    }
+    v[c] = x;
+  }
+  float sel_v[16];
+  int sel_i[16];
+  for (int r = 0; r < k; ++r) {
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int c = 0; c < MAXPER; ++c) {
+      const int e = c * 32 + lane;
+      if (e < E && !((taken >> c) & 1) && (v[c] > bv || (v[c] == bv && e < bi) || bi == 0x7fffffff)) {
+        bv = v[c];
+        bi = e;
+      }
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (oi != 0x7fffffff && (bi == 0x7fffffff || ov > bv || (ov == bv && oi < bi))) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    sel_v[r] = bv;
+    sel_i[r] = bi;
+    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+  }
+  if (lane == 0) {
+    float sum = 0.f;
+    float w[16];
+    for (int r = 0; r < k; ++r) {
+      w[r] = __expf(sel_v[r] - sel_v[0]);
+      sum += w[r];
+    }
+    for (int r = 0; r < k; ++r) {
+      idx_out[static_cast<size_t>(warp) * k + r] = sel_i[r];
+      gates_out[static_cast<size_t>(warp) * k + r] = w[r] / sum;
+      if (capture) capture[static_cast<size_t>(warp) * k + r] = sel_i[r];
+    }
+  }
+}
+
+// Stable permutation of the T*k (token, slot) pairs by expert, expert counts,
+// and the grouped GEMM tile lists (the shared expert is group E with all T
+// tokens).  One CTA of 1024 threads.
+//   perm_tok[pos]   token of permuted row pos
+//   inv_slot[p]     permuted row of pair p = t*k + j
+//   gu_tiles: {group, 64-row block, first row, rows}   (gate/up)
+//   dn_tiles: {group, 128-row block, first row, rows}  (down)
+//   counters[0] = gate/up tiles, counters[1] = down tiles, counters[2] = experts hit
+constexpr int PERM_THREADS = 1024;
+constexpr int PERM_MAXE = 256;
+
+__global__ void __launch_bounds__(PERM_THREADS) permute_kernel(const int32_t* __restrict__ idx, int T, int k,
+                                                               int E, int F, int Fs, int d,
+                                                               int32_t* __restrict__ perm_tok,
+                                                               int32_t* __restrict__ inv_slot,
+                                                               int4* __restrict__ gu_tiles,
+                                                               int4* __restrict__ dn_tiles,
+                                                               int32_t* __restrict__ counters) {
+  __shared__ int wcount[32][PERM_MAXE + 1];  // per-warp per-expert counts, then bases
+  __shared__ int offs[PERM_MAXE + 2];
+  __shared__ int gu_off[PERM_MAXE + 2];
+  __shared__ int dn_off[PERM_MAXE + 2];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int npairs = T * k;
+  const int per_warp = (npairs + 31) / 32;
+  const int p_begin = warp * per_warp;
+  const int p_end = min(npairs, p_begin + per_warp);
+  for (int e = lane; e < E; e += 32) wcount[warp][e] = 0;
+  __syncwarp();
+  const unsigned lt = (1u << lane) - 1u;
+  // pass 1: counts per (warp range, expert)
+  for (int c = p_begin; c < p_end; c += 32) {
+    const int p = c + lane;
+    const bool valid = p < p_end;
+    const unsigned act = __ballot_sync(0xffffffffu, valid);
+    if (valid) {
+      const int e = idx[p];
+      const unsigned m = __match_any_sync(act, e);
+      if ((m & lt) == 0) wcount[warp][e] += __popc(m);
+    }
+    __syncwarp();
+  }
+  __syncthreads();
+  // per-expert prefix over warps; totals
+  if (threadIdx.x < E) {
+    const int e = threadIdx.x;
+    int run = 0;
+    for (int w = 0; w < 32; ++w) {
+      const int c = wcount[w][e];
+      wcount[w][e] = run;
+      run += c;
+    }
+    offs[e] = run;  // count, scanned below
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int run = 0, gu = 0, dn = 0, hit = 0;
+    const int mb_gu = F / 64, mb_dn = d / 128;
+    for (int e = 0; e < E; ++e) {
+      const int c = offs[e];
+      offs[e] = run;
+      run += c;
+      const int chunks = (c + 127) / 128;
+      gu_off[e] = gu;
+      dn_off[e] = dn;
+      gu += chunks * mb_gu;
+      dn += chunks * mb_dn;
+      hit += c > 0;
+    }
+    offs[E] = run;
+    // shared expert: all T tokens
+    const int sch = (T + 127) / 128;
+    gu_off[E] = gu;
+    dn_off[E] = dn;
+    gu += sch * (Fs / 64);
+    dn += sch * mb_dn;
+    gu_off[E + 1] = gu;
+    dn_off[E + 1] = dn;
+    counters[0] = gu;
+    counters[1] = dn;
+    counters[2] = hit;
+  }
+  __syncthreads();
+  // pass 2: positions
+  for (int c = p_begin; c < p_end; c += 32) {
+    const int p = c + lane;
+    const bool valid = p < p_end;
+    const unsigned act = __ballot_sync(0xffffffffu, valid);
+    if (valid) {
+      const int e = idx[p];
+      const unsigned m = __match_any_sync(act, e);
+      const int pos = offs[e] + wcount[warp][e] + __popc(m & lt);
+      perm_tok[pos] = p / k;
+      inv_slot[p] = pos;
+      __syncwarp(act);
+      if ((m & lt) == 0) wcount[warp][e] += __popc(m);
+    }
+    __syncwarp();
+  }
+  // tile lists (one thread per group)
+  for (int g = threadIdx.x; g <= E; g += blockDim.x) {
+    const bool shared = g == E;
+    const int first = shared ? 0 : offs[g];
+    const int cnt = shared ? T : offs[g + 1] - offs[g];
+    const int mb_gu = (shared ? Fs : F) / 64, mb_dn = d / 128;
+    int gi = gu_off[g], di = dn_off[g];
+    for (int c0 = 0; c0 < cnt; c0 += 128) {
+      const int rows = min(128, cnt - c0);
+      for (int j = 0; j < mb_gu; ++j) gu_tiles[gi++] = make_int4(g, j, first + c0, rows);
+      for (int j = 0; j < mb_dn; ++j) dn_tiles[di++] = make_int4(g, j, first + c0, rows);
+    }
+  }
+}
+
+// xp[pos] = u[perm_tok[pos]] (bf16 rows of d elements, 16-byte vectors)
+__global__ void gather_rows_kernel(const uint16_t* __restrict__ u, const int32_t* __restrict__ perm_tok,
+                                   int rows, int d, uint16_t* __restrict__ xp) {
+  const int vec = d / 8;
+  const int64_t total = static_cast<int64_t>(rows) * vec;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int r = static_cast<int>(i / vec), c = static_cast<int>(i % vec);
+    const int t = perm_tok[r];
+    reinterpret_cast<uint4*>(xp)[static_cast<size_t>(r) * vec + c] =
+        reinterpret_cast<const uint4*>(u)[static_cast<size_t>(t) * vec + c];
+  }
+}
+
+// h[t] += y_shared[t] + sum_j gate[t][j] * y[inv_slot[t][j]]; u = RMSNorm(h)*gain
+__global__ void combine_norm_kernel(float* __restrict__ h, const float* __restrict__ yp,
+                                    const int32_t* __restrict__ inv_slot, const float* __restrict__ gates,
+                                    int k, int shared_base, int d, const uint16_t* __restrict__ gain, float eps,
+                                    uint16_t* __restrict__ u, float* __restrict__ capture) {
+  __shared__ float red[32];
+  __shared__ int slot[16];
+  __shared__ float gw[16];
+  const int row = blockIdx.x;
+  if (threadIdx.x < k) {
+    slot[threadIdx.x] = inv_slot[static_cast<size_t>(row) * k + threadIdx.x];
+    gw[threadIdx.x] = gates[static_cast<size_t>(row) * k + threadIdx.x];
+  }
+  __syncthreads();
+  float ss = 0.f;
+  for (int j = threadIdx.x; j < d; j += blockDim.x) {
+    float x = h[static_cast<size_t>(row) * d + j];
+    x += yp[static_cast<size_t>(shared_base + row) * d + j];
+    for (int s = 0; s < k; ++s) x += gw[s] * yp[static_cast<size_t>(slot[s]) * d + j];
+    h[static_cast<size_t>(row) * d + j] = x;
+    if (capture) capture[static_cast<size_t>(row) * d + j] = x;
+    ss += x * x;
+  }
+  ss = block_sum(ss, red);
+  const float r = rsqrtf(ss / d + eps);
+  for (int j = threadIdx.x; j < d; j += blockDim.x)
+    u[static_cast<size_t>(row) * d + j] = f32_to_bf16(h[static_cast<size_t>(row) * d + j] * r * bf16_to_f32(gain[j]));
+}
+
+// ---------------------------------------------------------------------------
+// LM-head partial merge + sampler.  Partials are in log2 units:
+// {m1, argmax, m2, sum 2^(x - m1)} per (vocabulary tile, token).
+// ---------------------------------------------------------------------------
+struct Top2 {
+  float m1;
+  int idx;
+  float m2;
+  float s;
+};
+
+__device__ __forceinline__ Top2 top2_merge(Top2 a, Top2 b) {
+  if (b.m1 == -INFINITY) return a;
+  if (a.m1 == -INFINITY) return b;
+  if (b.m1 > a.m1 || (b.m1 == a.m1 && b.idx < a.idx)) {
+    const Top2 t = a;
+    a = b;
+    b = t;
+  }
+  Top2 r;
+  r.m1 = a.m1;
+  r.idx = a.idx;
+  r.m2 = fmaxf(a.m2, b.m1);
+  r.s = a.s + b.s * exp2f(b.m1 - a.m1);
+  return r;
+}
+
+struct SampleArgs {
+  int n_vtiles, T, C, P, step, vocab;
+  uint32_t seed_lo, seed_hi;
+  float tau;
+  int32_t* canvas_out;
+  float* conf_out;
+  int32_t* settled;
+  int32_t* dbg_argmax;
+  float* dbg_lse;
+  float* dbg_conf;
+  float* dbg_margin;
+};
+
+__device__ __forceinline__ int sample_decision(int argmax, float conf, float tau, int pos, int step, int seq,
+                                               uint32_t seed_lo, uint32_t seed_hi, int vocab) {
+  if (conf >= tau) return argmax;  // NaN re-noises
+  const uint4 r = philox4x32_10(make_uint4(static_cast<uint32_t>(pos), static_cast<uint32_t>(step),
+                                           static_cast<uint32_t>(seq), 0u),
+                                make_uint2(seed_lo, seed_hi));
+  return uniform_token(r.x, vocab);
+}
+
+__global__ void lmhead_merge_sample_kernel(const float4* __restrict__ part, SampleArgs a) {
+  __shared__ Top2 sh[32];
+  const int t = blockIdx.x;
+  Top2 acc{-INFINITY, 0x7fffffff, -INFINITY, 0.f};
+  for (int v = threadIdx.x; v < a.n_vtiles; v += blockDim.x) {
+    const float4 p = part[static_cast<size_t>(v) * a.T + t];
+    acc = top2_merge(acc, Top2{p.x, __float_as_int(p.y), p.z, p.w});
+  }
+  for (int o = 16; o > 0; o >>= 1) {
+    Top2 other;
+    other.m1 = __shfl_xor_sync(0xffffffffu, acc.m1, o);
+    other.idx = __shfl_xor_sync(0xffffffffu, acc.idx, o);
+    other.m2 = __shfl_xor_sync(0xffffffffu, acc.m2, o);
+    other.s = __shfl_xor_sync(0xffffffffu, acc.s, o);
+    acc = top2_merge(acc, other);
+  }
+  if ((threadIdx.x & 31) == 0) sh[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < (blockDim.x >> 5); ++w) acc = top2_merge(acc, sh[w]);
+    const float conf = 1.f / acc.s;                      // exp(m1 - lse)
+    const float lse = (acc.m1 + log2f(acc.s)) * 0.69314718055994531f;
+    const float margin = (1.f - exp2f(acc.m2 - acc.m1)) / acc.s;
+    const int b = t / a.C, i = t % a.C;
+    const int out = sample_decision(acc.idx, conf, a.tau, a.P + i, a.step, b, a.seed_lo, a.seed_hi, a.vocab);
+    a.canvas_out[t] = out;
+    if (a.conf_out) a.conf_out[t] = conf;
+    if (a.settled && !(conf >= a.tau)) a.settled[b] = 0;
+    if (a.dbg_argmax) a.dbg_argmax[t] = acc.idx;
+    if (a.dbg_lse) a.dbg_lse[t] = lse;
+    if (a.dbg_conf) a.dbg_conf[t] = conf;
+    if (a.dbg_margin) a.dbg_margin[t] = margin;
+  }
+}
+
+// sampler alone (test hook): given argmax / conf
+__global__ void sample_only_kernel(const int32_t* __restrict__ argmax, const float* __restrict__ conf, int T,
+                                   int C, int P, int step, uint32_t seed_lo, uint32_t seed_hi, float tau,
+                                   int vocab, int32_t* __restrict__ out) {
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= T) return;
+  out[t] = sample_decision(argmax[t], conf[t], tau, P + t % C, step, t / C, seed_lo, seed_hi, vocab);
+}
+
+// waits on a barrier that is never signalled; the bounded wait must give up
+__global__ void wait_timeout_kernel(DevErr err) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, err);
+}
+
+}  // namespace dg

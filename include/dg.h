@@ -1,0 +1,221 @@
+/*
+ * dg.h — C ABI of the block discrete-diffusion denoising step (sm_100a).
+ *
+ * The method is the one described for "DiffusionGemma Technical Report":
+ *   - codemajin.net "DiffusionGemma architecture", section 3.2 (causal encoder
+ *     writes a KV cache; a weight-shared bidirectional decoder denoises the
+ *     256-token block while attending to it; finished blocks are appended to
+ *     the cache and never rewritten);
+ *   - same page, sections 3.1 and 3.3, and aibars.net "Uniform State
+ *     Diffusion" (confident tokens are kept, the rest are reset to uniformly
+ *     random vocabulary tokens);
+ *   - aiboss88.com "hybrid attention architecture" (prefill: causal attention
+ *     that writes the KV cache; denoising: bidirectional attention).
+ *
+ * Conventions common to every call
+ *   - All tensors are row-major.  "bf16" buffers hold IEEE bfloat16 bit
+ *     patterns (uint16_t).  Pointers named *_dev are CUDA device pointers,
+ *     *_host are host pointers.
+ *   - Weights are owned by the caller and must stay valid and unchanged until
+ *     dg_destroy.  The context owns the KV cache and every workspace buffer.
+ *   - Every call is asynchronous on the stream given to dg_create, except
+ *     dg_create, dg_destroy, dg_sync and dg_denoise_step_host, which
+ *     synchronise.  Arguments and capacities are checked on the host before
+ *     anything is launched; a rejected call returns an error and changes no
+ *     state.  Errors raised on the device (a bounded wait that ran out) are
+ *     reported by the next dg_sync as DG_ERR_DEVICE_TIMEOUT.
+ *   - dg_last_error() returns a message for the last failed call on ctx.
+ */
+#ifndef DG_H
+#define DG_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct dg_ctx dg_ctx;
+
+typedef enum dg_status {
+  DG_OK = 0,
+  DG_ERR_INVALID_ARG = 1,    /* a pointer, size or configuration value is out of range   */
+  DG_ERR_OOM = 2,            /* device allocation failed                                  */
+  DG_ERR_CAPACITY = 3,       /* batch or sequence length beyond what dg_create reserved   */
+  DG_ERR_CUDA = 4,           /* a CUDA runtime call failed (message in dg_last_error)     */
+  DG_ERR_DEVICE_TIMEOUT = 5, /* a kernel's bounded wait ran out; outputs are invalid      */
+  DG_ERR_STATE = 6,          /* call out of order (e.g. a step before any prefill)        */
+  DG_ERR_UNSUPPORTED = 7     /* shape the kernels do not support (see dg_config)          */
+} dg_status;
+
+/* Model shape and capacities.
+ * Supported shapes: d_model, expert_hidden and shared_hidden multiples of 64;
+ * head_dim in {64, 128, 176}; n_q_heads a multiple of n_kv_heads; vocab a
+ * multiple of 128; top_k <= 16 and <= n_experts <= 256; canvas a multiple of 16
+ * and <= 256.  The three output projections of a layer are the only places
+ * where a layer writes the residual stream. */
+typedef struct dg_config {
+  int32_t n_layers;
+  int32_t d_model;
+  int32_t n_q_heads;
+  int32_t n_kv_heads;
+  int32_t head_dim;
+  int32_t n_experts;       /* routed experts                                 */
+  int32_t top_k;           /* routed experts per token                       */
+  int32_t expert_hidden;   /* SwiGLU hidden width of a routed expert         */
+  int32_t shared_hidden;   /* SwiGLU hidden width of the shared expert       */
+  int32_t vocab;
+  float rope_base;         /* RoPE base (rotate-half pairs j, j + head_dim/2) */
+  float rms_eps;           /* RMSNorm epsilon                                */
+  float temperature;       /* logits are divided by this before the softmax  */
+  int32_t canvas;          /* tokens per block (256)                         */
+  int32_t max_batch;       /* sequences per call                             */
+  int32_t max_seq;         /* KV-cache capacity per sequence (tokens)        */
+  int32_t prefill_rows;    /* rows per causal chunk in dg_prefill (0: 2048)  */
+} dg_config;
+
+/* One layer's weights, bf16 device pointers, stored [out, in] (row = output).
+ *   attn_norm [d]              RMSNorm gain before attention
+ *   wqkv      [(Hq+2Hkv)*D, d] rows: Hq query heads, then Hkv key heads, then
+ *                              Hkv value heads, head-major, D rows per head
+ *   wo        [d, Hq*D]
+ *   ffn_norm  [d]
+ *   w_router  [E, d]
+ *   w_gate    [E, F, d], w_up [E, F, d], w_down [E, d, F]   routed experts
+ *   ws_gate   [Fs, d],   ws_up [Fs, d],   ws_down [d, Fs]   shared expert   */
+typedef struct dg_layer_weights {
+  const void* attn_norm;
+  const void* wqkv;
+  const void* wo;
+  const void* ffn_norm;
+  const void* w_router;
+  const void* w_gate;
+  const void* w_up;
+  const void* w_down;
+  const void* ws_gate;
+  const void* ws_up;
+  const void* ws_down;
+} dg_layer_weights;
+
+/* Model weights.  embed [V, d] bf16 is also the (tied) LM head.  router_bias
+ * [E] fp32 device pointer or NULL is added to every layer's router logits
+ * before top-k.  layers points to a HOST array of n_layers entries that is
+ * read during dg_create only. */
+typedef struct dg_weights {
+  const void* embed;
+  const void* final_norm;
+  const float* router_bias;
+  const dg_layer_weights* layers;
+} dg_weights;
+
+/* Create a context: validates cfg, allocates the KV cache
+ * ([n_layers][max_batch][n_kv_heads][max_seq][head_dim] bf16 for K and for V)
+ * and all workspaces, builds the RoPE table (angles in double precision) and
+ * the TMA descriptors of every weight.  cuda_stream is a cudaStream_t (NULL:
+ * legacy default stream).  On success *out receives the context. */
+dg_status dg_create(const dg_config* cfg, const dg_weights* weights, void* cuda_stream,
+                    dg_ctx** out);
+
+/* Release every resource of ctx (synchronises its stream first). */
+dg_status dg_destroy(dg_ctx* ctx);
+
+/* Causal encoder (aiboss88.com "hybrid attention architecture"; codemajin.net
+ * section 3.2): reset the cache and encode tokens_dev [batch, prefix_len]
+ * int32, every row attending to itself and the rows before it; keys/values of
+ * all layers are written to cache positions [0, prefix_len).
+ * Needs batch <= max_batch and prefix_len + canvas <= max_seq. */
+dg_status dg_prefill(dg_ctx* ctx, const int32_t* tokens_dev, int32_t batch, int32_t prefix_len);
+
+/* One denoising step over the canvas (codemajin.net sections 3.1-3.3):
+ * canvas_in_dev [batch, canvas] int32 tokens at positions [P, P+canvas) are
+ * run through every layer with bidirectional attention over cache[0,P) plus
+ * the whole canvas; the tied LM head gives, per position, the argmax token a
+ * and the confidence conf = max softmax probability (logits never leave the
+ * chip); the sampler then writes canvas_out = (conf >= tau) ? a : uniform
+ * token, the uniform token drawn by Philox4x32-10 with counter (P+i, step,
+ * sequence, 0) and key (seed low 32 bits, seed high 32 bits).
+ *   conf_dev        [batch, canvas] fp32 (written)
+ *   all_settled_dev [batch] int32 or NULL: 1 where every conf >= tau, else 0.
+ * The committed cache is not modified.  canvas_out_dev may equal
+ * canvas_in_dev; other outputs must not alias inputs.  batch is the batch of
+ * the last dg_prefill. */
+dg_status dg_denoise_step(dg_ctx* ctx, const int32_t* canvas_in_dev, int32_t step, uint64_t seed,
+                          float tau, int32_t* canvas_out_dev, float* conf_dev,
+                          int32_t* all_settled_dev);
+
+/* Same step with HOST buffers: copies canvas_in_host to the device, runs the
+ * step, copies canvas_out/conf/all_settled back and synchronises.  Any of
+ * conf_host and all_settled_host may be NULL. */
+dg_status dg_denoise_step_host(dg_ctx* ctx, const int32_t* canvas_in_host, int32_t step,
+                               uint64_t seed, float tau, int32_t* canvas_out_host,
+                               float* conf_host, int32_t* all_settled_host);
+
+/* Block commit (codemajin.net section 3.2 block-AR; section 5.1 counts it as
+ * one extra forward per block): one causal forward of block_dev
+ * [batch, canvas] int32 at positions [P, P+canvas), appending its keys/values
+ * to the cache; then P += canvas.  Needs P + 2*canvas <= max_seq. */
+dg_status dg_commit_block(dg_ctx* ctx, const int32_t* block_dev);
+
+/* Wait for all work of ctx and report device-side errors. */
+dg_status dg_sync(dg_ctx* ctx);
+
+/* Committed cache length P (tokens per sequence). */
+int32_t dg_cached_len(const dg_ctx* ctx);
+
+/* Message for the last failed call (never NULL). */
+const char* dg_last_error(const dg_ctx* ctx);
+
+/* ---------------------------------------------------------------------------
+ * Test hooks.  Exported for the parity tests; not part of the stable API.
+ * ------------------------------------------------------------------------- */
+
+/* Record, during the following denoising steps, the residual stream after
+ * every layer and the experts chosen in every layer (enable = 1), or stop
+ * recording and free the buffers (enable = 0). */
+dg_status dg_debug_capture(dg_ctx* ctx, int32_t enable);
+
+/* Residual stream of the last recorded step: layer 0 is the embedding, layer
+ * l > 0 the stream after layer l.  out_dev [batch*canvas, d] fp32. */
+dg_status dg_debug_hidden(dg_ctx* ctx, int32_t layer, float* out_dev);
+
+/* Experts of the last recorded step in layer l: out_dev [batch*canvas, top_k]
+ * int32, ordered by (logit desc, index asc). */
+dg_status dg_debug_experts(dg_ctx* ctx, int32_t layer, int32_t* out_dev);
+
+/* LM-head reduction of the last step: per position the argmax (lowest index
+ * of the maximum), log-sum-exp, confidence and top-1 minus top-2
+ * probability.  Each pointer [batch*canvas] or NULL. */
+dg_status dg_debug_lmhead(dg_ctx* ctx, int32_t* argmax_dev, float* lse_dev, float* conf_dev,
+                          float* margin_dev);
+
+/* Router decision alone on given fp32 logits [n_rows, n_experts] (router bias
+ * NOT added): idx_dev [n_rows, top_k] int32, gates_dev [n_rows, top_k] fp32. */
+dg_status dg_debug_router(dg_ctx* ctx, const float* logits_dev, int32_t n_rows, int32_t* idx_dev,
+                          float* gates_dev);
+
+/* Sampler decision alone on given argmax/conf [batch*canvas] (positions
+ * P + i of the current cache length). */
+dg_status dg_debug_sample(dg_ctx* ctx, const int32_t* argmax_dev, const float* conf_dev,
+                          int32_t batch, int32_t step, uint64_t seed, float tau, int32_t* out_dev);
+
+/* Launch a kernel that waits on a barrier nothing ever signals, with a wait
+ * limit of limit_ns nanoseconds; the following dg_sync must report
+ * DG_ERR_DEVICE_TIMEOUT and clear it.  Exercises the failure path of the
+ * bounded waits without faulting the device. */
+dg_status dg_debug_wait_timeout(dg_ctx* ctx, uint64_t limit_ns);
+
+/* One weight-streaming GEMM through the tcgen05 kernel alone:
+ * out_dev [splits, T, M] fp32 holds, for each split s of the K range, the
+ * partial sums of x_dev [T, K] bf16 times w_dev [M, K] bf16 transposed (the
+ * caller adds the splits).  K a multiple of 64, 1 <= splits <= K/64. */
+dg_status dg_debug_gemm(dg_ctx* ctx, const void* w_dev, int32_t M, int32_t K, const void* x_dev, int32_t T,
+                        int32_t splits, float* out_dev);
+
+/* Number of this library's kernel launches issued by ctx so far. */
+int64_t dg_debug_launch_count(const dg_ctx* ctx);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DG_H */

@@ -275,3 +275,18 @@ def uniform_tokens(w: Workload, what: str, n_rows: int, n_cols: int, block: int 
     else:
         t = (h * V) >> 32
     return t.to(torch.int32).view(n_rows, n_cols)
+
+
+def model_weights(w: Workload, device="cpu", layer_override=None, layers=None) -> dict:
+    """All weights of workload `w` as bf16 tensors on `device`, in the layout of
+    the C ABI (dg_weights / dg_layer_weights).  layer_override(l, dict) may
+    replace tensors of a layer (planted cases)."""
+    n = w.shape.n_layers if layers is None else layers
+    out = global_weights(w, device)
+    out["layers"] = []
+    for l in range(n):
+        t = layer_weights(w, l, device)
+        if layer_override is not None:
+            t = layer_override(l, t)
+        out["layers"].append(t)
+    return out

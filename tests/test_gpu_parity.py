@@ -1,0 +1,149 @@
+"""End-to-end parity of the CUDA denoising path with the fp64 oracle.
+
+Criteria (per step): residual stream after every layer within relative L2
+1e-2; expert sets identical except at router near-ties (k-th vs k+1-th logit
+gap < 1e-3); per-position log-probability within 5e-2; sampled tokens
+identical except where the top-1/top-2 probability margin or |conf - tau| is
+below 1e-3.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth_inputs as si
+
+from gpu_helpers import compare_step, gpu_step, make_context, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+
+def _run_workload(w, n_steps, temperature=1.0, report=None, seed=None):
+    """Prefill + n_steps denoising steps on both sides, each side fed its own
+    previous canvas; stops comparing once the two canvases legitimately part
+    (a decision inside the exclusion band)."""
+    seed = w.sample_seed if seed is None else seed
+    ctx, _ = make_context(w, temperature=temperature)
+    orc = oracle.for_workload(w)
+    prefix = si.uniform_tokens(w, "prefix", w.batch, w.prefix)
+    ctx.prefill(prefix.cuda())
+    orc.prefill(prefix.numpy())
+    canvas = si.uniform_tokens(w, "canvas", w.batch, w.canvas).numpy()
+    results = []
+    for s in range(n_steps):
+        tau = si.tau_schedule(w, s)
+        g = gpu_step(ctx, w, canvas, s, seed, tau, capture=True)
+        r = orc.denoise_step(canvas, s, seed, tau, temperature=temperature)
+        results.append(compare_step(g, r, tau, report=report))
+        if not np.array_equal(g["canvas_out"], r.canvas_out):
+            break
+        canvas = r.canvas_out
+    ctx.close()
+    return results
+
+
+def test_tiny_workload_all_steps():
+    rep = []
+    res = _run_workload(si.workload("tiny"), 8, report=rep)
+    print("tiny:", rep)
+    assert len(res) == 8
+
+
+def test_tiny_workload_sharpened_decisions_straddle_tau():
+    """At temperature 0.05 confidences spread across tau, so keep/re-noise
+    decisions of the sampler are exercised on real LM-head output."""
+    rep = []
+    _run_workload(si.workload("tiny"), 4, temperature=0.05, report=rep)
+    print("tiny T=0.05:", rep)
+
+
+def test_tiny_ragged_prefix_and_batch2():
+    w = si.workload("tiny").with_(prefix=200, batch=2)
+    rep = []
+    _run_workload(w, 2, report=rep)
+    print("tiny B2 P200:", rep)
+
+
+def test_small_workload_all_steps():
+    rep = []
+    res = _run_workload(si.workload("small"), 16, report=rep)
+    print("small:", rep)
+    assert len(res) == 16
+
+
+def test_small_workload_sharpened():
+    rep = []
+    _run_workload(si.workload("small"), 3, temperature=0.05, report=rep)
+    print("small T=0.05:", rep)
+
+
+def test_a4b_shape_two_layers_prefix_2048():
+    """Every kernel at the 26B-A4B shapes (d 2816, 128 experts top-8, head_dim
+    176, vocabulary 262144) and prefix 2048, depth reduced to 2 layers so the
+    fp64 oracle runs in seconds."""
+    w = si.workload("a4b_p2k").with_layers(2)
+    rep = []
+    _run_workload(w, 1, report=rep)
+    print("a4b L2:", rep)
+
+
+def test_commit_then_step_matches_oracle_and_prefill_of_concatenation():
+    w = si.workload("tiny").with_(prefix=64)
+    ctx, weights = make_context(w, temperature=0.05)
+    orc = oracle.for_workload(w)
+    prefix = si.uniform_tokens(w, "prefix", 1, 64)
+    block = si.uniform_tokens(w, "canvas", 1, 256, block=7)
+    ctx.prefill(prefix.cuda())
+    orc.prefill(prefix.numpy())
+    ctx.commit_block(block.cuda())
+    orc.commit_block(block.numpy())
+    assert ctx.cached_len == 320 and orc.P == 320
+    canvas = si.uniform_tokens(w, "canvas", 1, 256).numpy()
+    g1 = gpu_step(ctx, w, canvas, 0, 3, 0.9, capture=True)
+    r = orc.denoise_step(canvas, 0, 3, 0.9, temperature=0.05)
+    compare_step(g1, r, 0.9)
+    ctx2, _ = make_context(w, temperature=0.05, weights=weights)
+    ctx2.prefill(torch.cat([prefix, block], 1).cuda())
+    g2 = gpu_step(ctx2, w, canvas, 0, 3, 0.9, capture=True)
+    for l in range(len(g1["hidden"])):
+        assert rel_l2(g1["hidden"][l], g2["hidden"][l]) < 2e-3
+    ctx.close()
+    ctx2.close()
+
+
+def test_step_is_deterministic_and_host_variant_matches():
+    w = si.workload("small")
+    ctx, _ = make_context(w, temperature=0.05)
+    ctx.prefill(si.uniform_tokens(w, "prefix", 1, 1024).cuda())
+    canvas = si.uniform_tokens(w, "canvas", 1, 256).numpy()
+    a = gpu_step(ctx, w, canvas, 2, 5, 0.7)
+    b = gpu_step(ctx, w, canvas, 2, 5, 0.7)
+    np.testing.assert_array_equal(a["canvas_out"], b["canvas_out"])
+    np.testing.assert_array_equal(a["conf"], b["conf"])
+    out = np.empty((1, 256), np.int32)
+    conf = np.empty((1, 256), np.float32)
+    settled = np.empty(1, np.int32)
+    ctx.denoise_step_host(np.ascontiguousarray(canvas, dtype=np.int32), 2, 5, 0.7, out, conf, settled)
+    np.testing.assert_array_equal(out, a["canvas_out"])
+    np.testing.assert_array_equal(conf, a["conf"])
+    assert settled[0] == a["settled"][0]
+    ctx.close()
+
+
+def test_planted_identity_tiny():
+    w = si.workload("tiny").with_(prefix=32)
+
+    def zero_out(l, t):
+        t = dict(t)
+        for k in ("wo", "w_down", "ws_down"):
+            t[k] = torch.zeros_like(t[k])
+        return t
+
+    ctx, _ = make_context(w, temperature=0.05, layer_override=zero_out)
+    ctx.prefill(si.uniform_tokens(w, "prefix", 1, 32).cuda())
+    canvas = si.uniform_tokens(w, "canvas", 1, 256).numpy()
+    g = gpu_step(ctx, w, canvas, 0, 0, 0.9)
+    np.testing.assert_array_equal(g["argmax"], canvas)
+    assert (g["conf"] >= 0.9).all()
+    np.testing.assert_array_equal(g["canvas_out"], canvas)
+    ctx.close()
