@@ -1,0 +1,377 @@
+#!/usr/bin/env python3
+"""Throughput of the block discrete-diffusion denoising step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+
+One step = one dg_denoise_step call: embedding, 30 MoE transformer layers over
+the 256-token canvas with bidirectional attention against the prefix KV cache,
+the tied 262144-vocabulary LM head fused with the argmax / log-sum-exp
+reduction, and the Philox re-noising sampler.  Workload: the 26B-A4B-shaped
+model, batch 1, 2048-token uniform-random prefix (seeded synthetic weights
+and tokens).  Each step streams ~50 GB of weights, far more than the 126 MB
+L2, so no flush is needed between steps.
+
+Multi-GPU: independent replicas (one per rank, no collective on the data
+path); value = canvas tokens of all ranks / max-over-ranks time.
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "canvas tokens denoised/s (batch 1, 256-tok block) and % of step roofline"
+UNIT = "canvas tokens/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--workload", default="a4b_p2k")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained", d["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# algorithmic bytes / flops of one step
+# ---------------------------------------------------------------------------
+def step_cost(w, hits):
+    """bytes: every weight the step must read once (routed experts counted
+    from the experts actually hit, per layer) + the KV cache read; flops:
+    2 x active parameters per token + attention."""
+    s = w.shape
+    d, D, Hq, Hkv = s.d_model, s.head_dim, s.n_q_heads, s.n_kv_heads
+    B, C, P, L = w.batch, w.canvas, w.prefix, s.n_layers
+    attn_w = (s.qkv_dim * d + d * Hq * D) * 2
+    router_w = s.n_experts * d * 2
+    expert_w = 3 * s.expert_hidden * d * 2
+    shared_w = 3 * s.shared_hidden * d * 2
+    lm_w = s.vocab * d * 2
+    kv = L * B * (P + C) * Hkv * D * 2 * 2
+    by = sum(attn_w + router_w + hits[l] * expert_w + shared_w for l in range(L)) + lm_w + kv
+    active = L * (s.qkv_dim * d + d * Hq * D + s.n_experts * d + s.top_k * 3 * s.expert_hidden * d
+                  + 3 * s.shared_hidden * d) + s.vocab * d
+    fl = 2.0 * active * B * C + 4.0 * Hq * D * C * (P + C) * L * B
+    gateup_bytes = sum(hits[l] * 2 * s.expert_hidden * d * 2 + 2 * s.shared_hidden * d * 2
+                       for l in range(L)) / L
+    return by, fl, gateup_bytes
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class Clocks:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--id={index}", f"--query-gpu={self.Q}",
+                                       "--format=csv,noheader,nounits", "-lms", "200"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return None
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.p.kill()
+        self.f.flush()
+        rows = [r.split(",") for r in open(self.f.name).read().strip().splitlines() if r.count(",") >= 8]
+        os.unlink(self.f.name)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows]
+        mx = max(float(r[2]) for r in rows)
+        reasons = set()
+        for r in rows:
+            for name, col in (("hw_slowdown", 5), ("hw_thermal_slowdown", 6), ("sw_thermal_slowdown", 7),
+                              ("sw_power_cap", 8)):
+                if r[col].strip().lower().startswith("active"):
+                    reasons.add(name)
+        loaded = [x for x in sm if x > 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# oracle timing (host cores)
+# ---------------------------------------------------------------------------
+def _cores():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"),
+                default=0)
+        if n:
+            return n
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+class OracleSample:
+    """The fp64 oracle timed on a bounded sample of one step: layer 0 over the
+    whole canvas (scaled by the layer count) and the LM head over a fraction
+    of the vocabulary (scaled up).  Weight generation and the prefix cache are
+    set up once, outside the timing; bf16 -> fp64 weight conversion, which the
+    oracle does as part of its step, is inside."""
+
+    def __init__(self, w):
+        import oracle
+        import synth_inputs as si
+        self.w = w
+        self.orc = oracle.for_workload(w.with_layers(1), keep_layers=True)
+        self.orc.prefill(si.uniform_tokens(w, "prefix", w.batch, w.prefix).numpy())
+        self.canvas = si.uniform_tokens(w, "canvas", w.batch, w.canvas).numpy()
+
+    def run(self, vocab_frac):
+        import numpy as np
+        from oracle.model import _f64, _index, lm_head_stats, rms_norm
+        w, orc = self.w, self.orc
+        for lw in orc._layers.values():          # keep the generated bf16 tensors, redo conversions
+            lw._cache.clear()
+        t0 = time.perf_counter()
+        hs = []
+        for b in range(w.batch):
+            h = _f64(orc.embed[_index(self.canvas[b])])
+            h, _, _ = orc._layer_forward(0, h, b, orc.P, causal=False)
+            hs.append(h)
+        t_layer = time.perf_counter() - t0
+        z = rms_norm(np.concatenate(hs), orc.final_norm, w.shape.rms_eps)
+        V = w.shape.vocab
+        nv = max(128, int(V * vocab_frac)) // 128 * 128
+        t0 = time.perf_counter()
+        lm_head_stats(z, orc.embed[:nv], 1.0)
+        t_lm = (time.perf_counter() - t0) * V / nv
+        t_step = w.shape.n_layers * t_layer + t_lm
+        desc = (f"oracle (fp64 numpy) layer 0 of {w.shape.n_layers} over the {w.batch}x{w.canvas} canvas "
+                f"with the {w.prefix}-token cache ({t_layer:.2f} s, scaled x{w.shape.n_layers}) + LM head "
+                f"over {nv} of {V} vocabulary rows ({t_lm * nv / V:.2f} s, scaled to the full vocabulary)")
+        return w.batch * w.canvas / t_step, t_step, desc
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    vals = []
+    desc = ""
+    sample = OracleSample(w)
+    for i in range(args.warmup + args.steps):
+        v, t, desc = sample.run(vocab_frac=1.0 / 8)
+        if i >= args.warmup:
+            vals.append(t)
+    t = statistics.median(vals)
+    value = w.batch * w.canvas / t
+    cores = _cores()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{w.name}: {w.description}"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# native
+# ---------------------------------------------------------------------------
+def run_native(args, w):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import block_discrete_diffusion_denoise_b200 as dgp
+    import synth_inputs as si
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    stream = torch.cuda.current_stream()
+    weights = si.model_weights(w, "cuda")
+    torch.cuda.synchronize()
+    cfg = dgp.config_from_shape(w.shape, max_batch=w.batch, max_seq=w.prefix + 2 * w.canvas,
+                                canvas=w.canvas)
+    ctx = dgp.Context(cfg, weights, stream=stream.cuda_stream)
+    prefix = si.uniform_tokens(w, "prefix", w.batch, w.prefix, device="cuda")
+    ctx.prefill(prefix)
+    ctx.sync()
+    B, C = w.batch, w.canvas
+    cur = si.uniform_tokens(w, "canvas", B, C, device="cuda")
+    nxt = torch.empty_like(cur)
+    conf = torch.empty(B, C, dtype=torch.float32, device="cuda")
+    settled = torch.empty(B, dtype=torch.int32, device="cuda")
+    seed = w.sample_seed
+
+    # experts actually hit per layer (one recorded step, outside the timing)
+    ctx.debug_capture(True)
+    ctx.denoise_step(cur, 0, seed, w.tau0, nxt, conf, settled)
+    hits = []
+    for l in range(w.shape.n_layers):
+        e = torch.empty(B * C, w.shape.top_k, dtype=torch.int32, device="cuda")
+        ctx.debug_experts(l, e)
+        ctx.sync()
+        hits.append(int(torch.unique(e).numel()))
+    ctx.debug_capture(False)
+
+    for s in range(args.warmup):
+        ctx.denoise_step(cur, s, seed, si.tau_schedule(w, s), nxt, conf, settled)
+        cur, nxt = nxt, cur
+    ctx.sync()
+
+    # ---- timed region: K steps, the expert gate/up GEMM timed per launch ----
+    ctx.debug_profile(["expert_gateup"])
+    clocks = Clocks(local)
+    barrier()
+    torch.cuda.synchronize()
+    n0 = ctx.launch_count
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for s in range(args.steps):
+        ctx.denoise_step(cur, s, seed, si.tau_schedule(w, s % w.steps), nxt, conf, settled)
+        cur, nxt = nxt, cur
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    clk = clocks.stop()
+    launches = (ctx.launch_count - n0) // args.steps
+    prof = ctx.debug_profile_read()
+    ctx.sync()
+    if world > 1:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # ---- per-class breakdown (separate short pass, informational) ----
+    ctx.debug_profile(dgp.PROF_CLASSES)
+    for s in range(2):
+        ctx.denoise_step(cur, s, seed, w.tau0, nxt, conf, settled)
+        cur, nxt = nxt, cur
+    breakdown = {k: round(v[0] / 2, 4) for k, v in ctx.debug_profile_read().items()}
+    ctx.debug_profile([])
+
+    # ---- end to end through the host-buffer entry point ----
+    hin = np.ascontiguousarray(cur.cpu().numpy(), dtype=np.int32)
+    hout = np.empty_like(hin)
+    hconf = np.empty((B, C), np.float32)
+    hset = np.empty(B, np.int32)
+    ctx.denoise_step_host(hin, 0, seed, w.tau0, hout, hconf, hset)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for s in range(args.steps):
+        ctx.denoise_step_host(hin, s, seed, w.tau0, hout, hconf, hset)
+        hin, hout = hout, hin
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / args.steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+        barrier()
+
+    hbm, tf_burst, tf_sus, src = peaks()
+    by, fl, gu_bytes = step_cost(w, hits)
+    gu_ms, gu_n = prof["expert_gateup"]
+    gu_avg_ms = gu_ms / max(gu_n, 1)
+    achieved = gu_bytes / (gu_avg_ms * 1e-3) / 1e9
+    t_roof = max(by / (hbm * 1e9), fl / (tf_sus * 1e12))
+    traffic = None
+    tp = os.path.join(ROOT, "profiles", "expert_gateup_traffic.json")
+    if os.path.exists(tp):
+        try:
+            import hashlib
+            rec = json.load(open(tp))
+            src_hash = hashlib.sha256(open(os.path.join(ROOT, "block_discrete_diffusion_denoise_b200", "csrc",
+                                                        "gemm.cuh"), "rb").read()).hexdigest()
+            if rec.get("gemm_cuh_sha256") == src_hash and rec.get("workload") == w.name:
+                traffic = rec["bytes_per_launch"]
+        except Exception:
+            traffic = None
+    value = world * B * C / (ms * 1e-3)
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"{w.name}: {w.description}", "global_batch": world * B,
+                       "canvas": C, "prefix": w.prefix, "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2 (~50 GB of weights streamed per step)"},
+            "roofline": {"bound": "hbm", "kernel": "expert gate/up GEMM (tcgen05, SwiGLU epilogue)",
+                         "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                         "traffic": traffic, "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)",
+                         "bytes_per_launch": gu_bytes, "launch_ms": gu_avg_ms, "launches": gu_n},
+            "step_roofline": {"bytes": by, "flops": fl, "t_roof_ms": t_roof * 1e3,
+                              "frac": t_roof * 1e3 / ms,
+                              "peaks": f"{src}: HBM {hbm} GB/s, bf16 {tf_sus} TF/s sustained"},
+            "experts_hit_per_layer": hits,
+            "breakdown_ms_per_step": breakdown,
+            "e2e": {"value": world * B * C / (e2e_ms * 1e-3), "unit": UNIT,
+                    "h2d_bytes_per_step": B * C * 4, "d2h_bytes_per_step": B * C * 8 + B * 4,
+                    "ms_per_step": e2e_ms},
+            "gpu_launches": launches * args.steps,
+            "gpu_launches_per_step": launches,
+            "clocks": clk,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            v, t, desc = OracleSample(w).run(vocab_frac=1.0 / 4)
+            line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": _cores(), "kind": "oracle",
+                                    "sample": desc}
+        print(json.dumps(line), flush=True)
+    ctx.close()
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    import synth_inputs as si
+    w = si.workload(args.workload)
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_native(args, w)
+
+
+if __name__ == "__main__":
+    main()

@@ -21,7 +21,11 @@ STATUS = {0: "DG_OK", 1: "DG_ERR_INVALID_ARG", 2: "DG_ERR_OOM", 3: "DG_ERR_CAPAC
 EXPORTS = ["dg_create", "dg_destroy", "dg_prefill", "dg_denoise_step", "dg_denoise_step_host",
            "dg_commit_block", "dg_sync", "dg_cached_len", "dg_last_error", "dg_debug_capture",
            "dg_debug_hidden", "dg_debug_experts", "dg_debug_lmhead", "dg_debug_router",
-           "dg_debug_sample", "dg_debug_wait_timeout", "dg_debug_gemm", "dg_debug_launch_count"]
+           "dg_debug_sample", "dg_debug_wait_timeout", "dg_debug_gemm", "dg_debug_profile",
+           "dg_debug_profile_read", "dg_debug_launch_count"]
+
+# kernel classes of dg_debug_profile (DG_PROF_* in dg.h)
+PROF_CLASSES = ["expert_gateup", "expert_down", "lm_head", "attention", "dense_proj", "other"]
 
 
 class dg_config(ctypes.Structure):
@@ -85,6 +89,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "dg_debug_sample": ([P, P, P, I32, I32, U64, F32, P], I32),
         "dg_debug_wait_timeout": ([P, U64], I32),
         "dg_debug_gemm": ([P, P, I32, I32, P, I32, I32, P], I32),
+        "dg_debug_profile": ([P, I32], I32),
+        "dg_debug_profile_read": ([P, I32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(I64)], I32),
         "dg_debug_launch_count": ([P], I64),
     }
     for name, (args, res) in sig.items():
@@ -197,6 +203,20 @@ class Context:
     def debug_gemm(self, w, x, splits, out):
         M, K = w.shape
         self._check(self.lib.dg_debug_gemm(self.ctx, _ptr(w), M, K, _ptr(x), x.shape[0], int(splits), _ptr(out)))
+
+    def debug_profile(self, classes=()):
+        mask = 0
+        for c in classes:
+            mask |= 1 << (PROF_CLASSES.index(c) if isinstance(c, str) else int(c))
+        self._check(self.lib.dg_debug_profile(self.ctx, mask))
+
+    def debug_profile_read(self) -> dict:
+        out = {}
+        for i, name in enumerate(PROF_CLASSES):
+            ms, n = ctypes.c_double(), ctypes.c_int64()
+            self._check(self.lib.dg_debug_profile_read(self.ctx, i, ctypes.byref(ms), ctypes.byref(n)))
+            out[name] = (ms.value, n.value)
+        return out
 
     @property
     def launch_count(self) -> int:

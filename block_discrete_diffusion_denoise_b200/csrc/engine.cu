@@ -92,6 +92,11 @@ struct dg_ctx {
   uint64_t wait_limit_ns = 1000000000ull;
   int64_t launches = 0;
   std::string last_error;
+  // profiling hook: event pairs per kernel class
+  int prof_mask = 0;
+  std::vector<cudaEvent_t> ev_pool;
+  size_t ev_used = 0;
+  std::vector<std::pair<cudaEvent_t, cudaEvent_t>> prof_pairs[DG_PROF_CLASSES];
 };
 
 namespace {
@@ -149,6 +154,32 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
 
 DevErr dev_err(const dg_ctx* c) { return DevErr{c->err_word, c->wait_limit_ns}; }
 
+// Profiling hook: an event pair around the launches of one kernel class.
+struct ProfScope {
+  dg_ctx* c;
+  int cls;
+  cudaEvent_t stop = nullptr;
+  ProfScope(dg_ctx* ctx, int k) : c(ctx), cls(k) {
+    if (!(c->prof_mask >> cls & 1)) return;
+    if (c->ev_used + 2 > c->ev_pool.size()) {
+      for (int i = 0; i < 64; ++i) {
+        cudaEvent_t e;
+        if (cudaEventCreate(&e) != cudaSuccess) return;
+        c->ev_pool.push_back(e);
+      }
+    }
+    cudaEvent_t start = c->ev_pool[c->ev_used++];
+    stop = c->ev_pool[c->ev_used++];
+    cudaEventRecord(start, c->stream);
+    c->prof_pairs[cls].push_back({start, stop});
+  }
+  void end() {
+    if (stop) cudaEventRecord(stop, c->stream);
+    stop = nullptr;
+  }
+  ~ProfScope() { end(); }
+};
+
 int choose_splits(int tiles, int k_steps, int sms, size_t max_splits_by_cap) {
   int best = 1;
   double best_cost = 1e30;
@@ -183,8 +214,10 @@ dg_status gemm_dense(dg_ctx* c, const CUtensorMap& w, const CUtensorMap& x, int 
   p.out_f32 = c->part;
   p.err = dev_err(c);
   const int grid = std::min(c->sms, p.tiles_static);
+  ProfScope ps0(c, DG_PROF_DENSE);
   gemm_kernel<GEMM_DENSE><<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, c->stream>>>(p);
   DG_LAUNCHED(c);
+  ps0.end();
   *splits_out = p.splits;
   return DG_OK;
 }
@@ -220,6 +253,7 @@ dg_status attention(dg_ctx* c, int l, int B, int n, int pos0, bool causal) {
   p.chunk_len = chunk_len;
   p.n_chunks = n_chunks;
   dim3 grid(qblocks, B * c->Hkv, n_chunks);
+  ProfScope ps1(c, DG_PROF_ATTENTION);
   switch (c->D) {
     case 64:
       attn_kernel<64><<<grid, 128, att_smem_bytes<64>(), c->stream>>>(p);
@@ -234,10 +268,13 @@ dg_status attention(dg_ctx* c, int l, int B, int n, int pos0, bool causal) {
       return fail(c, DG_ERR_UNSUPPORTED, "head_dim %d", c->D);
   }
   DG_LAUNCHED(c);
+  ps1.end();
   if (n_chunks > 1) {
+    ProfScope ps2(c, DG_PROF_ATTENTION);
     attn_merge_kernel<<<static_cast<unsigned>(rows), 64, 0, c->stream>>>(c->opart, c->ml, n_chunks,
                                                                          static_cast<int>(rows), c->D, c->o);
     DG_LAUNCHED(c);
+    ps2.end();
   }
   return DG_OK;
 }
@@ -249,16 +286,22 @@ dg_status moe(dg_ctx* c, int l, int T) {
   dg_status st = gemm_dense(c, lm.wr, c->m_u16, c->E, T, c->d, &s3);
   if (st != DG_OK) return st;
   int32_t* cap = c->capture ? c->cap_idx + static_cast<size_t>(l) * c->R_step * c->k : nullptr;
+  ProfScope ps3(c, DG_PROF_OTHER);
   router_topk_kernel<<<(T * 32 + 255) / 256, 256, 0, c->stream>>>(c->part, s3, T, c->E, c->k, c->router_bias,
                                                                    c->idx, c->gates, cap);
   DG_LAUNCHED(c);
+  ps3.end();
+  ProfScope ps4(c, DG_PROF_OTHER);
   permute_kernel<<<1, PERM_THREADS, 0, c->stream>>>(c->idx, T, c->k, c->E, c->F, c->Fs, c->d, c->perm_tok,
                                                      c->inv_slot, c->gu_tiles, c->dn_tiles, c->counters);
   DG_LAUNCHED(c);
+  ps4.end();
   const int rows = T * c->k;
+  ProfScope ps5(c, DG_PROF_OTHER);
   gather_rows_kernel<<<std::min(4 * c->sms, (rows * (c->d / 8) + 255) / 256), 256, 0, c->stream>>>(
       c->u, c->perm_tok, rows, c->d, c->xp);
   DG_LAUNCHED(c);
+  ps5.end();
   (void)lw;
 
   GemmParams p;
@@ -280,8 +323,10 @@ dg_status moe(dg_ctx* c, int l, int T) {
   p.hs_out = c->hsbuf;
   p.hs_ld = c->Fs;
   p.err = dev_err(c);
+  ProfScope ps6(c, DG_PROF_EXPERT_GATEUP);
   gemm_kernel<GEMM_GATEUP><<<c->sms, GEMM_THREADS, GEMM_SMEM_BYTES, c->stream>>>(p);
   DG_LAUNCHED(c);
+  ps6.end();
 
   memset(&p, 0, sizeof(p));
   p.a_map[0] = lm.wd;
@@ -299,8 +344,10 @@ dg_status moe(dg_ctx* c, int l, int T) {
   p.out_ld = c->d;
   p.shared_row_base = rows;
   p.err = dev_err(c);
+  ProfScope ps7(c, DG_PROF_EXPERT_DOWN);
   gemm_kernel<GEMM_DOWN><<<c->sms, GEMM_THREADS, GEMM_SMEM_BYTES, c->stream>>>(p);
   DG_LAUNCHED(c);
+  ps7.end();
   return DG_OK;
 }
 
@@ -314,10 +361,12 @@ dg_status forward(dg_ctx* c, const int32_t* tokens, int tok_stride, int tok_off,
   const int T = B * n;
   const float eps = c->cfg.rms_eps;
   float* cap0 = (c->capture && !causal) ? c->cap_h : nullptr;
+  ProfScope ps8(c, DG_PROF_OTHER);
   embed_norm_kernel<<<T, 256, 0, c->stream>>>(tokens, tok_stride, tok_off, n, c->embed,
                                                static_cast<const uint16_t*>(c->layers[0].attn_norm), eps, c->d,
-                                               c->h, c->u, cap0, settled, B);
+                                               c->h, c->u, cap0, settled, B, c->V);
   DG_LAUNCHED(c);
+  ps8.end();
   for (int l = 0; l < c->L; ++l) {
     const LayerMaps& lm = c->lmaps[l];
     const dg_layer_weights& lw = c->layers[l];
@@ -325,26 +374,32 @@ dg_status forward(dg_ctx* c, const int32_t* tokens, int tok_stride, int tok_off,
     dg_status st = gemm_dense(c, lm.wqkv, c->m_u16, c->QKV, T, c->d, &s1);
     if (st != DG_OK) return st;
     const size_t layer_off = static_cast<size_t>(l) * c->cfg.max_batch * c->Hkv * c->cfg.max_seq * c->D;
+    ProfScope ps9(c, DG_PROF_OTHER);
     rope_qkv_kernel<<<T, 256, 0, c->stream>>>(c->part, s1, T, n, pos0, c->Hq, c->Hkv, c->D, c->rope, c->q,
                                                c->kcache + layer_off, c->vcache + layer_off, c->cfg.max_seq);
     DG_LAUNCHED(c);
+    ps9.end();
     if (causal && l == c->L - 1) break;  // only this layer's keys/values feed the cache
     st = attention(c, l, B, n, pos0, causal);
     if (st != DG_OK) return st;
     int s2 = 1;
     st = gemm_dense(c, lm.wo, c->m_o16, c->d, T, c->HD, &s2);
     if (st != DG_OK) return st;
+    ProfScope ps10(c, DG_PROF_OTHER);
     residual_norm_kernel<<<T, 256, 0, c->stream>>>(c->h, c->part, s2, T, c->d,
                                                     static_cast<const uint16_t*>(lw.ffn_norm), eps, c->u);
     DG_LAUNCHED(c);
+    ps10.end();
     st = moe(c, l, T);
     if (st != DG_OK) return st;
     const uint16_t* next_gain = l + 1 < c->L ? static_cast<const uint16_t*>(c->layers[l + 1].attn_norm)
                                              : c->final_norm;
     float* cap = (c->capture && !causal) ? c->cap_h + static_cast<size_t>(l + 1) * c->R_step * c->d : nullptr;
+    ProfScope ps11(c, DG_PROF_OTHER);
     combine_norm_kernel<<<T, 256, 0, c->stream>>>(c->h, c->yp, c->inv_slot, c->gates, c->k, T * c->k, c->d,
                                                    next_gain, eps, c->u, cap);
     DG_LAUNCHED(c);
+    ps11.end();
   }
   return DG_OK;
 }
@@ -365,8 +420,10 @@ dg_status lm_head_and_sample(dg_ctx* c, int B, int step, uint64_t seed, float ta
   p.lm_part = c->lm_part;
   p.logit_scale_log2 = static_cast<float>(1.4426950408889634 / static_cast<double>(c->cfg.temperature));
   p.err = dev_err(c);
+  ProfScope ps12(c, DG_PROF_LMHEAD);
   gemm_kernel<GEMM_LMHEAD><<<std::min(c->sms, p.tiles_static), GEMM_THREADS, GEMM_SMEM_BYTES, c->stream>>>(p);
   DG_LAUNCHED(c);
+  ps12.end();
   SampleArgs a;
   a.n_vtiles = n_vtiles;
   a.T = T;
@@ -384,8 +441,10 @@ dg_status lm_head_and_sample(dg_ctx* c, int B, int step, uint64_t seed, float ta
   a.dbg_lse = c->dbg_lse;
   a.dbg_conf = c->dbg_conf;
   a.dbg_margin = c->dbg_margin;
+  ProfScope ps13(c, DG_PROF_OTHER);
   lmhead_merge_sample_kernel<<<T, 256, 0, c->stream>>>(c->lm_part, a);
   DG_LAUNCHED(c);
+  ps13.end();
   return DG_OK;
 }
 
@@ -410,6 +469,8 @@ dg_status set_smem_attrs(dg_ctx* c) {
 }
 
 void free_all(dg_ctx* c) {
+  for (cudaEvent_t e : c->ev_pool) cudaEventDestroy(e);
+  c->ev_pool.clear();
   if (c->ws) cudaFree(c->ws);
   if (c->kcache) cudaFree(c->kcache);
   if (c->vcache) cudaFree(c->vcache);
@@ -810,6 +871,30 @@ dg_status dg_debug_gemm(dg_ctx* c, const void* w, int32_t M, int32_t K, const vo
   p.err = dev_err(c);
   gemm_kernel<GEMM_DENSE><<<std::min(c->sms, p.tiles_static), GEMM_THREADS, GEMM_SMEM_BYTES, c->stream>>>(p);
   DG_LAUNCHED(c);
+  return DG_OK;
+}
+
+dg_status dg_debug_profile(dg_ctx* c, int32_t mask) {
+  if (!c) return DG_ERR_INVALID_ARG;
+  DG_CUDA(c, cudaStreamSynchronize(c->stream));
+  for (auto& v : c->prof_pairs) v.clear();
+  c->ev_used = 0;
+  c->prof_mask = mask;
+  return DG_OK;
+}
+
+dg_status dg_debug_profile_read(dg_ctx* c, int32_t cls, double* total_ms, int64_t* launches) {
+  if (!c || cls < 0 || cls >= DG_PROF_CLASSES || !total_ms || !launches)
+    return fail(c, DG_ERR_INVALID_ARG, "profile_read");
+  DG_CUDA(c, cudaStreamSynchronize(c->stream));
+  double t = 0.0;
+  for (auto& pr : c->prof_pairs[cls]) {
+    float ms = 0.f;
+    DG_CUDA(c, cudaEventElapsedTime(&ms, pr.first, pr.second));
+    t += ms;
+  }
+  *total_ms = t;
+  *launches = static_cast<int64_t>(c->prof_pairs[cls].size());
   return DG_OK;
 }
 

@@ -38,12 +38,13 @@ __device__ __forceinline__ int uniform_token(uint32_t w, int vocab) {
 __global__ void embed_norm_kernel(const int32_t* __restrict__ tokens, int tok_stride, int tok_off, int n,
                                   const uint16_t* __restrict__ embed, const uint16_t* __restrict__ gain,
                                   float eps, int d, float* __restrict__ h, uint16_t* __restrict__ u,
-                                  float* __restrict__ capture, int32_t* settled, int n_settled) {
+                                  float* __restrict__ capture, int32_t* settled, int n_settled, int vocab) {
   __shared__ float red[32];
   const int row = blockIdx.x;
   const int b = row / n, i = row % n;
   if (settled != nullptr && row == 0 && threadIdx.x < n_settled) settled[threadIdx.x] = 1;
-  const int tok = tokens[static_cast<size_t>(b) * tok_stride + tok_off + i];
+  // out-of-range ids are clamped into the vocabulary rather than read out of bounds
+  const int tok = min(max(tokens[static_cast<size_t>(b) * tok_stride + tok_off + i], 0), vocab - 1);
   const uint16_t* e = embed + static_cast<size_t>(tok) * d;
   float ss = 0.f;
   for (int j = threadIdx.x; j < d; j += blockDim.x) {

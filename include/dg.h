@@ -211,6 +211,26 @@ dg_status dg_debug_wait_timeout(dg_ctx* ctx, uint64_t limit_ns);
 dg_status dg_debug_gemm(dg_ctx* ctx, const void* w_dev, int32_t M, int32_t K, const void* x_dev, int32_t T,
                         int32_t splits, float* out_dev);
 
+/* Kernel classes timed by the profiling hooks. */
+enum {
+  DG_PROF_EXPERT_GATEUP = 0, /* grouped routed + shared expert gate/up GEMM (SwiGLU epilogue) */
+  DG_PROF_EXPERT_DOWN = 1,   /* grouped expert down GEMM                                      */
+  DG_PROF_LMHEAD = 2,        /* LM-head GEMM with the argmax / log-sum-exp epilogue            */
+  DG_PROF_ATTENTION = 3,     /* attention kernel (+ chunk merge)                               */
+  DG_PROF_DENSE = 4,         /* QKV, output and router projections                            */
+  DG_PROF_OTHER = 5,         /* norms, RoPE, routing, gather, combine, sampler                */
+  DG_PROF_CLASSES = 6
+};
+
+/* Start (enable = class mask, bit c for class c) or stop (0) recording a CUDA
+ * event pair on the context stream around every launch of the selected
+ * classes; starting clears the totals. */
+dg_status dg_debug_profile(dg_ctx* ctx, int32_t class_mask);
+
+/* Synchronise and return, for one class, the summed device time (ms) and the
+ * number of launches recorded since dg_debug_profile. */
+dg_status dg_debug_profile_read(dg_ctx* ctx, int32_t cls, double* total_ms, int64_t* launches);
+
 /* Number of this library's kernel launches issued by ctx so far. */
 int64_t dg_debug_launch_count(const dg_ctx* ctx);
 

@@ -70,35 +70,84 @@ def gpu_step(ctx, w, canvas, step, seed, tau, capture=False):
     return res
 
 
-def compare_step(g: dict, r: "oracle.StepResult", tau: float, check_hidden=True, report=None):
-    """Apply the criteria; returns a dict of measured errors (asserts inside)."""
+def _rms_rows(h):
+    return np.sqrt(np.mean(h * h, axis=-1, keepdims=True) + 1e-6)
+
+
+def compare_step(g: dict, r: "oracle.StepResult", tau: float, orc=None, check_hidden=True, report=None,
+                 temperature: float = 1.0):
+    """Apply the criteria; returns a dict of measured errors (asserts at the end).
+
+    Router near-ties.  The GPU feeds the router bf16 operands derived from its
+    own fp32 residual stream, the oracle fp64 ones; where the oracle's k-th and
+    (k+1)-th logits are closer than the perturbation those input differences
+    can cause, the two may legitimately pick different experts.  The bound
+    used is Cauchy-Schwarz: |d(r_a - r_b)| <= ||W_r[a] - W_r[b]|| * ||du||, with
+    ||du|| = (drift of the normalised residual measured at the layer's input and
+    output) + the bf16 rounding bound 2^-8 ||u||.  A flip beyond the bound is a
+    failure; a token within it is counted and, from that layer on, left out of
+    the hidden-state and log-probability comparisons (its residual stream has
+    legitimately left the oracle's).
+    """
     out = {}
+    B, C = r.canvas_out.shape
+    diverged = np.zeros((B, C), dtype=bool)
+    fails = []
     if check_hidden and "hidden" in g:
-        errs = [rel_l2(g["hidden"][l], r.hidden[l]) for l in range(len(r.hidden))]
-        out["hidden_rel_l2_max"] = max(errs)
-        out["hidden_rel_l2"] = errs
-        # expert sets: equal wherever the oracle's k-th/k+1-th logit gap is not a near tie
+        errs = [rel_l2(g["hidden"][0], r.hidden[0])]
+        errs_all = list(errs)
         flips = 0
         for l in range(len(r.experts)):
             ge = np.sort(g["experts"][l], axis=-1)
             oe = np.sort(r.experts[l], axis=-1)
-            diff = (ge != oe).any(axis=-1)
-            near = r.router_margin[l] < EXCLUDE_BAND
-            bad = diff & ~near
+            diff = (ge != oe).any(axis=-1) & ~diverged
+            if diff.any():
+                assert orc is not None, "router flip found; pass the oracle to bound it"
+                wr = orc.layer(l)["w_router"]
+                du = np.zeros((B, C))
+                for hh in (l, l + 1):
+                    ug = g["hidden"][hh] / _rms_rows(g["hidden"][hh])
+                    uo = r.hidden[hh] / _rms_rows(r.hidden[hh])
+                    du = np.maximum(du, np.linalg.norm(ug - uo, axis=-1))
+                du = du + 2.0 ** -8 * np.sqrt(r.hidden[0].shape[-1])
+                srt = np.argsort(-r.router_logits[l], axis=-1, kind="stable")
+                k = r.experts[l].shape[-1]
+                for b, t in zip(*np.nonzero(diff)):
+                    ea, eb = srt[b, t, k - 1], srt[b, t, k]
+                    bound = np.linalg.norm(wr[ea] - wr[eb]) * du[b, t]
+                    gap = r.router_margin[l][b, t]
+                    if gap > bound:
+                        fails.append(f"layer {l} token {b},{t}: expert gap {gap:.4g} > bound {bound:.4g}")
             flips += int(diff.sum())
-            assert not bad.any(), f"layer {l}: {int(bad.sum())} tokens with different experts (no near tie)"
+            diverged |= diff
+            keep = ~diverged
+            errs.append(rel_l2(g["hidden"][l + 1][keep], r.hidden[l + 1][keep]))
+            errs_all.append(rel_l2(g["hidden"][l + 1], r.hidden[l + 1]))
+        out["hidden_rel_l2_max"] = max(errs)
+        out["hidden_rel_l2"] = errs
+        out["hidden_rel_l2_all_tokens"] = errs_all
         out["expert_flips"] = flips
-        assert out["hidden_rel_l2_max"] <= HIDDEN_REL_L2, errs
-    logp_g = -np.log(np.maximum(g["conf"].astype(np.float64), 1e-38))
-    logp_o = -r.logp
-    out["logp_abs_max"] = float(np.abs(logp_g - logp_o).max())
-    assert out["logp_abs_max"] <= LOGP_ABS, out["logp_abs_max"]
-    excl = (r.margin < EXCLUDE_BAND) | (np.abs(r.conf - tau) < EXCLUDE_BAND)
+        if out["hidden_rel_l2_max"] > HIDDEN_REL_L2:
+            fails.append(f"hidden rel-L2 {out['hidden_rel_l2_max']:.4g} > {HIDDEN_REL_L2}")
+    keep = ~diverged
+    logp_g = np.log(np.maximum(g["conf"].astype(np.float64), 1e-38))
+    dlogp = np.abs(logp_g - r.logp)
+    out["logp_abs_max"] = float(dlogp[keep].max()) if keep.any() else 0.0
+    out["logp_abs_max_all_tokens"] = float(dlogp.max())
+    # logits are divided by the temperature before the softmax, so their
+    # rounding error (and that of logp) scales with 1/T; the bound is stated at T=1
+    logp_tol = LOGP_ABS / min(1.0, temperature)
+    if out["logp_abs_max"] > logp_tol:
+        fails.append(f"logp max abs {out['logp_abs_max']:.4g} > {logp_tol:.4g}")
+    excl = (r.margin < EXCLUDE_BAND) | (np.abs(r.conf - tau) < EXCLUDE_BAND) | diverged
     mism = g["canvas_out"] != r.canvas_out
     out["token_mismatch"] = int((mism & ~excl).sum())
     out["excluded"] = int(excl.sum())
     out["excluded_mismatch"] = int((mism & excl).sum())
-    assert out["token_mismatch"] == 0, out
+    if out["token_mismatch"]:
+        fails.append(f"{out['token_mismatch']} token decisions differ outside the exclusion band")
     if report is not None:
         report.append(out)
+    print({k: v for k, v in out.items()})
+    assert not fails, fails
     return out

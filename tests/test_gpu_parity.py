@@ -1,10 +1,12 @@
 """End-to-end parity of the CUDA denoising path with the fp64 oracle.
 
 Criteria (per step): residual stream after every layer within relative L2
-1e-2; expert sets identical except at router near-ties (k-th vs k+1-th logit
-gap < 1e-3); per-position log-probability within 5e-2; sampled tokens
-identical except where the top-1/top-2 probability margin or |conf - tau| is
-below 1e-3.
+1e-2; per-position log-probability within 5e-2 (at temperature T the bound is
+5e-2/T, since logit rounding scales with 1/T); sampled tokens identical except
+where the top-1/top-2 probability margin or |conf - tau| is below 1e-3.  A
+token whose routed expert set differs from the oracle's must sit within the
+arithmetic perturbation bound of a router near-tie (see compare_step); it is
+then counted and left out of the later comparisons.
 """
 import numpy as np
 import pytest
@@ -34,7 +36,7 @@ def _run_workload(w, n_steps, temperature=1.0, report=None, seed=None):
         tau = si.tau_schedule(w, s)
         g = gpu_step(ctx, w, canvas, s, seed, tau, capture=True)
         r = orc.denoise_step(canvas, s, seed, tau, temperature=temperature)
-        results.append(compare_step(g, r, tau, report=report))
+        results.append(compare_step(g, r, tau, orc=orc, report=report, temperature=temperature))
         if not np.array_equal(g["canvas_out"], r.canvas_out):
             break
         canvas = r.canvas_out
@@ -101,7 +103,7 @@ def test_commit_then_step_matches_oracle_and_prefill_of_concatenation():
     canvas = si.uniform_tokens(w, "canvas", 1, 256).numpy()
     g1 = gpu_step(ctx, w, canvas, 0, 3, 0.9, capture=True)
     r = orc.denoise_step(canvas, 0, 3, 0.9, temperature=0.05)
-    compare_step(g1, r, 0.9)
+    compare_step(g1, r, 0.9, orc=orc, temperature=0.05)
     ctx2, _ = make_context(w, temperature=0.05, weights=weights)
     ctx2.prefill(torch.cat([prefix, block], 1).cuda())
     g2 = gpu_step(ctx2, w, canvas, 0, 3, 0.9, capture=True)
