@@ -22,7 +22,7 @@ EXPORTS = ["dg_create", "dg_destroy", "dg_prefill", "dg_denoise_step", "dg_denoi
            "dg_commit_block", "dg_sync", "dg_cached_len", "dg_last_error", "dg_debug_capture",
            "dg_debug_hidden", "dg_debug_experts", "dg_debug_lmhead", "dg_debug_router",
            "dg_debug_sample", "dg_debug_wait_timeout", "dg_debug_gemm", "dg_debug_profile",
-           "dg_debug_profile_read", "dg_debug_launch_count"]
+           "dg_debug_profile_read", "dg_debug_launch_count", "dg_lmhead_argmax_static"]
 
 # kernel classes of dg_debug_profile (DG_PROF_* in dg.h)
 PROF_CLASSES = ["expert_gateup", "expert_down", "lm_head", "attention", "dense_proj", "other"]
@@ -92,6 +92,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "dg_debug_profile": ([P, I32], I32),
         "dg_debug_profile_read": ([P, I32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(I64)], I32),
         "dg_debug_launch_count": ([P], I64),
+        "dg_lmhead_argmax_static": ([P, I32, I32, P, I32, F32, P, P, P, P], I32),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -231,3 +232,12 @@ def config_from_shape(shape, max_batch=1, max_seq=4096, canvas=256, temperature=
                 vocab=shape.vocab, rope_base=shape.rope_base, rms_eps=shape.rms_eps,
                 temperature=temperature, canvas=canvas, max_batch=max_batch, max_seq=max_seq,
                 prefill_rows=prefill_rows)
+
+
+def lmhead_argmax_static(z, embed, temperature, argmax=None, lse=None, conf=None, stream=None) -> int:
+    """dg_lmhead_argmax_static on torch CUDA tensors; returns the dg_status
+    code (0 = launched).  No device memory is allocated by the library."""
+    lib = load_library()
+    n_rows, d = z.shape
+    return lib.dg_lmhead_argmax_static(_ptr(z), n_rows, d, _ptr(embed), embed.shape[0], float(temperature),
+                                       _ptr(argmax), _ptr(lse), _ptr(conf), stream)

@@ -901,3 +901,108 @@ dg_status dg_debug_profile_read(dg_ctx* c, int32_t cls, double* total_ms, int64_
 int64_t dg_debug_launch_count(const dg_ctx* c) { return c ? c->launches : -1; }
 
 }  // extern "C"
+
+// =============================================================================
+// LM-head reduction that allocates nothing (dg_lmhead_argmax_static).
+//
+// Some callers cannot allocate device memory at the time they need this: code
+// that runs while another framework records a CUDA graph (allocation is not
+// allowed inside the capture), processes whose caching allocator has already
+// reserved the whole device, or embedded deployments that fix every byte of
+// device memory at start-up.  For them the per-(vocabulary tile, row)
+// partials of the LM-head reduction live in a fixed array in the library's
+// own device image instead of a context workspace.
+// =============================================================================
+namespace {
+
+constexpr size_t kLmStaticPartials = 524288;  // float4 entries = 8 MiB: n_rows * vocab / 128 <= this
+
+// Shared by every call on a device (the library image holds it until exit).
+static __device__ __align__(256) float4 g_lm_static_partials[kLmStaticPartials];
+static __device__ __align__(256) int g_lm_static_err[4];
+
+constexpr int kMaxDevices = 64;
+struct StaticSetup {
+  bool done = false;
+  float4* partials = nullptr;  // device address of g_lm_static_partials on this device
+  int* err = nullptr;          // device address of g_lm_static_err on this device
+  int sms = 0;
+};
+StaticSetup g_static_setup[kMaxDevices];
+
+// merge of the partials into argmax / lse / conf (rows flagged by a timed-out
+// wait get argmax -1 and NaN statistics)
+__global__ void lmhead_static_merge_kernel(const float4* __restrict__ part, int n_vtiles, int T,
+                                           const int* __restrict__ err, int32_t* __restrict__ argmax,
+                                           float* __restrict__ lse, float* __restrict__ conf) {
+  __shared__ Top2 sh[32];
+  const int t = blockIdx.x;
+  Top2 acc{-INFINITY, 0x7fffffff, -INFINITY, 0.f};
+  for (int v = threadIdx.x; v < n_vtiles; v += blockDim.x) {
+    const float4 p = part[static_cast<size_t>(v) * T + t];
+    acc = top2_merge(acc, Top2{p.x, __float_as_int(p.y), p.z, p.w});
+  }
+  for (int o = 16; o > 0; o >>= 1) {
+    Top2 other;
+    other.m1 = __shfl_xor_sync(0xffffffffu, acc.m1, o);
+    other.idx = __shfl_xor_sync(0xffffffffu, acc.idx, o);
+    other.m2 = __shfl_xor_sync(0xffffffffu, acc.m2, o);
+    other.s = __shfl_xor_sync(0xffffffffu, acc.s, o);
+    acc = top2_merge(acc, other);
+  }
+  if ((threadIdx.x & 31) == 0) sh[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < (blockDim.x >> 5); ++w) acc = top2_merge(acc, sh[w]);
+    const bool bad = err[0] != 0;
+    if (argmax) argmax[t] = bad ? -1 : acc.idx;
+    if (lse) lse[t] = bad ? NAN : (acc.m1 + log2f(acc.s)) * 0.69314718055994531f;
+    if (conf) conf[t] = bad ? NAN : 1.f / acc.s;
+  }
+}
+
+}  // namespace
+
+extern "C" dg_status dg_lmhead_argmax_static(const void* z, int32_t n_rows, int32_t d_model, const void* embed,
+                                             int32_t vocab, float temperature, int32_t* argmax_out,
+                                             float* lse_out, float* conf_out, void* cuda_stream) {
+  if (!z || !embed || n_rows <= 0 || d_model <= 0 || d_model % 64 || vocab <= 0 || vocab % GEMM_BN ||
+      !(temperature > 0.f) || !aligned16(z) || !aligned16(embed) || (!argmax_out && !lse_out && !conf_out))
+    return DG_ERR_INVALID_ARG;
+  const int n_vtiles = vocab / GEMM_BN;
+  if (static_cast<size_t>(n_vtiles) * static_cast<size_t>(n_rows) > kLmStaticPartials)
+    return DG_ERR_CAPACITY;  // n_rows * vocab / 128 beyond the fixed scratch
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DG_ERR_CUDA;
+  StaticSetup& su = g_static_setup[dev];
+  if (!su.done) {
+    // once per device, with that device current (the caller's current device)
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&su.partials), g_lm_static_partials) != cudaSuccess ||
+        cudaGetSymbolAddress(reinterpret_cast<void**>(&su.err), g_lm_static_err) != cudaSuccess ||
+        cudaDeviceGetAttribute(&su.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaFuncSetAttribute(gemm_kernel<GEMM_LMHEAD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             GEMM_SMEM_BYTES) != cudaSuccess)
+      return DG_ERR_CUDA;
+    su.done = true;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  GemmParams p;
+  memset(&p, 0, sizeof(p));
+  if (!make_map(&p.a_map[0], z, n_rows, d_model, 128) || !make_map(&p.b_map, embed, vocab, d_model, 128))
+    return DG_ERR_CUDA;
+  p.b_box_rows = 128;
+  p.M = n_rows;
+  p.k_steps = d_model / 64;
+  p.n_mtiles = (n_rows + GEMM_BM - 1) / GEMM_BM;
+  p.tiles_static = n_vtiles * p.n_mtiles;
+  p.lm_part = su.partials;
+  p.logit_scale_log2 = static_cast<float>(1.4426950408889634 / static_cast<double>(temperature));
+  p.err = DevErr{su.err, 1000000000ull};
+  if (cudaMemsetAsync(su.err, 0, sizeof(int), st) != cudaSuccess) return DG_ERR_CUDA;
+  gemm_kernel<GEMM_LMHEAD><<<std::min(su.sms, p.tiles_static), GEMM_THREADS, GEMM_SMEM_BYTES, st>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return DG_ERR_CUDA;
+  lmhead_static_merge_kernel<<<n_rows, 256, 0, st>>>(su.partials, n_vtiles, n_rows, su.err, argmax_out, lse_out,
+                                                     conf_out);
+  if (cudaGetLastError() != cudaSuccess) return DG_ERR_CUDA;
+  return DG_OK;
+}

@@ -234,6 +234,43 @@ dg_status dg_debug_profile_read(dg_ctx* ctx, int32_t cls, double* total_ms, int6
 /* Number of this library's kernel launches issued by ctx so far. */
 int64_t dg_debug_launch_count(const dg_ctx* ctx);
 
+/* ---------------------------------------------------------------------------
+ * LM-head reduction without any device allocation.
+ *
+ * The pages describe nothing like this; it is a deployment convenience.  It
+ * serves callers that cannot allocate device memory when they need the
+ * reduction: code running while another framework records a CUDA graph
+ * (allocation is forbidden inside the capture), processes whose caching
+ * allocator already holds the whole device, or embedded deployments that fix
+ * all device memory at start-up.
+ *
+ * Computes, for each of the n_rows rows of z_dev [n_rows, d_model] bf16, the
+ * logits z . embed^T / temperature over embed_dev [vocab, d_model] bf16 (the
+ * tied LM head) without writing them, and returns argmax_dev [n_rows] int32
+ * (lowest index of the maximum), lse_dev [n_rows] fp32 (log-sum-exp) and
+ * conf_dev [n_rows] fp32 (maximum softmax probability); any of the three may
+ * be NULL but not all.  It runs the same tcgen05 LM-head kernel as
+ * dg_denoise_step, asynchronously on cuda_stream (a cudaStream_t, NULL = the
+ * legacy default stream), with its partials in a fixed 8 MiB array inside the
+ * library (n_rows * vocab / 128 <= 524288, e.g. 256 rows of a 262144-token
+ * vocabulary).  Nothing is allocated and no context is needed.
+ *   - Larger problems are rejected with DG_ERR_CAPACITY before any launch;
+ *     malformed arguments (d_model not a multiple of 64, vocab not a multiple
+ *     of 128, unaligned pointers) with DG_ERR_INVALID_ARG.
+ *   - The first call on a device looks up the array's device address and sets
+ *     the kernel attributes for that device (the device current at the call);
+ *     make that first call before any stream capture.
+ *   - Every call on a device shares the one array, whose contents persist
+ *     between calls: each call writes every partial it later reads and clears
+ *     its own error flag first, but calls that overlap on the GPU (different
+ *     streams, or several host threads) race on the array and must be
+ *     serialised by the caller.
+ *   - If a bounded wait inside the kernel ran out, the rows come back with
+ *     argmax -1 and NaN statistics.  */
+dg_status dg_lmhead_argmax_static(const void* z_dev, int32_t n_rows, int32_t d_model, const void* embed_dev,
+                                  int32_t vocab, float temperature, int32_t* argmax_dev, float* lse_dev,
+                                  float* conf_dev, void* cuda_stream);
+
 #ifdef __cplusplus
 }
 #endif
