@@ -196,7 +196,8 @@ int choose_splits(int tiles, int k_steps, int sms, size_t max_splits_by_cap) {
 }
 
 // out[s][t][m] = partial sums over split s of W[m, :] . X[t, :]
-dg_status gemm_dense(dg_ctx* c, const CUtensorMap& w, const CUtensorMap& x, int M, int T, int K, int* splits_out) {
+dg_status gemm_dense(dg_ctx* c, const CUtensorMap& w, const CUtensorMap& x, int M, int T, int K, int* splits_out,
+                     int max_splits = 8) {
   GemmParams p;
   memset(&p, 0, sizeof(p));
   p.a_map[0] = w;
@@ -209,7 +210,7 @@ dg_status gemm_dense(dg_ctx* c, const CUtensorMap& w, const CUtensorMap& x, int 
   p.n_tiles_n = (T + p.bn - 1) / p.bn;
   const int m_tiles = (M + GEMM_BM - 1) / GEMM_BM;
   const size_t cap_s = c->part_cap / (static_cast<size_t>(T) * M);
-  p.splits = choose_splits(m_tiles * p.n_tiles_n, p.k_steps, c->sms, cap_s);
+  p.splits = choose_splits(m_tiles * p.n_tiles_n, p.k_steps, c->sms, std::min<size_t>(cap_s, max_splits));
   p.tiles_static = m_tiles * p.n_tiles_n * p.splits;
   p.out_f32 = c->part;
   p.err = dev_err(c);
@@ -283,7 +284,7 @@ dg_status moe(dg_ctx* c, int l, int T) {
   const LayerMaps& lm = c->lmaps[l];
   const dg_layer_weights& lw = c->layers[l];
   int s3 = 1;
-  dg_status st = gemm_dense(c, lm.wr, c->m_u16, c->E, T, c->d, &s3);
+  dg_status st = gemm_dense(c, lm.wr, c->m_u16, c->E, T, c->d, &s3, 4);
   if (st != DG_OK) return st;
   int32_t* cap = c->capture ? c->cap_idx + static_cast<size_t>(l) * c->R_step * c->k : nullptr;
   ProfScope ps3(c, DG_PROF_OTHER);
@@ -507,7 +508,7 @@ dg_status dg_create(const dg_config* cfg, const dg_weights* w, void* cuda_stream
       g.max_batch <= 0 || g.max_seq <= 0 || !(g.rms_eps >= 0.f) || !(g.temperature > 0.f) ||
       !(g.rope_base > 0.f))
     return reject(DG_ERR_INVALID_ARG, "non-positive dimension");
-  if (g.d_model % 128 || g.expert_hidden % 64 || g.shared_hidden % 64 || g.vocab % 128 ||
+  if (g.d_model % 128 || g.d_model > 4096 || g.expert_hidden % 64 || g.shared_hidden % 64 || g.vocab % 128 ||
       (g.head_dim != 64 && g.head_dim != 128 && g.head_dim != 176) || g.n_q_heads % g.n_kv_heads ||
       (g.n_q_heads * g.head_dim) % 64 || g.n_experts > PERM_MAXE || g.top_k > 16 || g.top_k > g.n_experts ||
       g.canvas % 16 || g.canvas > 256 || g.max_seq < g.canvas)

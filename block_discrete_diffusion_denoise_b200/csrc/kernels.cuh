@@ -31,101 +31,6 @@ __device__ __forceinline__ int uniform_token(uint32_t w, int vocab) {
   return static_cast<int>((static_cast<uint64_t>(w) * static_cast<uint64_t>(vocab)) >> 32);
 }
 
-// ---------------------------------------------------------------------------
-// embedding gather (bf16 -> fp32 residual) + RMSNorm -> bf16
-// tokens[b * tok_stride + tok_off + i], row = b * n + i
-// ---------------------------------------------------------------------------
-__global__ void embed_norm_kernel(const int32_t* __restrict__ tokens, int tok_stride, int tok_off, int n,
-                                  const uint16_t* __restrict__ embed, const uint16_t* __restrict__ gain,
-                                  float eps, int d, float* __restrict__ h, uint16_t* __restrict__ u,
-                                  float* __restrict__ capture, int32_t* settled, int n_settled, int vocab) {
-  __shared__ float red[32];
-  const int row = blockIdx.x;
-  const int b = row / n, i = row % n;
-  if (settled != nullptr && row == 0 && threadIdx.x < n_settled) settled[threadIdx.x] = 1;
-  // out-of-range ids are clamped into the vocabulary rather than read out of bounds
-  const int tok = min(max(tokens[static_cast<size_t>(b) * tok_stride + tok_off + i], 0), vocab - 1);
-  const uint16_t* e = embed + static_cast<size_t>(tok) * d;
-  float ss = 0.f;
-  for (int j = threadIdx.x; j < d; j += blockDim.x) {
-    const float x = bf16_to_f32(e[j]);
-    h[static_cast<size_t>(row) * d + j] = x;
-    if (capture) capture[static_cast<size_t>(row) * d + j] = x;
-    ss += x * x;
-  }
-  ss = block_sum(ss, red);
-  const float r = rsqrtf(ss / d + eps);
-  for (int j = threadIdx.x; j < d; j += blockDim.x) {
-    const float x = h[static_cast<size_t>(row) * d + j];
-    u[static_cast<size_t>(row) * d + j] = f32_to_bf16(x * r * bf16_to_f32(gain[j]));
-  }
-}
-
-// h[row] += sum_s part[s][row]; u[row] = RMSNorm(h[row]) * gain
-__global__ void residual_norm_kernel(float* __restrict__ h, const float* __restrict__ part, int splits,
-                                     int T, int d, const uint16_t* __restrict__ gain, float eps,
-                                     uint16_t* __restrict__ u) {
-  __shared__ float red[32];
-  const int row = blockIdx.x;
-  float ss = 0.f;
-  for (int j = threadIdx.x; j < d; j += blockDim.x) {
-    float x = h[static_cast<size_t>(row) * d + j];
-    for (int s = 0; s < splits; ++s) x += part[(static_cast<size_t>(s) * T + row) * d + j];
-    h[static_cast<size_t>(row) * d + j] = x;
-    ss += x * x;
-  }
-  ss = block_sum(ss, red);
-  const float r = rsqrtf(ss / d + eps);
-  for (int j = threadIdx.x; j < d; j += blockDim.x)
-    u[static_cast<size_t>(row) * d + j] = f32_to_bf16(h[static_cast<size_t>(row) * d + j] * r * bf16_to_f32(gain[j]));
-}
-
-// Reduce QKV split-K partials, rotate q and k (pairs j, j + D/2) at absolute
-// position pos0 + i, write q [row][Hq][D] bf16 and k, v into the cache rows.
-// cache layout: [B][Hkv][S_max][D] (this layer's base pointers).
-__global__ void rope_qkv_kernel(const float* __restrict__ part, int splits, int T, int n, int pos0, int Hq,
-                                int Hkv, int D, const float2* __restrict__ rope_tab,
-                                uint16_t* __restrict__ q, uint16_t* __restrict__ kc, uint16_t* __restrict__ vc,
-                                int S_max) {
-  const int row = blockIdx.x;
-  const int b = row / n, i = row % n;
-  const int pos = pos0 + i;
-  const int QKV = (Hq + 2 * Hkv) * D;
-  const int half = D / 2;
-  const float* base = part + static_cast<size_t>(row) * QKV;
-  const size_t sstride = static_cast<size_t>(T) * QKV;
-  // rotated heads: Hq query + Hkv key heads, half pairs each
-  for (int idx = threadIdx.x; idx < (Hq + Hkv) * half; idx += blockDim.x) {
-    const int hh = idx / half, j = idx % half;
-    const int c = hh * D + j;
-    float x1 = 0.f, x2 = 0.f;
-    for (int s = 0; s < splits; ++s) {
-      x1 += base[s * sstride + c];
-      x2 += base[s * sstride + c + half];
-    }
-    const float2 cs = rope_tab[static_cast<size_t>(pos) * half + j];
-    const float y1 = x1 * cs.x - x2 * cs.y;
-    const float y2 = x2 * cs.x + x1 * cs.y;
-    if (hh < Hq) {
-      uint16_t* dst = q + (static_cast<size_t>(row) * Hq + hh) * D;
-      dst[j] = f32_to_bf16(y1);
-      dst[j + half] = f32_to_bf16(y2);
-    } else {
-      const int g = hh - Hq;
-      uint16_t* dst = kc + ((static_cast<size_t>(b) * Hkv + g) * S_max + pos) * D;
-      dst[j] = f32_to_bf16(y1);
-      dst[j + half] = f32_to_bf16(y2);
-    }
-  }
-  for (int idx = threadIdx.x; idx < Hkv * D; idx += blockDim.x) {
-    const int g = idx / D, j = idx % D;
-    const int c = (Hq + Hkv) * D + idx;
-    float x = 0.f;
-    for (int s = 0; s < splits; ++s) x += base[s * sstride + c];
-    vc[((static_cast<size_t>(b) * Hkv + g) * S_max + pos) * D + j] = f32_to_bf16(x);
-  }
-}
-
 // Router: logits = sum_s part[s][row][e] (+ bias[e]); top-k by (logit desc,
 // index asc); gates = softmax over the k selected.  One warp per row.
 __global__ void router_topk_kernel(const float* __restrict__ part, int splits, int T, int E, int k,
@@ -316,11 +221,60 @@ __global__ void gather_rows_kernel(const uint16_t* __restrict__ u, const int32_t
   }
 }
 
-// h[t] += y_shared[t] + sum_j gate[t][j] * y[inv_slot[t][j]]; u = RMSNorm(h)*gain
-__global__ void combine_norm_kernel(float* __restrict__ h, const float* __restrict__ yp,
-                                    const int32_t* __restrict__ inv_slot, const float* __restrict__ gates,
-                                    int k, int shared_base, int d, const uint16_t* __restrict__ gain, float eps,
-                                    uint16_t* __restrict__ u, float* __restrict__ capture) {
+// ---------------------------------------------------------------------------
+// Row kernels: one CTA of ROW_THREADS per row; each thread keeps up to
+// ROW_MAXV float4 of the row in registers between the update and the norm.
+// ---------------------------------------------------------------------------
+constexpr int ROW_THREADS = 256;
+constexpr int ROW_MAXV = 4;  // d <= ROW_THREADS * ROW_MAXV * 4 = 4096
+
+__device__ __forceinline__ float4 load_bf16x4(const uint16_t* src) {
+  const uint2 i = *reinterpret_cast<const uint2*>(src);
+  return make_float4(bf16_to_f32(static_cast<uint16_t>(i.x & 0xffffu)), bf16_to_f32(static_cast<uint16_t>(i.x >> 16)),
+                     bf16_to_f32(static_cast<uint16_t>(i.y & 0xffffu)), bf16_to_f32(static_cast<uint16_t>(i.y >> 16)));
+}
+
+__device__ __forceinline__ void store_bf16x4(uint16_t* dst, float4 v) {
+  uint2 o;
+  o.x = pack_bf16x2(v.x, v.y);
+  o.y = pack_bf16x2(v.z, v.w);
+  *reinterpret_cast<uint2*>(dst) = o;
+}
+
+__device__ __forceinline__ float4 f4_add(float4 a, float4 b) {
+  return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+}
+
+__device__ __forceinline__ float4 f4_fma(float s, float4 a, float4 b) {  // b + s * a
+  return make_float4(fmaf(s, a.x, b.x), fmaf(s, a.y, b.y), fmaf(s, a.z, b.z), fmaf(s, a.w, b.w));
+}
+
+__device__ __forceinline__ float f4_sumsq(float4 a) { return a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w; }
+
+// u_row = RMSNorm(row held in v) * gain, as bf16
+__device__ __forceinline__ void norm_store_row(const float4 (&v)[ROW_MAXV], float ss, int d,
+                                               const uint16_t* __restrict__ gain, float eps,
+                                               uint16_t* __restrict__ urow, float* red) {
+  ss = block_sum(ss, red);
+  const float r = rsqrtf(ss / d + eps);
+  const int nv = d / 4;
+#pragma unroll
+  for (int i = 0; i < ROW_MAXV; ++i) {
+    const int c = threadIdx.x + i * ROW_THREADS;
+    if (c < nv) {
+      const float4 g = load_bf16x4(gain + 4 * c);
+      const float4 x = v[i];
+      store_bf16x4(urow + 4 * c, make_float4(x.x * r * g.x, x.y * r * g.y, x.z * r * g.z, x.w * r * g.w));
+    }
+  }
+}
+
+// h[t] += y_shared[t] + sum_j gate[t][j] * y[inv_slot[t][j]] (in that order);
+// u = RMSNorm(h) * gain
+__global__ void __launch_bounds__(ROW_THREADS) combine_norm_kernel(
+    float* __restrict__ h, const float* __restrict__ yp, const int32_t* __restrict__ inv_slot,
+    const float* __restrict__ gates, int k, int shared_base, int d, const uint16_t* __restrict__ gain, float eps,
+    uint16_t* __restrict__ u, float* __restrict__ capture) {
   __shared__ float red[32];
   __shared__ int slot[16];
   __shared__ float gw[16];
@@ -330,19 +284,127 @@ __global__ void combine_norm_kernel(float* __restrict__ h, const float* __restri
     gw[threadIdx.x] = gates[static_cast<size_t>(row) * k + threadIdx.x];
   }
   __syncthreads();
+  const int nv = d / 4;
+  float4* hrow = reinterpret_cast<float4*>(h + static_cast<size_t>(row) * d);
+  const float4* ys = reinterpret_cast<const float4*>(yp + static_cast<size_t>(shared_base + row) * d);
+  float4 v[ROW_MAXV];
   float ss = 0.f;
-  for (int j = threadIdx.x; j < d; j += blockDim.x) {
-    float x = h[static_cast<size_t>(row) * d + j];
-    x += yp[static_cast<size_t>(shared_base + row) * d + j];
-    for (int s = 0; s < k; ++s) x += gw[s] * yp[static_cast<size_t>(slot[s]) * d + j];
-    h[static_cast<size_t>(row) * d + j] = x;
-    if (capture) capture[static_cast<size_t>(row) * d + j] = x;
-    ss += x * x;
+#pragma unroll
+  for (int i = 0; i < ROW_MAXV; ++i) {
+    const int c = threadIdx.x + i * ROW_THREADS;
+    if (c < nv) {
+      float4 x = f4_add(hrow[c], ys[c]);
+      for (int s = 0; s < k; ++s)
+        x = f4_fma(gw[s], reinterpret_cast<const float4*>(yp + static_cast<size_t>(slot[s]) * d)[c], x);
+      hrow[c] = x;
+      if (capture) reinterpret_cast<float4*>(capture + static_cast<size_t>(row) * d)[c] = x;
+      v[i] = x;
+      ss += f4_sumsq(x);
+    }
   }
-  ss = block_sum(ss, red);
-  const float r = rsqrtf(ss / d + eps);
-  for (int j = threadIdx.x; j < d; j += blockDim.x)
-    u[static_cast<size_t>(row) * d + j] = f32_to_bf16(h[static_cast<size_t>(row) * d + j] * r * bf16_to_f32(gain[j]));
+  norm_store_row(v, ss, d, gain, eps, u + static_cast<size_t>(row) * d, red);
+}
+
+// Embedding gather (bf16 -> fp32 residual) + RMSNorm -> bf16.
+// Token of row b*n+i: tokens[b * tok_stride + tok_off + i]; ids outside the
+// vocabulary are clamped into it rather than read out of bounds.
+__global__ void __launch_bounds__(ROW_THREADS) embed_norm_kernel(
+    const int32_t* __restrict__ tokens, int tok_stride, int tok_off, int n, const uint16_t* __restrict__ embed,
+    const uint16_t* __restrict__ gain, float eps, int d, float* __restrict__ h, uint16_t* __restrict__ u,
+    float* __restrict__ capture, int32_t* settled, int n_settled, int vocab) {
+  __shared__ float red[32];
+  const int row = blockIdx.x;
+  const int b = row / n, i = row % n;
+  if (settled != nullptr && row == 0 && threadIdx.x < n_settled) settled[threadIdx.x] = 1;
+  const int tok = min(max(tokens[static_cast<size_t>(b) * tok_stride + tok_off + i], 0), vocab - 1);
+  const uint16_t* e = embed + static_cast<size_t>(tok) * d;
+  float4* hrow = reinterpret_cast<float4*>(h + static_cast<size_t>(row) * d);
+  const int nv = d / 4;
+  float4 v[ROW_MAXV];
+  float ss = 0.f;
+#pragma unroll
+  for (int j = 0; j < ROW_MAXV; ++j) {
+    const int c = threadIdx.x + j * ROW_THREADS;
+    if (c < nv) {
+      const float4 x = load_bf16x4(e + 4 * c);
+      hrow[c] = x;
+      if (capture) reinterpret_cast<float4*>(capture + static_cast<size_t>(row) * d)[c] = x;
+      v[j] = x;
+      ss += f4_sumsq(x);
+    }
+  }
+  norm_store_row(v, ss, d, gain, eps, u + static_cast<size_t>(row) * d, red);
+}
+
+// h[row] += sum_s part[s][row] (splits in order); u[row] = RMSNorm(h[row]) * gain
+__global__ void __launch_bounds__(ROW_THREADS) residual_norm_kernel(
+    float* __restrict__ h, const float* __restrict__ part, int splits, int T, int d,
+    const uint16_t* __restrict__ gain, float eps, uint16_t* __restrict__ u) {
+  __shared__ float red[32];
+  const int row = blockIdx.x;
+  const int nv = d / 4;
+  float4* hrow = reinterpret_cast<float4*>(h + static_cast<size_t>(row) * d);
+  float4 v[ROW_MAXV];
+  float ss = 0.f;
+#pragma unroll
+  for (int j = 0; j < ROW_MAXV; ++j) {
+    const int c = threadIdx.x + j * ROW_THREADS;
+    if (c < nv) {
+      float4 x = hrow[c];
+      for (int s = 0; s < splits; ++s)
+        x = f4_add(x, reinterpret_cast<const float4*>(part + (static_cast<size_t>(s) * T + row) * d)[c]);
+      hrow[c] = x;
+      v[j] = x;
+      ss += f4_sumsq(x);
+    }
+  }
+  norm_store_row(v, ss, d, gain, eps, u + static_cast<size_t>(row) * d, red);
+}
+
+// Reduce the QKV split-K partials (splits in order), rotate q and k pairs
+// (j, j + D/2) at absolute position pos0 + i, write q [row][Hq][D] bf16 and
+// k, v into this layer's cache [B][Hkv][S_max][D] at that position.  Four
+// consecutive j per thread (D/2 is a multiple of 4).
+__global__ void __launch_bounds__(ROW_THREADS) rope_qkv_kernel(
+    const float* __restrict__ part, int splits, int T, int n, int pos0, int Hq, int Hkv, int D,
+    const float2* __restrict__ rope_tab, uint16_t* __restrict__ q, uint16_t* __restrict__ kc,
+    uint16_t* __restrict__ vc, int S_max) {
+  const int row = blockIdx.x;
+  const int b = row / n, i = row % n;
+  const int pos = pos0 + i;
+  const int QKV = (Hq + 2 * Hkv) * D;
+  const int half = D / 2, hq4 = half / 4, d4 = D / 4;
+  const float* base = part + static_cast<size_t>(row) * QKV;
+  const size_t sstride = static_cast<size_t>(T) * QKV;
+  const int n_rot = (Hq + Hkv) * hq4;
+  for (int it = threadIdx.x; it < n_rot + Hkv * d4; it += ROW_THREADS) {
+    if (it < n_rot) {
+      const int hh = it / hq4, j = (it % hq4) * 4;
+      const int c = hh * D + j;
+      float4 x1 = make_float4(0.f, 0.f, 0.f, 0.f), x2 = x1;
+      for (int s = 0; s < splits; ++s) {
+        x1 = f4_add(x1, *reinterpret_cast<const float4*>(base + s * sstride + c));
+        x2 = f4_add(x2, *reinterpret_cast<const float4*>(base + s * sstride + c + half));
+      }
+      const float2* cs = rope_tab + static_cast<size_t>(pos) * half + j;
+      const float2 c0 = cs[0], c1 = cs[1], c2 = cs[2], c3 = cs[3];
+      const float4 y1 = make_float4(x1.x * c0.x - x2.x * c0.y, x1.y * c1.x - x2.y * c1.y,
+                                    x1.z * c2.x - x2.z * c2.y, x1.w * c3.x - x2.w * c3.y);
+      const float4 y2 = make_float4(x2.x * c0.x + x1.x * c0.y, x2.y * c1.x + x1.y * c1.y,
+                                    x2.z * c2.x + x1.z * c2.y, x2.w * c3.x + x1.w * c3.y);
+      uint16_t* dst = hh < Hq ? q + (static_cast<size_t>(row) * Hq + hh) * D
+                              : kc + ((static_cast<size_t>(b) * Hkv + (hh - Hq)) * S_max + pos) * D;
+      store_bf16x4(dst + j, y1);
+      store_bf16x4(dst + j + half, y2);
+    } else {
+      const int r = it - n_rot;
+      const int g = r / d4, j = (r % d4) * 4;
+      const int c = (Hq + Hkv) * D + g * D + j;
+      float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int s = 0; s < splits; ++s) x = f4_add(x, *reinterpret_cast<const float4*>(base + s * sstride + c));
+      store_bf16x4(vc + ((static_cast<size_t>(b) * Hkv + g) * S_max + pos) * D + j, x);
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------
