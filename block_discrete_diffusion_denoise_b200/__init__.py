@@ -11,7 +11,7 @@ import ctypes
 import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libdg.so")
+LIB_PATH = os.environ.get("DG_LIBRARY", os.path.join(HERE, "libdg.so"))
 
 DG_OK = 0
 STATUS = {0: "DG_OK", 1: "DG_ERR_INVALID_ARG", 2: "DG_ERR_OOM", 3: "DG_ERR_CAPACITY", 4: "DG_ERR_CUDA",
@@ -25,7 +25,7 @@ EXPORTS = ["dg_create", "dg_destroy", "dg_prefill", "dg_denoise_step", "dg_denoi
            "dg_debug_profile_read", "dg_debug_launch_count", "dg_lmhead_argmax_static"]
 
 # kernel classes of dg_debug_profile (DG_PROF_* in dg.h)
-PROF_CLASSES = ["expert_gateup", "expert_down", "lm_head", "attention", "dense_proj", "other"]
+PROF_CLASSES = ["experts", "routing", "lm_head", "attention", "dense_proj", "other"]
 
 
 class dg_config(ctypes.Structure):

@@ -23,9 +23,12 @@ struct AttnParams {
   int pos0;            // cached rows before the new rows
   int causal;
   int chunk_len;       // keys per chunk (multiple of 64)
-  int n_chunks;
+  int n_chunks;        // <= ATT_MAX_CHUNKS
   float scale_log2;    // log2(e) / sqrt(D)
+  int* qb_count;       // per query block: chunks finished (zero between launches)
 };
+
+constexpr int ATT_MAX_CHUNKS = 16;
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
@@ -263,6 +266,55 @@ __global__ void __launch_bounds__(128, 2) attn_kernel(const AttnParams p) {
         *reinterpret_cast<float2*>(orow + j * 8 + 2 * t4) = make_float2(o[j][2 * h], o[j][2 * h + 1]);
       if (t4 == 0) p.ml[blockIdx.z * nrows + rid] = make_float2(mrow[h], lrow[h]);
     }
+    // The last chunk of this query block to finish merges all of them:
+    // o = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c  (chunks in order).
+    __shared__ int is_last;
+    __shared__ float wgt[ATT_QROWS][ATT_MAX_CHUNKS];
+    __threadfence();
+    __syncthreads();
+    const int qb = blockIdx.y * gridDim.x + blockIdx.x;
+    if (threadIdx.x == 0) is_last = atomicAdd(p.qb_count + qb, 1) == p.n_chunks - 1;
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+    if (threadIdx.x < ATT_QROWS) {
+      const int r = row_base + threadIdx.x;
+      if (r < rows_total) {
+        const size_t rid = (static_cast<size_t>(b) * p.n + r / G) * p.Hq + kvh * G + r % G;
+        float M = -INFINITY;
+        for (int c = 0; c < p.n_chunks; ++c) M = fmaxf(M, __ldcg(&p.ml[c * nrows + rid].x));
+        const float Mref = M == -INFINITY ? 0.f : M;
+        float den = 0.f;
+        for (int c = 0; c < p.n_chunks; ++c) {
+          const float2 v = __ldcg(&p.ml[c * nrows + rid]);
+          const float wv = exp2f(v.x - Mref);
+          wgt[threadIdx.x][c] = wv;
+          den += v.y * wv;
+        }
+        const float inv = den > 0.f ? 1.f / den : 0.f;
+        for (int c = 0; c < p.n_chunks; ++c) wgt[threadIdx.x][c] *= inv;
+      }
+    }
+    __syncthreads();
+    constexpr int D4 = D / 4;
+    for (int it = threadIdx.x; it < ATT_QROWS * D4; it += blockDim.x) {
+      const int rr = it / D4, j = (it % D4) * 4;
+      const int r = row_base + rr;
+      if (r >= rows_total) continue;
+      const size_t rid = (static_cast<size_t>(b) * p.n + r / G) * p.Hq + kvh * G + r % G;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int c = 0; c < p.n_chunks; ++c) {
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(p.opart + (c * nrows + rid) * D + j));
+        const float wv = wgt[rr][c];
+        acc.x += wv * v.x;
+        acc.y += wv * v.y;
+        acc.z += wv * v.z;
+        acc.w += wv * v.w;
+      }
+      uint16_t* dst = p.o + rid * D + j;
+      *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+    }
+    if (threadIdx.x == 0) p.qb_count[qb] = 0;  // ready for the next launch
   }
 }
 

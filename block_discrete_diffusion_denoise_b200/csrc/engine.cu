@@ -59,8 +59,20 @@ struct dg_ctx {
   float* gates = nullptr;
   int32_t* perm_tok = nullptr;
   int32_t* inv_slot = nullptr;
-  int4* gu_tiles = nullptr;
-  int4* dn_tiles = nullptr;
+  int4* tiles = nullptr;        // fused expert GEMM tile list (gate/up, then down)
+  int32_t* chunk_done = nullptr;
+  int32_t* dense_work = nullptr;   // claim / exit counters of the dense GEMM
+  int32_t* qb_count = nullptr;     // attention: finished key chunks per query block
+  size_t qb_count_cap = 0;
+  // CUDA graph of the denoising step (per batch and cached length)
+  bool use_graphs = true;
+  cudaGraph_t step_graph = nullptr;
+  cudaGraphExec_t step_exec = nullptr;
+  int graph_B = -1, graph_P = -1;
+  cudaGraphNode_t embed_node = nullptr, sample_node = nullptr;
+  cudaKernelNodeParams embed_kp{}, sample_kp{};
+  std::vector<void*> embed_args, sample_args;
+  int64_t graph_launches = 0;
   int32_t* counters = nullptr;
   uint16_t* xp = nullptr;
   uint16_t* hbuf = nullptr;
@@ -77,14 +89,14 @@ struct dg_ctx {
   int32_t* io_canvas_out = nullptr;
   float* io_conf = nullptr;
   int32_t* io_settled = nullptr;
-  size_t max_gu_tiles = 0, max_dn_tiles = 0;
+  size_t max_gu_tiles = 0, max_dn_tiles = 0, max_chunks = 0;
   // capture (test hook)
   bool capture = false;
   float* cap_h = nullptr;
   int32_t* cap_idx = nullptr;
   // tensor maps
   std::vector<LayerMaps> lmaps;
-  CUtensorMap m_u16{}, m_u128{}, m_o16{}, m_xp16{}, m_h16{}, m_hs16{}, m_embed{};
+  CUtensorMap m_u16{}, m_u64{}, m_u128{}, m_o64{}, m_xp16{}, m_h16{}, m_hs16{}, m_embed{};
   // state
   int B = 0;
   int P = 0;
@@ -196,27 +208,29 @@ int choose_splits(int tiles, int k_steps, int sms, size_t max_splits_by_cap) {
 }
 
 // out[s][t][m] = partial sums over split s of W[m, :] . X[t, :]
+// x: token rows with 64-row TMA boxes
 dg_status gemm_dense(dg_ctx* c, const CUtensorMap& w, const CUtensorMap& x, int M, int T, int K, int* splits_out,
-                     int max_splits = 8) {
+                     int max_splits = 11) {
   GemmParams p;
   memset(&p, 0, sizeof(p));
   p.a_map[0] = w;
   p.b_map = x;
-  p.b_box_rows = 16;
+  p.b_box_rows = 64;
   p.M = M;
   p.T = T;
   p.k_steps = K / 64;
-  p.bn = std::min(GEMM_BN, (T + 15) / 16 * 16);
+  p.bn = std::min(DENSE_BN, (T + 15) / 16 * 16);
   p.n_tiles_n = (T + p.bn - 1) / p.bn;
   const int m_tiles = (M + GEMM_BM - 1) / GEMM_BM;
   const size_t cap_s = c->part_cap / (static_cast<size_t>(T) * M);
   p.splits = choose_splits(m_tiles * p.n_tiles_n, p.k_steps, c->sms, std::min<size_t>(cap_s, max_splits));
   p.tiles_static = m_tiles * p.n_tiles_n * p.splits;
   p.out_f32 = c->part;
+  p.work = c->dense_work;
   p.err = dev_err(c);
   const int grid = std::min(c->sms, p.tiles_static);
   ProfScope ps0(c, DG_PROF_DENSE);
-  gemm_kernel<GEMM_DENSE><<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, c->stream>>>(p);
+  gemm_kernel<GEMM_DENSE><<<grid, GEMM_THREADS, gemm_smem_bytes<GEMM_DENSE>(), c->stream>>>(p);
   DG_LAUNCHED(c);
   ps0.end();
   *splits_out = p.splits;
@@ -245,14 +259,18 @@ dg_status attention(dg_ctx* c, int l, int B, int n, int pos0, bool causal) {
   const int ctas = qblocks * B * c->Hkv;
   const int keys = pos0 + n;
   const size_t rows = static_cast<size_t>(B) * n * c->Hq;
-  int n_chunks = std::max(1, (2 * c->sms + ctas - 1) / ctas);
+  // split the keys so that all CTAs fit in one wave (two CTAs per SM)
+  int n_chunks = std::max(1, (2 * c->sms) / ctas);
   n_chunks = std::min(n_chunks, std::max(1, (keys + 255) / 256));
   n_chunks = std::min<int>(n_chunks, static_cast<int>(c->opart_rows_cap / rows));
+  n_chunks = std::min(n_chunks, ATT_MAX_CHUNKS);
   n_chunks = std::max(n_chunks, 1);
   int chunk_len = ((keys + n_chunks - 1) / n_chunks + ATT_KB - 1) / ATT_KB * ATT_KB;
   n_chunks = (keys + chunk_len - 1) / chunk_len;
+  if (static_cast<size_t>(ctas) > c->qb_count_cap) return fail(c, DG_ERR_CAPACITY, "attention: %d query blocks", ctas);
   p.chunk_len = chunk_len;
   p.n_chunks = n_chunks;
+  p.qb_count = c->qb_count;
   dim3 grid(qblocks, B * c->Hkv, n_chunks);
   ProfScope ps1(c, DG_PROF_ATTENTION);
   switch (c->D) {
@@ -270,13 +288,6 @@ dg_status attention(dg_ctx* c, int l, int B, int n, int pos0, bool causal) {
   }
   DG_LAUNCHED(c);
   ps1.end();
-  if (n_chunks > 1) {
-    ProfScope ps2(c, DG_PROF_ATTENTION);
-    attn_merge_kernel<<<static_cast<unsigned>(rows), 64, 0, c->stream>>>(c->opart, c->ml, n_chunks,
-                                                                         static_cast<int>(rows), c->D, c->o);
-    DG_LAUNCHED(c);
-    ps2.end();
-  }
   return DG_OK;
 }
 
@@ -284,27 +295,29 @@ dg_status moe(dg_ctx* c, int l, int T) {
   const LayerMaps& lm = c->lmaps[l];
   const dg_layer_weights& lw = c->layers[l];
   int s3 = 1;
-  dg_status st = gemm_dense(c, lm.wr, c->m_u16, c->E, T, c->d, &s3, 4);
+  dg_status st = gemm_dense(c, lm.wr, c->m_u64, c->E, T, c->d, &s3);
   if (st != DG_OK) return st;
   int32_t* cap = c->capture ? c->cap_idx + static_cast<size_t>(l) * c->R_step * c->k : nullptr;
-  ProfScope ps3(c, DG_PROF_OTHER);
+  ProfScope ps3(c, DG_PROF_ROUTING);
   router_topk_kernel<<<(T * 32 + 255) / 256, 256, 0, c->stream>>>(c->part, s3, T, c->E, c->k, c->router_bias,
                                                                    c->idx, c->gates, cap);
   DG_LAUNCHED(c);
   ps3.end();
-  ProfScope ps4(c, DG_PROF_OTHER);
+  ProfScope ps4(c, DG_PROF_ROUTING);
   permute_kernel<<<1, PERM_THREADS, 0, c->stream>>>(c->idx, T, c->k, c->E, c->F, c->Fs, c->d, c->perm_tok,
-                                                     c->inv_slot, c->gu_tiles, c->dn_tiles, c->counters);
+                                                     c->inv_slot, c->tiles, c->chunk_done, c->counters,
+                                                     MOE_CHUNK_ROWS);
   DG_LAUNCHED(c);
   ps4.end();
   const int rows = T * c->k;
-  ProfScope ps5(c, DG_PROF_OTHER);
+  ProfScope ps5(c, DG_PROF_ROUTING);
   gather_rows_kernel<<<std::min(4 * c->sms, (rows * (c->d / 8) + 255) / 256), 256, 0, c->stream>>>(
       c->u, c->perm_tok, rows, c->d, c->xp);
   DG_LAUNCHED(c);
   ps5.end();
   (void)lw;
 
+  // routed + shared experts, gate/up then down, one persistent launch
   GemmParams p;
   memset(&p, 0, sizeof(p));
   p.a_map[0] = lm.wg;
@@ -313,42 +326,29 @@ dg_status moe(dg_ctx* c, int l, int T) {
   p.as_map[1] = lm.wsu;
   p.b_map = c->m_xp16;
   p.bs_map = c->m_u16;
+  p.d_map = lm.wd;
+  p.ds_map = lm.wsd;
+  p.h_map = c->m_h16;
+  p.hs_map = c->m_hs16;
   p.b_box_rows = 16;
-  p.k_steps = c->d / 64;
-  p.tile_count = c->counters + 0;
-  p.tiles = c->gu_tiles;
+  p.counts = c->counters;
+  p.tiles = c->tiles;
+  p.work = c->counters + 3;
+  p.chunk_done = c->chunk_done;
   p.n_groups_routed = c->E;
-  p.a_rows_per_group = c->F;
+  p.F = c->F;
+  p.Fs = c->Fs;
+  p.d = c->d;
   p.h_out = c->hbuf;
-  p.h_ld = c->F;
   p.hs_out = c->hsbuf;
-  p.hs_ld = c->Fs;
-  p.err = dev_err(c);
-  ProfScope ps6(c, DG_PROF_EXPERT_GATEUP);
-  gemm_kernel<GEMM_GATEUP><<<c->sms, GEMM_THREADS, GEMM_SMEM_BYTES, c->stream>>>(p);
-  DG_LAUNCHED(c);
-  ps6.end();
-
-  memset(&p, 0, sizeof(p));
-  p.a_map[0] = lm.wd;
-  p.as_map[0] = lm.wsd;
-  p.b_map = c->m_h16;
-  p.bs_map = c->m_hs16;
-  p.b_box_rows = 16;
-  p.k_steps = c->F / 64;
-  p.k_steps_shared = c->Fs / 64;
-  p.tile_count = c->counters + 1;
-  p.tiles = c->dn_tiles;
-  p.n_groups_routed = c->E;
-  p.a_rows_per_group = c->d;
   p.out_f32 = c->yp;
   p.out_ld = c->d;
   p.shared_row_base = rows;
   p.err = dev_err(c);
-  ProfScope ps7(c, DG_PROF_EXPERT_DOWN);
-  gemm_kernel<GEMM_DOWN><<<c->sms, GEMM_THREADS, GEMM_SMEM_BYTES, c->stream>>>(p);
+  ProfScope ps6(c, DG_PROF_EXPERTS);
+  gemm_kernel<GEMM_MOE><<<c->sms, GEMM_THREADS, gemm_smem_bytes<GEMM_MOE>(), c->stream>>>(p);
   DG_LAUNCHED(c);
-  ps7.end();
+  ps6.end();
   return DG_OK;
 }
 
@@ -372,7 +372,7 @@ dg_status forward(dg_ctx* c, const int32_t* tokens, int tok_stride, int tok_off,
     const LayerMaps& lm = c->lmaps[l];
     const dg_layer_weights& lw = c->layers[l];
     int s1 = 1;
-    dg_status st = gemm_dense(c, lm.wqkv, c->m_u16, c->QKV, T, c->d, &s1);
+    dg_status st = gemm_dense(c, lm.wqkv, c->m_u64, c->QKV, T, c->d, &s1);
     if (st != DG_OK) return st;
     const size_t layer_off = static_cast<size_t>(l) * c->cfg.max_batch * c->Hkv * c->cfg.max_seq * c->D;
     ProfScope ps9(c, DG_PROF_OTHER);
@@ -384,7 +384,7 @@ dg_status forward(dg_ctx* c, const int32_t* tokens, int tok_stride, int tok_off,
     st = attention(c, l, B, n, pos0, causal);
     if (st != DG_OK) return st;
     int s2 = 1;
-    st = gemm_dense(c, lm.wo, c->m_o16, c->d, T, c->HD, &s2);
+    st = gemm_dense(c, lm.wo, c->m_o64, c->d, T, c->HD, &s2);
     if (st != DG_OK) return st;
     ProfScope ps10(c, DG_PROF_OTHER);
     residual_norm_kernel<<<T, 256, 0, c->stream>>>(c->h, c->part, s2, T, c->d,
@@ -422,7 +422,8 @@ dg_status lm_head_and_sample(dg_ctx* c, int B, int step, uint64_t seed, float ta
   p.logit_scale_log2 = static_cast<float>(1.4426950408889634 / static_cast<double>(c->cfg.temperature));
   p.err = dev_err(c);
   ProfScope ps12(c, DG_PROF_LMHEAD);
-  gemm_kernel<GEMM_LMHEAD><<<std::min(c->sms, p.tiles_static), GEMM_THREADS, GEMM_SMEM_BYTES, c->stream>>>(p);
+  gemm_kernel<GEMM_LMHEAD><<<std::min(c->sms, p.tiles_static), GEMM_THREADS, gemm_smem_bytes<GEMM_LMHEAD>(),
+                             c->stream>>>(p);
   DG_LAUNCHED(c);
   ps12.end();
   SampleArgs a;
@@ -459,17 +460,107 @@ T* carve(char*& cur, size_t count) {
 }
 
 dg_status set_smem_attrs(dg_ctx* c) {
-  DG_CUDA(c, cudaFuncSetAttribute(gemm_kernel<GEMM_DENSE>, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES));
-  DG_CUDA(c, cudaFuncSetAttribute(gemm_kernel<GEMM_GATEUP>, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES));
-  DG_CUDA(c, cudaFuncSetAttribute(gemm_kernel<GEMM_DOWN>, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES));
-  DG_CUDA(c, cudaFuncSetAttribute(gemm_kernel<GEMM_LMHEAD>, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES));
+  DG_CUDA(c, cudaFuncSetAttribute(gemm_kernel<GEMM_DENSE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  gemm_smem_bytes<GEMM_DENSE>()));
+  DG_CUDA(c, cudaFuncSetAttribute(gemm_kernel<GEMM_MOE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  gemm_smem_bytes<GEMM_MOE>()));
+  DG_CUDA(c, cudaFuncSetAttribute(gemm_kernel<GEMM_LMHEAD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  gemm_smem_bytes<GEMM_LMHEAD>()));
   DG_CUDA(c, cudaFuncSetAttribute(attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, att_smem_bytes<64>()));
   DG_CUDA(c, cudaFuncSetAttribute(attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, att_smem_bytes<128>()));
   DG_CUDA(c, cudaFuncSetAttribute(attn_kernel<176>, cudaFuncAttributeMaxDynamicSharedMemorySize, att_smem_bytes<176>()));
   return DG_OK;
 }
 
+void drop_step_graph(dg_ctx* c) {
+  if (c->step_exec) cudaGraphExecDestroy(c->step_exec);
+  if (c->step_graph) cudaGraphDestroy(c->step_graph);
+  c->step_exec = nullptr;
+  c->step_graph = nullptr;
+  c->graph_B = c->graph_P = -1;
+}
+
+// Capture the whole step (embedding .. sampler) once per (batch, cached
+// length) on the context stream; later calls only rebind the first kernel
+// (canvas, settled flags) and the last one (step, seed, tau, outputs).
+dg_status step_via_graph(dg_ctx* c, const int32_t* canvas_in, int32_t step, uint64_t seed, float tau,
+                         int32_t* canvas_out, float* conf, int32_t* settled) {
+  if (!c->step_exec || c->graph_B != c->B || c->graph_P != c->P) {
+    drop_step_graph(c);
+    const int64_t l0 = c->launches;
+    DG_CUDA(c, cudaStreamBeginCapture(c->stream, cudaStreamCaptureModeThreadLocal));
+    dg_status st = forward(c, c->io_canvas_in, c->cfg.canvas, 0, c->B, c->cfg.canvas, c->P, false, c->io_settled);
+    if (st == DG_OK)
+      st = lm_head_and_sample(c, c->B, 0, 0, 0.f, c->io_canvas_out, c->io_conf, c->io_settled);
+    cudaGraph_t g = nullptr;
+    const cudaError_t e = cudaStreamEndCapture(c->stream, &g);
+    if (st != DG_OK || e != cudaSuccess) {
+      if (g) cudaGraphDestroy(g);
+      cudaGetLastError();
+      return st != DG_OK ? st : fail(c, DG_ERR_CUDA, "step capture: %s", cudaGetErrorString(e));
+    }
+    c->step_graph = g;
+    DG_CUDA(c, cudaGraphInstantiate(&c->step_exec, g, 0));
+    size_t n = 0;
+    DG_CUDA(c, cudaGraphGetNodes(g, nullptr, &n));
+    std::vector<cudaGraphNode_t> nodes(n);
+    DG_CUDA(c, cudaGraphGetNodes(g, nodes.data(), &n));
+    c->embed_node = c->sample_node = nullptr;
+    for (cudaGraphNode_t nd : nodes) {
+      cudaGraphNodeType ty;
+      if (cudaGraphNodeGetType(nd, &ty) != cudaSuccess || ty != cudaGraphNodeTypeKernel) continue;
+      cudaKernelNodeParams kp;
+      if (cudaGraphKernelNodeGetParams(nd, &kp) != cudaSuccess) continue;
+      if (kp.func == reinterpret_cast<void*>(embed_norm_kernel)) {
+        c->embed_node = nd;
+        c->embed_kp = kp;
+      } else if (kp.func == reinterpret_cast<void*>(lmhead_merge_sample_kernel)) {
+        c->sample_node = nd;
+        c->sample_kp = kp;
+      }
+    }
+    if (!c->embed_node || !c->sample_node) {
+      drop_step_graph(c);
+      return fail(c, DG_ERR_CUDA, "step graph: entry/exit kernels not found");
+    }
+    // argument pointer arrays: point at the graph's stored values except the rebound ones
+    c->embed_args.assign(c->embed_kp.kernelParams, c->embed_kp.kernelParams + 14);
+    c->sample_args.assign(c->sample_kp.kernelParams, c->sample_kp.kernelParams + 2);
+    c->graph_launches = c->launches - l0;
+    c->launches = l0;
+    c->graph_B = c->B;
+    c->graph_P = c->P;
+  }
+  // embed_norm_kernel(tokens, tok_stride, tok_off, n, embed, gain, eps, d, h, u, capture, settled, n_settled, vocab)
+  const int32_t* tok = canvas_in;
+  int32_t* set0 = settled;
+  std::vector<void*> ea = c->embed_args;
+  ea[0] = &tok;
+  ea[11] = &set0;
+  cudaKernelNodeParams ekp = c->embed_kp;
+  ekp.kernelParams = ea.data();
+  DG_CUDA(c, cudaGraphExecKernelNodeSetParams(c->step_exec, c->embed_node, &ekp));
+  // lmhead_merge_sample_kernel(part, SampleArgs)
+  SampleArgs a = *static_cast<SampleArgs*>(c->sample_args[1]);
+  a.step = step;
+  a.seed_lo = static_cast<uint32_t>(seed & 0xFFFFFFFFull);
+  a.seed_hi = static_cast<uint32_t>(seed >> 32);
+  a.tau = tau;
+  a.canvas_out = canvas_out;
+  a.conf_out = conf;
+  a.settled = settled;
+  std::vector<void*> sa = c->sample_args;
+  sa[1] = &a;
+  cudaKernelNodeParams skp = c->sample_kp;
+  skp.kernelParams = sa.data();
+  DG_CUDA(c, cudaGraphExecKernelNodeSetParams(c->step_exec, c->sample_node, &skp));
+  DG_CUDA(c, cudaGraphLaunch(c->step_exec, c->stream));
+  c->launches += c->graph_launches;
+  return DG_OK;
+}
+
 void free_all(dg_ctx* c) {
+  drop_step_graph(c);
   for (cudaEvent_t e : c->ev_pool) cudaEventDestroy(e);
   c->ev_pool.clear();
   if (c->ws) cudaFree(c->ws);
@@ -510,7 +601,7 @@ dg_status dg_create(const dg_config* cfg, const dg_weights* w, void* cuda_stream
     return reject(DG_ERR_INVALID_ARG, "non-positive dimension");
   if (g.d_model % 128 || g.d_model > 4096 || g.expert_hidden % 64 || g.shared_hidden % 64 || g.vocab % 128 ||
       (g.head_dim != 64 && g.head_dim != 128 && g.head_dim != 176) || g.n_q_heads % g.n_kv_heads ||
-      (g.n_q_heads * g.head_dim) % 64 || g.n_experts > PERM_MAXE || g.top_k > 16 || g.top_k > g.n_experts ||
+      (g.n_q_heads * g.head_dim) % 64 || g.n_experts > PERM_MAXE || g.n_experts % 4 || g.top_k > 16 || g.top_k > g.n_experts ||
       g.canvas % 16 || g.canvas > 256 || g.max_seq < g.canvas)
     return reject(DG_ERR_UNSUPPORTED, "unsupported shape");
   if (!w->embed || !w->final_norm || !w->layers) return reject(DG_ERR_INVALID_ARG, "null weights");
@@ -559,9 +650,13 @@ dg_status dg_create(const dg_config* cfg, const dg_weights* w, void* cuda_stream
   const size_t mmax = std::max<size_t>({static_cast<size_t>(c->QKV), d, static_cast<size_t>(c->E)});
   c->part_cap = std::max<size_t>(R, 5 * 256) * mmax;
   c->opart_rows_cap = std::max<size_t>(16 * 256, 2 * R) * c->Hq;
-  const size_t chunks_max = (R * k + 127) / 128 + c->E;
-  c->max_gu_tiles = chunks_max * (c->F / 64) + ((R + 127) / 128) * (c->Fs / 64);
-  c->max_dn_tiles = (chunks_max + (R + 127) / 128) * (d / 128);
+  const size_t CH = MOE_CHUNK_ROWS;
+  const size_t chunks_max = (R * k + CH - 1) / CH + c->E;  // routed token chunks
+  const size_t chunks_shared = (R + CH - 1) / CH;
+  c->max_gu_tiles = chunks_max * (c->F / 64) + chunks_shared * (c->Fs / 64);
+  c->max_dn_tiles = (chunks_max + chunks_shared) * (d / 128);
+  c->max_chunks = chunks_max + chunks_shared;
+  c->qb_count_cap = static_cast<size_t>(c->Hkv) * ((R * (c->Hq / c->Hkv) + ATT_QROWS - 1) / ATT_QROWS + g.max_batch);
   size_t bytes = 0;
   auto add = [&](size_t n, size_t sz) { bytes += (n * sz + 255) / 256 * 256; };
   add(R * d, 4);                                  // h
@@ -575,8 +670,10 @@ dg_status dg_create(const dg_config* cfg, const dg_weights* w, void* cuda_stream
   add(R * k, 4);                                  // gates
   add(R * k, 4);                                  // perm_tok
   add(R * k, 4);                                  // inv_slot
-  add(c->max_gu_tiles, 16);                       // gu_tiles
-  add(c->max_dn_tiles, 16);                       // dn_tiles
+  add(c->max_gu_tiles + c->max_dn_tiles, 16);    // tiles
+  add(c->max_chunks, 4);                          // chunk_done
+  add(2, 4);                                      // dense_work
+  add(c->qb_count_cap, 4);                        // qb_count
   add(16, 4);                                     // counters
   add(R * k * d, 2);                              // xp
   add(R * k * c->F, 2);                           // hbuf
@@ -611,8 +708,10 @@ dg_status dg_create(const dg_config* cfg, const dg_weights* w, void* cuda_stream
   c->gates = carve<float>(cur, R * k);
   c->perm_tok = carve<int32_t>(cur, R * k);
   c->inv_slot = carve<int32_t>(cur, R * k);
-  c->gu_tiles = carve<int4>(cur, c->max_gu_tiles);
-  c->dn_tiles = carve<int4>(cur, c->max_dn_tiles);
+  c->tiles = carve<int4>(cur, c->max_gu_tiles + c->max_dn_tiles);
+  c->chunk_done = carve<int32_t>(cur, c->max_chunks);
+  c->dense_work = carve<int32_t>(cur, 2);
+  c->qb_count = carve<int32_t>(cur, c->qb_count_cap);
   c->counters = carve<int32_t>(cur, 16);
   c->xp = carve<uint16_t>(cur, R * k * d);
   c->hbuf = carve<uint16_t>(cur, R * k * c->F);
@@ -682,8 +781,9 @@ dg_status dg_create(const dg_config* cfg, const dg_weights* w, void* cuda_stream
     ok &= make_map(&m.wsd, lw.ws_down, d, c->Fs, 128);
   }
   ok &= make_map(&c->m_u16, c->u, R, d, 16);
+  ok &= make_map(&c->m_u64, c->u, R, d, 64);
   ok &= make_map(&c->m_u128, c->u, R, d, 128);
-  ok &= make_map(&c->m_o16, c->o, R, c->HD, 16);
+  ok &= make_map(&c->m_o64, c->o, R, c->HD, 64);
   ok &= make_map(&c->m_xp16, c->xp, R * k, d, 16);
   ok &= make_map(&c->m_h16, c->hbuf, R * k, c->F, 16);
   ok &= make_map(&c->m_hs16, c->hsbuf, R, c->Fs, 16);
@@ -731,6 +831,9 @@ dg_status dg_denoise_step(dg_ctx* c, const int32_t* canvas_in, int32_t step, uin
   if (!canvas_in || !canvas_out || !conf) return fail(c, DG_ERR_INVALID_ARG, "step: null buffer");
   if (!c->prefilled) return fail(c, DG_ERR_STATE, "step before prefill");
   if (c->P + c->cfg.canvas > c->cfg.max_seq) return fail(c, DG_ERR_CAPACITY, "step: cache full");
+  // test hooks (capture, profiling) need the eager launches
+  if (c->use_graphs && !c->capture && c->prof_mask == 0 && c->stream != nullptr)
+    return step_via_graph(c, canvas_in, step, seed, tau, canvas_out, conf, settled);
   dg_status st = forward(c, canvas_in, c->cfg.canvas, 0, c->B, c->cfg.canvas, c->P, false, settled);
   if (st != DG_OK) return st;
   return lm_head_and_sample(c, c->B, step, seed, tau, canvas_out, conf, settled);
@@ -858,19 +961,22 @@ dg_status dg_debug_gemm(dg_ctx* c, const void* w, int32_t M, int32_t K, const vo
     return fail(c, DG_ERR_INVALID_ARG, "debug_gemm");
   GemmParams p;
   memset(&p, 0, sizeof(p));
-  if (!make_map(&p.a_map[0], w, M, K, 128) || !make_map(&p.b_map, x, T, K, 16))
+  if (!make_map(&p.a_map[0], w, M, K, 128) || !make_map(&p.b_map, x, T, K, 64))
     return fail(c, DG_ERR_CUDA, "debug_gemm: tensor map");
-  p.b_box_rows = 16;
+  p.b_box_rows = 64;
   p.M = M;
   p.T = T;
   p.k_steps = K / 64;
-  p.bn = std::min(GEMM_BN, (T + 15) / 16 * 16);
+  p.bn = std::min(DENSE_BN, (T + 15) / 16 * 16);
   p.n_tiles_n = (T + p.bn - 1) / p.bn;
   p.splits = splits;
   p.tiles_static = ((M + GEMM_BM - 1) / GEMM_BM) * p.n_tiles_n * splits;
+  if (M % 4) return fail(c, DG_ERR_INVALID_ARG, "debug_gemm: M must be a multiple of 4");
   p.out_f32 = out;
+  p.work = c->dense_work;
   p.err = dev_err(c);
-  gemm_kernel<GEMM_DENSE><<<std::min(c->sms, p.tiles_static), GEMM_THREADS, GEMM_SMEM_BYTES, c->stream>>>(p);
+  gemm_kernel<GEMM_DENSE><<<std::min(c->sms, p.tiles_static), GEMM_THREADS, gemm_smem_bytes<GEMM_DENSE>(),
+                            c->stream>>>(p);
   DG_LAUNCHED(c);
   return DG_OK;
 }
@@ -982,7 +1088,7 @@ extern "C" dg_status dg_lmhead_argmax_static(const void* z, int32_t n_rows, int3
         cudaGetSymbolAddress(reinterpret_cast<void**>(&su.err), g_lm_static_err) != cudaSuccess ||
         cudaDeviceGetAttribute(&su.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
         cudaFuncSetAttribute(gemm_kernel<GEMM_LMHEAD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             GEMM_SMEM_BYTES) != cudaSuccess)
+                             gemm_smem_bytes<GEMM_LMHEAD>()) != cudaSuccess)
       return DG_ERR_CUDA;
     su.done = true;
   }
@@ -1000,7 +1106,8 @@ extern "C" dg_status dg_lmhead_argmax_static(const void* z, int32_t n_rows, int3
   p.logit_scale_log2 = static_cast<float>(1.4426950408889634 / static_cast<double>(temperature));
   p.err = DevErr{su.err, 1000000000ull};
   if (cudaMemsetAsync(su.err, 0, sizeof(int), st) != cudaSuccess) return DG_ERR_CUDA;
-  gemm_kernel<GEMM_LMHEAD><<<std::min(su.sms, p.tiles_static), GEMM_THREADS, GEMM_SMEM_BYTES, st>>>(p);
+  gemm_kernel<GEMM_LMHEAD><<<std::min(su.sms, p.tiles_static), GEMM_THREADS, gemm_smem_bytes<GEMM_LMHEAD>(),
+                             st>>>(p);
   if (cudaGetLastError() != cudaSuccess) return DG_ERR_CUDA;
   lmhead_static_merge_kernel<<<n_rows, 256, 0, st>>>(su.partials, n_vtiles, n_rows, su.err, argmax_out, lse_out,
                                                      conf_out);

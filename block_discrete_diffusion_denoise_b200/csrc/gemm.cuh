@@ -7,15 +7,21 @@
 // TMEM accumulators (128 lanes x 128 fp32 columns each), warps 2..5 drain the
 // other accumulator through the epilogue.  All waits are bounded.
 //
-// Four problem kinds share the pipeline (the tile decode and the epilogue
-// differ):
+// Three launch modes share the pipeline:
 //   DENSE   A = weight rows (output features), B = tokens; split-K partials
-//           out[split][token][feature] fp32 (deterministic, no atomics).
-//   GATEUP  grouped routed experts + the shared expert: A = 64 gate rows
-//           stacked on the same 64 up rows, B = the expert's tokens; the
-//           epilogue forms SiLU(gate) * up and stores bf16 hidden rows.
-//   DOWN    grouped: A = 128 rows of the down projection, B = hidden rows;
-//           fp32 output rows in permuted order.
+//           out[split][token][feature] fp32, summed in split order by the
+//           consumer kernel (deterministic, no atomics).  Tiles are claimed
+//           from an atomic counter.
+//   MOE     one launch for all experts of a layer, routed and shared: first the
+//           gate/up tiles (A = 64 gate rows stacked on the same 64 up rows, B =
+//           the expert's tokens; the epilogue forms SiLU(gate) * up and stores
+//           bf16 hidden rows), then the down tiles (A = 128 rows of the down
+//           projection, B = hidden rows; fp32 output rows in permuted order).
+//           Tiles are claimed from an atomic counter in list order; a down tile
+//           waits until every gate/up tile of its token chunk has published its
+//           hidden rows.  Every claimed tile's dependencies were claimed
+//           earlier by running CTAs and depend on nothing, so the wait always
+//           ends.
 //   LMHEAD  A = 128 tokens, B = 128 vocabulary rows of the tied embedding; the
 //           epilogue keeps, per token, the running top-2 logits, the argmax
 //           and the sum of exp, and writes one 16-byte partial per
@@ -28,43 +34,76 @@ namespace dg {
 
 constexpr int GEMM_BM = 128;
 constexpr int GEMM_BK = 64;
-constexpr int GEMM_BN = 128;
-constexpr int GEMM_STAGES = 6;
+constexpr int GEMM_BN = 128;                         // accumulator columns; dense / LM-head tile width
 constexpr int GEMM_A_BYTES = GEMM_BM * GEMM_BK * 2;  // 16 KB
-constexpr int GEMM_B_BYTES = GEMM_BN * GEMM_BK * 2;  // 16 KB
 constexpr int GEMM_THREADS = 192;
-constexpr int GEMM_TMEM_COLS = 2 * GEMM_BN;
-constexpr int GEMM_XCHG_FLOATS = 64 * 33;            // gate values of one 32-column chunk
-constexpr int GEMM_SMEM_BYTES = 1024 + GEMM_STAGES * (GEMM_A_BYTES + GEMM_B_BYTES) +
-                                GEMM_XCHG_FLOATS * 4 + 256;
+// epilogue staging: gate values of one 32-column chunk (64 x 33) or one
+// 32 x 128 fp32 block on its way to global memory
+constexpr int GEMM_XCHG_FLOATS = 32 * GEMM_BM;
+constexpr int GEMM_SCHED = 4;                        // claimed-tile ring
+constexpr int MOE_CHUNK_ROWS = 128;                  // tokens per expert tile
 
-enum GemmMode : int { GEMM_DENSE = 0, GEMM_GATEUP = 1, GEMM_DOWN = 2, GEMM_LMHEAD = 3 };
+enum GemmMode : int { GEMM_DENSE = 0, GEMM_MOE = 1, GEMM_LMHEAD = 3 };
+
+constexpr int DENSE_BN = 256;                        // tokens per dense tile: each weight tile streamed once
+
+// Stage ring depth (16 KB of A plus the B rows per stage).
+template <int MODE>
+constexpr int gemm_stages() {
+  return MODE == GEMM_DENSE ? 4 : 6;
+}
+// rows of B one stage holds
+template <int MODE>
+constexpr int gemm_b_rows() {
+  return MODE == GEMM_MOE ? MOE_CHUNK_ROWS : (MODE == GEMM_DENSE ? DENSE_BN : GEMM_BN);
+}
+template <int MODE>
+constexpr int gemm_b_bytes() {
+  return gemm_b_rows<MODE>() * GEMM_BK * 2;
+}
+// fp32 columns of one of the two TMEM accumulators (a power of two)
+template <int MODE>
+constexpr int gemm_acc_cols() {
+  return gemm_b_rows<MODE>() > 128 ? 256 : 128;
+}
+template <int MODE>
+constexpr int gemm_smem_bytes() {
+  return 1024 + gemm_stages<MODE>() * (GEMM_A_BYTES + gemm_b_bytes<MODE>()) + GEMM_XCHG_FLOATS * 4 + 512;
+}
+
+enum TileKind : int { KIND_DENSE = 0, KIND_GATEUP = 1, KIND_DOWN = 2, KIND_LMHEAD = 3 };
 
 struct GemmParams {
-  CUtensorMap a_map[2];   // DENSE/DOWN/LMHEAD: [0]; GATEUP: [0] gate, [1] up   (routed)
-  CUtensorMap as_map[2];  // shared expert A: GATEUP [0] gate, [1] up; DOWN [0]
-  CUtensorMap b_map;      // DENSE: tokens; GATEUP: gathered rows; DOWN: hidden; LMHEAD: embed
-  CUtensorMap bs_map;     // shared expert B: GATEUP: normed tokens; DOWN: shared hidden
-  int b_box_rows;         // rows per B box (16 or 128)
+  CUtensorMap a_map[2];   // DENSE/LMHEAD: [0]; MOE gate/up routed: [0] w_gate, [1] w_up
+  CUtensorMap as_map[2];  // MOE gate/up shared expert: [0] ws_gate, [1] ws_up
+  CUtensorMap b_map;      // DENSE: tokens; LMHEAD: embed; MOE gate/up routed: gathered rows
+  CUtensorMap bs_map;     // MOE gate/up shared: normed tokens
+  CUtensorMap d_map;      // MOE down routed A: w_down
+  CUtensorMap ds_map;     // MOE down shared A: ws_down
+  CUtensorMap h_map;      // MOE down routed B: routed hidden rows
+  CUtensorMap hs_map;     // MOE down shared B: shared hidden rows
+  int b_box_rows;         // rows per B box (16, or 128 for the LM head)
   int M;                  // DENSE: output features; LMHEAD: tokens
   int T;                  // DENSE: tokens
-  int k_steps;            // K / 64 (routed experts, dense, LM head)
-  int k_steps_shared;     // K / 64 of the shared expert's down projection
+  int k_steps;            // K / 64 (DENSE, LMHEAD)
   int splits;             // DENSE split-K
   int n_tiles_n;          // DENSE token tiles
   int bn;                 // DENSE token tile
   int n_mtiles;           // LMHEAD token tiles
   int tiles_static;       // DENSE / LMHEAD tile count
-  const int* tile_count;  // GATEUP / DOWN: tile count (device)
-  const int4* tiles;      // GATEUP / DOWN: {group, block, first row, rows}
+  // DENSE, MOE: claimed tiles
+  int* work;              // [0] claim counter, [1] exit counter; zero at launch, reset by the last CTA
+  // MOE
+  const int* counts;      // [0] gate/up tiles, [1] down tiles
+  const int4* tiles;      // gate/up tiles, then down tiles: {group | blk << 16, chunk, first row, rows}
+  int* chunk_done;        // finished gate/up tiles per token chunk, zero at launch
   int n_groups_routed;    // group == n_groups_routed is the shared expert
-  int a_rows_per_group;   // GATEUP: F; DOWN: d
-  float* out_f32;         // DENSE partials [splits][T][M]; DOWN rows [.][out_ld]
+  int F, Fs, d;
+  float* out_f32;         // DENSE partials [splits][T][M]; MOE down output rows [.][out_ld]
   int out_ld;
-  int shared_row_base;    // DOWN: output row of shared-expert token 0
-  uint16_t* h_out;        // GATEUP routed hidden [rows][h_ld]
-  uint16_t* hs_out;       // GATEUP shared hidden [tokens][hs_ld]
-  int h_ld, hs_ld;
+  int shared_row_base;    // MOE down: output row of shared-expert token 0
+  uint16_t* h_out;        // MOE routed hidden [rows][F]
+  uint16_t* hs_out;       // MOE shared hidden [tokens][Fs]
   float4* lm_part;        // LMHEAD partials [vocab tiles][M]
   float logit_scale_log2; // LMHEAD: log2(e) / temperature
   DevErr err;
@@ -72,26 +111,32 @@ struct GemmParams {
 
 struct GemmTile {
   const CUtensorMap* a0;
-  const CUtensorMap* a1;  // second 64-row A box (GATEUP) or nullptr
+  const CUtensorMap* a1;  // second 64-row A box (gate/up) or nullptr
   int a_row;
   const CUtensorMap* b;
   int b_row;
   int n;      // valid columns
   int nmma;   // MMA N (multiple of 16, <= 128)
   int k0, nk;
-  int split, group, blk;
+  int split, group, blk, chunk;
+  int kind;
+  bool shared;
   bool a_stream;  // A is read once (evict-first)
 };
 
 __device__ __forceinline__ int round16(int x) { return (x + 15) & ~15; }
 
+// rec: the MOE tile record (from the tile list); n_gu: number of gate/up tiles
 template <int MODE>
-__device__ __forceinline__ void decode_tile(const GemmParams& p, int tile, GemmTile& t) {
+__device__ __forceinline__ void decode_tile(const GemmParams& p, int tile, int4 rec, int n_gu, GemmTile& t) {
+  t.chunk = 0;
+  t.shared = false;
   if constexpr (MODE == GEMM_DENSE) {
     const int nt = tile % p.n_tiles_n;
     const int rest = tile / p.n_tiles_n;
     t.split = rest % p.splits;
     const int mt = rest / p.splits;
+    t.kind = KIND_DENSE;
     t.a0 = &p.a_map[0];
     t.a1 = nullptr;
     t.a_row = mt * GEMM_BM;
@@ -107,6 +152,7 @@ __device__ __forceinline__ void decode_tile(const GemmParams& p, int tile, GemmT
   } else if constexpr (MODE == GEMM_LMHEAD) {
     const int vt = tile / p.n_mtiles;
     const int mt = tile % p.n_mtiles;
+    t.kind = KIND_LMHEAD;
     t.a0 = &p.a_map[0];
     t.a1 = nullptr;
     t.a_row = mt * GEMM_BM;
@@ -121,62 +167,148 @@ __device__ __forceinline__ void decode_tile(const GemmParams& p, int tile, GemmT
     t.blk = mt;
     t.a_stream = false;
   } else {
-    const int4 e = p.tiles[tile];
-    const bool shared = e.x == p.n_groups_routed;
-    t.group = e.x;
-    t.blk = e.y;
+    const int4 e = rec;
+    const bool down = tile >= n_gu;
+    t.group = e.x & 0xffff;
+    t.blk = e.x >> 16;
+    t.chunk = e.y;
     t.b_row = e.z;
     t.n = e.w;
     t.nmma = round16(e.w);
     t.k0 = 0;
     t.split = 0;
-    t.a_stream = !shared;
-    if constexpr (MODE == GEMM_GATEUP) {
-      t.a0 = shared ? &p.as_map[0] : &p.a_map[0];
-      t.a1 = shared ? &p.as_map[1] : &p.a_map[1];
-      t.a_row = (shared ? 0 : e.x * p.a_rows_per_group) + e.y * 64;
-      t.b = shared ? &p.bs_map : &p.b_map;
-      t.nk = p.k_steps;
+    t.shared = t.group == p.n_groups_routed;
+    t.a_stream = !t.shared;
+    if (!down) {
+      t.kind = KIND_GATEUP;
+      t.a0 = t.shared ? &p.as_map[0] : &p.a_map[0];
+      t.a1 = t.shared ? &p.as_map[1] : &p.a_map[1];
+      t.a_row = (t.shared ? 0 : t.group * p.F) + t.blk * 64;
+      t.b = t.shared ? &p.bs_map : &p.b_map;
+      t.nk = p.d / GEMM_BK;
     } else {
-      t.a0 = shared ? &p.as_map[0] : &p.a_map[0];
+      t.kind = KIND_DOWN;
+      t.a0 = t.shared ? &p.ds_map : &p.d_map;
       t.a1 = nullptr;
-      t.a_row = (shared ? 0 : e.x * p.a_rows_per_group) + e.y * GEMM_BM;
-      t.b = shared ? &p.bs_map : &p.b_map;
-      t.nk = shared ? p.k_steps_shared : p.k_steps;
+      t.a_row = (t.shared ? 0 : t.group * p.d) + t.blk * GEMM_BM;
+      t.b = t.shared ? &p.hs_map : &p.h_map;
+      t.nk = (t.shared ? p.Fs : p.F) / GEMM_BK;
     }
   }
 }
 
 template <int MODE>
 __device__ __forceinline__ int tile_total(const GemmParams& p) {
-  if constexpr (MODE == GEMM_GATEUP || MODE == GEMM_DOWN) return *p.tile_count;
+  if constexpr (MODE == GEMM_MOE) return p.counts[0] + p.counts[1];
   return p.tiles_static;
 }
 
-// -----------------------------------------------------------------------------
-// epilogues: thread owns TMEM lane (row) `row` of the tile; v = 32 columns
-// -----------------------------------------------------------------------------
+__device__ __forceinline__ int ld_acquire_gpu(const int* ptr) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void red_release_gpu_add(int* ptr, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(ptr), "r"(v) : "memory");
+}
+
+// order this thread's earlier generic-proxy accesses with its later
+// async-proxy (TMA) accesses of global memory
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Wait (bounded) until every gate/up tile of `chunk` has published its rows.
+__device__ __forceinline__ bool wait_chunk_ready(const GemmParams& p, const GemmTile& t) {
+  const int need = (t.shared ? p.Fs : p.F) / 64;
+  const int* flag = p.chunk_done + t.chunk;
+  if (ld_acquire_gpu(flag) < need) {
+    const uint64_t t0 = globaltimer_ns();
+    while (ld_acquire_gpu(flag) < need) {
+      if (globaltimer_ns() - t0 > p.err.limit_ns) {
+        raise_error(p.err, ERR_TIMEOUT);
+        return false;
+      }
+      __nanosleep(64);
+    }
+  }
+  fence_proxy_async_global();
+  return true;
+}
+
+// Store a 128-column x 32-row fp32 block held one column per epilogue thread
+// (thread `col` has v[i] = element (row i, column col)) to dst[i * ld + col]
+// for i < nrows, col < ncols.  The block is transposed through shared memory
+// so each warp instruction writes 512 contiguous bytes as 16-byte vectors.
+// Called by all 128 epilogue threads; dst and ld keep 16-byte alignment.
+__device__ __forceinline__ void store_rows_via_smem(float* stage, const float (&v)[32], int col, int etid,
+                                                    float* dst, int ld, int nrows, int ncols) {
+#pragma unroll
+  for (int i = 0; i < 32; ++i) stage[i * GEMM_BM + col] = v[i];
+  named_bar_sync(1, 128);
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    const int idx = etid + 128 * r;
+    const int i = idx >> 5, c4 = (idx & 31) * 4;
+    if (i < nrows && c4 < ncols) {
+      const float4 x = *reinterpret_cast<const float4*>(stage + i * GEMM_BM + c4);
+      float* d = dst + static_cast<size_t>(i) * ld + c4;
+      if (c4 + 4 <= ncols) {
+        *reinterpret_cast<float4*>(d) = x;
+      } else {
+        d[0] = x.x;
+        if (c4 + 1 < ncols) d[1] = x.y;
+        if (c4 + 2 < ncols) d[2] = x.z;
+      }
+    }
+  }
+  named_bar_sync(1, 128);
+}
+
+template <int MODE>
+constexpr bool claims_tiles() {
+  return MODE == GEMM_MOE;
+}
+
+__device__ __forceinline__ int ld_relaxed_gpu(const int* ptr) {
+  int v;
+  asm volatile("ld.relaxed.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+
 template <int MODE>
 __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_constant__ GemmParams p) {
+  constexpr int STAGES = gemm_stages<MODE>();
+  constexpr int B_BYTES = gemm_b_bytes<MODE>();
+  constexpr int ACC_COLS = gemm_acc_cols<MODE>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
-  uint8_t* sB = sA + GEMM_STAGES * GEMM_A_BYTES;
-  float* xchg = reinterpret_cast<float*>(sB + GEMM_STAGES * GEMM_B_BYTES);
+  uint8_t* sB = sA + STAGES * GEMM_A_BYTES;
+  float* xchg = reinterpret_cast<float*>(sB + STAGES * B_BYTES);
   uint64_t* full = reinterpret_cast<uint64_t*>(xchg + GEMM_XCHG_FLOATS);
-  uint64_t* empty = full + GEMM_STAGES;
-  uint64_t* tfull = empty + GEMM_STAGES;
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* sched_full = drain + 1;
+  uint64_t* sched_empty = sched_full + GEMM_SCHED;
+  int4* sched_rec = reinterpret_cast<int4*>((reinterpret_cast<uintptr_t>(sched_empty + GEMM_SCHED) + 15) &
+                                            ~uintptr_t(15));
+  int* sched = reinterpret_cast<int*>(sched_rec + GEMM_SCHED);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sched + GEMM_SCHED);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int n_tiles = tile_total<MODE>(p);
+  const int n_gu = (MODE == GEMM_MOE) ? p.counts[0] : 0;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < GEMM_STAGES; ++s) {
+    for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -184,12 +316,16 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], 128);
     }
+    for (int s = 0; s < GEMM_SCHED; ++s) {
+      mbar_init(&sched_full[s], 1);
+      mbar_init(&sched_empty[s], 2);  // MMA issuer + epilogue leader
+    }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_holder, GEMM_TMEM_COLS);
+    tmem_alloc(tmem_holder, 2 * ACC_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -206,12 +342,64 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
       const uint64_t pol_last = policy_evict_last();
       int stage = 0;
       uint32_t phase = 0, issued = 0, issued_par = 0;
-      for (int tile = blockIdx.x; tile < n_tiles && !*abort_flag; tile += gridDim.x) {
+      // MOE: the claim of the next tile, its record and its dependency flag
+      // are fetched while the current tile's loads are being issued, so no
+      // global-memory round trip sits between two tiles.
+      int cur = -1, claim = 0, dep_hint = 0;
+      int4 cur_rec = make_int4(0, 0, 0, 0);
+      if constexpr (claims_tiles<MODE>()) {
+        cur = atomicAdd(p.work, 1);
+        if (cur < n_tiles) cur_rec = p.tiles[cur];
+        claim = atomicAdd(p.work, 1);
+      }
+      for (int it = 0;; ++it) {
+        int tile;
+        int4 rec = make_int4(0, 0, 0, 0);
+        int nxt = -1;
+        int4 nxt_rec = make_int4(0, 0, 0, 0);
+        if constexpr (claims_tiles<MODE>()) {
+          if (cur >= n_tiles || *abort_flag) cur = -1;
+          if (cur >= 0 && claim < n_tiles) {
+            nxt = claim;
+            nxt_rec = p.tiles[nxt];          // consumed in the next iteration
+            claim = atomicAdd(p.work, 1);
+          }
+          tile = cur;
+          rec = cur_rec;
+          const int slot = it % GEMM_SCHED;
+          if (!mbar_wait(&sched_empty[slot], ((it / GEMM_SCHED) & 1) ^ 1, p.err)) {
+            *abort_flag = 1;
+            break;
+          }
+          sched[slot] = tile;
+          sched_rec[slot] = rec;
+          mbar_arrive(&sched_full[slot]);
+          if (tile < 0) break;
+        } else {
+          tile = blockIdx.x + it * gridDim.x;
+          if (tile >= n_tiles || *abort_flag) break;
+        }
         GemmTile t;
-        decode_tile<MODE>(p, tile, t);
-        const uint32_t bytes = GEMM_A_BYTES + t.nmma * GEMM_BK * 2;
-        const uint64_t pol_a = (MODE == GEMM_LMHEAD) ? pol_last : (t.a_stream ? pol_first : pol_last);
-        const uint64_t pol_b = (MODE == GEMM_LMHEAD) ? pol_last : pol_last;
+        decode_tile<MODE>(p, tile, rec, n_gu, t);
+        const int cur_hint = dep_hint;
+        dep_hint = 0;
+        if constexpr (MODE == GEMM_MOE) {
+          if (t.kind == KIND_DOWN) {
+            const int need = (t.shared ? p.Fs : p.F) / 64;
+            if (cur_hint >= need) {
+              fence_acq_rel_gpu();          // the early relaxed read saw the release
+              fence_proxy_async_global();
+            } else if (!wait_chunk_ready(p, t)) {
+              *abort_flag = 1;
+              break;
+            }
+          }
+        }
+        // B arrives in whole boxes (rows past nmma are loaded, zero-filled
+        // past the tensor's end, and ignored by the MMA)
+        const int b_rows = (t.nmma + p.b_box_rows - 1) / p.b_box_rows * p.b_box_rows;
+        const uint32_t bytes = GEMM_A_BYTES + b_rows * GEMM_BK * 2;
+        const uint64_t pol_a = t.a_stream ? pol_first : pol_last;
         for (int k = 0; k < t.nk; ++k) {
           if (!mbar_wait(&empty[stage], phase ^ 1, p.err)) {
             *abort_flag = 1;
@@ -219,7 +407,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
           }
           mbar_arrive_expect_tx(&full[stage], bytes);
           uint8_t* a = sA + stage * GEMM_A_BYTES;
-          uint8_t* b = sB + stage * GEMM_B_BYTES;
+          uint8_t* b = sB + stage * B_BYTES;
           const int kx = (t.k0 + k) * GEMM_BK;
           if (t.a1 != nullptr) {
             tma_load_2d(a, t.a0, &full[stage], kx, t.a_row, pol_a);
@@ -228,17 +416,26 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
             tma_load_2d(a, t.a0, &full[stage], kx, t.a_row, pol_a);
           }
           for (int r = 0; r < t.nmma; r += p.b_box_rows)
-            tma_load_2d(b + r * (GEMM_BK * 2), t.b, &full[stage], kx, t.b_row + r, pol_b);
+            tma_load_2d(b + r * (GEMM_BK * 2), t.b, &full[stage], kx, t.b_row + r, pol_last);
+          if constexpr (claims_tiles<MODE>()) {
+            // halfway through this tile, read the next tile's dependency flag
+            if (k == (t.nk >> 1) && nxt >= n_gu) dep_hint = ld_relaxed_gpu(p.chunk_done + nxt_rec.y);
+          }
           issued |= 1u << stage;
           issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
-          if (++stage == GEMM_STAGES) {
+          if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
+        if (*abort_flag) break;
+        if constexpr (claims_tiles<MODE>()) {
+          cur = nxt;
+          cur_rec = nxt_rec;
+        }
       }
       // every copy this thread issued has landed before the CTA may exit
-      for (int s = 0; s < GEMM_STAGES; ++s)
+      for (int s = 0; s < STAGES; ++s)
         if ((issued >> s) & 1) mbar_wait(&full[s], (issued_par >> s) & 1, p.err);
     }
   } else if (warp == 1) {
@@ -247,14 +444,29 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
       int stage = 0;
       uint32_t phase = 0;
       bool aborted = false;
-      int it = 0;
-      for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
+      for (int it = 0;; ++it) {
+        int tile;
+        int4 rec = make_int4(0, 0, 0, 0);
+        if constexpr (claims_tiles<MODE>()) {
+          const int slot = it % GEMM_SCHED;
+          if (!mbar_wait(&sched_full[slot], (it / GEMM_SCHED) & 1, p.err)) {
+            aborted = true;
+            break;
+          }
+          tile = sched[slot];
+          rec = sched_rec[slot];
+          mbar_arrive(&sched_empty[slot]);
+          if (tile < 0) break;
+        } else {
+          tile = blockIdx.x + it * gridDim.x;
+          if (tile >= n_tiles) break;
+        }
         if (*abort_flag) {
           aborted = true;
           break;
         }
         GemmTile t;
-        decode_tile<MODE>(p, tile, t);
+        decode_tile<MODE>(p, tile, rec, n_gu, t);
         const int acc = it & 1;
         const uint32_t acc_par = (it >> 1) & 1;
         if (!mbar_wait(&tempty[acc], acc_par ^ 1, p.err)) {
@@ -262,7 +474,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * GEMM_BN;
+        const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
         const uint32_t idesc = umma_idesc_bf16(GEMM_BM, t.nmma);
         for (int k = 0; k < t.nk; ++k) {
           if (!mbar_wait(&full[stage], phase, p.err)) {
@@ -271,12 +483,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
           }
           tc_fence_after();
           const uint64_t ad = umma_desc_sw128(smem_u32(sA + stage * GEMM_A_BYTES));
-          const uint64_t bd = umma_desc_sw128(smem_u32(sB + stage * GEMM_B_BYTES));
+          const uint64_t bd = umma_desc_sw128(smem_u32(sB + stage * B_BYTES));
 #pragma unroll
           for (int kk = 0; kk < GEMM_BK / 16; ++kk)
             umma_bf16(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (k | kk) != 0);
           umma_commit(&empty[stage]);
-          if (++stage == GEMM_STAGES) {
+          if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
@@ -294,75 +506,97 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
     // ------------------------------ epilogue ----------------------------------
     const int q = warp & 3;              // TMEM lane quarter this warp may access
     const int row = q * 32 + lane;       // tile row owned by this thread
-    int it = 0;
-    for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
+    const int etid = threadIdx.x - 64;   // 0..127
+    for (int it = 0;; ++it) {
+      int tile = -1;
+      int4 rec = make_int4(0, 0, 0, 0);
+      bool ok = *abort_flag == 0;
+      if constexpr (claims_tiles<MODE>()) {
+        const int slot = it % GEMM_SCHED;
+        ok = ok && mbar_wait(&sched_full[slot], (it / GEMM_SCHED) & 1, p.err);
+        if (ok) {
+          tile = sched[slot];
+          rec = sched_rec[slot];
+        }
+      } else {
+        tile = blockIdx.x + it * gridDim.x;
+        if (tile >= n_tiles) tile = -1;
+      }
+      // the four epilogue warps leave together or not at all (they meet at
+      // named barriers inside the tile); the claimed-tile slot is released
+      // only after all of them have read it
+      ok = named_bar_and(2, 128, ok);
+      if constexpr (claims_tiles<MODE>()) {
+        if (ok && etid == 0) mbar_arrive(&sched_empty[it % GEMM_SCHED]);
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        break;
+      }
+      if (tile < 0) break;
       GemmTile t;
-      decode_tile<MODE>(p, tile, t);
+      decode_tile<MODE>(p, tile, rec, n_gu, t);
       const int acc = it & 1;
       const uint32_t acc_par = (it >> 1) & 1;
-      bool ok = (*abort_flag == 0) && mbar_wait(&tfull[acc], acc_par, p.err);
-      // the four epilogue warps leave together or not at all (they meet at
-      // named barriers inside the tile)
+      ok = mbar_wait(&tfull[acc], acc_par, p.err);
       ok = named_bar_and(2, 128, ok);
       if (!ok) {
         *abort_flag = 1;
         break;
       }
       tc_fence_after();
-      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * GEMM_BN;
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * ACC_COLS;
 
       if constexpr (MODE == GEMM_DENSE) {
-        const int m = t.a_row + row;
-        float* out = p.out_f32 + static_cast<size_t>(t.split) * p.T * p.M;
+        float* out = p.out_f32 + static_cast<size_t>(t.split) * p.T * p.M +
+                     static_cast<size_t>(t.b_row) * p.M + t.a_row;
         for (int c0 = 0; c0 < t.n; c0 += 32) {
           float v[32];
           tmem_ld32(tbase + c0, v);
-          if (m < p.M) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int c = c0 + i;
-              if (c < t.n) out[static_cast<size_t>(t.b_row + c) * p.M + m] = v[i];
-            }
-          }
+          store_rows_via_smem(xchg, v, row, etid, out + static_cast<size_t>(c0) * p.M, p.M, min(32, t.n - c0),
+                              p.M - t.a_row);
         }
-      } else if constexpr (MODE == GEMM_GATEUP) {
-        const bool shared = t.group == p.n_groups_routed;
-        uint16_t* hout = shared ? p.hs_out : p.h_out;
-        const int ld = shared ? p.hs_ld : p.h_ld;
-        const int col = t.blk * 64 + (row & 63);
-        for (int c0 = 0; c0 < t.n; c0 += 32) {
-          float v[32];
-          tmem_ld32(tbase + c0, v);
-          if (row < 64) {
+      } else if constexpr (MODE == GEMM_MOE) {
+        if (t.kind == KIND_GATEUP) {
+          uint16_t* hout = t.shared ? p.hs_out : p.h_out;
+          const int ld = t.shared ? p.Fs : p.F;
+          const int col = t.blk * 64 + (row & 63);
+          for (int c0 = 0; c0 < t.n; c0 += 32) {
+            float v[32];
+            tmem_ld32(tbase + c0, v);
+            if (row < 64) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) xchg[row * 33 + i] = v[i];
-          }
-          named_bar_sync(1, 128);
-          if (row >= 64) {
-            const float* gv = xchg + (row - 64) * 33;
+              for (int i = 0; i < 32; ++i) xchg[row * 33 + i] = v[i];
+            }
+            named_bar_sync(1, 128);
+            if (row >= 64) {
+              const float* gv = xchg + (row - 64) * 33;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int c = c0 + i;
-              if (c < t.n) {
-                const float g = gv[i];
-                const float h = g / (1.f + __expf(-g)) * v[i];
-                hout[static_cast<size_t>(t.b_row + c) * ld + col] = f32_to_bf16(h);
+              for (int i = 0; i < 32; ++i) {
+                const int c = c0 + i;
+                if (c < t.n) {
+                  const float g = gv[i];
+                  const float h = g / (1.f + __expf(-g)) * v[i];
+                  hout[static_cast<size_t>(t.b_row + c) * ld + col] = f32_to_bf16(h);
+                }
               }
             }
+            named_bar_sync(1, 128);
           }
+          // publish the hidden rows: every writer's stores are ordered before
+          // one release increment of the chunk's counter
+          __threadfence();
+          fence_proxy_async_global();
           named_bar_sync(1, 128);
-        }
-      } else if constexpr (MODE == GEMM_DOWN) {
-        const bool shared = t.group == p.n_groups_routed;
-        const int m = t.blk * GEMM_BM + row;
-        const int r0 = (shared ? p.shared_row_base : 0) + t.b_row;
-        for (int c0 = 0; c0 < t.n; c0 += 32) {
-          float v[32];
-          tmem_ld32(tbase + c0, v);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int c = c0 + i;
-            if (c < t.n) p.out_f32[static_cast<size_t>(r0 + c) * p.out_ld + m] = v[i];
+          if (etid == 0) red_release_gpu_add(p.chunk_done + t.chunk, 1);
+        } else {
+          const int r0 = (t.shared ? p.shared_row_base : 0) + t.b_row;
+          float* out = p.out_f32 + static_cast<size_t>(r0) * p.out_ld + t.blk * GEMM_BM;
+          for (int c0 = 0; c0 < t.n; c0 += 32) {
+            float v[32];
+            tmem_ld32(tbase + c0, v);
+            store_rows_via_smem(xchg, v, row, etid, out + static_cast<size_t>(c0) * p.out_ld, p.out_ld,
+                                min(32, t.n - c0), GEMM_BM);
           }
         }
       } else {  // GEMM_LMHEAD
@@ -398,7 +632,18 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, GEMM_TMEM_COLS);
+    tmem_dealloc(tmem_base, 2 * ACC_COLS);
+  }
+  if constexpr (claims_tiles<MODE>()) {
+    // the last CTA out resets the claim counter for the next launch (all
+    // claims of this launch were made before their CTA reached this point)
+    if (threadIdx.x == 0) {
+      __threadfence();
+      if (atomicAdd(p.work + 1, 1) == static_cast<int>(gridDim.x) - 1) {
+        atomicExch(p.work, 0);
+        atomicExch(p.work + 1, 0);
+      }
+    }
   }
 }
 

@@ -94,13 +94,16 @@ __global__ void router_topk_kernel(const float* __restrict__ part, int splits, i
 }
 
 // Stable permutation of the T*k (token, slot) pairs by expert, expert counts,
-// and the grouped GEMM tile lists (the shared expert is group E with all T
-// tokens).  One CTA of 1024 threads.
+// and the tile list of the fused expert GEMM (the shared expert is group E
+// with all T tokens).  One CTA of 1024 threads.
 //   perm_tok[pos]   token of permuted row pos
 //   inv_slot[p]     permuted row of pair p = t*k + j
-//   gu_tiles: {group, 64-row block, first row, rows}   (gate/up)
-//   dn_tiles: {group, 128-row block, first row, rows}  (down)
-//   counters[0] = gate/up tiles, counters[1] = down tiles, counters[2] = experts hit
+//   tiles           gate/up tiles, then down tiles, each
+//                   {group | block << 16, token chunk, first row, rows};
+//                   groups in the order shared, 0, 1, ..., E-1
+//   chunk_done[c]   zeroed (gate/up tiles of chunk c finished)
+//   counters[0] = gate/up tiles, [1] = down tiles, [2] = experts hit,
+//   counters[3] = tile claim counter (zeroed)
 constexpr int PERM_THREADS = 1024;
 constexpr int PERM_MAXE = 256;
 
@@ -108,9 +111,9 @@ __global__ void __launch_bounds__(PERM_THREADS) permute_kernel(const int32_t* __
                                                                int E, int F, int Fs, int d,
                                                                int32_t* __restrict__ perm_tok,
                                                                int32_t* __restrict__ inv_slot,
-                                                               int4* __restrict__ gu_tiles,
-                                                               int4* __restrict__ dn_tiles,
-                                                               int32_t* __restrict__ counters) {
+                                                               int4* __restrict__ tiles,
+                                                               int32_t* __restrict__ chunk_done,
+                                                               int32_t* __restrict__ counters, int chunk_rows) {
   __shared__ int wcount[32][PERM_MAXE + 1];  // per-warp per-expert counts, then bases
   __shared__ int offs[PERM_MAXE + 2];
   __shared__ int gu_off[PERM_MAXE + 2];
@@ -148,34 +151,39 @@ __global__ void __launch_bounds__(PERM_THREADS) permute_kernel(const int32_t* __
     offs[e] = run;  // count, scanned below
   }
   __syncthreads();
+  __shared__ int ch_off[PERM_MAXE + 2];
   if (threadIdx.x == 0) {
-    int run = 0, gu = 0, dn = 0, hit = 0;
     const int mb_gu = F / 64, mb_dn = d / 128;
+    // shared expert first (all T tokens), then the routed experts in order
+    const int sch = (T + chunk_rows - 1) / chunk_rows;
+    gu_off[E] = 0;
+    dn_off[E] = 0;
+    ch_off[E] = 0;
+    int gu = sch * (Fs / 64), dn = sch * mb_dn, ch = sch;
+    int run = 0, hit = 0;
     for (int e = 0; e < E; ++e) {
       const int c = offs[e];
       offs[e] = run;
       run += c;
-      const int chunks = (c + 127) / 128;
+      const int chunks = (c + chunk_rows - 1) / chunk_rows;
       gu_off[e] = gu;
       dn_off[e] = dn;
+      ch_off[e] = ch;
       gu += chunks * mb_gu;
       dn += chunks * mb_dn;
+      ch += chunks;
       hit += c > 0;
     }
     offs[E] = run;
-    // shared expert: all T tokens
-    const int sch = (T + 127) / 128;
-    gu_off[E] = gu;
-    dn_off[E] = dn;
-    gu += sch * (Fs / 64);
-    dn += sch * mb_dn;
-    gu_off[E + 1] = gu;
-    dn_off[E + 1] = dn;
+    gu_off[E + 1] = gu;  // total gate/up tiles: the down tiles follow them in the list
+    ch_off[E + 1] = ch;
     counters[0] = gu;
     counters[1] = dn;
     counters[2] = hit;
+    counters[3] = 0;
   }
   __syncthreads();
+  for (int c = threadIdx.x; c < ch_off[E + 1]; c += blockDim.x) chunk_done[c] = 0;
   // pass 2: positions
   for (int c = p_begin; c < p_end; c += 32) {
     const int p = c + lane;
@@ -192,18 +200,25 @@ __global__ void __launch_bounds__(PERM_THREADS) permute_kernel(const int32_t* __
     }
     __syncwarp();
   }
-  // tile lists (one thread per group)
+  // tile list (one thread per group)
+  const int n_gu = gu_off[E + 1];
   for (int g = threadIdx.x; g <= E; g += blockDim.x) {
     const bool shared = g == E;
     const int first = shared ? 0 : offs[g];
     const int cnt = shared ? T : offs[g + 1] - offs[g];
     const int mb_gu = (shared ? Fs : F) / 64, mb_dn = d / 128;
-    int gi = gu_off[g], di = dn_off[g];
-    for (int c0 = 0; c0 < cnt; c0 += 128) {
-      const int rows = min(128, cnt - c0);
-      for (int j = 0; j < mb_gu; ++j) gu_tiles[gi++] = make_int4(g, j, first + c0, rows);
-      for (int j = 0; j < mb_dn; ++j) dn_tiles[di++] = make_int4(g, j, first + c0, rows);
-    }
+    const int nch = (cnt + chunk_rows - 1) / chunk_rows;
+    int gi = gu_off[g], di = n_gu + dn_off[g];
+    // block-major: the chunk tiles of one weight block sit next to each other,
+    // so the re-reads of that block hit L2
+    for (int j = 0; j < mb_gu; ++j)
+      for (int ch = 0; ch < nch; ++ch)
+        tiles[gi++] = make_int4(g | (j << 16), ch_off[g] + ch, first + ch * chunk_rows,
+                                min(chunk_rows, cnt - ch * chunk_rows));
+    for (int j = 0; j < mb_dn; ++j)
+      for (int ch = 0; ch < nch; ++ch)
+        tiles[di++] = make_int4(g | (j << 16), ch_off[g] + ch, first + ch * chunk_rows,
+                                min(chunk_rows, cnt - ch * chunk_rows));
   }
 }
 

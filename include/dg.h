@@ -51,7 +51,8 @@ typedef enum dg_status {
 /* Model shape and capacities.
  * Supported shapes: d_model, expert_hidden and shared_hidden multiples of 64;
  * head_dim in {64, 128, 176}; n_q_heads a multiple of n_kv_heads; vocab a
- * multiple of 128; top_k <= 16 and <= n_experts <= 256; canvas a multiple of 16
+ * multiple of 128; top_k <= 16 and <= n_experts <= 256, n_experts a multiple
+ * of 4; d_model a multiple of 128 and <= 4096; canvas a multiple of 16
  * and <= 256.  The three output projections of a layer are the only places
  * where a layer writes the residual stream. */
 typedef struct dg_config {
@@ -207,18 +208,19 @@ dg_status dg_debug_wait_timeout(dg_ctx* ctx, uint64_t limit_ns);
 /* One weight-streaming GEMM through the tcgen05 kernel alone:
  * out_dev [splits, T, M] fp32 holds, for each split s of the K range, the
  * partial sums of x_dev [T, K] bf16 times w_dev [M, K] bf16 transposed (the
- * caller adds the splits).  K a multiple of 64, 1 <= splits <= K/64. */
+ * caller adds the splits).  K a multiple of 64, M a multiple of 4,
+ * 1 <= splits <= K/64. */
 dg_status dg_debug_gemm(dg_ctx* ctx, const void* w_dev, int32_t M, int32_t K, const void* x_dev, int32_t T,
                         int32_t splits, float* out_dev);
 
 /* Kernel classes timed by the profiling hooks. */
 enum {
-  DG_PROF_EXPERT_GATEUP = 0, /* grouped routed + shared expert gate/up GEMM (SwiGLU epilogue) */
-  DG_PROF_EXPERT_DOWN = 1,   /* grouped expert down GEMM                                      */
+  DG_PROF_EXPERTS = 0,       /* fused routed + shared expert GEMM: gate/up (SwiGLU) and down   */
+  DG_PROF_ROUTING = 1,       /* router top-k, token permutation and row gather                 */
   DG_PROF_LMHEAD = 2,        /* LM-head GEMM with the argmax / log-sum-exp epilogue            */
   DG_PROF_ATTENTION = 3,     /* attention kernel (+ chunk merge)                               */
   DG_PROF_DENSE = 4,         /* QKV, output and router projections                            */
-  DG_PROF_OTHER = 5,         /* norms, RoPE, routing, gather, combine, sampler                */
+  DG_PROF_OTHER = 5,         /* norms, RoPE, combine, LM-head merge + sampler                 */
   DG_PROF_CLASSES = 6
 };
 

@@ -22,14 +22,14 @@ def rel_l2(a, b) -> float:
 
 
 def make_context(w: si.Workload, temperature: float = 1.0, layer_override=None, max_seq: int | None = None,
-                 prefill_rows: int = 0, weights=None):
+                 prefill_rows: int = 0, weights=None, stream=None):
     if weights is None:
         weights = si.model_weights(w, "cuda", layer_override)
     if max_seq is None:
         max_seq = w.prefix + w.canvas * (w.blocks + 1)
     cfg = dgp.config_from_shape(w.shape, max_batch=w.batch, max_seq=max_seq, canvas=w.canvas,
                                 temperature=temperature, prefill_rows=prefill_rows)
-    return dgp.Context(cfg, weights), weights
+    return dgp.Context(cfg, weights, stream=stream), weights
 
 
 def gpu_step(ctx, w, canvas, step, seed, tau, capture=False):
@@ -140,6 +140,15 @@ def compare_step(g: dict, r: "oracle.StepResult", tau: float, orc=None, check_hi
     if out["logp_abs_max"] > logp_tol:
         fails.append(f"logp max abs {out['logp_abs_max']:.4g} > {logp_tol:.4g}")
     excl = (r.margin < EXCLUDE_BAND) | (np.abs(r.conf - tau) < EXCLUDE_BAND) | diverged
+    if temperature < 1.0:
+        # Below T = 1 a confidence moves by up to conf * (e^{logp error} - 1),
+        # far beyond the 1e-3 band; a position whose two confidences fall on
+        # opposite sides of tau while its logp agrees within the tolerance is
+        # exempt.  (The decision given a confidence is checked bit-exact by
+        # the sampler hook test.)
+        straddle = ((g["conf"] >= tau) != (r.conf >= tau)) & (dlogp <= logp_tol)
+        out["straddle_exempt"] = int(straddle.sum())
+        excl = excl | straddle
     mism = g["canvas_out"] != r.canvas_out
     out["token_mismatch"] = int((mism & ~excl).sum())
     out["excluded"] = int(excl.sum())

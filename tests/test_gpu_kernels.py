@@ -33,7 +33,7 @@ def test_tcgen05_gemm_matches_fp64_matmul(tiny_ctx, M, K, T, splits):
     g = torch.Generator().manual_seed(M * 7 + K + T)
     w = _bf16(torch.randn(M, K, generator=g) * 0.05)
     x = _bf16(torch.randn(T, K, generator=g))
-    out = torch.empty(splits, T, M, dtype=torch.float32, device="cuda")
+    out = torch.full((splits, T, M), float("nan"), dtype=torch.float32, device="cuda")
     ctx.debug_gemm(w.cuda(), x.cuda(), splits, out)
     ctx.sync()
     got = out.sum(0).cpu().double()

@@ -132,6 +132,47 @@ def test_step_is_deterministic_and_host_variant_matches():
     ctx.close()
 
 
+def test_graph_step_matches_eager_launches():
+    """On a non-default stream the step runs as one captured CUDA graph whose
+    first and last kernels are rebound per call; it must give the same bits
+    as the kernels launched one by one, across changes of step, seed, tau and
+    buffers, and again after a block commit (which changes the cached length)."""
+    w = si.workload("small").with_(prefix=512)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        ctx, _ = make_context(w, temperature=0.05, stream=s.cuda_stream)
+        ctx.prefill(si.uniform_tokens(w, "prefix", 1, 512, device="cuda"))
+        canvas = si.uniform_tokens(w, "canvas", 1, 256, device="cuda")
+
+        def run(step, seed, tau, eager):
+            out = torch.empty_like(canvas)
+            conf = torch.empty(1, 256, dtype=torch.float32, device="cuda")
+            settled = torch.empty(1, dtype=torch.int32, device="cuda")
+            if eager:
+                ctx.debug_profile(["other"])       # any profiling forces one-by-one launches
+            ctx.denoise_step(canvas, step, seed, tau, out, conf, settled)
+            if eager:
+                ctx.debug_profile([])
+            ctx.sync()
+            return out.cpu(), conf.cpu(), settled.cpu()
+
+        for step, seed, tau in ((0, 1, 0.9), (3, 77, 0.5), (3, 77, 0.5), (9, 2 ** 40 + 5, 0.0)):
+            g = run(step, seed, tau, eager=False)
+            e = run(step, seed, tau, eager=True)
+            for a, b in zip(g, e):
+                assert torch.equal(a, b)
+        n0 = ctx.launch_count
+        run(1, 1, 0.9, eager=False)
+        per_step = ctx.launch_count - n0
+        assert per_step > 0
+        ctx.commit_block(canvas)
+        g = run(1, 5, 0.7, eager=False)
+        e = run(1, 5, 0.7, eager=True)
+        for a, b in zip(g, e):
+            assert torch.equal(a, b)
+        ctx.close()
+
+
 def test_planted_identity_tiny():
     w = si.workload("tiny").with_(prefix=32)
 
