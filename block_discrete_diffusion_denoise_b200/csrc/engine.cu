@@ -11,7 +11,7 @@
 #include <vector>
 
 #include "../../include/dg.h"
-#include "attention.cuh"
+#include "attention_tc.cuh"
 #include "common.cuh"
 #include "gemm.cuh"
 #include "kernels.cuh"
@@ -26,6 +26,7 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
 
 struct LayerMaps {
   CUtensorMap wqkv, wo, wr, wg, wu, wd, wsg, wsu, wsd;
+  CUtensorMap kc, vc;  // this layer's K / V cache rows, 64 x 64 boxes
 };
 
 }  // namespace
@@ -43,7 +44,7 @@ struct dg_ctx {
   int d = 0, D = 0, Hq = 0, Hkv = 0, E = 0, k = 0, F = 0, Fs = 0, V = 0, L = 0, QKV = 0, HD = 0;
   int R = 0;        // workspace rows (max of step rows and prefill rows)
   int R_step = 0;   // max_batch * canvas
-  size_t part_cap = 0, opart_rows_cap = 0;
+  size_t part_cap = 0;
   // device buffers
   void* ws = nullptr;
   uint16_t* kcache = nullptr;
@@ -53,8 +54,6 @@ struct dg_ctx {
   float* part = nullptr;
   uint16_t* q = nullptr;
   uint16_t* o = nullptr;
-  float* opart = nullptr;
-  float2* ml = nullptr;
   int32_t* idx = nullptr;
   float* gates = nullptr;
   int32_t* perm_tok = nullptr;
@@ -62,8 +61,7 @@ struct dg_ctx {
   int4* tiles = nullptr;        // fused expert GEMM tile list (gate/up, then down)
   int32_t* chunk_done = nullptr;
   int32_t* dense_work = nullptr;   // claim / exit counters of the dense GEMM
-  int32_t* qb_count = nullptr;     // attention: finished key chunks per query block
-  size_t qb_count_cap = 0;
+  int attn_max_clusters[ATC_MAX_CHUNKS + 1] = {};  // co-resident attention clusters per cluster size
   // CUDA graph of the denoising step (per batch and cached length)
   bool use_graphs = true;
   cudaGraph_t step_graph = nullptr;
@@ -97,6 +95,7 @@ struct dg_ctx {
   // tensor maps
   std::vector<LayerMaps> lmaps;
   CUtensorMap m_u16{}, m_u64{}, m_u128{}, m_o64{}, m_xp16{}, m_h16{}, m_hs16{}, m_embed{};
+  CUtensorMap m_q4{};  // queries as (D, G, Hkv, token): one GQA group's rows per box
   // state
   int B = 0;
   int P = 0;
@@ -160,6 +159,22 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
   cuuint32_t box[2] = {64, box_rows};
   cuuint32_t es[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Queries [token][Hq][D] seen as 4-D (D, G, Hkv, token): a box of 64 columns x
+// G heads x 1 kv head x 128/G tokens is the 128 packed rows (row = token * G +
+// head) of one GQA group, 128-byte swizzled.  Requires 128 % G == 0.
+bool make_map_q4(CUtensorMap* m, const void* base, uint64_t tokens, int Hkv, int G, int D) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc || base == nullptr) return false;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(G), static_cast<cuuint64_t>(Hkv), tokens};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(G) * D * 2,
+                           static_cast<cuuint64_t>(Hkv) * G * D * 2};
+  cuuint32_t box[4] = {64, static_cast<cuuint32_t>(G), 1, static_cast<cuuint32_t>(ATC_BQ / G)};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -237,15 +252,51 @@ dg_status gemm_dense(dg_ctx* c, const CUtensorMap& w, const CUtensorMap& x, int 
   return DG_OK;
 }
 
+template <int D>
+cudaError_t launch_attention(const AttnTcParams& p, dim3 grid, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(ATC_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = AtcCfg<D>::SMEM;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = grid.z;  // the key chunks of one query block
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, attn_tc_kernel<D>, p);
+}
+
+template <int D>
+cudaError_t attention_cluster_limits(dg_ctx* c) {
+  for (int nc = 1; nc <= ATC_MAX_CHUNKS; ++nc) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(1, 1, nc);
+    cfg.blockDim = dim3(ATC_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = AtcCfg<D>::SMEM;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = nc;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int num = 0;
+    cudaError_t e = cudaOccupancyMaxActiveClusters(&num, attn_tc_kernel<D>, &cfg);
+    if (e != cudaSuccess) return e;
+    c->attn_max_clusters[nc] = num;
+  }
+  return cudaSuccess;
+}
+
 dg_status attention(dg_ctx* c, int l, int B, int n, int pos0, bool causal) {
-  const size_t layer_off = static_cast<size_t>(l) * c->cfg.max_batch * c->Hkv * c->cfg.max_seq * c->D;
-  AttnParams p;
-  p.q = c->q;
-  p.kc = c->kcache + layer_off;
-  p.vc = c->vcache + layer_off;
+  AttnTcParams p;
+  p.q_map = c->m_q4;
+  p.k_map = c->lmaps[l].kc;
+  p.v_map = c->lmaps[l].vc;
   p.o = c->o;
-  p.opart = c->opart;
-  p.ml = c->ml;
   p.n = n;
   p.B = B;
   p.Hq = c->Hq;
@@ -254,38 +305,40 @@ dg_status attention(dg_ctx* c, int l, int B, int n, int pos0, bool causal) {
   p.pos0 = pos0;
   p.causal = causal ? 1 : 0;
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c->D)));
+  p.err = dev_err(c);
   const int G = c->Hq / c->Hkv;
-  const int qblocks = (n * G + ATT_QROWS - 1) / ATT_QROWS;
-  const int ctas = qblocks * B * c->Hkv;
+  const int qblocks = (n * G + ATC_BQ - 1) / ATC_BQ;
+  const int clusters = qblocks * B * c->Hkv;
   const int keys = pos0 + n;
-  const size_t rows = static_cast<size_t>(B) * n * c->Hq;
-  // split the keys so that all CTAs fit in one wave (two CTAs per SM)
-  int n_chunks = std::max(1, (2 * c->sms) / ctas);
-  n_chunks = std::min(n_chunks, std::max(1, (keys + 255) / 256));
-  n_chunks = std::min<int>(n_chunks, static_cast<int>(c->opart_rows_cap / rows));
-  n_chunks = std::min(n_chunks, ATT_MAX_CHUNKS);
-  n_chunks = std::max(n_chunks, 1);
-  int chunk_len = ((keys + n_chunks - 1) / n_chunks + ATT_KB - 1) / ATT_KB * ATT_KB;
+  // Split the keys into the largest cluster of chunks (at least 256 keys
+  // each) for which every cluster is resident at once; one chunk otherwise.
+  int n_chunks = 1;
+  for (int nc = std::min(ATC_MAX_CHUNKS, std::max(1, keys / 256)); nc > 1; --nc)
+    if (clusters <= c->attn_max_clusters[nc]) {
+      n_chunks = nc;
+      break;
+    }
+  const int chunk_len = ((keys + n_chunks - 1) / n_chunks + ATC_BK - 1) / ATC_BK * ATC_BK;
   n_chunks = (keys + chunk_len - 1) / chunk_len;
-  if (static_cast<size_t>(ctas) > c->qb_count_cap) return fail(c, DG_ERR_CAPACITY, "attention: %d query blocks", ctas);
   p.chunk_len = chunk_len;
   p.n_chunks = n_chunks;
-  p.qb_count = c->qb_count;
-  dim3 grid(qblocks, B * c->Hkv, n_chunks);
+  const dim3 grid(qblocks, B * c->Hkv, n_chunks);
   ProfScope ps1(c, DG_PROF_ATTENTION);
+  cudaError_t e;
   switch (c->D) {
     case 64:
-      attn_kernel<64><<<grid, 128, att_smem_bytes<64>(), c->stream>>>(p);
+      e = launch_attention<64>(p, grid, c->stream);
       break;
     case 128:
-      attn_kernel<128><<<grid, 128, att_smem_bytes<128>(), c->stream>>>(p);
+      e = launch_attention<128>(p, grid, c->stream);
       break;
     case 176:
-      attn_kernel<176><<<grid, 128, att_smem_bytes<176>(), c->stream>>>(p);
+      e = launch_attention<176>(p, grid, c->stream);
       break;
     default:
       return fail(c, DG_ERR_UNSUPPORTED, "head_dim %d", c->D);
   }
+  if (e != cudaSuccess) return fail(c, DG_ERR_CUDA, "attention launch: %s", cudaGetErrorString(e));
   DG_LAUNCHED(c);
   ps1.end();
   return DG_OK;
@@ -466,9 +519,9 @@ dg_status set_smem_attrs(dg_ctx* c) {
                                   gemm_smem_bytes<GEMM_MOE>()));
   DG_CUDA(c, cudaFuncSetAttribute(gemm_kernel<GEMM_LMHEAD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   gemm_smem_bytes<GEMM_LMHEAD>()));
-  DG_CUDA(c, cudaFuncSetAttribute(attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, att_smem_bytes<64>()));
-  DG_CUDA(c, cudaFuncSetAttribute(attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, att_smem_bytes<128>()));
-  DG_CUDA(c, cudaFuncSetAttribute(attn_kernel<176>, cudaFuncAttributeMaxDynamicSharedMemorySize, att_smem_bytes<176>()));
+  DG_CUDA(c, cudaFuncSetAttribute(attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, AtcCfg<64>::SMEM));
+  DG_CUDA(c, cudaFuncSetAttribute(attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, AtcCfg<128>::SMEM));
+  DG_CUDA(c, cudaFuncSetAttribute(attn_tc_kernel<176>, cudaFuncAttributeMaxDynamicSharedMemorySize, AtcCfg<176>::SMEM));
   return DG_OK;
 }
 
@@ -601,7 +654,7 @@ dg_status dg_create(const dg_config* cfg, const dg_weights* w, void* cuda_stream
     return reject(DG_ERR_INVALID_ARG, "non-positive dimension");
   if (g.d_model % 128 || g.d_model > 4096 || g.expert_hidden % 64 || g.shared_hidden % 64 || g.vocab % 128 ||
       (g.head_dim != 64 && g.head_dim != 128 && g.head_dim != 176) || g.n_q_heads % g.n_kv_heads ||
-      (g.n_q_heads * g.head_dim) % 64 || g.n_experts > PERM_MAXE || g.n_experts % 4 || g.top_k > 16 || g.top_k > g.n_experts ||
+      (g.n_q_heads * g.head_dim) % 64 || ATC_BQ % (g.n_q_heads / g.n_kv_heads) || g.n_experts > PERM_MAXE || g.n_experts % 4 || g.top_k > 16 || g.top_k > g.n_experts ||
       g.canvas % 16 || g.canvas > 256 || g.max_seq < g.canvas)
     return reject(DG_ERR_UNSUPPORTED, "unsupported shape");
   if (!w->embed || !w->final_norm || !w->layers) return reject(DG_ERR_INVALID_ARG, "null weights");
@@ -644,19 +697,23 @@ dg_status dg_create(const dg_config* cfg, const dg_weights* w, void* cuda_stream
     delete c;
     return DG_ERR_CUDA;
   }
+  e = c->D == 64 ? attention_cluster_limits<64>(c)
+                 : c->D == 128 ? attention_cluster_limits<128>(c) : attention_cluster_limits<176>(c);
+  if (e != cudaSuccess) {
+    delete c;
+    return DG_ERR_CUDA;
+  }
 
   // ---- workspace plan ----
   const size_t R = c->R, d = c->d, k = c->k;
   const size_t mmax = std::max<size_t>({static_cast<size_t>(c->QKV), d, static_cast<size_t>(c->E)});
   c->part_cap = std::max<size_t>(R, 5 * 256) * mmax;
-  c->opart_rows_cap = std::max<size_t>(16 * 256, 2 * R) * c->Hq;
   const size_t CH = MOE_CHUNK_ROWS;
   const size_t chunks_max = (R * k + CH - 1) / CH + c->E;  // routed token chunks
   const size_t chunks_shared = (R + CH - 1) / CH;
   c->max_gu_tiles = chunks_max * (c->F / 64) + chunks_shared * (c->Fs / 64);
   c->max_dn_tiles = (chunks_max + chunks_shared) * (d / 128);
   c->max_chunks = chunks_max + chunks_shared;
-  c->qb_count_cap = static_cast<size_t>(c->Hkv) * ((R * (c->Hq / c->Hkv) + ATT_QROWS - 1) / ATT_QROWS + g.max_batch);
   size_t bytes = 0;
   auto add = [&](size_t n, size_t sz) { bytes += (n * sz + 255) / 256 * 256; };
   add(R * d, 4);                                  // h
@@ -664,8 +721,6 @@ dg_status dg_create(const dg_config* cfg, const dg_weights* w, void* cuda_stream
   add(c->part_cap, 4);                            // part
   add(R * c->HD, 2);                              // q
   add(R * c->HD, 2);                              // o
-  add(c->opart_rows_cap * c->D, 4);               // opart
-  add(c->opart_rows_cap, 8);                      // ml
   add(R * k, 4);                                  // idx
   add(R * k, 4);                                  // gates
   add(R * k, 4);                                  // perm_tok
@@ -673,7 +728,6 @@ dg_status dg_create(const dg_config* cfg, const dg_weights* w, void* cuda_stream
   add(c->max_gu_tiles + c->max_dn_tiles, 16);    // tiles
   add(c->max_chunks, 4);                          // chunk_done
   add(2, 4);                                      // dense_work
-  add(c->qb_count_cap, 4);                        // qb_count
   add(16, 4);                                     // counters
   add(R * k * d, 2);                              // xp
   add(R * k * c->F, 2);                           // hbuf
@@ -702,8 +756,6 @@ dg_status dg_create(const dg_config* cfg, const dg_weights* w, void* cuda_stream
   c->part = carve<float>(cur, c->part_cap);
   c->q = carve<uint16_t>(cur, R * c->HD);
   c->o = carve<uint16_t>(cur, R * c->HD);
-  c->opart = carve<float>(cur, c->opart_rows_cap * c->D);
-  c->ml = carve<float2>(cur, c->opart_rows_cap);
   c->idx = carve<int32_t>(cur, R * k);
   c->gates = carve<float>(cur, R * k);
   c->perm_tok = carve<int32_t>(cur, R * k);
@@ -711,7 +763,6 @@ dg_status dg_create(const dg_config* cfg, const dg_weights* w, void* cuda_stream
   c->tiles = carve<int4>(cur, c->max_gu_tiles + c->max_dn_tiles);
   c->chunk_done = carve<int32_t>(cur, c->max_chunks);
   c->dense_work = carve<int32_t>(cur, 2);
-  c->qb_count = carve<int32_t>(cur, c->qb_count_cap);
   c->counters = carve<int32_t>(cur, 16);
   c->xp = carve<uint16_t>(cur, R * k * d);
   c->hbuf = carve<uint16_t>(cur, R * k * c->F);
@@ -779,7 +830,12 @@ dg_status dg_create(const dg_config* cfg, const dg_weights* w, void* cuda_stream
     ok &= make_map(&m.wsg, lw.ws_gate, c->Fs, d, 64);
     ok &= make_map(&m.wsu, lw.ws_up, c->Fs, d, 64);
     ok &= make_map(&m.wsd, lw.ws_down, d, c->Fs, 128);
+    const size_t layer_off = static_cast<size_t>(l) * g.max_batch * c->Hkv * g.max_seq * c->D;
+    const uint64_t cache_rows = static_cast<uint64_t>(g.max_batch) * c->Hkv * g.max_seq;
+    ok &= make_map(&m.kc, c->kcache + layer_off, cache_rows, c->D, 64);
+    ok &= make_map(&m.vc, c->vcache + layer_off, cache_rows, c->D, 64);
   }
+  ok &= make_map_q4(&c->m_q4, c->q, R, c->Hkv, c->Hq / c->Hkv, c->D);
   ok &= make_map(&c->m_u16, c->u, R, d, 16);
   ok &= make_map(&c->m_u64, c->u, R, d, 64);
   ok &= make_map(&c->m_u128, c->u, R, d, 128);
