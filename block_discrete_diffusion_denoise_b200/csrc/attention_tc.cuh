@@ -371,21 +371,39 @@ __global__ void __launch_bounds__(ATC_THREADS, 1) attn_tc_kernel(const __grid_co
     const int r_lo = rank * rpr, r_hi = min(ATC_BQ, r_lo + rpr);
     constexpr int D4 = D / 4;
     const uint32_t os_at = smem_u32(osm);
-    for (int it = threadIdx.x - 64; it < (r_hi - r_lo) * D4; it += 256) {
-      const int rr = r_lo + it / D4, c4 = (it % D4) * 4;
-      const int rg = row_base + rr;
-      if (rg >= rows_total) continue;
-      const uint32_t off = static_cast<uint32_t>((rr * C::OS_LD + c4) * 4);
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int q = 0; q < nc; ++q) {
-        const float4 v = ld_dsmem_f4(mapa_shared(os_at + off, q));
-        acc.x += v.x;
-        acc.y += v.y;
-        acc.z += v.z;
-        acc.w += v.w;
+    // two items per pass, all their peer loads issued before any is used
+    const int n_items = (r_hi - r_lo) * D4;
+    for (int it0 = threadIdx.x - 64; it0 < n_items; it0 += 512) {
+      float4 acc[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
+      float4 v[2][ATC_MAX_CHUNKS];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int it = it0 + 256 * h;
+        const int rr = r_lo + it / D4, c4 = (it % D4) * 4;
+        const uint32_t off = static_cast<uint32_t>((rr * C::OS_LD + c4) * 4);
+#pragma unroll
+        for (int q = 0; q < ATC_MAX_CHUNKS; ++q)
+          if (q < nc && it < n_items) v[h][q] = ld_dsmem_f4(mapa_shared(os_at + off, q));
       }
-      const size_t rid = (static_cast<size_t>(b) * p.n + rg / G) * p.Hq + kvh * G + rg % G;
-      *reinterpret_cast<uint2*>(p.o + rid * D + c4) = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int it = it0 + 256 * h;
+        if (it >= n_items) continue;
+#pragma unroll
+        for (int q = 0; q < ATC_MAX_CHUNKS; ++q)
+          if (q < nc) {
+            acc[h].x += v[h][q].x;
+            acc[h].y += v[h][q].y;
+            acc[h].z += v[h][q].z;
+            acc[h].w += v[h][q].w;
+          }
+        const int rr = r_lo + it / D4, c4 = (it % D4) * 4;
+        const int rg = row_base + rr;
+        if (rg >= rows_total) continue;
+        const size_t rid = (static_cast<size_t>(b) * p.n + rg / G) * p.Hq + kvh * G + rg % G;
+        *reinterpret_cast<uint2*>(p.o + rid * D + c4) =
+            make_uint2(pack_bf16x2(acc[h].x, acc[h].y), pack_bf16x2(acc[h].z, acc[h].w));
+      }
     }
   }
   cluster_sync_all();  // no CTA leaves while a peer may still read its shared memory

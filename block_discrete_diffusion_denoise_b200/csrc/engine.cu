@@ -60,6 +60,7 @@ struct dg_ctx {
   int32_t* inv_slot = nullptr;
   int4* tiles = nullptr;        // fused expert GEMM tile list (gate/up, then down)
   int32_t* chunk_done = nullptr;
+  int32_t* route = nullptr;        // routing: expert counts [E], cursors [E], finished CTAs [1]
   int32_t* dense_work = nullptr;   // claim / exit counters of the dense GEMM
   int attn_max_clusters[ATC_MAX_CHUNKS + 1] = {};  // co-resident attention clusters per cluster size
   // CUDA graph of the denoising step (per batch and cached length)
@@ -179,6 +180,25 @@ bool make_map_q4(CUtensorMap* m, const void* base, uint64_t tokens, int Hkv, int
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Launch on the context's stream (arguments converted to the kernel's types).
+template <typename... KArgs, typename... Args>
+cudaError_t launch(dg_ctx* c, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = c->stream;
+  cfg.numAttrs = 0;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+#define DG_LAUNCH(c, kern, grid, block, smem, ...)                                                           \
+  do {                                                                                                      \
+    const cudaError_t le_ = launch((c), kern, dim3(grid), dim3(block), (smem), __VA_ARGS__);               \
+    if (le_ != cudaSuccess) return fail((c), DG_ERR_CUDA, "launch %s: %s", #kern, cudaGetErrorString(le_)); \
+    DG_LAUNCHED(c);                                                                                         \
+  } while (0)
+
 DevErr dev_err(const dg_ctx* c) { return DevErr{c->err_word, c->wait_limit_ns}; }
 
 // Profiling hook: an event pair around the launches of one kernel class.
@@ -245,20 +265,19 @@ dg_status gemm_dense(dg_ctx* c, const CUtensorMap& w, const CUtensorMap& x, int 
   p.err = dev_err(c);
   const int grid = std::min(c->sms, p.tiles_static);
   ProfScope ps0(c, DG_PROF_DENSE);
-  gemm_kernel<GEMM_DENSE><<<grid, GEMM_THREADS, gemm_smem_bytes<GEMM_DENSE>(), c->stream>>>(p);
-  DG_LAUNCHED(c);
+  DG_LAUNCH(c, gemm_kernel<GEMM_DENSE>, grid, GEMM_THREADS, gemm_smem_bytes<GEMM_DENSE>(), p);
   ps0.end();
   *splits_out = p.splits;
   return DG_OK;
 }
 
 template <int D>
-cudaError_t launch_attention(const AttnTcParams& p, dim3 grid, cudaStream_t stream) {
+cudaError_t launch_attention(const dg_ctx* c, const AttnTcParams& p, dim3 grid) {
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(ATC_THREADS, 1, 1);
   cfg.dynamicSmemBytes = AtcCfg<D>::SMEM;
-  cfg.stream = stream;
+  cfg.stream = c->stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 1;
@@ -327,13 +346,13 @@ dg_status attention(dg_ctx* c, int l, int B, int n, int pos0, bool causal) {
   cudaError_t e;
   switch (c->D) {
     case 64:
-      e = launch_attention<64>(p, grid, c->stream);
+      e = launch_attention<64>(c, p, grid);
       break;
     case 128:
-      e = launch_attention<128>(p, grid, c->stream);
+      e = launch_attention<128>(c, p, grid);
       break;
     case 176:
-      e = launch_attention<176>(p, grid, c->stream);
+      e = launch_attention<176>(c, p, grid);
       break;
     default:
       return fail(c, DG_ERR_UNSUPPORTED, "head_dim %d", c->D);
@@ -351,23 +370,19 @@ dg_status moe(dg_ctx* c, int l, int T) {
   dg_status st = gemm_dense(c, lm.wr, c->m_u64, c->E, T, c->d, &s3);
   if (st != DG_OK) return st;
   int32_t* cap = c->capture ? c->cap_idx + static_cast<size_t>(l) * c->R_step * c->k : nullptr;
+  // routing: top-k with expert counts (8 rows per CTA), then the permutation
+  // by expert, the row gather and the expert tile list (rows spread over up
+  // to 2 CTAs per SM)
+  const int pg_ctas = std::min(T, 2 * c->sms);
+  const int pg_rows = (T + pg_ctas - 1) / pg_ctas;
   ProfScope ps3(c, DG_PROF_ROUTING);
-  router_topk_kernel<<<(T * 32 + 255) / 256, 256, 0, c->stream>>>(c->part, s3, T, c->E, c->k, c->router_bias,
-                                                                   c->idx, c->gates, cap);
-  DG_LAUNCHED(c);
+  DG_LAUNCH(c, router_topk_kernel, (T + 7) / 8, 256, 0, static_cast<const float*>(c->part), s3, T, c->E, c->k,
+            c->router_bias, c->idx, c->gates, cap, 8, c->route);
+  DG_LAUNCH(c, permute_gather_kernel, (T + pg_rows - 1) / pg_rows, 256, 0, static_cast<const int32_t*>(c->idx),
+            c->route, pg_rows, T, c->k, c->E, c->F, c->Fs, c->d, static_cast<const uint16_t*>(c->u), c->perm_tok,
+            c->inv_slot, c->xp, c->tiles, c->chunk_done, c->counters, MOE_CHUNK_ROWS);
   ps3.end();
-  ProfScope ps4(c, DG_PROF_ROUTING);
-  permute_kernel<<<1, PERM_THREADS, 0, c->stream>>>(c->idx, T, c->k, c->E, c->F, c->Fs, c->d, c->perm_tok,
-                                                     c->inv_slot, c->tiles, c->chunk_done, c->counters,
-                                                     MOE_CHUNK_ROWS);
-  DG_LAUNCHED(c);
-  ps4.end();
   const int rows = T * c->k;
-  ProfScope ps5(c, DG_PROF_ROUTING);
-  gather_rows_kernel<<<std::min(4 * c->sms, (rows * (c->d / 8) + 255) / 256), 256, 0, c->stream>>>(
-      c->u, c->perm_tok, rows, c->d, c->xp);
-  DG_LAUNCHED(c);
-  ps5.end();
   (void)lw;
 
   // routed + shared experts, gate/up then down, one persistent launch
@@ -399,8 +414,7 @@ dg_status moe(dg_ctx* c, int l, int T) {
   p.shared_row_base = rows;
   p.err = dev_err(c);
   ProfScope ps6(c, DG_PROF_EXPERTS);
-  gemm_kernel<GEMM_MOE><<<c->sms, GEMM_THREADS, gemm_smem_bytes<GEMM_MOE>(), c->stream>>>(p);
-  DG_LAUNCHED(c);
+  DG_LAUNCH(c, gemm_kernel<GEMM_MOE>, c->sms, GEMM_THREADS, gemm_smem_bytes<GEMM_MOE>(), p);
   ps6.end();
   return DG_OK;
 }
@@ -416,10 +430,8 @@ dg_status forward(dg_ctx* c, const int32_t* tokens, int tok_stride, int tok_off,
   const float eps = c->cfg.rms_eps;
   float* cap0 = (c->capture && !causal) ? c->cap_h : nullptr;
   ProfScope ps8(c, DG_PROF_OTHER);
-  embed_norm_kernel<<<T, 256, 0, c->stream>>>(tokens, tok_stride, tok_off, n, c->embed,
-                                               static_cast<const uint16_t*>(c->layers[0].attn_norm), eps, c->d,
-                                               c->h, c->u, cap0, settled, B, c->V);
-  DG_LAUNCHED(c);
+  DG_LAUNCH(c, embed_norm_kernel, T, 256, 0, tokens, tok_stride, tok_off, n, c->embed,
+            static_cast<const uint16_t*>(c->layers[0].attn_norm), eps, c->d, c->h, c->u, cap0, settled, B, c->V);
   ps8.end();
   for (int l = 0; l < c->L; ++l) {
     const LayerMaps& lm = c->lmaps[l];
@@ -429,9 +441,9 @@ dg_status forward(dg_ctx* c, const int32_t* tokens, int tok_stride, int tok_off,
     if (st != DG_OK) return st;
     const size_t layer_off = static_cast<size_t>(l) * c->cfg.max_batch * c->Hkv * c->cfg.max_seq * c->D;
     ProfScope ps9(c, DG_PROF_OTHER);
-    rope_qkv_kernel<<<T, 256, 0, c->stream>>>(c->part, s1, T, n, pos0, c->Hq, c->Hkv, c->D, c->rope, c->q,
-                                               c->kcache + layer_off, c->vcache + layer_off, c->cfg.max_seq);
-    DG_LAUNCHED(c);
+    DG_LAUNCH(c, rope_qkv_kernel, T, 256, 0, static_cast<const float*>(c->part), s1, T, n, pos0, c->Hq, c->Hkv,
+              c->D, static_cast<const float2*>(c->rope), c->q, c->kcache + layer_off, c->vcache + layer_off,
+              c->cfg.max_seq);
     ps9.end();
     if (causal && l == c->L - 1) break;  // only this layer's keys/values feed the cache
     st = attention(c, l, B, n, pos0, causal);
@@ -440,9 +452,8 @@ dg_status forward(dg_ctx* c, const int32_t* tokens, int tok_stride, int tok_off,
     st = gemm_dense(c, lm.wo, c->m_o64, c->d, T, c->HD, &s2);
     if (st != DG_OK) return st;
     ProfScope ps10(c, DG_PROF_OTHER);
-    residual_norm_kernel<<<T, 256, 0, c->stream>>>(c->h, c->part, s2, T, c->d,
-                                                    static_cast<const uint16_t*>(lw.ffn_norm), eps, c->u);
-    DG_LAUNCHED(c);
+    DG_LAUNCH(c, residual_norm_kernel, T, 256, 0, c->h, static_cast<const float*>(c->part), s2, T, c->d,
+              static_cast<const uint16_t*>(lw.ffn_norm), eps, c->u);
     ps10.end();
     st = moe(c, l, T);
     if (st != DG_OK) return st;
@@ -450,9 +461,9 @@ dg_status forward(dg_ctx* c, const int32_t* tokens, int tok_stride, int tok_off,
                                              : c->final_norm;
     float* cap = (c->capture && !causal) ? c->cap_h + static_cast<size_t>(l + 1) * c->R_step * c->d : nullptr;
     ProfScope ps11(c, DG_PROF_OTHER);
-    combine_norm_kernel<<<T, 256, 0, c->stream>>>(c->h, c->yp, c->inv_slot, c->gates, c->k, T * c->k, c->d,
-                                                   next_gain, eps, c->u, cap);
-    DG_LAUNCHED(c);
+    DG_LAUNCH(c, combine_norm_kernel, T, 256, 0, c->h, static_cast<const float*>(c->yp),
+              static_cast<const int32_t*>(c->inv_slot), static_cast<const float*>(c->gates), c->k, T * c->k, c->d,
+              next_gain, eps, c->u, cap);
     ps11.end();
   }
   return DG_OK;
@@ -475,9 +486,8 @@ dg_status lm_head_and_sample(dg_ctx* c, int B, int step, uint64_t seed, float ta
   p.logit_scale_log2 = static_cast<float>(1.4426950408889634 / static_cast<double>(c->cfg.temperature));
   p.err = dev_err(c);
   ProfScope ps12(c, DG_PROF_LMHEAD);
-  gemm_kernel<GEMM_LMHEAD><<<std::min(c->sms, p.tiles_static), GEMM_THREADS, gemm_smem_bytes<GEMM_LMHEAD>(),
-                             c->stream>>>(p);
-  DG_LAUNCHED(c);
+  DG_LAUNCH(c, gemm_kernel<GEMM_LMHEAD>, std::min(c->sms, p.tiles_static), GEMM_THREADS,
+            gemm_smem_bytes<GEMM_LMHEAD>(), p);
   ps12.end();
   SampleArgs a;
   a.n_vtiles = n_vtiles;
@@ -497,8 +507,7 @@ dg_status lm_head_and_sample(dg_ctx* c, int B, int step, uint64_t seed, float ta
   a.dbg_conf = c->dbg_conf;
   a.dbg_margin = c->dbg_margin;
   ProfScope ps13(c, DG_PROF_OTHER);
-  lmhead_merge_sample_kernel<<<T, 256, 0, c->stream>>>(c->lm_part, a);
-  DG_LAUNCHED(c);
+  DG_LAUNCH(c, lmhead_merge_sample_kernel, T, 256, 0, static_cast<const float4*>(c->lm_part), a);
   ps13.end();
   return DG_OK;
 }
@@ -727,6 +736,7 @@ dg_status dg_create(const dg_config* cfg, const dg_weights* w, void* cuda_stream
   add(R * k, 4);                                  // inv_slot
   add(c->max_gu_tiles + c->max_dn_tiles, 16);    // tiles
   add(c->max_chunks, 4);                          // chunk_done
+  add(2 * PERM_MAXE + 1, 4);                     // route
   add(2, 4);                                      // dense_work
   add(16, 4);                                     // counters
   add(R * k * d, 2);                              // xp
@@ -762,6 +772,7 @@ dg_status dg_create(const dg_config* cfg, const dg_weights* w, void* cuda_stream
   c->inv_slot = carve<int32_t>(cur, R * k);
   c->tiles = carve<int4>(cur, c->max_gu_tiles + c->max_dn_tiles);
   c->chunk_done = carve<int32_t>(cur, c->max_chunks);
+  c->route = carve<int32_t>(cur, 2 * PERM_MAXE + 1);
   c->dense_work = carve<int32_t>(cur, 2);
   c->counters = carve<int32_t>(cur, 16);
   c->xp = carve<uint16_t>(cur, R * k * d);
@@ -986,8 +997,8 @@ dg_status dg_debug_lmhead(dg_ctx* c, int32_t* argmax, float* lse, float* conf, f
 
 dg_status dg_debug_router(dg_ctx* c, const float* logits, int32_t n_rows, int32_t* idx, float* gates) {
   if (!c || !logits || !idx || !gates || n_rows <= 0) return fail(c, DG_ERR_INVALID_ARG, "debug_router");
-  router_topk_kernel<<<(n_rows * 32 + 255) / 256, 256, 0, c->stream>>>(logits, 1, n_rows, c->E, c->k, nullptr, idx,
-                                                                        gates, nullptr);
+  router_topk_kernel<<<(n_rows + 7) / 8, 256, 0, c->stream>>>(logits, 1, n_rows, c->E, c->k, nullptr, idx, gates,
+                                                               nullptr, 8, nullptr);
   DG_LAUNCHED(c);
   return DG_OK;
 }

@@ -39,7 +39,7 @@ constexpr int GEMM_A_BYTES = GEMM_BM * GEMM_BK * 2;  // 16 KB
 constexpr int GEMM_THREADS = 192;
 // epilogue staging: gate values of one 32-column chunk (64 x 33) or one
 // 32 x 128 fp32 block on its way to global memory
-constexpr int GEMM_XCHG_FLOATS = 32 * GEMM_BM;
+constexpr int GEMM_XCHG_FLOATS = 2 * 32 * GEMM_BM;
 constexpr int GEMM_SCHED = 4;                        // claimed-tile ring
 constexpr int MOE_CHUNK_ROWS = 128;                  // tokens per expert tile
 
@@ -242,8 +242,12 @@ __device__ __forceinline__ bool wait_chunk_ready(const GemmParams& p, const Gemm
 // for i < nrows, col < ncols.  The block is transposed through shared memory
 // so each warp instruction writes 512 contiguous bytes as 16-byte vectors.
 // Called by all 128 epilogue threads; dst and ld keep 16-byte alignment.
-__device__ __forceinline__ void store_rows_via_smem(float* stage, const float (&v)[32], int col, int etid,
-                                                    float* dst, int ld, int nrows, int ncols) {
+// Successive calls within a tile alternate between the two halves of the
+// exchange area: the next call's barrier orders this call's reads before
+// its half is written again, and the barriers at the start of every tile
+// do the same across tiles.
+__device__ __forceinline__ void store_rows_via_smem(float* stage, const float* v, int col, int etid, float* dst,
+                                                    int ld, int nrows, int ncols) {
 #pragma unroll
   for (int i = 0; i < 32; ++i) stage[i * GEMM_BM + col] = v[i];
   named_bar_sync(1, 128);
@@ -263,7 +267,6 @@ __device__ __forceinline__ void store_rows_via_smem(float* stage, const float (&
       }
     }
   }
-  named_bar_sync(1, 128);
 }
 
 template <int MODE>
@@ -304,8 +307,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int n_tiles = tile_total<MODE>(p);
-  const int n_gu = (MODE == GEMM_MOE) ? p.counts[0] : 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -332,6 +333,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  const int n_tiles = tile_total<MODE>(p);
+  const int n_gu = (MODE == GEMM_MOE) ? p.counts[0] : 0;
 
   if (warp == 0) {
     // ------------------------------ TMA producer ------------------------------
@@ -409,12 +412,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
           uint8_t* a = sA + stage * GEMM_A_BYTES;
           uint8_t* b = sB + stage * B_BYTES;
           const int kx = (t.k0 + k) * GEMM_BK;
-          if (t.a1 != nullptr) {
-            tma_load_2d(a, t.a0, &full[stage], kx, t.a_row, pol_a);
-            tma_load_2d(a + GEMM_A_BYTES / 2, t.a1, &full[stage], kx, t.a_row, pol_a);
-          } else {
-            tma_load_2d(a, t.a0, &full[stage], kx, t.a_row, pol_a);
-          }
+          tma_load_2d(a, t.a0, &full[stage], kx, t.a_row, pol_a);
+          if (t.a1 != nullptr) tma_load_2d(a + GEMM_A_BYTES / 2, t.a1, &full[stage], kx, t.a_row, pol_a);
           for (int r = 0; r < t.nmma; r += p.b_box_rows)
             tma_load_2d(b + r * (GEMM_BK * 2), t.b, &full[stage], kx, t.b_row + r, pol_last);
           if constexpr (claims_tiles<MODE>()) {
@@ -550,11 +549,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
       if constexpr (MODE == GEMM_DENSE) {
         float* out = p.out_f32 + static_cast<size_t>(t.split) * p.T * p.M +
                      static_cast<size_t>(t.b_row) * p.M + t.a_row;
-        for (int c0 = 0; c0 < t.n; c0 += 32) {
-          float v[32];
-          tmem_ld32(tbase + c0, v);
-          store_rows_via_smem(xchg, v, row, etid, out + static_cast<size_t>(c0) * p.M, p.M, min(32, t.n - c0),
-                              p.M - t.a_row);
+        for (int c0 = 0; c0 < t.n; c0 += 64) {
+          float v[64];
+          tmem_ld64(tbase + c0, v);
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            if (c0 + 32 * h < t.n)
+              store_rows_via_smem(xchg + h * 32 * GEMM_BM, v + 32 * h, row, etid,
+                                  out + static_cast<size_t>(c0 + 32 * h) * p.M, p.M, min(32, t.n - c0 - 32 * h),
+                                  p.M - t.a_row);
         }
       } else if constexpr (MODE == GEMM_MOE) {
         if (t.kind == KIND_GATEUP) {
@@ -592,11 +595,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
         } else {
           const int r0 = (t.shared ? p.shared_row_base : 0) + t.b_row;
           float* out = p.out_f32 + static_cast<size_t>(r0) * p.out_ld + t.blk * GEMM_BM;
-          for (int c0 = 0; c0 < t.n; c0 += 32) {
-            float v[32];
-            tmem_ld32(tbase + c0, v);
-            store_rows_via_smem(xchg, v, row, etid, out + static_cast<size_t>(c0) * p.out_ld, p.out_ld,
-                                min(32, t.n - c0), GEMM_BM);
+          for (int c0 = 0; c0 < t.n; c0 += 64) {
+            float v[64];
+            tmem_ld64(tbase + c0, v);
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+              if (c0 + 32 * h < t.n)
+                store_rows_via_smem(xchg + h * 32 * GEMM_BM, v + 32 * h, row, etid,
+                                    out + static_cast<size_t>(c0 + 32 * h) * p.out_ld, p.out_ld,
+                                    min(32, t.n - c0 - 32 * h), GEMM_BM);
           }
         }
       } else {  // GEMM_LMHEAD
@@ -631,6 +638,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
+    __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem_base, 2 * ACC_COLS);
   }

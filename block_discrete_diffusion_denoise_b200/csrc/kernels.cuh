@@ -32,207 +32,249 @@ __device__ __forceinline__ int uniform_token(uint32_t w, int vocab) {
 }
 
 // Router: logits = sum_s part[s][row][e] (+ bias[e]); top-k by (logit desc,
-// index asc); gates = softmax over the k selected.  One warp per row.
-__global__ void router_topk_kernel(const float* __restrict__ part, int splits, int T, int E, int k,
-                                   const float* __restrict__ bias, int32_t* __restrict__ idx_out,
-                                   float* __restrict__ gates_out, int32_t* __restrict__ capture) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (warp >= T) return;
-  constexpr int MAXPER = 8;  // E <= 256
-  float v[MAXPER];
-  uint32_t taken = 0;
-#pragma unroll
-  for (int c = 0; c < MAXPER; ++c) {
-    const int e = c * 32 + lane;
-    float x = -INFINITY;
-    if (e < E) {
-      x = 0.f;
-      for (int s = 0; s < splits; ++s) x += part[(static_cast<size_t>(s) * T + warp) * E + e];
-      if (bias) x += bias[e];
-    }
-    v[c] = x;
+// index asc); gates = softmax over the k selected.  One warp per row; CTA c
+// owns rows [c * rows_per_cta, (c + 1) * rows_per_cta).  With `counts`, the
+// (row, slot) pairs choosing each expert are added to counts[e] (zero before
+// the launch).
+constexpr int PERM_MAXE = 256;
+
+__global__ void __launch_bounds__(256) router_topk_kernel(const float* __restrict__ part, int splits, int T, int E,
+                                                          int k, const float* __restrict__ bias,
+                                                          int32_t* __restrict__ idx_out,
+                                                          float* __restrict__ gates_out,
+                                                          int32_t* __restrict__ capture, int rows_per_cta,
+                                                          int32_t* __restrict__ counts) {
+  __shared__ int s_hist[PERM_MAXE];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (counts) {
+    for (int e = threadIdx.x; e < E; e += blockDim.x) s_hist[e] = 0;
+    __syncthreads();
   }
-  float sel_v[16];
-  int sel_i[16];
-  for (int r = 0; r < k; ++r) {
-    float bv = -INFINITY;
-    int bi = 0x7fffffff;
+  const int row_end = min(T, (blockIdx.x + 1) * rows_per_cta);
+  for (int row = blockIdx.x * rows_per_cta + warp; row < row_end; row += blockDim.x >> 5) {
+    constexpr int MAXPER = PERM_MAXE / 32;
+    float v[MAXPER];
+    uint32_t taken = 0;
 #pragma unroll
     for (int c = 0; c < MAXPER; ++c) {
       const int e = c * 32 + lane;
-      if (e < E && !((taken >> c) & 1) && (v[c] > bv || (v[c] == bv && e < bi) || bi == 0x7fffffff)) {
-        bv = v[c];
-        bi = e;
+      float x = -INFINITY;
+      if (e < E) {
+        x = 0.f;
+        for (int s = 0; s < splits; ++s) x += part[(static_cast<size_t>(s) * T + row) * E + e];
+        if (bias) x += bias[e];
       }
+      v[c] = x;
     }
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (oi != 0x7fffffff && (bi == 0x7fffffff || ov > bv || (ov == bv && oi < bi))) {
-        bv = ov;
-        bi = oi;
+    // lane r keeps the r-th selection (k <= 16 < 32)
+    float my_v = -INFINITY, top_v = -INFINITY;
+    int my_i = 0;
+    for (int r = 0; r < k; ++r) {
+      float bv = -INFINITY;
+      int bi = 0x7fffffff;
+#pragma unroll
+      for (int c = 0; c < MAXPER; ++c) {
+        const int e = c * 32 + lane;
+        if (e < E && !((taken >> c) & 1) && (v[c] > bv || (v[c] == bv && e < bi) || bi == 0x7fffffff)) {
+          bv = v[c];
+          bi = e;
+        }
       }
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (oi != 0x7fffffff && (bi == 0x7fffffff || ov > bv || (ov == bv && oi < bi))) {
+          bv = ov;
+          bi = oi;
+        }
+      }
+      if (r == 0) top_v = bv;
+      if (lane == r) {
+        my_v = bv;
+        my_i = bi;
+      }
+      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
     }
-    sel_v[r] = bv;
-    sel_i[r] = bi;
-    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-  }
-  if (lane == 0) {
+    // gates: softmax over the k selected logits, summed in slot order
+    const float w = lane < k ? __expf(my_v - top_v) : 0.f;
     float sum = 0.f;
-    float w[16];
-    for (int r = 0; r < k; ++r) {
-      w[r] = __expf(sel_v[r] - sel_v[0]);
-      sum += w[r];
+    for (int r = 0; r < k; ++r) sum += __shfl_sync(0xffffffffu, w, r);
+    if (lane < k) {
+      idx_out[static_cast<size_t>(row) * k + lane] = my_i;
+      gates_out[static_cast<size_t>(row) * k + lane] = w / sum;
+      if (capture) capture[static_cast<size_t>(row) * k + lane] = my_i;
+      if (counts) atomicAdd(&s_hist[my_i], 1);
     }
-    for (int r = 0; r < k; ++r) {
-      idx_out[static_cast<size_t>(warp) * k + r] = sel_i[r];
-      gates_out[static_cast<size_t>(warp) * k + r] = w[r] / sum;
-      if (capture) capture[static_cast<size_t>(warp) * k + r] = sel_i[r];
-    }
+  }
+  if (counts) {
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x)
+      if (s_hist[e] > 0) atomicAdd(&counts[e], s_hist[e]);
   }
 }
 
-// Stable permutation of the T*k (token, slot) pairs by expert, expert counts,
-// and the tile list of the fused expert GEMM (the shared expert is group E
-// with all T tokens).  One CTA of 1024 threads.
-//   perm_tok[pos]   token of permuted row pos
-//   inv_slot[p]     permuted row of pair p = t*k + j
+// exclusive scan over the 256 threads of a block; `tmp` >= 8 ints
+__device__ __forceinline__ int block_excl_scan256(int v, int* tmp, int& total) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) tmp[warp] = x;
+  __syncthreads();
+  int wbase = 0;
+  total = 0;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) {
+    const int t = tmp[w];
+    if (w < warp) wbase += t;
+    total += t;
+  }
+  __syncthreads();
+  return wbase + x - v;
+}
+
+// Permutation of the T*k (row, slot) pairs by expert, the gather of the
+// routed rows, and the tile list of the fused expert GEMM.  Expert e owns
+// positions [start_e, start_e + counts[e]); pairs claim positions in it from
+// cursor[e].  The order of rows within an expert does not change any value
+// (every row of a tile is an independent dot product and the combine sums a
+// token's slots in slot order through inv_slot), so the claim order is free.
+//   perm_tok[pos]   row of permuted position pos;  xp[pos] = u[perm_tok[pos]]
+//   inv_slot[p]     permuted position of pair p = t*k + j
 //   tiles           gate/up tiles, then down tiles, each
 //                   {group | block << 16, token chunk, first row, rows};
-//                   groups in the order shared, 0, 1, ..., E-1
+//                   groups in the order shared (= E, all T rows), 0, ..., E-1;
+//                   within a group block-major, so re-reads of a weight block
+//                   by its chunks hit L2
 //   chunk_done[c]   zeroed (gate/up tiles of chunk c finished)
 //   counters[0] = gate/up tiles, [1] = down tiles, [2] = experts hit,
 //   counters[3] = tile claim counter (zeroed)
-constexpr int PERM_THREADS = 1024;
-constexpr int PERM_MAXE = 256;
-
-__global__ void __launch_bounds__(PERM_THREADS) permute_kernel(const int32_t* __restrict__ idx, int T, int k,
-                                                               int E, int F, int Fs, int d,
-                                                               int32_t* __restrict__ perm_tok,
-                                                               int32_t* __restrict__ inv_slot,
-                                                               int4* __restrict__ tiles,
-                                                               int32_t* __restrict__ chunk_done,
-                                                               int32_t* __restrict__ counters, int chunk_rows) {
-  __shared__ int wcount[32][PERM_MAXE + 1];  // per-warp per-expert counts, then bases
-  __shared__ int offs[PERM_MAXE + 2];
-  __shared__ int gu_off[PERM_MAXE + 2];
-  __shared__ int dn_off[PERM_MAXE + 2];
+//   route[0..E) = counts, route[E..2E) = cursors, route[2E] = finished CTAs:
+//   the last CTA to finish zeroes them for the next launch.
+__global__ void __launch_bounds__(256) permute_gather_kernel(
+    const int32_t* __restrict__ idx, int32_t* __restrict__ route, int rows_per_cta, int T, int k, int E, int F,
+    int Fs, int d, const uint16_t* __restrict__ u, int32_t* __restrict__ perm_tok, int32_t* __restrict__ inv_slot,
+    uint16_t* __restrict__ xp, int4* __restrict__ tiles, int32_t* __restrict__ chunk_done,
+    int32_t* __restrict__ counters, int chunk_rows) {
+  __shared__ int s_start[PERM_MAXE];   // first position of each expert
+  __shared__ int s_cnt[PERM_MAXE];
+  __shared__ int s_pos[256];
+  __shared__ int tmp[8];
+  __shared__ int s_last;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int npairs = T * k;
-  const int per_warp = (npairs + 31) / 32;
-  const int p_begin = warp * per_warp;
-  const int p_end = min(npairs, p_begin + per_warp);
-  for (int e = lane; e < E; e += 32) wcount[warp][e] = 0;
-  __syncwarp();
+  int32_t* cursor = route + E;
+  {
+    const int c = threadIdx.x < E ? __ldcg(&route[threadIdx.x]) : 0;
+    int total;
+    const int ex = block_excl_scan256(c, tmp, total);
+    if (threadIdx.x < E) {
+      s_start[threadIdx.x] = ex;
+      s_cnt[threadIdx.x] = c;
+    }
+  }
+  __syncthreads();
+
+  if (blockIdx.x == 0) {
+    // Tile list.  Slot s = 0 is the shared expert, slot s >= 1 expert s - 1;
+    // each thread takes slots 2t and 2t + 1 of the scans.
+    const int mb_dn = d / 128;
+    int nch[2], gu[2], dn[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int sl = 2 * threadIdx.x + h;
+      const int cnt = sl == 0 ? T : (sl <= E ? s_cnt[sl - 1] : 0);
+      nch[h] = (cnt + chunk_rows - 1) / chunk_rows;
+      gu[h] = nch[h] * ((sl == 0 ? Fs : F) / 64);
+      dn[h] = nch[h] * mb_dn;
+    }
+    int tot_ch, tot_gu, tot_dn;
+    const int ch0 = block_excl_scan256(nch[0] + nch[1], tmp, tot_ch);
+    const int gu0 = block_excl_scan256(gu[0] + gu[1], tmp, tot_gu);
+    const int dn0 = block_excl_scan256(dn[0] + dn[1], tmp, tot_dn);
+    const int hit = __syncthreads_count(threadIdx.x < E && s_cnt[threadIdx.x] > 0) +
+                    __syncthreads_count(threadIdx.x + 256 < E && s_cnt[threadIdx.x + 256] > 0);
+    if (threadIdx.x == 0) {
+      counters[0] = tot_gu;
+      counters[1] = tot_dn;
+      counters[2] = hit;
+      counters[3] = 0;
+    }
+    for (int c = threadIdx.x; c < tot_ch; c += 256) chunk_done[c] = 0;
+    int ch_at = ch0, gu_at = gu0, dn_at = tot_gu + dn0;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int sl = 2 * threadIdx.x + h;
+      if (sl <= E) {
+        const int g = sl == 0 ? E : sl - 1;
+        const int cnt = sl == 0 ? T : s_cnt[g];
+        const int first = sl == 0 ? 0 : s_start[g];
+        const int mb_gu = (sl == 0 ? Fs : F) / 64;
+        for (int j = 0; j < mb_gu; ++j)
+          for (int ch = 0; ch < nch[h]; ++ch)
+            tiles[gu_at++] = make_int4(g | (j << 16), ch_at + ch, first + ch * chunk_rows,
+                                       min(chunk_rows, cnt - ch * chunk_rows));
+        for (int j = 0; j < mb_dn; ++j)
+          for (int ch = 0; ch < nch[h]; ++ch)
+            tiles[dn_at++] = make_int4(g | (j << 16), ch_at + ch, first + ch * chunk_rows,
+                                       min(chunk_rows, cnt - ch * chunk_rows));
+        ch_at += nch[h];
+      }
+    }
+  }
+
+  // positions of this CTA's pairs, 256 at a time (one warp-aggregated claim
+  // per expert and warp), then the gather of their rows
   const unsigned lt = (1u << lane) - 1u;
-  // pass 1: counts per (warp range, expert)
-  for (int c = p_begin; c < p_end; c += 32) {
-    const int p = c + lane;
+  const int p_begin = blockIdx.x * rows_per_cta * k;
+  const int p_end = min(T, (blockIdx.x + 1) * rows_per_cta) * k;
+  const int vec = d / 8;
+  for (int c0 = p_begin; c0 < p_end; c0 += 256) {
+    const int p = c0 + threadIdx.x;
     const bool valid = p < p_end;
-    const unsigned act = __ballot_sync(0xffffffffu, valid);
+    const int e = valid ? idx[p] : -1;
+    const unsigned m = __match_any_sync(0xffffffffu, e);
+    const int leader = __ffs(m) - 1;
+    int base = 0;
+    if (valid && lane == leader) base = atomicAdd(&cursor[e], __popc(m));
+    base = __shfl_sync(0xffffffffu, base, leader);
     if (valid) {
-      const int e = idx[p];
-      const unsigned m = __match_any_sync(act, e);
-      if ((m & lt) == 0) wcount[warp][e] += __popc(m);
-    }
-    __syncwarp();
-  }
-  __syncthreads();
-  // per-expert prefix over warps; totals
-  if (threadIdx.x < E) {
-    const int e = threadIdx.x;
-    int run = 0;
-    for (int w = 0; w < 32; ++w) {
-      const int c = wcount[w][e];
-      wcount[w][e] = run;
-      run += c;
-    }
-    offs[e] = run;  // count, scanned below
-  }
-  __syncthreads();
-  __shared__ int ch_off[PERM_MAXE + 2];
-  if (threadIdx.x == 0) {
-    const int mb_gu = F / 64, mb_dn = d / 128;
-    // shared expert first (all T tokens), then the routed experts in order
-    const int sch = (T + chunk_rows - 1) / chunk_rows;
-    gu_off[E] = 0;
-    dn_off[E] = 0;
-    ch_off[E] = 0;
-    int gu = sch * (Fs / 64), dn = sch * mb_dn, ch = sch;
-    int run = 0, hit = 0;
-    for (int e = 0; e < E; ++e) {
-      const int c = offs[e];
-      offs[e] = run;
-      run += c;
-      const int chunks = (c + chunk_rows - 1) / chunk_rows;
-      gu_off[e] = gu;
-      dn_off[e] = dn;
-      ch_off[e] = ch;
-      gu += chunks * mb_gu;
-      dn += chunks * mb_dn;
-      ch += chunks;
-      hit += c > 0;
-    }
-    offs[E] = run;
-    gu_off[E + 1] = gu;  // total gate/up tiles: the down tiles follow them in the list
-    ch_off[E + 1] = ch;
-    counters[0] = gu;
-    counters[1] = dn;
-    counters[2] = hit;
-    counters[3] = 0;
-  }
-  __syncthreads();
-  for (int c = threadIdx.x; c < ch_off[E + 1]; c += blockDim.x) chunk_done[c] = 0;
-  // pass 2: positions
-  for (int c = p_begin; c < p_end; c += 32) {
-    const int p = c + lane;
-    const bool valid = p < p_end;
-    const unsigned act = __ballot_sync(0xffffffffu, valid);
-    if (valid) {
-      const int e = idx[p];
-      const unsigned m = __match_any_sync(act, e);
-      const int pos = offs[e] + wcount[warp][e] + __popc(m & lt);
+      const int pos = s_start[e] + base + __popc(m & lt);
       perm_tok[pos] = p / k;
       inv_slot[p] = pos;
-      __syncwarp(act);
-      if ((m & lt) == 0) wcount[warp][e] += __popc(m);
+      s_pos[threadIdx.x] = pos;
     }
-    __syncwarp();
+    __syncthreads();
+    // one warp per pair; each lane keeps 4 row loads in flight
+    const int n_here = min(256, p_end - c0);
+    for (int pr = warp; pr < n_here; pr += 8) {
+      const uint4* src = reinterpret_cast<const uint4*>(u) + static_cast<size_t>((c0 + pr) / k) * vec;
+      uint4* dst = reinterpret_cast<uint4*>(xp) + static_cast<size_t>(s_pos[pr]) * vec;
+      for (int cv = lane; cv < vec; cv += 128) {
+        uint4 r[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (cv + 32 * q < vec) r[q] = src[cv + 32 * q];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (cv + 32 * q < vec) dst[cv + 32 * q] = r[q];
+      }
+    }
+    __syncthreads();
   }
-  // tile list (one thread per group)
-  const int n_gu = gu_off[E + 1];
-  for (int g = threadIdx.x; g <= E; g += blockDim.x) {
-    const bool shared = g == E;
-    const int first = shared ? 0 : offs[g];
-    const int cnt = shared ? T : offs[g + 1] - offs[g];
-    const int mb_gu = (shared ? Fs : F) / 64, mb_dn = d / 128;
-    const int nch = (cnt + chunk_rows - 1) / chunk_rows;
-    int gi = gu_off[g], di = n_gu + dn_off[g];
-    // block-major: the chunk tiles of one weight block sit next to each other,
-    // so the re-reads of that block hit L2
-    for (int j = 0; j < mb_gu; ++j)
-      for (int ch = 0; ch < nch; ++ch)
-        tiles[gi++] = make_int4(g | (j << 16), ch_off[g] + ch, first + ch * chunk_rows,
-                                min(chunk_rows, cnt - ch * chunk_rows));
-    for (int j = 0; j < mb_dn; ++j)
-      for (int ch = 0; ch < nch; ++ch)
-        tiles[di++] = make_int4(g | (j << 16), ch_off[g] + ch, first + ch * chunk_rows,
-                                min(chunk_rows, cnt - ch * chunk_rows));
-  }
-}
 
-// xp[pos] = u[perm_tok[pos]] (bf16 rows of d elements, 16-byte vectors)
-__global__ void gather_rows_kernel(const uint16_t* __restrict__ u, const int32_t* __restrict__ perm_tok,
-                                   int rows, int d, uint16_t* __restrict__ xp) {
-  const int vec = d / 8;
-  const int64_t total = static_cast<int64_t>(rows) * vec;
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int r = static_cast<int>(i / vec), c = static_cast<int>(i % vec);
-    const int t = perm_tok[r];
-    reinterpret_cast<uint4*>(xp)[static_cast<size_t>(r) * vec + c] =
-        reinterpret_cast<const uint4*>(u)[static_cast<size_t>(t) * vec + c];
+  // the last CTA out zeroes the counts and cursors (every CTA has read the
+  // counts and made its claims before it counts itself out)
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = atomicAdd(&route[2 * E], 1) == static_cast<int>(gridDim.x) - 1;
+  __syncthreads();
+  if (s_last) {
+    for (int e = threadIdx.x; e < 2 * E; e += 256) route[e] = 0;
+    __syncthreads();
+    if (threadIdx.x == 0) route[2 * E] = 0;
   }
 }
 
