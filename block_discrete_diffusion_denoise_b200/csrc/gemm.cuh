@@ -82,7 +82,12 @@ struct GemmParams {
   CUtensorMap ds_map;     // MOE down shared A: ws_down
   CUtensorMap h_map;      // MOE down routed B: routed hidden rows
   CUtensorMap hs_map;     // MOE down shared B: shared hidden rows
-  int b_box_rows;         // rows per B box (16, or 128 for the LM head)
+  // MOE: the same B tensors in 64-row boxes; whole 64-row groups go in one
+  // copy each, the rest in b_box_rows boxes (fewer copies measured faster;
+  // 128-row boxes measured slower than two 64-row ones)
+  CUtensorMap b_mid_map, bs_mid_map, h_mid_map, hs_mid_map;
+  int b_box_rows;         // rows per B box (16 MOE, 64 DENSE, 128 LM head)
+  int b_mid_rows;         // 0 = none (64 MOE)
   int M;                  // DENSE: output features; LMHEAD: tokens
   int T;                  // DENSE: tokens
   int k_steps;            // K / 64 (DENSE, LMHEAD)
@@ -114,6 +119,7 @@ struct GemmTile {
   const CUtensorMap* a1;  // second 64-row A box (gate/up) or nullptr
   int a_row;
   const CUtensorMap* b;
+  const CUtensorMap* b_mid;  // the same tensor in b_mid_rows boxes
   int b_row;
   int n;      // valid columns
   int nmma;   // MMA N (multiple of 16, <= 128)
@@ -141,6 +147,7 @@ __device__ __forceinline__ void decode_tile(const GemmParams& p, int tile, int4 
     t.a1 = nullptr;
     t.a_row = mt * GEMM_BM;
     t.b = &p.b_map;
+    t.b_mid = &p.b_mid_map;
     t.b_row = nt * p.bn;
     t.n = min(p.bn, p.T - t.b_row);
     t.nmma = round16(t.n);
@@ -157,6 +164,7 @@ __device__ __forceinline__ void decode_tile(const GemmParams& p, int tile, int4 
     t.a1 = nullptr;
     t.a_row = mt * GEMM_BM;
     t.b = &p.b_map;
+    t.b_mid = &p.b_mid_map;
     t.b_row = vt * GEMM_BN;
     t.n = GEMM_BN;
     t.nmma = GEMM_BN;
@@ -185,6 +193,7 @@ __device__ __forceinline__ void decode_tile(const GemmParams& p, int tile, int4 
       t.a1 = t.shared ? &p.as_map[1] : &p.a_map[1];
       t.a_row = (t.shared ? 0 : t.group * p.F) + t.blk * 64;
       t.b = t.shared ? &p.bs_map : &p.b_map;
+      t.b_mid = t.shared ? &p.bs_mid_map : &p.b_mid_map;
       t.nk = p.d / GEMM_BK;
     } else {
       t.kind = KIND_DOWN;
@@ -192,6 +201,7 @@ __device__ __forceinline__ void decode_tile(const GemmParams& p, int tile, int4 
       t.a1 = nullptr;
       t.a_row = (t.shared ? 0 : t.group * p.d) + t.blk * GEMM_BM;
       t.b = t.shared ? &p.hs_map : &p.h_map;
+      t.b_mid = t.shared ? &p.hs_mid_map : &p.h_mid_map;
       t.nk = (t.shared ? p.Fs : p.F) / GEMM_BK;
     }
   }
@@ -414,7 +424,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
           const int kx = (t.k0 + k) * GEMM_BK;
           tma_load_2d(a, t.a0, &full[stage], kx, t.a_row, pol_a);
           if (t.a1 != nullptr) tma_load_2d(a + GEMM_A_BYTES / 2, t.a1, &full[stage], kx, t.a_row, pol_a);
-          for (int r = 0; r < t.nmma; r += p.b_box_rows)
+          int r = 0;
+          if (p.b_mid_rows > 0)
+            for (; r + p.b_mid_rows <= t.nmma; r += p.b_mid_rows)
+              tma_load_2d(b + r * (GEMM_BK * 2), t.b_mid, &full[stage], kx, t.b_row + r, pol_last);
+          for (; r < t.nmma; r += p.b_box_rows)
             tma_load_2d(b + r * (GEMM_BK * 2), t.b, &full[stage], kx, t.b_row + r, pol_last);
           if constexpr (claims_tiles<MODE>()) {
             // halfway through this tile, read the next tile's dependency flag
