@@ -18,6 +18,7 @@ Prints one JSON line on rank 0.
 from __future__ import annotations
 
 import argparse
+import datetime
 import json
 import math
 import os
@@ -83,7 +84,9 @@ def step_cost(w, hits):
 # clocks during the timed region
 # ---------------------------------------------------------------------------
 class Clocks:
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi sampler started before the warm-up; stop(t0, t1) keeps the
+    samples whose timestamps fall in the timed window [t0, t1] (host clock)."""
+    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -97,26 +100,37 @@ class Clocks:
         except OSError:
             self.p = None
 
-    def stop(self):
+    def stop(self, t0=None, t1=None):
         if self.p is None:
             return None
+        time.sleep(0.1)  # let the sampler record the end of the window
         self.p.terminate()
         try:
             self.p.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.p.kill()
         self.f.flush()
-        rows = [r.split(",") for r in open(self.f.name).read().strip().splitlines() if r.count(",") >= 8]
+        rows = [[x.strip() for x in r.split(",")] for r in open(self.f.name).read().strip().splitlines()
+                if r.count(",") >= 9]
         os.unlink(self.f.name)
+
+        def stamp(r):
+            try:
+                return datetime.datetime.strptime(r[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            except ValueError:
+                return None
+        if t0 is not None and t1 is not None:
+            inside = [r for r in rows if (stamp(r) is not None and t0 - 0.06 <= stamp(r) <= t1 + 0.06)]
+            rows = inside or rows
         if not rows:
             return None
-        sm = [float(r[1]) for r in rows]
-        mx = max(float(r[2]) for r in rows)
+        sm = [float(r[2]) for r in rows]
+        mx = max(float(r[3]) for r in rows)
         reasons = set()
         for r in rows:
-            for name, col in (("hw_slowdown", 5), ("hw_thermal_slowdown", 6), ("sw_thermal_slowdown", 7),
-                              ("sw_power_cap", 8)):
-                if r[col].strip().lower().startswith("active"):
+            for name, col in (("hw_slowdown", 6), ("hw_thermal_slowdown", 7), ("sw_thermal_slowdown", 8),
+                              ("sw_power_cap", 9)):
+                if r[col].lower().startswith("active"):
                     reasons.add(name)
         loaded = [x for x in sm if x > 0.5 * mx] or sm
         return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
@@ -218,7 +232,6 @@ def run_native(args, w):
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     if world > 1:
-        import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
 
@@ -256,15 +269,16 @@ def run_native(args, w):
         hits.append(int(torch.unique(e).numel()))
     ctx.debug_capture(False)
 
+    clocks = Clocks(local)  # sampling from before the warm-up on
     for s in range(args.warmup):
         ctx.denoise_step(cur, s, seed, si.tau_schedule(w, s), nxt, conf, settled)
         cur, nxt = nxt, cur
     ctx.sync()
 
     # ---- timed region: K steps (the step runs as one CUDA graph) ----
-    clocks = Clocks(local)
     barrier()
     torch.cuda.synchronize()
+    t_wall0 = time.time()
     n0 = ctx.launch_count
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record(stream)
@@ -274,8 +288,9 @@ def run_native(args, w):
     ev1.record(stream)
     torch.cuda.synchronize()
     barrier()
+    t_wall1 = time.time()
     ms = ev0.elapsed_time(ev1) / args.steps
-    clk = clocks.stop()
+    clk = clocks.stop(t_wall0, t_wall1)
     launches = (ctx.launch_count - n0) // args.steps
     ctx.sync()
     if world > 1:
