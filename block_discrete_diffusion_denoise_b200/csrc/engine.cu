@@ -96,6 +96,7 @@ struct dg_ctx {
   // tensor maps
   std::vector<LayerMaps> lmaps;
   CUtensorMap m_u16{}, m_u64{}, m_u128{}, m_o64{}, m_xp16{}, m_h16{}, m_hs16{}, m_embed{};
+  CUtensorMap m_xp64{}, m_h64{}, m_hs64{};         // 64-row boxes (expert GEMM B)
   CUtensorMap m_q4{};  // queries as (D, G, Hkv, token): one GQA group's rows per box
   // state
   int B = 0;
@@ -254,18 +255,21 @@ dg_status gemm_dense(dg_ctx* c, const CUtensorMap& w, const CUtensorMap& x, int 
   p.M = M;
   p.T = T;
   p.k_steps = K / 64;
-  p.bn = std::min(DENSE_BN, (T + 15) / 16 * 16);
-  p.n_tiles_n = (T + p.bn - 1) / p.bn;
   const int m_tiles = (M + GEMM_BM - 1) / GEMM_BM;
+  p.bn = std::min(DENSE_BN, (T + 15) / 16 * 16);
+  // few output rows (the router): narrower token tiles, so more CTAs share
+  // the work and each tile's epilogue is shorter
+  if (m_tiles * 8 < c->sms && p.bn > 64) p.bn = 64;
+  p.n_tiles_n = (T + p.bn - 1) / p.bn;
   const size_t cap_s = c->part_cap / (static_cast<size_t>(T) * M);
   p.splits = choose_splits(m_tiles * p.n_tiles_n, p.k_steps, c->sms, std::min<size_t>(cap_s, max_splits));
   p.tiles_static = m_tiles * p.n_tiles_n * p.splits;
   p.out_f32 = c->part;
   p.work = c->dense_work;
   p.err = dev_err(c);
-  const int grid = std::min(c->sms, p.tiles_static);
   ProfScope ps0(c, DG_PROF_DENSE);
-  DG_LAUNCH(c, gemm_kernel<GEMM_DENSE>, grid, GEMM_THREADS, gemm_smem_bytes<GEMM_DENSE>(), p);
+  DG_LAUNCH(c, gemm_kernel<GEMM_DENSE>, std::min(c->sms, p.tiles_static), GEMM_THREADS,
+            gemm_smem_bytes<GEMM_DENSE>(), p);
   ps0.end();
   *splits_out = p.splits;
   return DG_OK;
@@ -398,6 +402,11 @@ dg_status moe(dg_ctx* c, int l, int T) {
   p.ds_map = lm.wsd;
   p.h_map = c->m_h16;
   p.hs_map = c->m_hs16;
+  p.b_mid_map = c->m_xp64;
+  p.bs_mid_map = c->m_u64;
+  p.h_mid_map = c->m_h64;
+  p.hs_mid_map = c->m_hs64;
+  p.b_mid_rows = 64;
   p.b_box_rows = 16;
   p.counts = c->counters;
   p.tiles = c->tiles;
@@ -852,6 +861,9 @@ dg_status dg_create(const dg_config* cfg, const dg_weights* w, void* cuda_stream
   ok &= make_map(&c->m_u128, c->u, R, d, 128);
   ok &= make_map(&c->m_o64, c->o, R, c->HD, 64);
   ok &= make_map(&c->m_xp16, c->xp, R * k, d, 16);
+  ok &= make_map(&c->m_xp64, c->xp, R * k, d, 64);
+  ok &= make_map(&c->m_h64, c->hbuf, R * k, c->F, 64);
+  ok &= make_map(&c->m_hs64, c->hsbuf, R, c->Fs, 64);
   ok &= make_map(&c->m_h16, c->hbuf, R * k, c->F, 16);
   ok &= make_map(&c->m_hs16, c->hsbuf, R, c->Fs, 16);
   ok &= make_map(&c->m_embed, c->embed, c->V, d, 128);

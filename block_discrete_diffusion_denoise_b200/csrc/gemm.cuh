@@ -2,16 +2,16 @@
 //
 //   D[m, n] = sum_k A[m, k] * B[n, k]        (A, B bf16 K-major; D fp32 in TMEM)
 //
-// One CTA per SM.  Warp 0 (one lane) issues TMA loads into a 6-stage ring of
-// shared-memory stages, warp 1 (one lane) issues tcgen05.mma into one of two
-// TMEM accumulators (128 lanes x 128 fp32 columns each), warps 2..5 drain the
-// other accumulator through the epilogue.  All waits are bounded.
+// One CTA per SM.  Warp 0 (one lane) issues TMA loads into a ring of
+// shared-memory stages (4 for DENSE, 6 otherwise), warp 1 (one lane) issues
+// tcgen05.mma into one of two TMEM accumulators (128 lanes x 128 or 256 fp32
+// columns each), warps 2..5 drain the other accumulator through the epilogue.
+// All waits are bounded.
 //
 // Three launch modes share the pipeline:
-//   DENSE   A = weight rows (output features), B = tokens; split-K partials
-//           out[split][token][feature] fp32, summed in split order by the
-//           consumer kernel (deterministic, no atomics).  Tiles are claimed
-//           from an atomic counter.
+//   DENSE   A = weight rows (output features), B = up to 256 tokens; split-K
+//           partials out[split][token][feature] fp32, summed in split order by
+//           the consumer kernel (deterministic, no atomics).  Static tiles.
 //   MOE     one launch for all experts of a layer, routed and shared: first the
 //           gate/up tiles (A = 64 gate rows stacked on the same 64 up rows, B =
 //           the expert's tokens; the epilogue forms SiLU(gate) * up and stores
@@ -250,7 +250,8 @@ __device__ __forceinline__ bool wait_chunk_ready(const GemmParams& p, const Gemm
 // Store a 128-column x 32-row fp32 block held one column per epilogue thread
 // (thread `col` has v[i] = element (row i, column col)) to dst[i * ld + col]
 // for i < nrows, col < ncols.  The block is transposed through shared memory
-// so each warp instruction writes 512 contiguous bytes as 16-byte vectors.
+// so each warp instruction writes 512 contiguous bytes as 16-byte vectors;
+// all eight shared-memory reads are issued before the first global store.
 // Called by all 128 epilogue threads; dst and ld keep 16-byte alignment.
 // Successive calls within a tile alternate between the two halves of the
 // exchange area: the next call's barrier orders this call's reads before
@@ -258,22 +259,35 @@ __device__ __forceinline__ bool wait_chunk_ready(const GemmParams& p, const Gemm
 // do the same across tiles.
 __device__ __forceinline__ void store_rows_via_smem(float* stage, const float* v, int col, int etid, float* dst,
                                                     int ld, int nrows, int ncols) {
+  const uint32_t sb = smem_u32(stage);
 #pragma unroll
-  for (int i = 0; i < 32; ++i) stage[i * GEMM_BM + col] = v[i];
+  for (int i = 0; i < 32; ++i)
+    asm volatile("st.shared.f32 [%0], %1;" ::"r"(sb + (i * GEMM_BM + col) * 4), "f"(v[i]) : "memory");
   named_bar_sync(1, 128);
+  float4 x[8];
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    const int idx = etid + 128 * r;
+    const int i = idx >> 5, c4 = (idx & 31) * 4;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(x[r].x), "=f"(x[r].y), "=f"(x[r].z), "=f"(x[r].w)
+                 : "r"(sb + (i * GEMM_BM + c4) * 4)
+                 : "memory");
+  }
 #pragma unroll
   for (int r = 0; r < 8; ++r) {
     const int idx = etid + 128 * r;
     const int i = idx >> 5, c4 = (idx & 31) * 4;
     if (i < nrows && c4 < ncols) {
-      const float4 x = *reinterpret_cast<const float4*>(stage + i * GEMM_BM + c4);
       float* d = dst + static_cast<size_t>(i) * ld + c4;
       if (c4 + 4 <= ncols) {
-        *reinterpret_cast<float4*>(d) = x;
+        asm volatile("st.global.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(__cvta_generic_to_global(d)), "f"(x[r].x),
+                     "f"(x[r].y), "f"(x[r].z), "f"(x[r].w)
+                     : "memory");
       } else {
-        d[0] = x.x;
-        if (c4 + 1 < ncols) d[1] = x.y;
-        if (c4 + 2 < ncols) d[2] = x.z;
+        d[0] = x[r].x;
+        if (c4 + 1 < ncols) d[1] = x[r].y;
+        if (c4 + 2 < ncols) d[2] = x[r].z;
       }
     }
   }
