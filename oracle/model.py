@@ -293,7 +293,12 @@ class Oracle:
 
     # -- one transformer layer over new rows of one sequence --
     def _layer_forward(self, l: int, h: np.ndarray, b: int, pos0: int, causal: bool,
-                       need_ffn: bool = True, dbg: dict | None = None):
+                       need_ffn: bool = True, dbg: dict | None = None, need_attn: bool = True):
+        """One layer over n new rows at positions [pos0, pos0 + n).  Returns the
+        updated residual and the rows' keys/values.  need_attn=False returns
+        after the keys/values (h unchanged): the causal encoder's last layer
+        only feeds the cache (codemajin.net "DiffusionGemma architecture",
+        section 3.2)."""
         s = self.s
         lw = self.layer(l)
         n = h.shape[0]
@@ -306,6 +311,8 @@ class Oracle:
         cos, sin = rope_angles(np.arange(pos0, pos0 + n), D, s.rope_base)
         q = apply_rope(q, cos, sin)
         k = apply_rope(k, cos, sin)
+        if not need_attn:
+            return h, k, v
         keys = np.concatenate([self.k_cache[l][b][:, :pos0], k], axis=1)
         vals = np.concatenate([self.v_cache[l][b][:, :pos0], v], axis=1)
         if causal:
@@ -340,7 +347,8 @@ class Oracle:
             h = _f64(self.embed[_index(tokens[b])])
             for l in range(s.n_layers):
                 last = l == s.n_layers - 1
-                h, k, v = self._layer_forward(l, h, b, self.P, causal=True, need_ffn=not last)
+                h, k, v = self._layer_forward(l, h, b, self.P, causal=True, need_ffn=not last,
+                                              need_attn=not last)
                 self.k_cache[l][b] = np.concatenate([self.k_cache[l][b][:, :self.P], k], axis=1)
                 self.v_cache[l][b] = np.concatenate([self.v_cache[l][b][:, :self.P], v], axis=1)
         self.P += n

@@ -89,6 +89,45 @@ def test_a4b_shape_two_layers_prefix_2048():
     print("a4b L2:", rep)
 
 
+def test_a4b_p32k_one_layer_prefix_32768():
+    """The 32k-prefix configuration: the step's bidirectional attention runs
+    over 33,024 keys per (sequence, kv head), split into key chunks merged
+    inside a cluster.  Depth 1, so the causal encoder only projects the prefix
+    to keys/values and the fp64 oracle stays within seconds."""
+    w = si.workload("a4b_p32k").with_layers(1)
+    rep = []
+    _run_workload(w, 1, report=rep)
+    print("a4b p32k L1:", rep)
+
+
+def test_a4b_blockar_b8_step_commit_step():
+    """Batch 8, 4096-token prefix, Zipf-skewed router bias: a step, the block
+    commit (cache advanced by 256 for every sequence) and a step of the next
+    block, each step against the oracle.  Depth 1 keeps the fp64 oracle near a
+    minute; causal attention at these shapes is covered at depth 2 with the
+    2048-token prefix."""
+    w = si.workload("a4b_blockar_b8").with_layers(1)
+    ctx, _ = make_context(w)
+    orc = oracle.for_workload(w)
+    prefix = si.uniform_tokens(w, "prefix", w.batch, w.prefix)
+    ctx.prefill(prefix.cuda())
+    orc.prefill(prefix.numpy())
+    tau = si.tau_schedule(w, 0)
+    canvas = si.uniform_tokens(w, "canvas", w.batch, w.canvas).numpy()
+    g = gpu_step(ctx, w, canvas, 0, w.sample_seed, tau, capture=True)
+    r = orc.denoise_step(canvas, 0, w.sample_seed, tau)
+    compare_step(g, r, tau, orc=orc)
+    block = r.canvas_out
+    ctx.commit_block(torch.as_tensor(block, dtype=torch.int32).cuda())
+    orc.commit_block(block)
+    assert ctx.cached_len == w.prefix + w.canvas == orc.P
+    canvas2 = si.uniform_tokens(w, "canvas", w.batch, w.canvas, block=1).numpy()
+    g2 = gpu_step(ctx, w, canvas2, 0, w.sample_seed, tau, capture=True)
+    r2 = orc.denoise_step(canvas2, 0, w.sample_seed, tau)
+    compare_step(g2, r2, tau, orc=orc)
+    ctx.close()
+
+
 def test_commit_then_step_matches_oracle_and_prefill_of_concatenation():
     w = si.workload("tiny").with_(prefix=64)
     ctx, weights = make_context(w, temperature=0.05)
