@@ -228,21 +228,6 @@ struct ProfScope {
   ~ProfScope() { end(); }
 };
 
-int choose_splits(int tiles, int k_steps, int sms, size_t max_splits_by_cap) {
-  int best = 1;
-  double best_cost = 1e30;
-  for (int s = 1; s <= 8; ++s) {
-    if (k_steps / s < 4 || static_cast<size_t>(s) > max_splits_by_cap) break;
-    const double rounds = std::ceil(static_cast<double>(tiles) * s / sms);
-    const double cost = rounds / s + 0.03 * s;
-    if (cost < best_cost - 1e-9) {
-      best_cost = cost;
-      best = s;
-    }
-  }
-  return best;
-}
-
 // out[s][t][m] = partial sums over split s of W[m, :] . X[t, :]
 // x: token rows with 64-row TMA boxes
 dg_status gemm_dense(dg_ctx* c, const CUtensorMap& w, const CUtensorMap& x, int M, int T, int K, int* splits_out,
@@ -256,13 +241,35 @@ dg_status gemm_dense(dg_ctx* c, const CUtensorMap& w, const CUtensorMap& x, int 
   p.T = T;
   p.k_steps = K / 64;
   const int m_tiles = (M + GEMM_BM - 1) / GEMM_BM;
-  p.bn = std::min(DENSE_BN, (T + 15) / 16 * 16);
-  // few output rows (the router): narrower token tiles, so more CTAs share
-  // the work and each tile's epilogue is shorter
-  if (m_tiles * 8 < c->sms && p.bn > 64) p.bn = 64;
-  p.n_tiles_n = (T + p.bn - 1) / p.bn;
   const size_t cap_s = c->part_cap / (static_cast<size_t>(T) * M);
-  p.splits = choose_splits(m_tiles * p.n_tiles_n, p.k_steps, c->sms, std::min<size_t>(cap_s, max_splits));
+  // Token-tile width and split count from a per-CTA cost model fitted to
+  // in-kernel phase stamps of these GEMMs on B200 (µs): ~2.3 to the first
+  // operands, 0.12 + 0.28*bn/256 per 64-wide k-step, 4.4*bn/256 for the
+  // epilogue, plus ~0.3 per split for the consumer that sums the partials.
+  const int widths[3] = {std::min(DENSE_BN, (T + 15) / 16 * 16), 128, 64};
+  double best = 1e30;
+  int best_bn = widths[0], best_s = 1;
+  for (int wi = 0; wi < 3; ++wi) {
+    const int bnc = widths[wi];
+    if (wi > 0 && bnc >= widths[0]) continue;
+    const int nt = (T + bnc - 1) / bnc;
+    for (int sp = 1; sp <= 8; ++sp) {
+      if (p.k_steps / sp < 4 || static_cast<size_t>(sp) > std::min<size_t>(cap_s, max_splits)) break;
+      const int ctas = m_tiles * nt * sp;
+      const double rounds = std::ceil(static_cast<double>(ctas) / c->sms);
+      const double per_cta = 2.3 + (static_cast<double>(p.k_steps) / sp) * (0.12 + 0.28 * bnc / 256.0) +
+                             4.4 * bnc / 256.0;
+      const double cost = rounds * per_cta + 0.3 * sp;
+      if (cost < best - 1e-9) {
+        best = cost;
+        best_bn = bnc;
+        best_s = sp;
+      }
+    }
+  }
+  p.bn = best_bn;
+  p.n_tiles_n = (T + p.bn - 1) / p.bn;
+  p.splits = best_s;
   p.tiles_static = m_tiles * p.n_tiles_n * p.splits;
   p.out_f32 = c->part;
   p.work = c->dense_work;
