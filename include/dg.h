@@ -50,10 +50,11 @@ typedef enum dg_status {
 
 /* Model shape and capacities.
  * Supported shapes: d_model, expert_hidden and shared_hidden multiples of 64;
- * head_dim in {64, 128, 176}; n_q_heads a multiple of n_kv_heads; vocab a
- * multiple of 128; top_k <= 16 and <= n_experts <= 256, n_experts a multiple
- * of 4; d_model a multiple of 128 and <= 4096; canvas a multiple of 16
- * and <= 256.  The three output projections of a layer are the only places
+ * head_dim in {64, 128, 176}; n_q_heads a multiple of n_kv_heads, and the
+ * group size n_q_heads / n_kv_heads a divisor of 128 (one attention tile
+ * holds whole groups); vocab a multiple of 128; top_k <= 16 and <= n_experts
+ * <= 256, n_experts a multiple of 4; d_model a multiple of 128 and <= 4096;
+ * canvas a multiple of 16 and <= 256.  The three output projections of a layer are the only places
  * where a layer writes the residual stream. */
 typedef struct dg_config {
   int32_t n_layers;
@@ -218,7 +219,7 @@ enum {
   DG_PROF_EXPERTS = 0,       /* fused routed + shared expert GEMM: gate/up (SwiGLU) and down   */
   DG_PROF_ROUTING = 1,       /* router top-k, token permutation and row gather                 */
   DG_PROF_LMHEAD = 2,        /* LM-head GEMM with the argmax / log-sum-exp epilogue            */
-  DG_PROF_ATTENTION = 3,     /* attention kernel (+ chunk merge)                               */
+  DG_PROF_ATTENTION = 3,     /* attention kernel (key chunks merged inside the kernel)         */
   DG_PROF_DENSE = 4,         /* QKV, output and router projections                            */
   DG_PROF_OTHER = 5,         /* norms, RoPE, combine, LM-head merge + sampler                 */
   DG_PROF_CLASSES = 6
