@@ -138,6 +138,26 @@ class Clocks:
 
 
 # ---------------------------------------------------------------------------
+# replicas: one process per GPU, no collective on the data path
+# ---------------------------------------------------------------------------
+def max_over_ranks(value: float, world: int, device) -> float:
+    """The slowest rank's value; every rank must call it (a no-op on one rank)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replicas_value(world: int, batch: int, canvas: int, ms: float) -> float:
+    """Whole-job canvas tokens/s: each of `world` ranks denoises its own batch
+    of `batch` sequences in `ms` milliseconds (the slowest rank's time)."""
+    return world * batch * canvas / (ms * 1e-3)
+
+
+# ---------------------------------------------------------------------------
 # oracle timing (host cores)
 # ---------------------------------------------------------------------------
 def _cores():
@@ -293,10 +313,7 @@ def run_native(args, w):
     clk = clocks.stop(t_wall0, t_wall1)
     launches = (ctx.launch_count - n0) // args.steps
     ctx.sync()
-    if world > 1:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, world, "cuda")
 
     # ---- second timed region, K steps with launches issued one by one: a CUDA
     # event pair on the library stream around every fused expert GEMM launch
@@ -332,12 +349,8 @@ def run_native(args, w):
         hin, hout = hout, hin
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / args.steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-        barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, "cuda")
+    barrier()
 
     hbm, tf_burst, tf_sus, src = peaks()
     by, fl, gu_bytes = step_cost(w, hits)
@@ -357,7 +370,7 @@ def run_native(args, w):
                 traffic = rec["bytes_per_launch"]
         except Exception:
             traffic = None
-    value = world * B * C / (ms * 1e-3)
+    value = replicas_value(world, B, C, ms)
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -377,7 +390,7 @@ def run_native(args, w):
                               "peaks": f"{src}: HBM {hbm} GB/s, bf16 {tf_sus} TF/s sustained"},
             "experts_hit_per_layer": hits,
             "breakdown_ms_per_step": breakdown,
-            "e2e": {"value": world * B * C / (e2e_ms * 1e-3), "unit": UNIT,
+            "e2e": {"value": replicas_value(world, B, C, e2e_ms), "unit": UNIT,
                     "h2d_bytes_per_step": B * C * 4, "d2h_bytes_per_step": B * C * 8 + B * 4,
                     "ms_per_step": e2e_ms},
             "gpu_launches": launches * args.steps,
