@@ -657,18 +657,35 @@ void free_all(dg_ctx* c) {
 // =============================================================================
 // C ABI
 // =============================================================================
+namespace {
+
+// The calling thread's last dg_create failure (a failed create has no
+// context to carry it); dg_last_error(NULL) returns it.
+thread_local std::string g_create_error;
+
+// free a context that dg_create gives up on, keeping its message
+void discard(dg_ctx* c) {
+  g_create_error = "dg_create: " + c->last_error;
+  delete c;
+}
+
+}  // namespace
+
 extern "C" {
 
 dg_status dg_create(const dg_config* cfg, const dg_weights* w, void* cuda_stream, dg_ctx** out) {
-  if (!cfg || !w || !out) return DG_ERR_INVALID_ARG;
+  if (!cfg || !w || !out) {
+    g_create_error = "dg_create: null argument";
+    return DG_ERR_INVALID_ARG;
+  }
+  g_create_error.clear();
   *out = nullptr;
   dg_ctx* c = new dg_ctx();
   c->cfg = *cfg;
   dg_config& g = c->cfg;
   if (g.prefill_rows <= 0) g.prefill_rows = 2048;
   auto reject = [&](dg_status s, const char* why) {
-    static thread_local std::string msg;
-    msg = why;
+    g_create_error = std::string("dg_create: ") + why;
     delete c;
     return s;
   };
@@ -714,18 +731,19 @@ dg_status dg_create(const dg_config* cfg, const dg_weights* w, void* cuda_stream
   cudaError_t e = cudaGetDevice(&c->dev);
   if (e != cudaSuccess) {
     dg_status st = fail(c, DG_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
-    delete c;
+    discard(c);
     return st;
   }
   cudaDeviceGetAttribute(&c->sms, cudaDevAttrMultiProcessorCount, c->dev);
   if (set_smem_attrs(c) != DG_OK) {
-    delete c;
+    discard(c);
     return DG_ERR_CUDA;
   }
   e = c->D == 64 ? attention_cluster_limits<64>(c)
                  : c->D == 128 ? attention_cluster_limits<128>(c) : attention_cluster_limits<176>(c);
   if (e != cudaSuccess) {
-    delete c;
+    fail(c, DG_ERR_CUDA, "cluster occupancy query: %s", cudaGetErrorString(e));
+    discard(c);
     return DG_ERR_CUDA;
   }
 
@@ -773,7 +791,7 @@ dg_status dg_create(const dg_config* cfg, const dg_weights* w, void* cuda_stream
   e = cudaMalloc(&c->ws, bytes);
   if (e != cudaSuccess) {
     dg_status st = fail(c, DG_ERR_OOM, "workspace %zu bytes: %s", bytes, cudaGetErrorString(e));
-    delete c;
+    discard(c);
     return st;
   }
   char* cur = static_cast<char*>(c->ws);
@@ -813,7 +831,7 @@ dg_status dg_create(const dg_config* cfg, const dg_weights* w, void* cuda_stream
   if (e != cudaSuccess) {
     dg_status st = fail(c, DG_ERR_OOM, "KV cache 2 x %zu bytes: %s", cache_elems * 2, cudaGetErrorString(e));
     free_all(c);
-    delete c;
+    discard(c);
     return st;
   }
   // zero everything once: stale rows of token-side operands then hold finite values
@@ -837,7 +855,7 @@ dg_status dg_create(const dg_config* cfg, const dg_weights* w, void* cuda_stream
     if (e != cudaSuccess) {
       dg_status st = fail(c, DG_ERR_CUDA, "rope upload: %s", cudaGetErrorString(e));
       free_all(c);
-      delete c;
+      discard(c);
       return st;
     }
   }
@@ -877,7 +895,7 @@ dg_status dg_create(const dg_config* cfg, const dg_weights* w, void* cuda_stream
   if (!ok) {
     dg_status st = fail(c, DG_ERR_CUDA, "cuTensorMapEncodeTiled failed");
     free_all(c);
-    delete c;
+    discard(c);
     return st;
   }
   *out = c;
@@ -969,7 +987,10 @@ dg_status dg_sync(dg_ctx* c) {
 
 int32_t dg_cached_len(const dg_ctx* c) { return c ? c->P : -1; }
 
-const char* dg_last_error(const dg_ctx* c) { return c ? c->last_error.c_str() : "null context"; }
+const char* dg_last_error(const dg_ctx* c) {
+  if (c) return c->last_error.c_str();
+  return g_create_error.empty() ? "null context" : g_create_error.c_str();
+}
 
 dg_status dg_debug_capture(dg_ctx* c, int32_t enable) {
   if (!c) return DG_ERR_INVALID_ARG;

@@ -24,7 +24,8 @@
  *     anything is launched; a rejected call returns an error and changes no
  *     state.  Errors raised on the device (a bounded wait that ran out) are
  *     reported by the next dg_sync as DG_ERR_DEVICE_TIMEOUT.
- *   - dg_last_error() returns a message for the last failed call on ctx.
+ *   - dg_last_error() returns a message for the last failed call on ctx
+ *     (or, for ctx == NULL, for this thread's last failed dg_create).
  */
 #ifndef DG_H
 #define DG_H
@@ -164,7 +165,9 @@ dg_status dg_sync(dg_ctx* ctx);
 /* Committed cache length P (tokens per sequence). */
 int32_t dg_cached_len(const dg_ctx* ctx);
 
-/* Message for the last failed call (never NULL). */
+/* Message for the last failed call on ctx (never NULL).  With ctx == NULL:
+ * the calling thread's last dg_create failure (a failed create returns no
+ * context), or "null context" if it has none; a successful dg_create clears it. */
 const char* dg_last_error(const dg_ctx* ctx);
 
 /* ---------------------------------------------------------------------------

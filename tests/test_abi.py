@@ -42,3 +42,65 @@ def test_config_struct_matches_header_field_order():
     body = src[src.index("typedef struct dg_layer_weights"):src.index("} dg_layer_weights;")]
     names = re.findall(r"const void\*\s+([a-z_]+);", body)
     assert names == dgp.LAYER_FIELDS
+
+
+def _tiny_config(**over):
+    import synth_inputs as si
+    cfg = dgp.config_from_shape(si.workload("tiny").shape, max_batch=1, max_seq=512, canvas=256)
+    cfg.update(over)
+    c = dgp.dg_config()
+    for name, _ in dgp.dg_config._fields_:
+        setattr(c, name, cfg[name])
+    return c
+
+
+def _fake_weights(n_layers, null_field=None):
+    """Host addresses, 16-byte aligned and never dereferenced: dg_create checks
+    shapes and pointers before it touches a device."""
+    layers = (dgp.dg_layer_weights * n_layers)()
+    for i in range(n_layers):
+        for j, f in enumerate(dgp.LAYER_FIELDS):
+            setattr(layers[i], f, None if f == null_field else 0x10000 + 0x100 * (i * 16 + j))
+    w = dgp.dg_weights(embed=0x200000, final_norm=0x300000, router_bias=None,
+                       layers=ctypes.cast(layers, ctypes.POINTER(dgp.dg_layer_weights)))
+    return w, layers
+
+
+def _create(cfg, w):
+    lib = dgp.load_library()
+    out = ctypes.c_void_p()
+    st = lib.dg_create(ctypes.byref(cfg), ctypes.byref(w), None, ctypes.byref(out))
+    return st, out.value, lib.dg_last_error(None).decode()
+
+
+def test_create_rejects_unsupported_shapes_without_a_device():
+    w, keep = _fake_weights(2)
+    cases = {
+        "head_dim": dict(head_dim=96),                      # not in {64, 128, 176}
+        "gqa group vs attention tile": dict(n_q_heads=6, n_kv_heads=2),   # group 3 does not divide 128
+        "experts": dict(n_experts=300, top_k=2),            # > 256
+        "canvas": dict(canvas=200),                         # not a multiple of 16
+        "d_model": dict(d_model=320),                       # not a multiple of 128
+        "max_seq": dict(max_seq=128),                       # shorter than the canvas
+    }
+    for what, over in cases.items():
+        st, ctx, msg = _create(_tiny_config(**over), w)
+        assert st == 7 and ctx is None, (what, st)          # DG_ERR_UNSUPPORTED, no context
+        assert msg == "dg_create: unsupported shape", (what, msg)
+
+
+def test_create_rejects_bad_arguments_without_a_device():
+    w, keep = _fake_weights(2)
+    st, ctx, msg = _create(_tiny_config(n_layers=0), w)
+    assert (st, ctx) == (1, None) and "non-positive" in msg
+    st, ctx, msg = _create(_tiny_config(temperature=0.0), w)
+    assert (st, ctx) == (1, None) and "non-positive" in msg
+    w2, keep2 = _fake_weights(2, null_field="w_down")
+    st, ctx, msg = _create(_tiny_config(), w2)
+    assert (st, ctx) == (1, None) and "layer weight" in msg
+    w3 = dgp.dg_weights(embed=None, final_norm=0x300000, router_bias=None, layers=w.layers)
+    st, ctx, msg = _create(_tiny_config(), w3)
+    assert (st, ctx) == (1, None) and "null weights" in msg
+    lib = dgp.load_library()
+    assert lib.dg_create(None, ctypes.byref(w), None, None) == 1
+    assert lib.dg_last_error(None) == b"dg_create: null argument"
