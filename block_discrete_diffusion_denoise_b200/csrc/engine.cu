@@ -537,6 +537,15 @@ T* carve(char*& cur, size_t count) {
   return p;
 }
 
+// every kernel's dynamic shared memory fits the 227 KB a CTA may opt into
+constexpr int kMaxSmemPerCta = 232448;
+static_assert(gemm_smem_bytes<GEMM_DENSE>() <= kMaxSmemPerCta, "dense GEMM shared memory");
+static_assert(gemm_smem_bytes<GEMM_MOE>() <= kMaxSmemPerCta, "expert GEMM shared memory");
+static_assert(gemm_smem_bytes<GEMM_LMHEAD>() <= kMaxSmemPerCta, "LM-head GEMM shared memory");
+static_assert(AtcCfg<64>::SMEM <= kMaxSmemPerCta && AtcCfg<128>::SMEM <= kMaxSmemPerCta &&
+                  AtcCfg<176>::SMEM <= kMaxSmemPerCta,
+              "attention shared memory");
+
 dg_status set_smem_attrs(dg_ctx* c) {
   DG_CUDA(c, cudaFuncSetAttribute(gemm_kernel<GEMM_DENSE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   gemm_smem_bytes<GEMM_DENSE>()));
