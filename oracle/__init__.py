@@ -10,7 +10,7 @@ seeded input generator module `synth_inputs`.
 Parity status of each function is recorded beside its pin in tests/.
 """
 from .model import (Oracle, Shape, StepResult, apply_rope, attention, lm_head_stats, moe,
-                    renoise_tokens, rms_norm, rope_angles, route_top_k, sample, silu,
+                    renoise_tokens, rms_norm, rope_angles, route_top_k, sample, selected_gates, silu,
                     swiglu_ffn, tokens_per_forward, tokens_per_second)
 from .philox import philox4x32_10, uniform_token
 

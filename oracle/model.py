@@ -100,10 +100,15 @@ def route_top_k(logits: np.ndarray, k: int):
     for i in range(n):
         order = sorted(range(E), key=lambda e: (-logits[i, e], e))
         idx[i] = order[:k]
-    sel = np.take_along_axis(logits.astype(np.float64), idx, axis=1)
+    return idx, selected_gates(logits, idx)
+
+
+def selected_gates(logits: np.ndarray, idx: np.ndarray) -> np.ndarray:
+    """Softmax over the logits of the experts listed in idx [n, k]."""
+    sel = np.take_along_axis(logits.astype(np.float64), np.asarray(idx, dtype=np.int64), axis=1)
     sel = sel - sel.max(axis=1, keepdims=True)
     g = np.exp(sel)
-    return idx, g / g.sum(axis=1, keepdims=True)
+    return g / g.sum(axis=1, keepdims=True)
 
 
 def swiglu_ffn(x: np.ndarray, wg: np.ndarray, wu: np.ndarray, wd: np.ndarray) -> np.ndarray:
@@ -125,12 +130,13 @@ def moe(u: np.ndarray, lw, idx: np.ndarray, gates: np.ndarray) -> np.ndarray:
 def lm_head_stats(z: np.ndarray, embed, temperature: float, row_chunk: int = 64,
                   vocab_chunk: int = 32768):
     """Per row of logits s = z E^T / T: max m, lowest argmax a, log-sum-exp,
-    confidence exp(m - lse), log-probability m - lse and the top-1/top-2
-    probability margin.  `embed` is the [V, d] tied embedding (any array or
-    bf16 tensor); whole logit rows are formed before any statistic is taken."""
+    confidence exp(m - lse), log-probability m - lse, the top-1/top-2
+    probability margin and the top-1/top-2 logit gap m - m2.  `embed` is the
+    [V, d] tied embedding (any array or bf16 tensor); whole logit rows are
+    formed before any statistic is taken."""
     n = z.shape[0]
     V = embed.shape[0]
-    res = {k: np.empty(n) for k in ("max", "lse", "conf", "logp", "margin")}
+    res = {k: np.empty(n) for k in ("max", "lse", "conf", "logp", "margin", "gap")}
     res["argmax"] = np.empty(n, dtype=np.int64)
     logits = np.empty((min(n, row_chunk), V))
     for r0 in range(0, n, row_chunk):
@@ -152,6 +158,7 @@ def lm_head_stats(z: np.ndarray, embed, temperature: float, row_chunk: int = 64,
         res["conf"][sl] = np.exp(m - lse)
         res["logp"][sl] = m - lse
         res["margin"][sl] = np.exp(m - lse) - np.exp(m2 - lse)
+        res["gap"][sl] = m - m2
     return res
 
 
@@ -256,6 +263,8 @@ class StepResult:
     experts: list = field(default_factory=list)     # per layer, [B, C, k]
     router_logits: list = field(default_factory=list)
     router_margin: list = field(default_factory=list)  # k-th minus (k+1)-th logit
+    gap: np.ndarray | None = None                    # top-1 minus top-2 logit (after /T)
+    forced_hidden: list = field(default_factory=list)  # teacher-forced layer outputs, [B, C, d]
 
 
 class Oracle:
@@ -293,12 +302,16 @@ class Oracle:
 
     # -- one transformer layer over new rows of one sequence --
     def _layer_forward(self, l: int, h: np.ndarray, b: int, pos0: int, causal: bool,
-                       need_ffn: bool = True, dbg: dict | None = None, need_attn: bool = True):
+                       need_ffn: bool = True, dbg: dict | None = None, need_attn: bool = True,
+                       forced_idx: np.ndarray | None = None):
         """One layer over n new rows at positions [pos0, pos0 + n).  Returns the
         updated residual and the rows' keys/values.  need_attn=False returns
         after the keys/values (h unchanged): the causal encoder's last layer
         only feeds the cache (codemajin.net "DiffusionGemma architecture",
-        section 3.2)."""
+        section 3.2).  forced_idx [n, k], when given, replaces the layer's own
+        top-k choice by these experts (gates are still the softmax of this
+        layer's logits at them): a test measures one layer's error on inputs
+        and routing taken from elsewhere."""
         s = self.s
         lw = self.layer(l)
         n = h.shape[0]
@@ -326,7 +339,11 @@ class Oracle:
             r = u2 @ lw["w_router"].T
             if self.router_bias is not None:
                 r = r + self.router_bias
-            idx, gates = route_top_k(r, s.top_k)
+            if forced_idx is None:
+                idx, gates = route_top_k(r, s.top_k)
+            else:
+                idx = np.asarray(forced_idx, dtype=np.int64)
+                gates = selected_gates(r, idx)
             h = h + moe(u2, lw, idx, gates)
             if dbg is not None:
                 dbg["idx"], dbg["logits"] = idx, r
@@ -369,7 +386,15 @@ class Oracle:
 
     # -- bidirectional decoder + sampler --
     def denoise_step(self, canvas: np.ndarray, step: int, seed: int, tau: float,
-                     temperature: float = 1.0, record: bool = True) -> StepResult:
+                     temperature: float = 1.0, record: bool = True,
+                     teacher: dict | None = None) -> StepResult:
+        """One denoising step of the canvas [B, C] (cache unchanged).
+
+        teacher = {"hidden": [L+1 of [B, C, d]], "experts": [L of [B, C, k]]},
+        when given, also runs every layer l on teacher["hidden"][l] with the
+        experts teacher["experts"][l] and returns those outputs as
+        forced_hidden[l + 1] (forced_hidden[0] is teacher["hidden"][0]): the
+        error of each layer alone, free of the drift accumulated before it."""
         canvas = np.asarray(canvas)
         B, C = canvas.shape
         s = self.s
@@ -378,6 +403,10 @@ class Oracle:
         rlog = [np.empty((B, C, s.n_experts)) for _ in range(s.n_layers)] if record else []
         rmar = [np.empty((B, C)) for _ in range(s.n_layers)] if record else []
         z = np.empty((B, C, s.d_model))
+        forced = []
+        if teacher is not None:
+            forced = [np.asarray(teacher["hidden"][0], dtype=np.float64)]
+            forced += [np.empty((B, C, s.d_model)) for _ in range(s.n_layers)]
         for b in range(B):
             h = _f64(self.embed[_index(canvas[b])])
             if record:
@@ -385,6 +414,11 @@ class Oracle:
             for l in range(s.n_layers):
                 dbg = {}
                 h, _, _ = self._layer_forward(l, h, b, self.P, causal=False, dbg=dbg)
+                if teacher is not None:
+                    hf, _, _ = self._layer_forward(
+                        l, np.asarray(teacher["hidden"][l][b], dtype=np.float64), b, self.P,
+                        causal=False, forced_idx=teacher["experts"][l][b])
+                    forced[l + 1][b] = hf
                 if record:
                     hidden[l + 1][b] = h
                     experts[l][b] = dbg["idx"]
@@ -400,4 +434,4 @@ class Oracle:
         return StepResult(canvas_out=rs(out), conf=rs(st["conf"]), argmax=rs(st["argmax"]),
                           lse=rs(st["lse"]), logp=rs(st["logp"]), margin=rs(st["margin"]),
                           hidden=hidden, experts=experts, router_logits=rlog,
-                          router_margin=rmar)
+                          router_margin=rmar, gap=rs(st["gap"]), forced_hidden=forced)

@@ -211,12 +211,15 @@ def test_lm_head_stats_match_logsumexp_and_ties():
     np.testing.assert_allclose(st["lse"], logsumexp(s, axis=1), rtol=1e-13)
     assert st["argmax"][0] == 3                  # lowest index of the tied max
     assert st["margin"][0] == 0.0
+    assert st["gap"][0] == 0.0
     for i in range(5):
         p = np.exp(s[i] - logsumexp(s[i]))
         srt = np.sort(p)[::-1]
         assert st["argmax"][i] == min(j for j in range(37) if s[i, j] == s[i].max())
         assert abs(st["conf"][i] - srt[0]) < 1e-14
         assert abs(st["margin"][i] - (srt[0] - srt[1])) < 1e-14
+        ls = sorted(s[i], reverse=True)           # brute-force top-1 minus top-2 logit
+        assert abs(st["gap"][i] - (ls[0] - ls[1])) < 1e-12
 
 
 # --- sampler: fixed positions kept, re-noised tokens uniform (chi-square) ---
