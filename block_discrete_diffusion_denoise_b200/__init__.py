@@ -20,7 +20,7 @@ STATUS = {0: "DG_OK", 1: "DG_ERR_INVALID_ARG", 2: "DG_ERR_OOM", 3: "DG_ERR_CAPAC
 # every function declared in include/dg.h
 EXPORTS = ["dg_create", "dg_destroy", "dg_prefill", "dg_denoise_step", "dg_denoise_step_host",
            "dg_commit_block", "dg_sync", "dg_cached_len", "dg_last_error", "dg_debug_capture",
-           "dg_debug_hidden", "dg_debug_experts", "dg_debug_lmhead", "dg_debug_router",
+           "dg_debug_hidden", "dg_debug_experts", "dg_debug_norm_rows", "dg_debug_lmhead", "dg_debug_router",
            "dg_debug_sample", "dg_debug_wait_timeout", "dg_debug_gemm", "dg_debug_profile",
            "dg_debug_profile_read", "dg_debug_launch_count", "dg_lmhead_argmax_static"]
 
@@ -84,6 +84,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "dg_debug_capture": ([P, I32], I32),
         "dg_debug_hidden": ([P, I32, P], I32),
         "dg_debug_experts": ([P, I32, P], I32),
+        "dg_debug_norm_rows": ([P, I32, P], I32),
         "dg_debug_lmhead": ([P, P, P, P, P], I32),
         "dg_debug_router": ([P, P, I32, P, P], I32),
         "dg_debug_sample": ([P, P, P, I32, I32, U64, F32, P], I32),
@@ -188,6 +189,9 @@ class Context:
     def debug_experts(self, layer, out):
         self._check(self.lib.dg_debug_experts(self.ctx, layer, _ptr(out)))
 
+    def debug_norm_rows(self, layer, out):
+        self._check(self.lib.dg_debug_norm_rows(self.ctx, layer, _ptr(out)))
+
     def debug_lmhead(self, argmax=None, lse=None, conf=None, margin=None):
         self._check(self.lib.dg_debug_lmhead(self.ctx, _ptr(argmax), _ptr(lse), _ptr(conf), _ptr(margin)))
 
@@ -236,8 +240,77 @@ def config_from_shape(shape, max_batch=1, max_seq=4096, canvas=256, temperature=
 
 def lmhead_argmax_static(z, embed, temperature, argmax=None, lse=None, conf=None, stream=None) -> int:
     """dg_lmhead_argmax_static on torch CUDA tensors; returns the dg_status
-    code (0 = launched).  No device memory is allocated by the library."""
+    code (0 = launched).  No device memory is allocated by the library.
+
+    The library sees raw pointers and sizes only, so the tensors are checked
+    here first and DG_ERR_INVALID_ARG (1) is returned, with nothing launched,
+    when z or embed is not a contiguous bf16 CUDA matrix, their widths differ,
+    or an output is not a contiguous CUDA tensor of its type (int32 argmax,
+    float32 lse / conf) with at least one element per row of z."""
+    import torch
     lib = load_library()
+
+    def dense_cuda(t, dtype, ndim=None):
+        return (isinstance(t, torch.Tensor) and t.is_cuda and t.dtype == dtype and t.is_contiguous()
+                and (ndim is None or t.dim() == ndim))
+    if not (dense_cuda(z, torch.bfloat16, 2) and dense_cuda(embed, torch.bfloat16, 2)):
+        return 1
     n_rows, d = z.shape
+    if embed.shape[1] != d or embed.device != z.device:
+        return 1
+    for t, dtype in ((argmax, torch.int32), (lse, torch.float32), (conf, torch.float32)):
+        if t is not None and not (dense_cuda(t, dtype) and t.numel() >= n_rows and t.device == z.device):
+            return 1
     return lib.dg_lmhead_argmax_static(_ptr(z), n_rows, d, _ptr(embed), embed.shape[0], float(temperature),
                                        _ptr(argmax), _ptr(lse), _ptr(conf), stream)
+
+
+def generate_blocks(ctx: Context, prefix, init_canvas, n_blocks: int, max_steps: int, tau, seed: int,
+                    commit_last: bool = False, before_step=None, after_step=None) -> dict:
+    """Block-autoregressive generation through the C ABI (codemajin.net
+    "DiffusionGemma architecture", section 3.2, block-AR; aibars.net, block
+    commit): prefill the prompt causally, then for each block start from
+    init_canvas(k) (an int32 CUDA tensor [batch, canvas], e.g. uniform noise),
+    run up to max_steps denoising steps, stop as soon as every position of
+    every sequence is settled (conf >= tau, read from the all-settled flags),
+    and commit the block to the KV cache.  The last block is committed only
+    with commit_last, matching the K - 1 commit forwards that codemajin.net
+    section 5.1 counts in TPF.
+
+    tau is a float or a function of the step index.  before_step(k, s) and
+    after_step(k, s, canvas_in, canvas_out, conf, settled) are optional hooks
+    (tests use them to record a step).  Host control only: every step of the
+    path runs in the library's kernels; the one device-to-host read per step is
+    the batch's all-settled flags.
+
+    Returns {"blocks": [final canvas of each block], "steps": [steps taken per
+    block], "settled": [whether each block stopped early]}."""
+    import torch
+    B, C = int(prefix.shape[0]), int(ctx.cfg["canvas"])
+    ctx.prefill(prefix)
+    out = {"blocks": [], "steps": [], "settled": []}
+    for k in range(n_blocks):
+        cur = init_canvas(k).to(torch.int32).contiguous()
+        nxt = torch.empty_like(cur)
+        conf = torch.empty(B, C, dtype=torch.float32, device=cur.device)
+        settled = torch.empty(B, dtype=torch.int32, device=cur.device)
+        steps, done = 0, False
+        for s in range(max_steps):
+            if before_step is not None:
+                before_step(k, s)
+            t = tau(s) if callable(tau) else tau
+            ctx.denoise_step(cur, s, seed, t, nxt, conf, settled)
+            if after_step is not None:
+                after_step(k, s, cur, nxt, conf, settled)
+            cur, nxt = nxt, cur
+            steps += 1
+            ctx.sync()                       # the flags are written on the context's stream
+            if bool((settled.cpu() != 0).all()):
+                done = True
+                break
+        out["blocks"].append(cur.clone())
+        out["steps"].append(steps)
+        out["settled"].append(done)
+        if k + 1 < n_blocks or commit_last:
+            ctx.commit_block(cur)
+    return out

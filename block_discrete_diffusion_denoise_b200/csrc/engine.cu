@@ -7,6 +7,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -93,6 +94,7 @@ struct dg_ctx {
   bool capture = false;
   float* cap_h = nullptr;
   int32_t* cap_idx = nullptr;
+  uint16_t* cap_u = nullptr;    // [L + 1][R_step][d]: router inputs per layer, then the LM-head input
   // tensor maps
   std::vector<LayerMaps> lmaps;
   CUtensorMap m_u16{}, m_u64{}, m_u128{}, m_o64{}, m_xp16{}, m_h16{}, m_hs16{}, m_embed{};
@@ -471,6 +473,9 @@ dg_status forward(dg_ctx* c, const int32_t* tokens, int tok_stride, int tok_off,
     DG_LAUNCH(c, residual_norm_kernel, T, 256, 0, c->h, static_cast<const float*>(c->part), s2, T, c->d,
               static_cast<const uint16_t*>(lw.ffn_norm), eps, c->u);
     ps10.end();
+    if (c->capture && !causal)
+      DG_CUDA(c, cudaMemcpyAsync(c->cap_u + static_cast<size_t>(l) * c->R_step * c->d, c->u,
+                                 static_cast<size_t>(T) * c->d * 2, cudaMemcpyDeviceToDevice, c->stream));
     st = moe(c, l, T);
     if (st != DG_OK) return st;
     const uint16_t* next_gain = l + 1 < c->L ? static_cast<const uint16_t*>(c->layers[l + 1].attn_norm)
@@ -481,6 +486,9 @@ dg_status forward(dg_ctx* c, const int32_t* tokens, int tok_stride, int tok_off,
               static_cast<const int32_t*>(c->inv_slot), static_cast<const float*>(c->gates), c->k, T * c->k, c->d,
               next_gain, eps, c->u, cap);
     ps11.end();
+    if (c->capture && !causal && l == c->L - 1)
+      DG_CUDA(c, cudaMemcpyAsync(c->cap_u + static_cast<size_t>(c->L) * c->R_step * c->d, c->u,
+                                 static_cast<size_t>(T) * c->d * 2, cudaMemcpyDeviceToDevice, c->stream));
   }
   return DG_OK;
 }
@@ -655,10 +663,12 @@ void free_all(dg_ctx* c) {
   if (c->vcache) cudaFree(c->vcache);
   if (c->cap_h) cudaFree(c->cap_h);
   if (c->cap_idx) cudaFree(c->cap_idx);
+  if (c->cap_u) cudaFree(c->cap_u);
   c->ws = nullptr;
   c->kcache = c->vcache = nullptr;
   c->cap_h = nullptr;
   c->cap_idx = nullptr;
+  c->cap_u = nullptr;
 }
 
 }  // namespace
@@ -1006,13 +1016,16 @@ dg_status dg_debug_capture(dg_ctx* c, int32_t enable) {
   if (enable && !c->cap_h) {
     DG_CUDA(c, cudaMalloc(&c->cap_h, static_cast<size_t>(c->L + 1) * c->R_step * c->d * 4));
     DG_CUDA(c, cudaMalloc(&c->cap_idx, static_cast<size_t>(c->L) * c->R_step * c->k * 4));
+    DG_CUDA(c, cudaMalloc(&c->cap_u, static_cast<size_t>(c->L + 1) * c->R_step * c->d * 2));
   }
   if (!enable && c->cap_h) {
     cudaStreamSynchronize(c->stream);
     cudaFree(c->cap_h);
     cudaFree(c->cap_idx);
+    cudaFree(c->cap_u);
     c->cap_h = nullptr;
     c->cap_idx = nullptr;
+    c->cap_u = nullptr;
   }
   c->capture = enable != 0;
   return DG_OK;
@@ -1030,6 +1043,14 @@ dg_status dg_debug_experts(dg_ctx* c, int32_t layer, int32_t* out) {
   if (!c || !out || !c->cap_idx || layer < 0 || layer >= c->L) return fail(c, DG_ERR_INVALID_ARG, "debug_experts");
   const size_t n = static_cast<size_t>(c->B) * c->cfg.canvas * c->k;
   DG_CUDA(c, cudaMemcpyAsync(out, c->cap_idx + static_cast<size_t>(layer) * c->R_step * c->k, n * 4,
+                             cudaMemcpyDeviceToDevice, c->stream));
+  return DG_OK;
+}
+
+dg_status dg_debug_norm_rows(dg_ctx* c, int32_t layer, void* out) {
+  if (!c || !out || !c->cap_u || layer < 0 || layer > c->L) return fail(c, DG_ERR_INVALID_ARG, "debug_norm_rows");
+  const size_t n = static_cast<size_t>(c->B) * c->cfg.canvas * c->d;
+  DG_CUDA(c, cudaMemcpyAsync(out, c->cap_u + static_cast<size_t>(layer) * c->R_step * c->d, n * 2,
                              cudaMemcpyDeviceToDevice, c->stream));
   return DG_OK;
 }
@@ -1152,6 +1173,7 @@ struct StaticSetup {
   int sms = 0;
 };
 StaticSetup g_static_setup[kMaxDevices];
+std::mutex g_static_setup_mutex;  // the first calls on a device may come from several threads
 
 // merge of the partials into argmax / lse / conf (rows flagged by a timed-out
 // wait get argmax -1 and NaN statistics)
@@ -1197,16 +1219,23 @@ extern "C" dg_status dg_lmhead_argmax_static(const void* z, int32_t n_rows, int3
     return DG_ERR_CAPACITY;  // n_rows * vocab / 128 beyond the fixed scratch
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DG_ERR_CUDA;
-  StaticSetup& su = g_static_setup[dev];
-  if (!su.done) {
+  StaticSetup su;
+  {
     // once per device, with that device current (the caller's current device)
-    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&su.partials), g_lm_static_partials) != cudaSuccess ||
-        cudaGetSymbolAddress(reinterpret_cast<void**>(&su.err), g_lm_static_err) != cudaSuccess ||
-        cudaDeviceGetAttribute(&su.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-        cudaFuncSetAttribute(gemm_kernel<GEMM_LMHEAD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             gemm_smem_bytes<GEMM_LMHEAD>()) != cudaSuccess)
-      return DG_ERR_CUDA;
-    su.done = true;
+    std::lock_guard<std::mutex> lock(g_static_setup_mutex);
+    StaticSetup& g = g_static_setup[dev];
+    if (!g.done) {
+      StaticSetup n;
+      if (cudaGetSymbolAddress(reinterpret_cast<void**>(&n.partials), g_lm_static_partials) != cudaSuccess ||
+          cudaGetSymbolAddress(reinterpret_cast<void**>(&n.err), g_lm_static_err) != cudaSuccess ||
+          cudaDeviceGetAttribute(&n.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+          cudaFuncSetAttribute(gemm_kernel<GEMM_LMHEAD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               gemm_smem_bytes<GEMM_LMHEAD>()) != cudaSuccess)
+        return DG_ERR_CUDA;
+      n.done = true;
+      g = n;
+    }
+    su = g;
   }
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
   GemmParams p;
@@ -1222,11 +1251,21 @@ extern "C" dg_status dg_lmhead_argmax_static(const void* z, int32_t n_rows, int3
   p.logit_scale_log2 = static_cast<float>(1.4426950408889634 / static_cast<double>(temperature));
   p.err = DevErr{su.err, 1000000000ull};
   if (cudaMemsetAsync(su.err, 0, sizeof(int), st) != cudaSuccess) return DG_ERR_CUDA;
-  gemm_kernel<GEMM_LMHEAD><<<std::min(su.sms, p.tiles_static), GEMM_THREADS, gemm_smem_bytes<GEMM_LMHEAD>(),
-                             st>>>(p);
-  if (cudaGetLastError() != cudaSuccess) return DG_ERR_CUDA;
-  lmhead_static_merge_kernel<<<n_rows, 256, 0, st>>>(su.partials, n_vtiles, n_rows, su.err, argmax_out, lse_out,
-                                                     conf_out);
-  if (cudaGetLastError() != cudaSuccess) return DG_ERR_CUDA;
+  // each launch's own status (cudaLaunchKernelEx), so an error the caller
+  // left pending from its own earlier work is neither reported nor cleared here
+  cudaLaunchConfig_t lc{};
+  lc.gridDim = dim3(std::min(su.sms, p.tiles_static));
+  lc.blockDim = dim3(GEMM_THREADS);
+  lc.dynamicSmemBytes = gemm_smem_bytes<GEMM_LMHEAD>();
+  lc.stream = st;
+  if (cudaLaunchKernelEx(&lc, gemm_kernel<GEMM_LMHEAD>, p) != cudaSuccess) return DG_ERR_CUDA;
+  lc.gridDim = dim3(n_rows);
+  lc.blockDim = dim3(256);
+  lc.dynamicSmemBytes = 0;
+  const float4* parts = su.partials;
+  const int* errp = su.err;
+  if (cudaLaunchKernelEx(&lc, lmhead_static_merge_kernel, parts, n_vtiles, static_cast<int>(n_rows), errp,
+                         argmax_out, lse_out, conf_out) != cudaSuccess)
+    return DG_ERR_CUDA;
   return DG_OK;
 }

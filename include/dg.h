@@ -187,6 +187,14 @@ dg_status dg_debug_hidden(dg_ctx* ctx, int32_t layer, float* out_dev);
  * int32, ordered by (logit desc, index asc). */
 dg_status dg_debug_experts(dg_ctx* ctx, int32_t layer, int32_t* out_dev);
 
+/* bf16 rows [batch*canvas, d] of the last recorded step, exactly as the
+ * kernels consumed them: for 0 <= layer < n_layers the rows fed to that
+ * layer's router and experts (RMSNorm of the residual after attention), for
+ * layer == n_layers the rows fed to the LM head (the final RMSNorm).  Lets a
+ * test give the oracle the very operands of a decision (expert choice,
+ * argmax) the kernels took. */
+dg_status dg_debug_norm_rows(dg_ctx* ctx, int32_t layer, void* out_dev);
+
 /* LM-head reduction of the last step: per position the argmax (lowest index
  * of the maximum), log-sum-exp, confidence and top-1 minus top-2
  * probability.  Each pointer [batch*canvas] or NULL. */
@@ -265,7 +273,10 @@ int64_t dg_debug_launch_count(const dg_ctx* ctx);
  *     of 128, unaligned pointers) with DG_ERR_INVALID_ARG.
  *   - The first call on a device looks up the array's device address and sets
  *     the kernel attributes for that device (the device current at the call);
- *     make that first call before any stream capture.
+ *     make that first call before any stream capture.  That set-up runs under
+ *     a lock, so first calls may come from any thread.
+ *   - Only the two launches' own status is checked: a CUDA error the caller
+ *     left pending from earlier work is neither reported nor cleared.
  *   - Every call on a device shares the one array, whose contents persist
  *     between calls: each call writes every partial it later reads and clears
  *     its own error flag first, but calls that overlap on the GPU (different

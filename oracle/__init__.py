@@ -24,10 +24,11 @@ def shape_of(w) -> Shape:
                  vocab=s.vocab, rope_base=s.rope_base, rms_eps=s.rms_eps)
 
 
-def for_workload(w, keep_layers: bool = True, layer_override=None) -> Oracle:
+def for_workload(w, keep_layers: bool = True, layer_override=None, seq_ids=None) -> Oracle:
     """Oracle over the seeded weights of workload `w` (generated on the CPU).
 
-    layer_override(l, tensors) may edit a layer's tensors (planted cases)."""
+    layer_override(l, tensors) may edit a layer's tensors (planted cases);
+    seq_ids gives the batch index of each of the oracle's sequences."""
     import synth_inputs as si
 
     def layer_fn(l):
@@ -38,4 +39,4 @@ def for_workload(w, keep_layers: bool = True, layer_override=None) -> Oracle:
 
     g = si.global_weights(w, "cpu")
     return Oracle(shape_of(w), layer_fn, g["embed"], g["final_norm"], g["router_bias"],
-                  batch=w.batch, keep_layers=keep_layers)
+                  batch=w.batch, keep_layers=keep_layers, seq_ids=seq_ids)

@@ -265,6 +265,9 @@ class StepResult:
     router_margin: list = field(default_factory=list)  # k-th minus (k+1)-th logit
     gap: np.ndarray | None = None                    # top-1 minus top-2 logit (after /T)
     forced_hidden: list = field(default_factory=list)  # teacher-forced layer outputs, [B, C, d]
+    forced_experts: list = field(default_factory=list)  # top-k of given router rows, [B, C, k]
+    forced_router_margin: list = field(default_factory=list)  # their k-th minus (k+1)-th logit
+    forced_lm: dict | None = None                    # lm_head_stats of given LM-head rows, [B, C]
 
 
 class Oracle:
@@ -275,13 +278,16 @@ class Oracle:
     """
 
     def __init__(self, shape: Shape, layer_fn, embed, final_norm, router_bias=None,
-                 batch: int = 1, keep_layers: bool = True):
+                 batch: int = 1, keep_layers: bool = True, seq_ids=None):
         self.s = shape
         self.layer_fn = layer_fn
         self.embed = embed            # kept in storage precision; rows converted on use
         self.final_norm = _f64(final_norm)
         self.router_bias = None if router_bias is None else _f64(router_bias)
         self.B = batch
+        # index of each of the oracle's sequences in the caller's batch (the
+        # sampler's counter carries it): a subset of a batch can be checked
+        self.seq_ids = np.arange(batch) if seq_ids is None else np.asarray(seq_ids)
         self.keep_layers = keep_layers
         self._layers = {}
         # KV cache per layer: list over sequences of (K [Hkv, P, D], V [Hkv, P, D])
@@ -295,9 +301,14 @@ class Oracle:
     def layer(self, l: int) -> LayerWeights:
         if l in self._layers:
             return self._layers[l]
+        last = getattr(self, "_last_layer", None)
+        if last is not None and last[0] == l:
+            return last[1]
         lw = LayerWeights(self.layer_fn(l))
         if self.keep_layers:
             self._layers[l] = lw
+        else:
+            self._last_layer = (l, lw)   # only the layer in use is held
         return lw
 
     # -- one transformer layer over new rows of one sequence --
@@ -394,7 +405,12 @@ class Oracle:
         when given, also runs every layer l on teacher["hidden"][l] with the
         experts teacher["experts"][l] and returns those outputs as
         forced_hidden[l + 1] (forced_hidden[0] is teacher["hidden"][0]): the
-        error of each layer alone, free of the drift accumulated before it."""
+        error of each layer alone, free of the drift accumulated before it.
+        Optional teacher["router_rows"] (L of [B, C, d], the normalised rows a
+        layer's router consumed) give forced_experts / forced_router_margin,
+        the top-k of those rows' logits; teacher["lm_rows"] ([B, C, d], the
+        normalised rows the LM head consumed) give forced_lm, the LM-head
+        statistics of those rows."""
         canvas = np.asarray(canvas)
         B, C = canvas.shape
         s = self.s
@@ -403,10 +419,13 @@ class Oracle:
         rlog = [np.empty((B, C, s.n_experts)) for _ in range(s.n_layers)] if record else []
         rmar = [np.empty((B, C)) for _ in range(s.n_layers)] if record else []
         z = np.empty((B, C, s.d_model))
-        forced = []
+        forced, f_exp, f_mar, f_lm = [], [], [], None
         if teacher is not None:
             forced = [np.asarray(teacher["hidden"][0], dtype=np.float64)]
             forced += [np.empty((B, C, s.d_model)) for _ in range(s.n_layers)]
+            if teacher.get("router_rows") is not None:
+                f_exp = [np.empty((B, C, s.top_k), dtype=np.int64) for _ in range(s.n_layers)]
+                f_mar = [np.empty((B, C)) for _ in range(s.n_layers)]
         for b in range(B):
             h = _f64(self.embed[_index(canvas[b])])
             if record:
@@ -419,6 +438,16 @@ class Oracle:
                         l, np.asarray(teacher["hidden"][l][b], dtype=np.float64), b, self.P,
                         causal=False, forced_idx=teacher["experts"][l][b])
                     forced[l + 1][b] = hf
+                    if teacher.get("router_rows") is not None:
+                        rr = np.asarray(teacher["router_rows"][l][b], dtype=np.float64) @ \
+                            self.layer(l)["w_router"].T
+                        if self.router_bias is not None:
+                            rr = rr + self.router_bias
+                        fi, _ = route_top_k(rr, s.top_k)
+                        srt = -np.sort(-rr, axis=1)
+                        f_exp[l][b] = fi
+                        f_mar[l][b] = (srt[:, s.top_k - 1] - srt[:, s.top_k] if s.top_k < s.n_experts
+                                       else np.inf)
                 if record:
                     hidden[l + 1][b] = h
                     experts[l][b] = dbg["idx"]
@@ -426,12 +455,16 @@ class Oracle:
                     rmar[l][b] = dbg["margin"]
             z[b] = rms_norm(h, self.final_norm, s.rms_eps)
         st = lm_head_stats(z.reshape(B * C, s.d_model), self.embed, temperature)
+        if teacher is not None and teacher.get("lm_rows") is not None:
+            zf = np.asarray(teacher["lm_rows"], dtype=np.float64).reshape(B * C, s.d_model)
+            f_lm = {k: v.reshape(B, C) for k, v in lm_head_stats(zf, self.embed, temperature).items()}
         pos = np.tile(np.arange(self.P, self.P + C), B)
-        seq = np.repeat(np.arange(B), C)
+        seq = np.repeat(self.seq_ids[:B], C)
         noise = renoise_tokens(pos, step, seq, seed, s.vocab)
         out = sample(st["argmax"], st["conf"], tau, noise)
         rs = lambda a: a.reshape(B, C)
         return StepResult(canvas_out=rs(out), conf=rs(st["conf"]), argmax=rs(st["argmax"]),
                           lse=rs(st["lse"]), logp=rs(st["logp"]), margin=rs(st["margin"]),
                           hidden=hidden, experts=experts, router_logits=rlog,
-                          router_margin=rmar, gap=rs(st["gap"]), forced_hidden=forced)
+                          router_margin=rmar, gap=rs(st["gap"]), forced_hidden=forced,
+                          forced_experts=f_exp, forced_router_margin=f_mar, forced_lm=f_lm)

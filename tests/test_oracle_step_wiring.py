@@ -161,22 +161,38 @@ def test_batch_rows_are_independent():
     both.prefill(prompt)
     rb = both.denoise_step(canvas, 3, 9, 0.9)
     for b in range(2):
-        one = oracle.for_workload(w.with_(batch=1))
+        # one sequence alone, told its index in the batch (the sampler's counter carries it)
+        one = oracle.for_workload(w.with_(batch=1), seq_ids=[b])
         one.prefill(prompt[b:b + 1])
         r1 = one.denoise_step(canvas[b:b + 1], 3, 9, 0.9)
         np.testing.assert_allclose(rb.hidden[-1][b], r1.hidden[-1][0], rtol=1e-12, atol=1e-14)
         np.testing.assert_array_equal(rb.argmax[b], r1.argmax[0])
+        np.testing.assert_array_equal(rb.canvas_out[b], r1.canvas_out[0])
 
 
 def test_teacher_forced_layer_reproduces_free_running_layer(setup):
-    """Fed its own hidden states and expert choices, the teacher-forced
-    layers give the free-running ones back (the forced mode changes where a
-    layer's inputs come from, not what it computes)."""
+    """Fed its own hidden states, expert choices, router rows and LM-head rows,
+    the teacher-forced mode gives the free-running results back (it changes
+    where a layer's inputs come from, not what it computes)."""
     w, weights, prompt, canvas, seq, orc, r = setup
-    teacher = {"hidden": r.hidden, "experts": r.experts}
+    s = w.shape
+    router_rows = []
+    for l in range(s.n_layers):
+        # the router's input: RMSNorm of the residual after this layer's attention
+        lw = orc.layer(l)
+        hh, _, _ = orc._layer_forward(l, r.hidden[l][0], 0, orc.P, causal=False, need_ffn=False)
+        router_rows.append(oracle.rms_norm(hh, lw["ffn_norm"], s.rms_eps)[None])
+    lm_rows = oracle.rms_norm(r.hidden[-1], orc.final_norm, s.rms_eps)
+    teacher = {"hidden": r.hidden, "experts": r.experts, "router_rows": router_rows, "lm_rows": lm_rows}
     rf = orc.denoise_step(canvas.numpy(), 0, 1, 0.9, temperature=0.5, teacher=teacher)
-    for l in range(w.shape.n_layers + 1):
+    for l in range(s.n_layers + 1):
         np.testing.assert_array_equal(rf.forced_hidden[l], r.hidden[l])
+    for l in range(s.n_layers):
+        np.testing.assert_array_equal(rf.forced_experts[l], r.experts[l])
+        np.testing.assert_allclose(rf.forced_router_margin[l], r.router_margin[l], rtol=1e-12, atol=1e-14)
+    np.testing.assert_array_equal(rf.forced_lm["argmax"], r.argmax)
+    np.testing.assert_allclose(rf.forced_lm["lse"], r.lse, rtol=1e-14)
+    np.testing.assert_allclose(rf.forced_lm["gap"], r.gap, rtol=1e-12, atol=1e-14)
 
 
 @pytest.mark.parametrize("plant", ["rope_from_zero", "canvas_sees_only_itself", "causal_step",
