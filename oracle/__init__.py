@@ -9,7 +9,8 @@ seeded input generator module `synth_inputs`.
 
 Parity status of each function is recorded beside its pin in tests/.
 """
-from .model import (Oracle, Shape, StepResult, apply_rope, attention, lm_head_stats, moe,
+from .model import (Oracle, Shape, StepResult, anneal_temperature, apply_rope, attention, entropy_accept,
+                    entropy_sample, lm_head_stats, mean_entropy, moe,
                     renoise_tokens, rms_norm, rope_angles, route_top_k, sample, selected_gates, silu,
                     swiglu_ffn, tokens_per_forward, tokens_per_second)
 from .philox import philox4x32_10, uniform_token

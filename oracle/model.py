@@ -131,12 +131,13 @@ def lm_head_stats(z: np.ndarray, embed, temperature: float, row_chunk: int = 64,
                   vocab_chunk: int = 32768):
     """Per row of logits s = z E^T / T: max m, lowest argmax a, log-sum-exp,
     confidence exp(m - lse), log-probability m - lse, the top-1/top-2
-    probability margin and the top-1/top-2 logit gap m - m2.  `embed` is the
-    [V, d] tied embedding (any array or bf16 tensor); whole logit rows are
+    probability margin, the top-1/top-2 logit gap m - m2 and the entropy of
+    the softmax, -sum_v p_v ln p_v = lse - sum_v p_v s_v (nats).  `embed` is
+    the [V, d] tied embedding (any array or bf16 tensor); whole logit rows are
     formed before any statistic is taken."""
     n = z.shape[0]
     V = embed.shape[0]
-    res = {k: np.empty(n) for k in ("max", "lse", "conf", "logp", "margin", "gap")}
+    res = {k: np.empty(n) for k in ("max", "lse", "conf", "logp", "margin", "gap", "entropy")}
     res["argmax"] = np.empty(n, dtype=np.int64)
     logits = np.empty((min(n, row_chunk), V))
     for r0 in range(0, n, row_chunk):
@@ -149,6 +150,8 @@ def lm_head_stats(z: np.ndarray, embed, temperature: float, row_chunk: int = 64,
         a = np.argmax(s, axis=1)                      # first (lowest) index of the max
         m = s[rows, a]
         lse = m + np.log(np.exp(s - m[:, None]).sum(axis=1))
+        prob = np.exp(s - lse[:, None])
+        ent = lse - (prob * s).sum(axis=1)
         s[rows, a] = -np.inf
         m2 = s.max(axis=1)
         sl = slice(r0, r0 + s.shape[0])
@@ -159,6 +162,7 @@ def lm_head_stats(z: np.ndarray, embed, temperature: float, row_chunk: int = 64,
         res["logp"][sl] = m - lse
         res["margin"][sl] = np.exp(m - lse) - np.exp(m2 - lse)
         res["gap"][sl] = m - m2
+        res["entropy"][sl] = ent
     return res
 
 
@@ -178,6 +182,67 @@ def sample(argmax: np.ndarray, conf: np.ndarray, tau: float, noise: np.ndarray) 
     confidence re-noises)."""
     keep = np.asarray(conf) >= tau
     return np.where(keep, argmax, noise)
+
+
+# ---------------------------------------------------------------------------
+# entropy-constrained sampler (codemajin.net "DiffusionGemma architecture",
+# section 3.3).  The page states: stop adaptively once the canvas's mean
+# predicted entropy falls below a threshold AND the most likely token at every
+# position is the one predicted at the previous step; otherwise accept tokens
+# in order of low entropy and reset the rest to uniformly random tokens; the
+# temperature falls linearly from 0.8 to 0.4; at most 48 steps.  It does not
+# say how many tokens a step accepts; the sampler is called
+# "entropy-constrained", read here as: the longest run of the lowest-entropy
+# positions whose summed entropy stays within a budget gamma (at least one).
+# Sums and comparisons are taken in float32, in the stated order, so that a
+# decision is the same wherever it is taken from the same float32 entropies.
+# ---------------------------------------------------------------------------
+def anneal_temperature(step: int, max_steps: int = 48, t_first: float = 0.8, t_last: float = 0.4) -> float:
+    """Temperature of denoising step `step` (0-based): linear from t_first at
+    the first step to t_last at step max_steps - 1."""
+    if max_steps <= 1:
+        return t_first
+    return t_first + (t_last - t_first) * step / (max_steps - 1)
+
+
+def entropy_accept(entropy: np.ndarray, gamma: float) -> np.ndarray:
+    """Boolean mask of the accepted positions of one canvas: positions taken
+    in ascending (entropy, position) order while the float32 running sum of
+    their entropies stays <= gamma; the first position is always taken."""
+    e = np.asarray(entropy, dtype=np.float32)
+    order = sorted(range(len(e)), key=lambda i: (e[i], i))
+    acc = np.zeros(len(e), dtype=bool)
+    run = np.float32(0.0)
+    g = np.float32(gamma)
+    for rank, i in enumerate(order):
+        run = np.float32(run + e[i])
+        if rank > 0 and not (run <= g):
+            break
+        acc[i] = True
+    return acc
+
+
+def mean_entropy(entropy: np.ndarray) -> np.float32:
+    """Mean of one canvas's entropies: float32 sum in position order, / C."""
+    run = np.float32(0.0)
+    for x in np.asarray(entropy, dtype=np.float32):
+        run = np.float32(run + x)
+    return np.float32(run / np.float32(len(entropy)))
+
+
+def entropy_sample(argmax: np.ndarray, entropy: np.ndarray, prev_argmax, gamma: float, stop_entropy: float,
+                   noise: np.ndarray):
+    """One canvas: returns (tokens, stopped).  stopped when prev_argmax is
+    given (not the first step), the mean entropy is < stop_entropy and the
+    argmax equals prev_argmax everywhere; then every position takes its
+    argmax.  Otherwise the accepted positions take their argmax and the rest
+    the uniform draws `noise`."""
+    argmax = np.asarray(argmax)
+    stopped = (prev_argmax is not None and bool(mean_entropy(entropy) < np.float32(stop_entropy))
+               and bool(np.array_equal(argmax, np.asarray(prev_argmax))))
+    if stopped:
+        return argmax.copy(), True
+    return np.where(entropy_accept(entropy, gamma), argmax, noise), False
 
 
 def tokens_per_forward(total_tokens: int, total_steps: int, n_blocks: int) -> float:
@@ -264,6 +329,8 @@ class StepResult:
     router_logits: list = field(default_factory=list)
     router_margin: list = field(default_factory=list)  # k-th minus (k+1)-th logit
     gap: np.ndarray | None = None                    # top-1 minus top-2 logit (after /T)
+    entropy: np.ndarray | None = None                # softmax entropy per position (nats)
+    stopped: np.ndarray | None = None                # entropy sampler: adaptive stop per sequence
     forced_hidden: list = field(default_factory=list)  # teacher-forced layer outputs, [B, C, d]
     forced_experts: list = field(default_factory=list)  # top-k of given router rows, [B, C, k]
     forced_router_margin: list = field(default_factory=list)  # their k-th minus (k+1)-th logit
@@ -466,5 +533,31 @@ class Oracle:
         return StepResult(canvas_out=rs(out), conf=rs(st["conf"]), argmax=rs(st["argmax"]),
                           lse=rs(st["lse"]), logp=rs(st["logp"]), margin=rs(st["margin"]),
                           hidden=hidden, experts=experts, router_logits=rlog,
-                          router_margin=rmar, gap=rs(st["gap"]), forced_hidden=forced,
+                          router_margin=rmar, gap=rs(st["gap"]), entropy=rs(st["entropy"]),
+                          forced_hidden=forced,
                           forced_experts=f_exp, forced_router_margin=f_mar, forced_lm=f_lm)
+
+
+def _entropy_step(self, canvas, step: int, seed: int, temperature: float, gamma: float, stop_entropy: float,
+                  prev_argmax=None, record: bool = True, teacher: dict | None = None) -> StepResult:
+    """One denoising step with the entropy-constrained sampler (codemajin.net
+    section 3.3): the forward pass at this step's temperature, then per
+    sequence the adaptive stop test against prev_argmax [B, C] (None at the
+    first step of a block) or the entropy-ordered acceptance; re-noised
+    positions take the same Philox draws as the threshold sampler."""
+    r = self.denoise_step(canvas, step, seed, np.inf, temperature=temperature, record=record, teacher=teacher)
+    B, C = r.argmax.shape
+    noise = renoise_tokens(np.tile(np.arange(self.P, self.P + C), B), step, np.repeat(self.seq_ids[:B], C),
+                           seed, self.s.vocab).reshape(B, C)
+    out = np.empty_like(r.argmax)
+    stopped = np.zeros(B, dtype=bool)
+    for b in range(B):
+        prev = None if prev_argmax is None else np.asarray(prev_argmax)[b]
+        out[b], stopped[b] = entropy_sample(r.argmax[b], r.entropy[b].astype(np.float32), prev, gamma,
+                                            stop_entropy, noise[b])
+    r.canvas_out = out
+    r.stopped = stopped
+    return r
+
+
+Oracle.denoise_step_entropy = _entropy_step

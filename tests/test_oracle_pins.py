@@ -336,3 +336,79 @@ def test_synth_slices_and_moments():
     assert abs(wo.std().item() - 0.02 / 2) < 5e-4      # 1/sqrt(2*layers) on the tiny model
     t = si.uniform_tokens(w, "canvas", 1, 256)
     assert t.dtype == torch.int32 and int(t.min()) >= 0 and int(t.max()) < 8192
+
+
+# --- entropy-constrained sampler (codemajin.net section 3.3) -----------------
+def test_lm_head_entropy_matches_scipy():
+    from scipy.special import softmax
+    from scipy.stats import entropy
+    z = rng.standard_normal((6, 8))
+    E = rng.standard_normal((41, 8))
+    st = om.lm_head_stats(z, E, 0.6, row_chunk=4, vocab_chunk=16)
+    ref = entropy(softmax(z @ E.T / 0.6, axis=1), axis=1)
+    np.testing.assert_allclose(st["entropy"], ref, rtol=1e-12, atol=1e-14)
+    # a one-hot distribution has zero entropy, a uniform one ln V
+    st2 = om.lm_head_stats(np.zeros((1, 8)), E, 1.0)
+    assert abs(st2["entropy"][0] - math.log(41)) < 1e-12
+
+
+def test_entropy_accept_is_the_longest_low_entropy_prefix_within_budget():
+    r2 = np.random.default_rng(7)
+    for trial in range(300):
+        n = int(r2.integers(1, 12))
+        e = r2.choice([0.1, 0.25, 0.5, 1.0, 2.0], size=n).astype(np.float32)  # many exact ties
+        gamma = float(r2.choice([0.0, 0.3, 0.75, 1.5, 100.0]))
+        acc = om.entropy_accept(e, gamma)
+        # brute force over the (entropy, position) order
+        order = sorted(range(n), key=lambda i: (float(e[i]), i))
+        k = 1
+        while k < n and float(np.sum(e[order[:k + 1]], dtype=np.float64)) <= gamma + 1e-6:
+            k += 1
+        expect = np.zeros(n, dtype=bool)
+        expect[order[:k]] = True
+        np.testing.assert_array_equal(acc, expect)
+    assert om.entropy_accept(np.array([3.0, 1.0, 1.0], np.float32), 0.0).tolist() == [False, True, False]
+    assert om.entropy_accept(np.array([3.0, 1.0, 1.0], np.float32), 1e9).all()
+
+
+def test_entropy_sample_stop_rule():
+    a = np.array([5, 6, 7, 8])
+    noise = np.array([100, 101, 102, 103])
+    low = np.full(4, 0.01, np.float32)
+    # first step of a block: no previous prediction, never stops
+    out, stop = om.entropy_sample(a, low, None, 0.0, 1.0, noise)
+    assert not stop and out.tolist() == [5, 101, 102, 103]
+    # mean entropy below the threshold and argmax unchanged: stop, keep every argmax
+    out, stop = om.entropy_sample(a, low, a.copy(), 0.0, 1.0, noise)
+    assert stop and out.tolist() == [5, 6, 7, 8]
+    # one argmax changed: no stop
+    out, stop = om.entropy_sample(a, low, np.array([5, 6, 7, 9]), 0.0, 1.0, noise)
+    assert not stop
+    # mean entropy at the threshold: no stop (strictly below is required)
+    out, stop = om.entropy_sample(a, np.full(4, 0.5, np.float32), a.copy(), 1.0, 0.5, noise)
+    assert not stop and out.tolist() == [5, 6, 102, 103]
+
+
+def test_anneal_temperature_linear_08_to_04():
+    assert om.anneal_temperature(0, 48) == 0.8
+    assert abs(om.anneal_temperature(47, 48) - 0.4) < 1e-15
+    assert abs(om.anneal_temperature(23.5, 48) - 0.6) < 1e-15
+    ts = [om.anneal_temperature(s, 48) for s in range(48)]
+    assert all(b < a for a, b in zip(ts, ts[1:]))
+
+
+def test_entropy_step_reuses_forward_and_noise():
+    """The entropy step is the threshold step's forward pass plus another
+    sampler: same argmax and entropies, re-noised positions take the same
+    Philox draws."""
+    w = _tiny(prefix=16)
+    o = oracle.for_workload(w)
+    o.prefill(si.uniform_tokens(w, "prefix", 1, 16).numpy())
+    cv = si.uniform_tokens(w, "canvas", 1, 256).numpy()
+    r1 = o.denoise_step(cv, 3, 11, 2.0, temperature=0.7)          # tau > 1: every position re-noised
+    r2 = o.denoise_step_entropy(cv, 3, 11, 0.7, 0.5, 0.1)
+    np.testing.assert_array_equal(r1.argmax, r2.argmax)
+    acc = om.entropy_accept(r2.entropy[0].astype(np.float32), 0.5)
+    np.testing.assert_array_equal(r2.canvas_out[0][acc], r2.argmax[0][acc])
+    np.testing.assert_array_equal(r2.canvas_out[0][~acc], r1.canvas_out[0][~acc])
+    assert not r2.stopped[0]
