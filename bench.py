@@ -45,6 +45,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=0,
                     help="reduced depth (profiling captures only; not a bench number)")
+    ap.add_argument("--batch-sweep", default="",
+                    help="comma-separated batch sizes: step throughput and roofline bound per batch "
+                         "(one JSON line of its own, not the bench line)")
     return ap.parse_args()
 
 
@@ -187,7 +190,12 @@ class OracleSample:
         self.orc.prefill(si.uniform_tokens(w, "prefix", w.batch, w.prefix).numpy())
         self.canvas = si.uniform_tokens(w, "canvas", w.batch, w.canvas).numpy()
 
-    def run(self, vocab_frac):
+    VOCAB_FRAC = 1.0 / 8          # one sample definition for both the cpu_baseline and the reference arm
+
+    def run(self, vocab_frac=VOCAB_FRAC):
+        """Returns (canvas tokens/s of the full step extrapolated from the
+        sample, extrapolated full-step seconds, seconds the sample took,
+        description)."""
         import numpy as np
         from oracle.model import _f64, _index, lm_head_stats, rms_norm
         w, orc = self.w, self.orc
@@ -205,30 +213,36 @@ class OracleSample:
         nv = max(128, int(V * vocab_frac)) // 128 * 128
         t0 = time.perf_counter()
         lm_head_stats(z, orc.embed[:nv], 1.0)
-        t_lm = (time.perf_counter() - t0) * V / nv
+        t_lm_sample = time.perf_counter() - t0
+        t_lm = t_lm_sample * V / nv
         t_step = w.shape.n_layers * t_layer + t_lm
         desc = (f"oracle (fp64 numpy) layer 0 of {w.shape.n_layers} over the {w.batch}x{w.canvas} canvas "
                 f"with the {w.prefix}-token cache ({t_layer:.2f} s, scaled x{w.shape.n_layers}) + LM head "
-                f"over {nv} of {V} vocabulary rows ({t_lm * nv / V:.2f} s, scaled to the full vocabulary)")
-        return w.batch * w.canvas / t_step, t_step, desc
+                f"over {nv} of {V} vocabulary rows ({t_lm_sample:.2f} s, scaled to the full vocabulary); "
+                f"extrapolated full step {t_step:.1f} s")
+        return w.batch * w.canvas / t_step, t_step, t_layer + t_lm_sample, desc
 
 
 def run_reference(args, w):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    vals = []
+    vals, spent = [], []
     desc = ""
     sample = OracleSample(w)
     for i in range(args.warmup + args.steps):
-        v, t, desc = sample.run(vocab_frac=1.0 / 8)
+        v, t, t_sample, desc = sample.run()
         if i >= args.warmup:
             vals.append(t)
+            spent.append(t_sample)
     t = statistics.median(vals)
     value = w.batch * w.canvas / t
     cores = _cores()
+    # each timed step is one bounded sample of the step (ms_per_step: the time
+    # it took); value is the full step's throughput extrapolated from it
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": statistics.median(spent) * 1e3,
+            "extrapolated_ms_per_full_step": t * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": f"{w.name}: {w.description}"},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
@@ -398,7 +412,7 @@ def run_native(args, w):
             "clocks": clk,
         }
         if world == 1 and not args.no_cpu_baseline:
-            v, t, desc = OracleSample(w).run(vocab_frac=1.0 / 4)
+            v, t, _, desc = OracleSample(w).run()
             line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": _cores(), "kind": "oracle",
                                     "sample": desc}
         print(json.dumps(line), flush=True)
@@ -407,13 +421,77 @@ def run_native(args, w):
         dist.destroy_process_group()
 
 
+def run_batch_sweep(args, w):
+    """Where the step turns from HBM-bound to tensor-bound as the batch grows
+    (codemajin.net section 5.4: above about 32 concurrent requests the
+    diffusion step loses its advantage to compute load).  One context sized
+    for the largest batch; per batch B: prefill B sequences, warm up, time
+    `steps` graph-replayed steps with CUDA events, and count the experts hit
+    for the step's algorithmic bytes."""
+    import torch
+
+    import block_discrete_diffusion_denoise_b200 as dgp
+    import synth_inputs as si
+
+    batches = [int(b) for b in args.batch_sweep.split(",") if b]
+    stream = torch.cuda.Stream()
+    torch.cuda.set_stream(stream)
+    weights = si.model_weights(w, "cuda")
+    cfg = dgp.config_from_shape(w.shape, max_batch=max(batches), max_seq=w.prefix + 2 * w.canvas,
+                                canvas=w.canvas)
+    ctx = dgp.Context(cfg, weights, stream=stream.cuda_stream)
+    hbm, tf_burst, tf_sus, src = peaks()
+    rows = []
+    for B in batches:
+        wb = w.with_(batch=B)
+        ctx.prefill(si.uniform_tokens(wb, "prefix", B, w.prefix, device="cuda"))
+        cur = si.uniform_tokens(wb, "canvas", B, w.canvas, device="cuda")
+        nxt = torch.empty_like(cur)
+        conf = torch.empty(B, w.canvas, dtype=torch.float32, device="cuda")
+        ctx.debug_capture(True)
+        ctx.denoise_step(cur, 0, w.sample_seed, w.tau0, nxt, conf)
+        hits = []
+        for l in range(w.shape.n_layers):
+            e = torch.empty(B * w.canvas, w.shape.top_k, dtype=torch.int32, device="cuda")
+            ctx.debug_experts(l, e)
+            ctx.sync()
+            hits.append(int(torch.unique(e).numel()))
+        ctx.debug_capture(False)
+        for s in range(args.warmup):
+            ctx.denoise_step(cur, s, w.sample_seed, w.tau0, nxt, conf)
+            cur, nxt = nxt, cur
+        ctx.sync()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for s in range(args.steps):
+            ctx.denoise_step(cur, s, w.sample_seed, w.tau0, nxt, conf)
+            cur, nxt = nxt, cur
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / args.steps
+        by, fl, _ = step_cost(wb, hits)
+        t_hbm, t_tc = by / (hbm * 1e9) * 1e3, fl / (tf_sus * 1e12) * 1e3
+        rows.append({"batch": B, "ms_per_step": ms, "canvas_tok_s": B * w.canvas / (ms * 1e-3),
+                     "bytes": by, "flops": fl, "t_hbm_ms": t_hbm, "t_tensor_ms": t_tc,
+                     "bound": "hbm" if t_hbm >= t_tc else "tensor", "roofline_frac": max(t_hbm, t_tc) / ms,
+                     "experts_hit_mean": sum(hits) / len(hits)})
+        print(json.dumps(rows[-1]), file=sys.stderr, flush=True)
+    ctx.close()
+    print(json.dumps({"metric": "canvas tokens denoised/s vs batch", "workload": f"{w.name}: {w.description}",
+                      "steps": args.steps, "warmup": args.warmup, "dtype": "bf16",
+                      "peaks": f"{src}: HBM {hbm} GB/s, bf16 {tf_sus} TF/s sustained", "sweep": rows}),
+          flush=True)
+
+
 def main():
     args = parse()
     import synth_inputs as si
     w = si.workload(args.workload)
     if args.layers:
         w = w.with_layers(args.layers)
-    if args.impl == "reference":
+    if args.batch_sweep:
+        run_batch_sweep(args, w)
+    elif args.impl == "reference":
         run_reference(args, w)
     else:
         run_native(args, w)

@@ -18,10 +18,12 @@ STATUS = {0: "DG_OK", 1: "DG_ERR_INVALID_ARG", 2: "DG_ERR_OOM", 3: "DG_ERR_CAPAC
           5: "DG_ERR_DEVICE_TIMEOUT", 6: "DG_ERR_STATE", 7: "DG_ERR_UNSUPPORTED"}
 
 # every function declared in include/dg.h
-EXPORTS = ["dg_create", "dg_destroy", "dg_prefill", "dg_denoise_step", "dg_denoise_step_host",
+EXPORTS = ["dg_create", "dg_destroy", "dg_prefill", "dg_denoise_step", "dg_denoise_step_entropy",
+           "dg_denoise_step_host",
            "dg_commit_block", "dg_sync", "dg_cached_len", "dg_last_error", "dg_debug_capture",
            "dg_debug_hidden", "dg_debug_experts", "dg_debug_norm_rows", "dg_debug_lmhead", "dg_debug_router",
-           "dg_debug_sample", "dg_debug_wait_timeout", "dg_debug_gemm", "dg_debug_profile",
+           "dg_debug_sample", "dg_debug_entropy_sample", "dg_debug_entropy", "dg_debug_wait_timeout",
+           "dg_debug_gemm", "dg_debug_profile",
            "dg_debug_profile_read", "dg_debug_launch_count", "dg_lmhead_argmax_static"]
 
 # kernel classes of dg_debug_profile (DG_PROF_* in dg.h)
@@ -53,6 +55,10 @@ class dg_weights(ctypes.Structure):
                 ("router_bias", ctypes.c_void_p), ("layers", ctypes.POINTER(dg_layer_weights))]
 
 
+class dg_entropy_args(ctypes.Structure):
+    _fields_ = [("temperature", ctypes.c_float), ("gamma", ctypes.c_float), ("stop_entropy", ctypes.c_float)]
+
+
 class DGError(RuntimeError):
     def __init__(self, status: int, msg: str):
         super().__init__(f"{STATUS.get(status, status)}: {msg}")
@@ -77,6 +83,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "dg_prefill": ([P, P, I32, I32], I32),
         "dg_denoise_step": ([P, P, I32, U64, F32, P, P, P], I32),
         "dg_denoise_step_host": ([P, P, I32, U64, F32, P, P, P], I32),
+        "dg_denoise_step_entropy": ([P, P, I32, U64, ctypes.POINTER(dg_entropy_args), P, P, P, P, P], I32),
+        "dg_debug_entropy_sample": ([P, P, P, P, I32, I32, U64, F32, F32, P, P], I32),
+        "dg_debug_entropy": ([P, P], I32),
         "dg_commit_block": ([P, P], I32),
         "dg_sync": ([P], I32),
         "dg_cached_len": ([P], I32),
@@ -160,6 +169,13 @@ class Context:
         self._check(self.lib.dg_denoise_step(self.ctx, _ptr(canvas_in), int(step), int(seed), float(tau),
                                              _ptr(canvas_out), _ptr(conf), _ptr(settled)))
 
+    def denoise_step_entropy(self, canvas_in, step, seed, temperature, gamma, stop_entropy, canvas_out,
+                             prev_argmax=None, argmax_out=None, entropy=None, stopped=None):
+        a = dg_entropy_args(float(temperature), float(gamma), float(stop_entropy))
+        self._check(self.lib.dg_denoise_step_entropy(self.ctx, _ptr(canvas_in), int(step), int(seed), ctypes.byref(a),
+                                                     _ptr(prev_argmax), _ptr(argmax_out), _ptr(canvas_out),
+                                                     _ptr(entropy), _ptr(stopped)))
+
     def denoise_step_host(self, canvas_in, step, seed, tau, canvas_out, conf=None, settled=None):
         """Host-buffer variant: numpy int32/float32 arrays (or pinned CPU tensors)."""
         def hp(a):
@@ -201,6 +217,15 @@ class Context:
     def debug_sample(self, argmax, conf, batch, step, seed, tau, out):
         self._check(self.lib.dg_debug_sample(self.ctx, _ptr(argmax), _ptr(conf), batch, int(step), int(seed),
                                              float(tau), _ptr(out)))
+
+    def debug_entropy_sample(self, argmax, entropy, prev_argmax, batch, step, seed, gamma, stop_entropy, out,
+                             stopped=None):
+        self._check(self.lib.dg_debug_entropy_sample(self.ctx, _ptr(argmax), _ptr(entropy), _ptr(prev_argmax), batch,
+                                                     int(step), int(seed), float(gamma), float(stop_entropy),
+                                                     _ptr(out), _ptr(stopped)))
+
+    def debug_entropy(self, out):
+        self._check(self.lib.dg_debug_entropy(self.ctx, _ptr(out)))
 
     def debug_wait_timeout(self, limit_ns: int):
         self._check(self.lib.dg_debug_wait_timeout(self.ctx, int(limit_ns)))
@@ -265,8 +290,17 @@ def lmhead_argmax_static(z, embed, temperature, argmax=None, lse=None, conf=None
                                        _ptr(argmax), _ptr(lse), _ptr(conf), stream)
 
 
+def anneal_temperature(step: int, max_steps: int = 48, t_first: float = 0.8, t_last: float = 0.4) -> float:
+    """Temperature of step `step` of a block: linear from 0.8 at the first
+    step to 0.4 at step max_steps - 1 (codemajin.net "DiffusionGemma
+    architecture", section 3.3)."""
+    if max_steps <= 1:
+        return t_first
+    return t_first + (t_last - t_first) * step / (max_steps - 1)
+
+
 def generate_blocks(ctx: Context, prefix, init_canvas, n_blocks: int, max_steps: int, tau, seed: int,
-                    commit_last: bool = False, before_step=None, after_step=None) -> dict:
+                    commit_last: bool = False, before_step=None, after_step=None, entropy=None) -> dict:
     """Block-autoregressive generation through the C ABI (codemajin.net
     "DiffusionGemma architecture", section 3.2, block-AR; aibars.net, block
     commit): prefill the prompt causally, then for each block start from
@@ -277,9 +311,14 @@ def generate_blocks(ctx: Context, prefix, init_canvas, n_blocks: int, max_steps:
     with commit_last, matching the K - 1 commit forwards that codemajin.net
     section 5.1 counts in TPF.
 
-    tau is a float or a function of the step index.  before_step(k, s) and
+    tau is a float or a function of the step index.  With entropy =
+    {"gamma": ..., "stop_entropy": ...} the steps use the entropy-constrained
+    sampler instead (dg_denoise_step_entropy) at the temperatures of
+    anneal_temperature(step, max_steps), and a block ends when every sequence
+    reports the adaptive stop (section 3.3).  before_step(k, s) and
     after_step(k, s, canvas_in, canvas_out, conf, settled) are optional hooks
-    (tests use them to record a step).  Host control only: every step of the
+    (tests use them to record a step; with the entropy sampler conf holds the
+    entropies and settled the stop flags).  Host control only: every step of the
     path runs in the library's kernels; the one device-to-host read per step is
     the batch's all-settled flags.
 
@@ -294,12 +333,18 @@ def generate_blocks(ctx: Context, prefix, init_canvas, n_blocks: int, max_steps:
         nxt = torch.empty_like(cur)
         conf = torch.empty(B, C, dtype=torch.float32, device=cur.device)
         settled = torch.empty(B, dtype=torch.int32, device=cur.device)
+        argmax = torch.empty(B, C, dtype=torch.int32, device=cur.device)
         steps, done = 0, False
         for s in range(max_steps):
             if before_step is not None:
                 before_step(k, s)
-            t = tau(s) if callable(tau) else tau
-            ctx.denoise_step(cur, s, seed, t, nxt, conf, settled)
+            if entropy is not None:
+                ctx.denoise_step_entropy(cur, s, seed, anneal_temperature(s, max_steps), entropy["gamma"],
+                                         entropy["stop_entropy"], nxt, prev_argmax=argmax if s > 0 else None,
+                                         argmax_out=argmax, entropy=conf, stopped=settled)
+            else:
+                t = tau(s) if callable(tau) else tau
+                ctx.denoise_step(cur, s, seed, t, nxt, conf, settled)
             if after_step is not None:
                 after_step(k, s, cur, nxt, conf, settled)
             cur, nxt = nxt, cur

@@ -5,34 +5,42 @@
 // fills the KV cache, the bidirectional decoder reads it while updating the
 // whole canvas; aiboss88.com "hybrid attention architecture" names both modes.)
 //
-// One CTA = (sequence, kv head, 128 packed query rows, key chunk).  The G
+// One CTA = (sequence, kv head, 256 packed query rows, key chunk).  The G
 // query heads of a GQA group are packed as consecutive rows (row = i*G + h)
-// so each K/V block feeds all of them; a 4-D TMA box pulls exactly those rows
-// out of the [token][head][D] query layout.  The key chunks of one query block
-// form a thread-block cluster and are merged through distributed shared memory.
+// so each K/V block feeds all of them; the 256 rows are two 128-row query
+// tiles, each pulled by one 4-D TMA box out of the [token][head][D] query
+// layout, and every K/V block is read once for both.  The key chunks of one
+// query block form a thread-block cluster and are merged through distributed
+// shared memory.
 //
-// Warp 0 issues TMA loads (Q once; 64-key K blocks into a 3-deep ring; V blocks
-// into a 2-deep ring).  Warp 1 issues tcgen05.mma: S = Q K^T into one of two
-// TMEM buffers (128 x 64 fp32), and O += P V into TMEM (128 x D fp32; V used as
-// an MN-major operand).  Warps 2..5 and 6..9 are two softmax warpgroups; each
-// owns one S buffer (even / odd S tiles) and one query row per thread.
+// Warp 0 issues TMA loads (both Q tiles once; 64-key K and V blocks into
+// 2-deep rings).  Warp 1 issues tcgen05.mma: S_q = Q_q K^T into tile q's TMEM
+// buffer (128 x 64 fp32) and O_q += P_q V into tile q's TMEM accumulator
+// (128 x D fp32; V used as an MN-major operand).  Warps 2..5 and 6..9 are the
+// softmax warpgroups of tiles 0 and 1, one query row per thread, so every row
+// statistic is thread-local.  While one warpgroup turns its S into P the
+// tensor core works on the other tile.
 //
-// Two passes over the key blocks: pass 1 only finds each row's maximum score;
-// pass 2 recomputes S, forms P = 2^(s*scale - max) (bf16, written to shared
-// memory in the swizzled K-major operand layout) and the row sums.  With the
-// final maximum known up front, O never needs rescaling inside TMEM.
+// Single pass with online softmax: P = 2^(s * scale - m_ref), where m_ref is a
+// per-row reference maximum.  It is raised only when a block's maximum
+// exceeds it by more than RESCALE_LOG2 (then O and the row sum are scaled by
+// 2^(old - new) in TMEM), so P stays below 2^RESCALE_LOG2 and rescaling is
+// rare after the first block.
 #pragma once
 
 #include "common.cuh"
 
 namespace dg {
 
-constexpr int ATC_BQ = 128;        // packed query rows per CTA (MMA M)
+constexpr int ATC_BQ = 128;        // packed query rows per tile (MMA M)
+constexpr int ATC_NQ = 2;          // query tiles per CTA
+constexpr int ATC_ROWS = ATC_BQ * ATC_NQ;
 constexpr int ATC_BK = 64;         // keys per block (MMA N of Q K^T, K of P V)
-constexpr int ATC_KSTAGES = 3;
+constexpr int ATC_KSTAGES = 2;
 constexpr int ATC_VSTAGES = 2;
 constexpr int ATC_THREADS = 320;   // producer warp, MMA warp, two softmax warpgroups
-constexpr int ATC_MAX_CHUNKS = 8;  // key chunks = cluster size (portable limit)
+constexpr int ATC_MAX_CHUNKS = 16; // key chunks = cluster size (above 8 needs the non-portable opt-in)
+constexpr float ATC_RESCALE_LOG2 = 8.f;
 
 struct AttnTcParams {
   CUtensorMap q_map;   // 4-D (D, G, Hkv, tokens) over q [token][Hq][D]; box (64, G, 1, 128/G)
@@ -47,15 +55,19 @@ struct AttnTcParams {
 template <int D>
 struct AtcCfg {
   static constexpr int DK = (D + 63) / 64;             // 64-column boxes along the head dimension
-  static constexpr int Q_BYTES = DK * ATC_BQ * 128;
+  static constexpr int Q_BYTES = DK * ATC_BQ * 128;    // one query tile
   static constexpr int KV_BYTES = DK * ATC_BK * 128;
-  static constexpr int P_BYTES = ATC_BQ * ATC_BK * 2;
-  static constexpr int O_COL = 128;                    // TMEM: S buffers in columns [0, 128), O after them
-  static constexpr int TMEM_COLS = O_COL + D <= 256 ? 256 : 512;
+  static constexpr int P_BYTES = ATC_BQ * ATC_BK * 2;  // one tile's P
+  static constexpr int REGION = ATC_NQ * Q_BYTES + (ATC_KSTAGES + ATC_VSTAGES) * KV_BYTES + ATC_NQ * P_BYTES;
+  static constexpr int S_COL = 0;                      // TMEM: S_q at q * 64, O_q at 128 + q * D
+  static constexpr int O_COL = ATC_NQ * ATC_BK;
+  static constexpr int TMEM_COLS = O_COL + ATC_NQ * D <= 256 ? 256 : 512;
   static constexpr int OS_LD = D + 4;                  // fp32 row stride of the merged-O staging tile
-  static constexpr int TAIL = 4096;                    // barriers, flags, row statistics
-  static constexpr int SMEM = 1024 + Q_BYTES + (ATC_KSTAGES + ATC_VSTAGES) * KV_BYTES + 2 * P_BYTES + TAIL;
-  static_assert(ATC_BQ * OS_LD * 4 <= (ATC_KSTAGES + ATC_VSTAGES) * KV_BYTES, "O staging must fit the K/V ring");
+  static constexpr int ML_BYTES = ATC_ROWS * 8;        // per-row (max, sum), at the end of the region
+  static constexpr int TAIL = 512;                     // barriers, flags
+  static constexpr int SMEM = 1024 + REGION + TAIL;
+  static_assert(ATC_ROWS * OS_LD * 4 <= REGION - ML_BYTES, "merged-O staging must fit below the row statistics");
+  static_assert(O_COL + ATC_NQ * D <= 512, "S and O accumulators must fit TMEM");
   static_assert(D % 16 == 0 && D <= 256, "head_dim must be a multiple of 16, at most 256");
 };
 
@@ -64,37 +76,35 @@ __global__ void __launch_bounds__(ATC_THREADS, 1) attn_tc_kernel(const __grid_co
   using C = AtcCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sQ = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sK = sQ + C::Q_BYTES;
+  uint8_t* sK = sQ + ATC_NQ * C::Q_BYTES;
   uint8_t* sV = sK + ATC_KSTAGES * C::KV_BYTES;
   uint8_t* sP = sV + ATC_VSTAGES * C::KV_BYTES;
-  uint8_t* tail = sP + 2 * C::P_BYTES;
+  uint8_t* tail = sQ + C::REGION;
   uint64_t* bars = reinterpret_cast<uint64_t*>(tail);
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;
   uint64_t* k_empty = k_full + ATC_KSTAGES;
   uint64_t* v_full = k_empty + ATC_KSTAGES;
   uint64_t* v_empty = v_full + ATC_VSTAGES;
-  uint64_t* s_full = v_empty + ATC_VSTAGES;
-  uint64_t* s_empty = s_full + 2;
-  uint64_t* p_full = s_empty + 2;
-  uint64_t* p_empty = p_full + 2;
-  uint64_t* o_full = p_empty + 2;
-  uint64_t* drain = o_full + 1;
+  uint64_t* s_full = v_empty + ATC_VSTAGES;   // [NQ] MMA -> warpgroup q: S_q of the next block ready
+  uint64_t* s_free = s_full + ATC_NQ;         // [NQ] warpgroup q -> MMA: S_q read into registers
+  uint64_t* p_full = s_free + ATC_NQ;         // [NQ] warpgroup q -> MMA: P_q written
+  uint64_t* o_done = p_full + ATC_NQ;         // [NQ] MMA -> warpgroup q: O_q += P_q V complete
+  uint64_t* drain = o_done + ATC_NQ;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tail + 256);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tail + 260);
-  float* red_m = reinterpret_cast<float*>(tail + 512);           // [2][128] per-warpgroup row maxima
-  float* red_l = red_m + 2 * ATC_BQ;                             // [2][128] per-warpgroup row sums
-  float2* ml_s = reinterpret_cast<float2*>(red_l + 2 * ATC_BQ);  // [128] (max, sum) of this chunk
-  float* osm = reinterpret_cast<float*>(sK);                     // [128][OS_LD] scaled O, after all MMAs
+  float2* ml_s = reinterpret_cast<float2*>(sQ + C::REGION - C::ML_BYTES);  // [256] (max, sum), after the mainloop
+  float* osm = reinterpret_cast<float*>(sQ);                             // [256][OS_LD] scaled O, after the mainloop
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.Hq / p.Hkv;
   const int b = blockIdx.y / p.Hkv, kvh = blockIdx.y % p.Hkv;
   const int rows_total = p.n * G;
-  const int row_base = blockIdx.x * ATC_BQ;
+  const int row_base = blockIdx.x * ATC_ROWS;
+  const int nq = rows_total - row_base > ATC_BQ ? 2 : 1;   // query tiles holding live rows
   int kend_cta;
   if (p.causal) {
-    const int i_last = min((row_base + ATC_BQ - 1) / G, p.n - 1);
+    const int i_last = min((row_base + nq * ATC_BQ - 1) / G, p.n - 1);
     kend_cta = p.pos0 + i_last + 1;
   } else {
     kend_cta = p.pos0 + p.n;
@@ -114,13 +124,12 @@ __global__ void __launch_bounds__(ATC_THREADS, 1) attn_tc_kernel(const __grid_co
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&s_full[s], 1);
-      mbar_init(&s_empty[s], 128);
-      mbar_init(&p_full[s], 128);
-      mbar_init(&p_empty[s], 1);
+    for (int q = 0; q < ATC_NQ; ++q) {
+      mbar_init(&s_full[q], 1);
+      mbar_init(&s_free[q], ATC_BQ);
+      mbar_init(&p_full[q], ATC_BQ);
+      mbar_init(&o_done[q], 1);
     }
-    mbar_init(o_full, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -135,11 +144,11 @@ __global__ void __launch_bounds__(ATC_THREADS, 1) attn_tc_kernel(const __grid_co
   const uint32_t tmem_base = *tmem_holder;
 
   // softmax state of this thread's row (warps 2..9)
-  const int wg = (warp - 2) >> 2;                // softmax warpgroup 0 / 1
+  const int wg = (warp - 2) >> 2;                // softmax warpgroup = query tile
   const int quarter = warp & 3;                  // TMEM lanes this warp may access
-  const int rloc = quarter * 32 + lane;          // packed row of the tile = TMEM lane
+  const int rloc = quarter * 32 + lane;          // row of the tile = TMEM lane
   const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
-  const int r = row_base + rloc;
+  const int r = row_base + wg * ATC_BQ + rloc;
   const bool live = r < rows_total;
   float mref = -INFINITY, lsum = 0.f;
   bool ok = true;
@@ -152,41 +161,36 @@ __global__ void __launch_bounds__(ATC_THREADS, 1) attn_tc_kernel(const __grid_co
       tma_prefetch_desc(&p.v_map);
       const uint64_t pol = policy_evict_last();  // K/V blocks are shared by the head's query blocks
       uint32_t k_issued = 0, k_par = 0, v_issued = 0, v_par = 0;
-      mbar_arrive_expect_tx(q_full, C::Q_BYTES);
-      for (int db = 0; db < C::DK; ++db)
-        tma_load_4d(sQ + db * ATC_BQ * 128, &p.q_map, q_full, db * 64, 0, kvh, b * p.n + row_base / G, pol);
-      int uk = 0, uv = 0;
-      for (int pass = 0; pass < 2 && !*abort_flag; ++pass) {
-        for (int j = 0; j < nb; ++j) {
-          const int s = uk % ATC_KSTAGES;
-          const uint32_t ph = (uk / ATC_KSTAGES) & 1;
-          if (!mbar_wait(&k_empty[s], ph ^ 1, p.err)) {
-            *abort_flag = 1;
-            break;
-          }
-          mbar_arrive_expect_tx(&k_full[s], C::KV_BYTES);
-          for (int db = 0; db < C::DK; ++db)
-            tma_load_2d(sK + s * C::KV_BYTES + db * ATC_BK * 128, &p.k_map, &k_full[s], db * 64,
-                        kv_row0 + j * ATC_BK, pol);
-          k_issued |= 1u << s;
-          k_par = (k_par & ~(1u << s)) | (ph << s);
-          ++uk;
-          if (pass == 1) {
-            const int sv = uv % ATC_VSTAGES;
-            const uint32_t phv = (uv / ATC_VSTAGES) & 1;
-            if (!mbar_wait(&v_empty[sv], phv ^ 1, p.err)) {
-              *abort_flag = 1;
-              break;
-            }
-            mbar_arrive_expect_tx(&v_full[sv], C::KV_BYTES);
-            for (int db = 0; db < C::DK; ++db)
-              tma_load_2d(sV + sv * C::KV_BYTES + db * ATC_BK * 128, &p.v_map, &v_full[sv], db * 64,
-                          kv_row0 + j * ATC_BK, pol);
-            v_issued |= 1u << sv;
-            v_par = (v_par & ~(1u << sv)) | (phv << sv);
-            ++uv;
-          }
+      mbar_arrive_expect_tx(q_full, nq * C::Q_BYTES);
+      for (int q = 0; q < nq; ++q)
+        for (int db = 0; db < C::DK; ++db)
+          tma_load_4d(sQ + q * C::Q_BYTES + db * ATC_BQ * 128, &p.q_map, q_full, db * 64, 0, kvh,
+                      b * p.n + (row_base + q * ATC_BQ) / G, pol);
+      for (int j = 0; j < nb && !*abort_flag; ++j) {
+        const int s = j % ATC_KSTAGES;
+        const uint32_t ph = (j / ATC_KSTAGES) & 1;
+        if (!mbar_wait(&k_empty[s], ph ^ 1, p.err)) {
+          *abort_flag = 1;
+          break;
         }
+        mbar_arrive_expect_tx(&k_full[s], C::KV_BYTES);
+        for (int db = 0; db < C::DK; ++db)
+          tma_load_2d(sK + s * C::KV_BYTES + db * ATC_BK * 128, &p.k_map, &k_full[s], db * 64, kv_row0 + j * ATC_BK,
+                      pol);
+        k_issued |= 1u << s;
+        k_par = (k_par & ~(1u << s)) | (ph << s);
+        const int sv = j % ATC_VSTAGES;
+        const uint32_t phv = (j / ATC_VSTAGES) & 1;
+        if (!mbar_wait(&v_empty[sv], phv ^ 1, p.err)) {
+          *abort_flag = 1;
+          break;
+        }
+        mbar_arrive_expect_tx(&v_full[sv], C::KV_BYTES);
+        for (int db = 0; db < C::DK; ++db)
+          tma_load_2d(sV + sv * C::KV_BYTES + db * ATC_BK * 128, &p.v_map, &v_full[sv], db * 64,
+                      kv_row0 + j * ATC_BK, pol);
+        v_issued |= 1u << sv;
+        v_par = (v_par & ~(1u << sv)) | (phv << sv);
       }
       // every copy issued here has landed before its buffer is reused or the CTA exits
       mbar_wait(q_full, 0, p.err);
@@ -202,77 +206,78 @@ __global__ void __launch_bounds__(ATC_THREADS, 1) attn_tc_kernel(const __grid_co
       constexpr uint32_t IDESC_PV = umma_idesc_bf16(ATC_BQ, D) | (1u << 16);    // V is MN-major
       const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK);
       const uint32_t v_addr = smem_u32(sV), p_addr = smem_u32(sP);
-      // S tile u (u < nb: pass 1, block u; u >= nb: pass 2, block u - nb) into TMEM buffer u & 1
-      auto issue_s = [&](int u) -> bool {
-        const int sb = u & 1, ks = u % ATC_KSTAGES;
-        if (!mbar_wait(&s_empty[sb], ((u >> 1) & 1) ^ 1, p.err)) return false;
-        if (!mbar_wait(&k_full[ks], (u / ATC_KSTAGES) & 1, p.err)) return false;
+      // S_q(j) = Q_q K_j^T into tile q's S buffer (freed by the warpgroup for j > 0)
+      auto issue_s = [&](int q, int j) -> bool {
+        if (j > 0 && !mbar_wait(&s_free[q], (j - 1) & 1, p.err)) return false;
         tc_fence_after();
-        const uint32_t kb = k_addr + ks * C::KV_BYTES;
+        const uint32_t kb = k_addr + (j % ATC_KSTAGES) * C::KV_BYTES, qb = q_addr + q * C::Q_BYTES;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t a_at = q_addr + (kk >> 2) * (ATC_BQ * 128) + (kk & 3) * 32;
+          const uint32_t a_at = qb + (kk >> 2) * (ATC_BQ * 128) + (kk & 3) * 32;
           const uint32_t b_at = kb + (kk >> 2) * (ATC_BK * 128) + (kk & 3) * 32;
-          umma_bf16(tmem_base + sb * ATC_BK, umma_desc_sw128(a_at), umma_desc_sw128(b_at), IDESC_S,
+          umma_bf16(tmem_base + C::S_COL + q * ATC_BK, umma_desc_sw128(a_at), umma_desc_sw128(b_at), IDESC_S,
                     kk > 0 ? 1u : 0u);
         }
-        umma_commit(&k_empty[ks]);
-        umma_commit(&s_full[sb]);
+        umma_commit(&s_full[q]);
         return true;
       };
-      // O += P_j V_j (P buffer j & 1, written by the warpgroup that owns S tile nb + j)
-      auto issue_pv = [&](int j) -> bool {
-        const int vs = j % ATC_VSTAGES, pb = j & 1;
-        if (!mbar_wait(&v_full[vs], (j / ATC_VSTAGES) & 1, p.err)) return false;
-        if (!mbar_wait(&p_full[pb], (j >> 1) & 1, p.err)) return false;
+      // O_q += P_q(j) V_j
+      auto issue_pv = [&](int q, int j) -> bool {
+        if (!mbar_wait(&p_full[q], j & 1, p.err)) return false;
         tc_fence_after();
-        const uint32_t vb = v_addr + vs * C::KV_BYTES, pbuf = p_addr + pb * C::P_BYTES;
+        const uint32_t vb = v_addr + (j % ATC_VSTAGES) * C::KV_BYTES, pb = p_addr + q * C::P_BYTES;
 #pragma unroll
         for (int kk = 0; kk < ATC_BK / 16; ++kk)
-          umma_bf16(tmem_base + C::O_COL, umma_desc_sw128(pbuf + kk * 32),
+          umma_bf16(tmem_base + C::O_COL + q * D, umma_desc_sw128(pb + kk * 32),
                     umma_desc_sw128_mn(vb + kk * 2048, ATC_BK * 128), IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(&v_empty[vs]);
-        umma_commit(&p_empty[pb]);
+        umma_commit(&o_done[q]);
         return true;
       };
-      bool mok = mbar_wait(q_full, 0, p.err);
-      tc_fence_after();
-      for (int u = 0; u < nb && mok; ++u) mok = issue_s(u);
-      // pass 2 keeps two S tiles ahead of the P V products: the tile for block
-      // j + 2 reuses the buffer that block j's warpgroup released before it
-      // produced P_j, so issuing it right after P_j V_j never waits
-      if (mok) mok = issue_s(nb);
-      if (mok && nb > 1) mok = issue_s(nb + 1);
+      bool mok = mbar_wait(q_full, 0, p.err) && mbar_wait(&k_full[0], 0, p.err);
+      for (int q = 0; q < nq && mok; ++q) mok = issue_s(q, 0);
+      if (mok) umma_commit(&k_empty[0]);
+      // block j + 1's scores are issued before block j's P V products, so the
+      // tensor core works on one tile while the other tile's warpgroup turns
+      // its scores into probabilities
       for (int j = 0; j < nb && mok; ++j) {
-        mok = issue_pv(j);
-        if (mok && j + 2 < nb) mok = issue_s(nb + j + 2);
+        if (j + 1 < nb) {
+          const int ks = (j + 1) % ATC_KSTAGES;
+          mok = mbar_wait(&k_full[ks], ((j + 1) / ATC_KSTAGES) & 1, p.err);
+          for (int q = 0; q < nq && mok; ++q) mok = issue_s(q, j + 1);
+          if (mok) umma_commit(&k_empty[ks]);
+        }
+        const int vs = j % ATC_VSTAGES;
+        mok = mok && mbar_wait(&v_full[vs], (j / ATC_VSTAGES) & 1, p.err);
+        for (int q = 0; q < nq && mok; ++q) mok = issue_pv(q, j);
+        if (mok) umma_commit(&v_empty[vs]);
         if (*abort_flag) mok = false;
       }
-      if (mok) umma_commit(o_full);
       if (!mok) *abort_flag = 1;
       // every MMA issued has completed before TMEM or its operands are reused
       umma_commit(drain);
       mbar_wait(drain, 0, p.err);
     }
-  } else {
-    // ----------------------- softmax warpgroups (warps 2..9) -----------------------
+  } else if (wg < nq && nb > 0) {
+    // ----------------------- softmax warpgroup of tile wg -----------------------
     const int i = live ? r / G : 0;
     // keys of this chunk the row sees: [0, lim) relative to kbeg
     const int lim = (live ? min(p.causal ? p.pos0 + i + 1 : p.pos0 + p.n, kend) : 0) - kbeg;
+    const uint32_t s_col = t_row + C::S_COL + wg * ATC_BK;
+    const uint32_t o_col = t_row + C::O_COL + wg * D;
+    uint8_t* pdst = sP + wg * C::P_BYTES + rloc * 128;
     float s[64];
-    // pass 1: row maximum of the raw scores over this warpgroup's S tiles
-    float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-    for (int u = wg; u < nb && ok; u += 2) {
+    for (int j = 0; j < nb && ok; ++j) {
       // warp-uniform decision: tcgen05.ld below is a warp-collective
-      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[wg], (u >> 1) & 1, p.err) && !*abort_flag)) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[wg], j & 1, p.err) && !*abort_flag)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      tmem_ld64(t_row + wg * ATC_BK, s);
+      tmem_ld64(s_col, s);
       tc_fence_before();
-      mbar_arrive(&s_empty[wg]);
-      const int lj = lim - u * ATC_BK;
+      mbar_arrive(&s_free[wg]);
+      const int lj = lim - j * ATC_BK;
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
       if (lj >= ATC_BK) {
 #pragma unroll
         for (int c = 0; c < ATC_BK; ++c) mx[c & 3] = fmaxf(mx[c & 3], s[c]);
@@ -281,24 +286,13 @@ __global__ void __launch_bounds__(ATC_THREADS, 1) attn_tc_kernel(const __grid_co
         for (int c = 0; c < ATC_BK; ++c)
           if (c < lj) mx[c & 3] = fmaxf(mx[c & 3], s[c]);
       }
-    }
-    red_m[wg * ATC_BQ + rloc] = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-    named_bar_sync(1, 256);
-    // scale > 0, so the maximum of the scaled scores is the scaled maximum
-    mref = fmaxf(red_m[rloc], red_m[ATC_BQ + rloc]) * p.scale_log2;
-    // pass 2: P = 2^(s * scale - max) in bf16 to shared memory, row sums
-    float l = 0.f;
-    for (int j = (wg + nb) & 1; j < nb && ok; j += 2) {
-      const int u = nb + j, pb = j & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[wg], (u >> 1) & 1, p.err) && !*abort_flag)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      tmem_ld64(t_row + wg * ATC_BK, s);
-      tc_fence_before();
-      mbar_arrive(&s_empty[wg]);
-      const int lj = lim - j * ATC_BK;
+      // scale > 0, so the maximum of the scaled scores is the scaled maximum
+      const float mblk = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * p.scale_log2;
+      const bool resc = mblk > mref + ATC_RESCALE_LOG2;          // false while nothing is visible
+      const float factor = resc ? ex2_approx(mref - mblk) : 1.f;  // 0 when mref = -inf
+      if (resc) mref = mblk;
+      lsum *= factor;
+      float l = 0.f;
       uint32_t pk[ATC_BK / 2];
 #pragma unroll
       for (int c = 0; c < ATC_BK / 2; ++c) {
@@ -307,29 +301,40 @@ __global__ void __launch_bounds__(ATC_THREADS, 1) attn_tc_kernel(const __grid_co
         l += p0 + p1;
         pk[c] = pack_bf16x2(p0, p1);
       }
-      if (!__all_sync(0xffffffffu, mbar_wait(&p_empty[pb], ((j >> 1) & 1) ^ 1, p.err))) {
-        ok = false;
-        break;
+      lsum += l;
+      if (j > 0) {
+        // O_q += P_q(j-1) V_{j-1} has completed: O_q is stable and P_q's buffer free
+        if (!__all_sync(0xffffffffu, mbar_wait(&o_done[wg], (j - 1) & 1, p.err))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, resc)) {
+#pragma unroll 1
+          for (int c0 = 0; c0 < D; c0 += 16) {
+            float v[16];
+            tmem_ld16(o_col + c0, v);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[e] *= factor;
+            tmem_st16(o_col + c0, v);
+          }
+          tmem_st_wait();
+        }
       }
       // row rloc of a K-major 128-byte-swizzled tile: 16-byte chunk c lands at c ^ (row & 7)
-      uint8_t* dst = sP + pb * C::P_BYTES + rloc * 128;
 #pragma unroll
       for (int ch = 0; ch < 8; ++ch)
-        *reinterpret_cast<uint4*>(dst + ((ch ^ (rloc & 7)) << 4)) =
+        *reinterpret_cast<uint4*>(pdst + ((ch ^ (rloc & 7)) << 4)) =
             make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
       fence_proxy_async_smem();
-      mbar_arrive(&p_full[pb]);
+      tc_fence_before();
+      mbar_arrive(&p_full[wg]);
     }
-    red_l[wg * ATC_BQ + rloc] = l;
-    if (!ok) *abort_flag = 1;
-    named_bar_sync(1, 256);
-    lsum = red_l[rloc] + red_l[ATC_BQ + rloc];
-    if (nb > 0 && ok) {
-      ok = __all_sync(0xffffffffu, mbar_wait(o_full, 0, p.err) && !*abort_flag);
+    if (ok) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&o_done[wg], (nb - 1) & 1, p.err) && !*abort_flag);
       tc_fence_after();
     }
-    if (nb == 0) mref = -INFINITY;
-    if (wg == 0) ml_s[rloc] = make_float2(mref, lsum);
+    if (!ok) *abort_flag = 1;
   }
 
   // ---------- merge the key chunks of this query block (one cluster) ----------
@@ -337,9 +342,19 @@ __global__ void __launch_bounds__(ATC_THREADS, 1) attn_tc_kernel(const __grid_co
   // scales its own rows into shared memory, then every chunk sums a slice of
   // the rows over all chunks' tiles (distributed shared memory) and stores it.
   const int nc = p.n_chunks;
+  if (warp >= 2) {
+    named_bar_sync(1, 256);  // both tiles' MMAs are complete: the operand region may be reused
+    const bool have = wg < nq && nb > 0 && ok;
+    if (!have) {
+      mref = -INFINITY;
+      lsum = 0.f;
+    }
+    ml_s[wg * ATC_BQ + rloc] = make_float2(mref, lsum);
+  }
   cluster_sync_all();  // every chunk's (max, sum) is visible
   if (warp >= 2) {
-    const uint32_t ml_at = smem_u32(&ml_s[rloc]);
+    const int row = wg * ATC_BQ + rloc;
+    const uint32_t ml_at = smem_u32(&ml_s[row]);
     float M = -INFINITY;
     for (int q = 0; q < nc; ++q) M = fmaxf(M, ld_dsmem_f2(mapa_shared(ml_at, q)).x);
     const float Mref = M == -INFINITY ? 0.f : M;
@@ -349,17 +364,17 @@ __global__ void __launch_bounds__(ATC_THREADS, 1) attn_tc_kernel(const __grid_co
       den += v.y * ex2_approx(v.x - Mref);
     }
     const float w = (den > 0.f && mref != -INFINITY) ? ex2_approx(mref - Mref) / den : 0.f;
-    const bool have_o = nb > 0 && ok;  // warp-uniform
-#pragma unroll
-    for (int k = wg; k < D / 16; k += 2) {
+    const bool have_o = wg < nq && nb > 0 && __all_sync(0xffffffffu, ok);  // warp-uniform
+#pragma unroll 1
+    for (int c0 = 0; c0 < D; c0 += 16) {
       float v[16];
       if (have_o) {
-        tmem_ld16(t_row + C::O_COL + k * 16, v);
+        tmem_ld16(t_row + C::O_COL + wg * D + c0, v);
       } else {
 #pragma unroll
         for (int e = 0; e < 16; ++e) v[e] = 0.f;
       }
-      float4* dst = reinterpret_cast<float4*>(osm + rloc * C::OS_LD + k * 16);
+      float4* dst = reinterpret_cast<float4*>(osm + row * C::OS_LD + c0);
 #pragma unroll
       for (int e = 0; e < 4; ++e) dst[e] = make_float4(v[4 * e] * w, v[4 * e + 1] * w, v[4 * e + 2] * w, v[4 * e + 3] * w);
     }
@@ -367,43 +382,35 @@ __global__ void __launch_bounds__(ATC_THREADS, 1) attn_tc_kernel(const __grid_co
   cluster_sync_all();  // every chunk's scaled tile is complete
   if (warp >= 2) {
     const int rank = static_cast<int>(cluster_ctarank());
-    const int rpr = (ATC_BQ + nc - 1) / nc;
-    const int r_lo = rank * rpr, r_hi = min(ATC_BQ, r_lo + rpr);
+    const int rpr = (ATC_ROWS + nc - 1) / nc;
+    const int r_lo = rank * rpr, r_hi = min(ATC_ROWS, r_lo + rpr);
     constexpr int D4 = D / 4;
     const uint32_t os_at = smem_u32(osm);
-    // two items per pass, all their peer loads issued before any is used
-    const int n_items = (r_hi - r_lo) * D4;
-    for (int it0 = threadIdx.x - 64; it0 < n_items; it0 += 512) {
-      float4 acc[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
-      float4 v[2][ATC_MAX_CHUNKS];
+    const int n_items = max(0, r_hi - r_lo) * D4;
+    for (int it = threadIdx.x - 64; it < n_items; it += 256) {
+      const int rr = r_lo + it / D4, c4 = (it % D4) * 4;
+      const uint32_t off = static_cast<uint32_t>((rr * C::OS_LD + c4) * 4);
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      // peers in groups of eight, all loads of a group issued before any is used
+      for (int q0 = 0; q0 < nc; q0 += 8) {
+        float4 v[8];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int it = it0 + 256 * h;
-        const int rr = r_lo + it / D4, c4 = (it % D4) * 4;
-        const uint32_t off = static_cast<uint32_t>((rr * C::OS_LD + c4) * 4);
+        for (int u = 0; u < 8; ++u)
+          if (q0 + u < nc) v[u] = ld_dsmem_f4(mapa_shared(os_at + off, q0 + u));
 #pragma unroll
-        for (int q = 0; q < ATC_MAX_CHUNKS; ++q)
-          if (q < nc && it < n_items) v[h][q] = ld_dsmem_f4(mapa_shared(os_at + off, q));
-      }
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int it = it0 + 256 * h;
-        if (it >= n_items) continue;
-#pragma unroll
-        for (int q = 0; q < ATC_MAX_CHUNKS; ++q)
-          if (q < nc) {
-            acc[h].x += v[h][q].x;
-            acc[h].y += v[h][q].y;
-            acc[h].z += v[h][q].z;
-            acc[h].w += v[h][q].w;
+        for (int u = 0; u < 8; ++u)
+          if (q0 + u < nc) {
+            acc.x += v[u].x;
+            acc.y += v[u].y;
+            acc.z += v[u].z;
+            acc.w += v[u].w;
           }
-        const int rr = r_lo + it / D4, c4 = (it % D4) * 4;
-        const int rg = row_base + rr;
-        if (rg >= rows_total) continue;
-        const size_t rid = (static_cast<size_t>(b) * p.n + rg / G) * p.Hq + kvh * G + rg % G;
-        *reinterpret_cast<uint2*>(p.o + rid * D + c4) =
-            make_uint2(pack_bf16x2(acc[h].x, acc[h].y), pack_bf16x2(acc[h].z, acc[h].w));
       }
+      const int rg = row_base + rr;
+      if (rg >= rows_total) continue;
+      const size_t rid = (static_cast<size_t>(b) * p.n + rg / G) * p.Hq + kvh * G + rg % G;
+      *reinterpret_cast<uint2*>(p.o + rid * D + c4) =
+          make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
     }
   }
   cluster_sync_all();  // no CTA leaves while a peer may still read its shared memory

@@ -30,6 +30,21 @@ struct LayerMaps {
   CUtensorMap kc, vc;  // this layer's K / V cache rows, 64 x 64 boxes
 };
 
+// the sampler that ends a step
+enum Sampler : int { SAMPLER_TAU = 0, SAMPLER_ENTROPY = 1, SAMPLER_COUNT = 2 };
+
+// Step as one captured CUDA graph; a call rebinds the nodes whose arguments
+// change: the embedding (canvas), the LM head (temperature) and the sampler.
+struct StepGraph {
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t exec = nullptr;
+  int B = -1, P = -1;
+  cudaGraphNode_t embed_node = nullptr, lm_node = nullptr, sample_node = nullptr;
+  cudaKernelNodeParams embed_kp{}, lm_kp{}, sample_kp{};
+  std::vector<void*> embed_args, sample_args;
+  int64_t launches = 0;
+};
+
 }  // namespace
 
 struct dg_ctx {
@@ -57,23 +72,15 @@ struct dg_ctx {
   uint16_t* o = nullptr;
   int32_t* idx = nullptr;
   float* gates = nullptr;
-  int32_t* perm_tok = nullptr;
-  int32_t* inv_slot = nullptr;
-  int4* tiles = nullptr;        // fused expert GEMM tile list (gate/up, then down)
-  int32_t* chunk_done = nullptr;
-  int32_t* route = nullptr;        // routing: expert counts [E], cursors [E], finished CTAs [1]
+  int32_t* inv_slot = nullptr;     // routed row of each (token, slot) pair
+  int32_t* chunk_done = nullptr;   // finished gate/up tiles per expert token chunk
+  int32_t* expert_rows = nullptr;  // [E] rows routed to each expert (dispatch cursors)
+  int32_t* moe_work = nullptr;     // claim / exit counters of the expert GEMM
   int32_t* dense_work = nullptr;   // claim / exit counters of the dense GEMM
   int attn_max_clusters[ATC_MAX_CHUNKS + 1] = {};  // co-resident attention clusters per cluster size
-  // CUDA graph of the denoising step (per batch and cached length)
+  // CUDA graphs of the denoising step, one per sampler (per batch and cached length)
   bool use_graphs = true;
-  cudaGraph_t step_graph = nullptr;
-  cudaGraphExec_t step_exec = nullptr;
-  int graph_B = -1, graph_P = -1;
-  cudaGraphNode_t embed_node = nullptr, sample_node = nullptr;
-  cudaKernelNodeParams embed_kp{}, sample_kp{};
-  std::vector<void*> embed_args, sample_args;
-  int64_t graph_launches = 0;
-  int32_t* counters = nullptr;
+  StepGraph graphs[SAMPLER_COUNT];
   uint16_t* xp = nullptr;
   uint16_t* hbuf = nullptr;
   uint16_t* hsbuf = nullptr;
@@ -85,11 +92,13 @@ struct dg_ctx {
   float* dbg_lse = nullptr;
   float* dbg_conf = nullptr;
   float* dbg_margin = nullptr;
+  float* dbg_entropy = nullptr;
+  float* lm_s1 = nullptr;          // LM-head entropy partials [V/128][R_step]
   int32_t* io_canvas_in = nullptr;
   int32_t* io_canvas_out = nullptr;
   float* io_conf = nullptr;
   int32_t* io_settled = nullptr;
-  size_t max_gu_tiles = 0, max_dn_tiles = 0, max_chunks = 0;
+  size_t max_chunks = 0;
   // capture (test hook)
   bool capture = false;
   float* cap_h = nullptr;
@@ -105,6 +114,7 @@ struct dg_ctx {
   int P = 0;
   bool prefilled = false;
   uint64_t wait_limit_ns = 1000000000ull;
+  bool trace = false;          // DG_TRACE=1: launch shapes to stderr
   int64_t launches = 0;
   std::string last_error;
   // profiling hook: event pairs per kernel class
@@ -256,7 +266,9 @@ dg_status gemm_dense(dg_ctx* c, const CUtensorMap& w, const CUtensorMap& x, int 
     if (wi > 0 && bnc >= widths[0]) continue;
     const int nt = (T + bnc - 1) / bnc;
     for (int sp = 1; sp <= 8; ++sp) {
-      if (p.k_steps / sp < 4 || static_cast<size_t>(sp) > std::min<size_t>(cap_s, max_splits)) break;
+      if (p.k_steps / sp < 4 || static_cast<size_t>(sp) > std::min<size_t>({cap_s, static_cast<size_t>(max_splits),
+                                                                             static_cast<size_t>(ROW_MAX_SPLITS)}))
+        break;
       const int ctas = m_tiles * nt * sp;
       const double rounds = std::ceil(static_cast<double>(ctas) / c->sms);
       const double per_cta = 2.3 + (static_cast<double>(p.k_steps) / sp) * (0.12 + 0.28 * bnc / 256.0) +
@@ -317,7 +329,11 @@ cudaError_t attention_cluster_limits(dg_ctx* c) {
     cfg.numAttrs = 1;
     int num = 0;
     cudaError_t e = cudaOccupancyMaxActiveClusters(&num, attn_tc_kernel<D>, &cfg);
-    if (e != cudaSuccess) return e;
+    if (e != cudaSuccess) {
+      if (nc <= 8) return e;
+      cudaGetLastError();  // a non-portable size this device does not offer: not used
+      num = 0;
+    }
     c->attn_max_clusters[nc] = num;
   }
   return cudaSuccess;
@@ -339,21 +355,28 @@ dg_status attention(dg_ctx* c, int l, int B, int n, int pos0, bool causal) {
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c->D)));
   p.err = dev_err(c);
   const int G = c->Hq / c->Hkv;
-  const int qblocks = (n * G + ATC_BQ - 1) / ATC_BQ;
-  const int clusters = qblocks * B * c->Hkv;
+  const int qblocks = (n * G + ATC_ROWS - 1) / ATC_ROWS;
+  const int units = qblocks * B * c->Hkv;
   const int keys = pos0 + n;
-  // Split the keys into the largest cluster of chunks (at least 256 keys
-  // each) for which every cluster is resident at once; one chunk otherwise.
-  int n_chunks = 1;
-  for (int nc = std::min(ATC_MAX_CHUNKS, std::max(1, keys / 256)); nc > 1; --nc)
-    if (clusters <= c->attn_max_clusters[nc]) {
+  // Split the keys into the cluster of chunks that gives each CTA the fewest
+  // 64-key blocks while every cluster is resident at once (fewer chunks on
+  // ties: each chunk adds a merge share); one chunk when nothing fits.
+  int n_chunks = 1, best_blocks = (keys + ATC_BK - 1) / ATC_BK;
+  for (int nc = 2; nc <= ATC_MAX_CHUNKS; ++nc) {
+    if (units > c->attn_max_clusters[nc] || keys < nc * ATC_BK) continue;
+    const int blocks = ((keys + nc - 1) / nc + ATC_BK - 1) / ATC_BK;
+    if (blocks < best_blocks) {
+      best_blocks = blocks;
       n_chunks = nc;
-      break;
     }
-  const int chunk_len = ((keys + n_chunks - 1) / n_chunks + ATC_BK - 1) / ATC_BK * ATC_BK;
+  }
+  const int chunk_len = best_blocks * ATC_BK;
   n_chunks = (keys + chunk_len - 1) / chunk_len;
   p.chunk_len = chunk_len;
   p.n_chunks = n_chunks;
+  if (c->trace && l == 0)
+    fprintf(stderr, "[dg] attention: keys %d, units %d, chunks %d x %d keys (resident clusters of that size %d)\n",
+            keys, units, n_chunks, chunk_len, c->attn_max_clusters[n_chunks]);
   const dim3 grid(qblocks, B * c->Hkv, n_chunks);
   ProfScope ps1(c, DG_PROF_ATTENTION);
   cudaError_t e;
@@ -376,27 +399,22 @@ dg_status attention(dg_ctx* c, int l, int B, int n, int pos0, bool causal) {
   return DG_OK;
 }
 
-dg_status moe(dg_ctx* c, int l, int T) {
+// record: capture the expert choices (denoising steps only: the capture
+// buffers hold R_step rows per layer)
+dg_status moe(dg_ctx* c, int l, int T, bool record) {
   const LayerMaps& lm = c->lmaps[l];
-  const dg_layer_weights& lw = c->layers[l];
   int s3 = 1;
   dg_status st = gemm_dense(c, lm.wr, c->m_u64, c->E, T, c->d, &s3);
   if (st != DG_OK) return st;
-  int32_t* cap = c->capture ? c->cap_idx + static_cast<size_t>(l) * c->R_step * c->k : nullptr;
-  // routing: top-k with expert counts (8 rows per CTA), then the permutation
-  // by expert, the row gather and the expert tile list (rows spread over up
-  // to 2 CTAs per SM)
-  const int pg_ctas = std::min(T, 2 * c->sms);
-  const int pg_rows = (T + pg_ctas - 1) / pg_ctas;
+  int32_t* cap = (record && c->capture) ? c->cap_idx + static_cast<size_t>(l) * c->R_step * c->k : nullptr;
+  // routing: the top-k decision of every token with the claim of its rows in
+  // the experts' regions and the copy of its activations (one warp per token)
   ProfScope ps3(c, DG_PROF_ROUTING);
-  DG_LAUNCH(c, router_topk_kernel, (T + 7) / 8, 256, 0, static_cast<const float*>(c->part), s3, T, c->E, c->k,
-            c->router_bias, c->idx, c->gates, cap, 8, c->route);
-  DG_LAUNCH(c, permute_gather_kernel, (T + pg_rows - 1) / pg_rows, 256, 0, static_cast<const int32_t*>(c->idx),
-            c->route, pg_rows, T, c->k, c->E, c->F, c->Fs, c->d, static_cast<const uint16_t*>(c->u), c->perm_tok,
-            c->inv_slot, c->xp, c->tiles, c->chunk_done, c->counters, MOE_CHUNK_ROWS);
+  // expert e's rows: [e * T, e * T + rows_e) (a region per expert, T rows each)
+  DG_LAUNCH(c, route_dispatch_kernel, (T + 7) / 8, 256, 0, static_cast<const float*>(c->part), s3, T, c->E, c->k,
+            c->router_bias, c->idx, c->gates, cap, c->expert_rows, T, c->d, static_cast<const uint16_t*>(c->u),
+            c->xp, c->inv_slot);
   ps3.end();
-  const int rows = T * c->k;
-  (void)lw;
 
   // routed + shared experts, gate/up then down, one persistent launch
   GemmParams p;
@@ -417,9 +435,10 @@ dg_status moe(dg_ctx* c, int l, int T) {
   p.hs_mid_map = c->m_hs64;
   p.b_mid_rows = 64;
   p.b_box_rows = 16;
-  p.counts = c->counters;
-  p.tiles = c->tiles;
-  p.work = c->counters + 3;
+  p.T = T;
+  p.expert_rows = c->expert_rows;
+  p.region = T;
+  p.work = c->moe_work;
   p.chunk_done = c->chunk_done;
   p.n_groups_routed = c->E;
   p.F = c->F;
@@ -429,7 +448,7 @@ dg_status moe(dg_ctx* c, int l, int T) {
   p.hs_out = c->hsbuf;
   p.out_f32 = c->yp;
   p.out_ld = c->d;
-  p.shared_row_base = rows;
+  p.shared_row_base = c->E * T;
   p.err = dev_err(c);
   ProfScope ps6(c, DG_PROF_EXPERTS);
   DG_LAUNCH(c, gemm_kernel<GEMM_MOE>, c->sms, GEMM_THREADS, gemm_smem_bytes<GEMM_MOE>(), p);
@@ -448,7 +467,7 @@ dg_status forward(dg_ctx* c, const int32_t* tokens, int tok_stride, int tok_off,
   const float eps = c->cfg.rms_eps;
   float* cap0 = (c->capture && !causal) ? c->cap_h : nullptr;
   ProfScope ps8(c, DG_PROF_OTHER);
-  DG_LAUNCH(c, embed_norm_kernel, T, 256, 0, tokens, tok_stride, tok_off, n, c->embed,
+  DG_LAUNCH(c, embed_norm_kernel, T, row_threads(c->d), 0, tokens, tok_stride, tok_off, n, c->embed,
             static_cast<const uint16_t*>(c->layers[0].attn_norm), eps, c->d, c->h, c->u, cap0, settled, B, c->V);
   ps8.end();
   for (int l = 0; l < c->L; ++l) {
@@ -459,7 +478,11 @@ dg_status forward(dg_ctx* c, const int32_t* tokens, int tok_stride, int tok_off,
     if (st != DG_OK) return st;
     const size_t layer_off = static_cast<size_t>(l) * c->cfg.max_batch * c->Hkv * c->cfg.max_seq * c->D;
     ProfScope ps9(c, DG_PROF_OTHER);
-    DG_LAUNCH(c, rope_qkv_kernel, T, 256, 0, static_cast<const float*>(c->part), s1, T, n, pos0, c->Hq, c->Hkv,
+    DG_LAUNCH(c, rope_qkv_kernel, dim3(T, ROPE_CTAS_PER_ROW),
+              std::min(ROPE_MAX_THREADS,
+                       (rope_items(c->Hq, c->Hkv, c->D) + ROPE_CTAS_PER_ROW * 32 - 1) / (ROPE_CTAS_PER_ROW * 32) * 32),
+              0,
+              static_cast<const float*>(c->part), s1, T, n, pos0, c->Hq, c->Hkv,
               c->D, static_cast<const float2*>(c->rope), c->q, c->kcache + layer_off, c->vcache + layer_off,
               c->cfg.max_seq);
     ps9.end();
@@ -470,21 +493,21 @@ dg_status forward(dg_ctx* c, const int32_t* tokens, int tok_stride, int tok_off,
     st = gemm_dense(c, lm.wo, c->m_o64, c->d, T, c->HD, &s2);
     if (st != DG_OK) return st;
     ProfScope ps10(c, DG_PROF_OTHER);
-    DG_LAUNCH(c, residual_norm_kernel, T, 256, 0, c->h, static_cast<const float*>(c->part), s2, T, c->d,
+    DG_LAUNCH(c, residual_norm_kernel, T, row_threads(c->d), 0, c->h, static_cast<const float*>(c->part), s2, T, c->d,
               static_cast<const uint16_t*>(lw.ffn_norm), eps, c->u);
     ps10.end();
     if (c->capture && !causal)
       DG_CUDA(c, cudaMemcpyAsync(c->cap_u + static_cast<size_t>(l) * c->R_step * c->d, c->u,
                                  static_cast<size_t>(T) * c->d * 2, cudaMemcpyDeviceToDevice, c->stream));
-    st = moe(c, l, T);
+    st = moe(c, l, T, !causal);
     if (st != DG_OK) return st;
     const uint16_t* next_gain = l + 1 < c->L ? static_cast<const uint16_t*>(c->layers[l + 1].attn_norm)
                                              : c->final_norm;
     float* cap = (c->capture && !causal) ? c->cap_h + static_cast<size_t>(l + 1) * c->R_step * c->d : nullptr;
     ProfScope ps11(c, DG_PROF_OTHER);
-    DG_LAUNCH(c, combine_norm_kernel, T, 256, 0, c->h, static_cast<const float*>(c->yp),
-              static_cast<const int32_t*>(c->inv_slot), static_cast<const float*>(c->gates), c->k, T * c->k, c->d,
-              next_gain, eps, c->u, cap);
+    DG_LAUNCH(c, combine_norm_kernel, T, row_threads(c->d), 0, c->h, static_cast<const float*>(c->yp),
+              static_cast<const int32_t*>(c->inv_slot), static_cast<const float*>(c->gates), c->k, c->E * T,
+              c->d, next_gain, eps, c->u, cap);
     ps11.end();
     if (c->capture && !causal && l == c->L - 1)
       DG_CUDA(c, cudaMemcpyAsync(c->cap_u + static_cast<size_t>(c->L) * c->R_step * c->d, c->u,
@@ -493,9 +516,9 @@ dg_status forward(dg_ctx* c, const int32_t* tokens, int tok_stride, int tok_off,
   return DG_OK;
 }
 
-dg_status lm_head_and_sample(dg_ctx* c, int B, int step, uint64_t seed, float tau, int32_t* canvas_out,
-                             float* conf_out, int32_t* settled) {
-  const int T = B * c->cfg.canvas;
+// LM head over the B*C canvas rows with the per-(vocabulary tile, row)
+// statistics, at the given temperature
+dg_status lm_head(dg_ctx* c, int T, float temperature) {
   GemmParams p;
   memset(&p, 0, sizeof(p));
   p.a_map[0] = c->m_u128;
@@ -504,34 +527,98 @@ dg_status lm_head_and_sample(dg_ctx* c, int B, int step, uint64_t seed, float ta
   p.M = T;
   p.k_steps = c->d / 64;
   p.n_mtiles = (T + GEMM_BM - 1) / GEMM_BM;
-  const int n_vtiles = c->V / GEMM_BN;
-  p.tiles_static = n_vtiles * p.n_mtiles;
+  p.tiles_static = (c->V / GEMM_BN) * p.n_mtiles;
   p.lm_part = c->lm_part;
-  p.logit_scale_log2 = static_cast<float>(1.4426950408889634 / static_cast<double>(c->cfg.temperature));
+  p.lm_s1 = c->lm_s1;
+  p.logit_scale_log2 = static_cast<float>(1.4426950408889634 / static_cast<double>(temperature));
   p.err = dev_err(c);
   ProfScope ps12(c, DG_PROF_LMHEAD);
   DG_LAUNCH(c, gemm_kernel<GEMM_LMHEAD>, std::min(c->sms, p.tiles_static), GEMM_THREADS,
             gemm_smem_bytes<GEMM_LMHEAD>(), p);
   ps12.end();
+  return DG_OK;
+}
+
+SampleArgs merge_args(const dg_ctx* c, int T, bool stats_only) {
   SampleArgs a;
-  a.n_vtiles = n_vtiles;
+  memset(&a, 0, sizeof(a));
+  a.n_vtiles = c->V / GEMM_BN;
   a.T = T;
   a.C = c->cfg.canvas;
   a.P = c->P;
-  a.step = step;
   a.vocab = c->V;
+  a.stats_only = stats_only ? 1 : 0;
+  a.dbg_argmax = c->dbg_argmax;
+  a.dbg_lse = c->dbg_lse;
+  a.dbg_conf = c->dbg_conf;
+  a.dbg_margin = c->dbg_margin;
+  a.dbg_entropy = c->dbg_entropy;
+  a.s1 = c->lm_s1;
+  return a;
+}
+
+// threshold sampler: merge of the LM-head statistics + Philox re-noising
+dg_status lm_head_and_sample(dg_ctx* c, int B, int step, uint64_t seed, float tau, int32_t* canvas_out,
+                             float* conf_out, int32_t* settled) {
+  const int T = B * c->cfg.canvas;
+  dg_status st = lm_head(c, T, c->cfg.temperature);
+  if (st != DG_OK) return st;
+  SampleArgs a = merge_args(c, T, false);
+  a.step = step;
   a.seed_lo = static_cast<uint32_t>(seed & 0xFFFFFFFFull);
   a.seed_hi = static_cast<uint32_t>(seed >> 32);
   a.tau = tau;
   a.canvas_out = canvas_out;
   a.conf_out = conf_out;
   a.settled = settled;
-  a.dbg_argmax = c->dbg_argmax;
-  a.dbg_lse = c->dbg_lse;
-  a.dbg_conf = c->dbg_conf;
-  a.dbg_margin = c->dbg_margin;
   ProfScope ps13(c, DG_PROF_OTHER);
   DG_LAUNCH(c, lmhead_merge_sample_kernel, T, 256, 0, static_cast<const float4*>(c->lm_part), a);
+  ps13.end();
+  return DG_OK;
+}
+
+struct EntropyCall {
+  int step;
+  uint64_t seed;
+  dg_entropy_args args;
+  const int32_t* prev_argmax;
+  int32_t* argmax_out;
+  int32_t* canvas_out;
+  float* entropy_out;
+  int32_t* stopped;
+};
+
+EntropyArgs entropy_args(const dg_ctx* c, const EntropyCall& e) {
+  EntropyArgs a;
+  memset(&a, 0, sizeof(a));
+  a.C = c->cfg.canvas;
+  a.P = c->P;
+  a.step = e.step;
+  a.vocab = c->V;
+  a.seed_lo = static_cast<uint32_t>(e.seed & 0xFFFFFFFFull);
+  a.seed_hi = static_cast<uint32_t>(e.seed >> 32);
+  a.gamma = e.args.gamma;
+  a.stop_entropy = e.args.stop_entropy;
+  a.argmax = c->dbg_argmax;
+  a.entropy = c->dbg_entropy;
+  a.prev_argmax = e.prev_argmax;
+  a.argmax_out = e.argmax_out;
+  a.canvas_out = e.canvas_out;
+  a.entropy_out = e.entropy_out;
+  a.stopped = e.stopped;
+  return a;
+}
+
+// entropy-constrained sampler: LM head at this step's temperature, merged
+// statistics, then the per-sequence ordering / budget / stop rule
+dg_status lm_head_and_entropy_sample(dg_ctx* c, int B, const EntropyCall& e) {
+  const int T = B * c->cfg.canvas;
+  dg_status st = lm_head(c, T, e.args.temperature);
+  if (st != DG_OK) return st;
+  SampleArgs a = merge_args(c, T, true);
+  ProfScope ps13(c, DG_PROF_OTHER);
+  DG_LAUNCH(c, lmhead_merge_sample_kernel, T, 256, 0, static_cast<const float4*>(c->lm_part), a);
+  DG_LAUNCH(c, entropy_sample_kernel, B, 256, 0, entropy_args(c, e));
   ps13.end();
   return DG_OK;
 }
@@ -544,6 +631,11 @@ T* carve(char*& cur, size_t count) {
   cur += (count * sizeof(T) + 255) / 256 * 256;
   return p;
 }
+
+// rows of one forward (tokens of a step or of a prefill chunk): the expert
+// GEMM's tile tables count rows and chunks in 16 bits
+constexpr int kMaxRows = 32768;
+static_assert(PERM_MAXE == MOE_MAX_EXPERTS, "routing and expert GEMM agree on the expert limit");
 
 // every kernel's dynamic shared memory fits the 227 KB a CTA may opt into
 constexpr int kMaxSmemPerCta = 232448;
@@ -564,79 +656,120 @@ dg_status set_smem_attrs(dg_ctx* c) {
   DG_CUDA(c, cudaFuncSetAttribute(attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, AtcCfg<64>::SMEM));
   DG_CUDA(c, cudaFuncSetAttribute(attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, AtcCfg<128>::SMEM));
   DG_CUDA(c, cudaFuncSetAttribute(attn_tc_kernel<176>, cudaFuncAttributeMaxDynamicSharedMemorySize, AtcCfg<176>::SMEM));
+  // clusters of up to 16 key chunks (above the portable 8)
+  DG_CUDA(c, cudaFuncSetAttribute(attn_tc_kernel<64>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
+  DG_CUDA(c, cudaFuncSetAttribute(attn_tc_kernel<128>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
+  DG_CUDA(c, cudaFuncSetAttribute(attn_tc_kernel<176>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
   return DG_OK;
 }
 
-void drop_step_graph(dg_ctx* c) {
-  if (c->step_exec) cudaGraphExecDestroy(c->step_exec);
-  if (c->step_graph) cudaGraphDestroy(c->step_graph);
-  c->step_exec = nullptr;
-  c->step_graph = nullptr;
-  c->graph_B = c->graph_P = -1;
+void drop_step_graph(StepGraph& g) {
+  if (g.exec) cudaGraphExecDestroy(g.exec);
+  if (g.graph) cudaGraphDestroy(g.graph);
+  g = StepGraph();
 }
 
-// Capture the whole step (embedding .. sampler) once per (batch, cached
-// length) on the context stream; later calls only rebind the first kernel
-// (canvas, settled flags) and the last one (step, seed, tau, outputs).
-dg_status step_via_graph(dg_ctx* c, const int32_t* canvas_in, int32_t step, uint64_t seed, float tau,
-                         int32_t* canvas_out, float* conf, int32_t* settled) {
-  if (!c->step_exec || c->graph_B != c->B || c->graph_P != c->P) {
-    drop_step_graph(c);
-    const int64_t l0 = c->launches;
-    DG_CUDA(c, cudaStreamBeginCapture(c->stream, cudaStreamCaptureModeThreadLocal));
-    dg_status st = forward(c, c->io_canvas_in, c->cfg.canvas, 0, c->B, c->cfg.canvas, c->P, false, c->io_settled);
-    if (st == DG_OK)
+void drop_step_graphs(dg_ctx* c) {
+  for (StepGraph& g : c->graphs) drop_step_graph(g);
+}
+
+// Capture the whole step (embedding .. sampler) with the given sampler once
+// per (batch, cached length) on the context stream.
+dg_status capture_step(dg_ctx* c, int mode) {
+  StepGraph& sg = c->graphs[mode];
+  drop_step_graph(sg);
+  const int64_t l0 = c->launches;
+  DG_CUDA(c, cudaStreamBeginCapture(c->stream, cudaStreamCaptureModeThreadLocal));
+  dg_status st = forward(c, c->io_canvas_in, c->cfg.canvas, 0, c->B, c->cfg.canvas, c->P, false,
+                         mode == SAMPLER_TAU ? c->io_settled : nullptr);
+  if (st == DG_OK) {
+    if (mode == SAMPLER_TAU) {
       st = lm_head_and_sample(c, c->B, 0, 0, 0.f, c->io_canvas_out, c->io_conf, c->io_settled);
-    cudaGraph_t g = nullptr;
-    const cudaError_t e = cudaStreamEndCapture(c->stream, &g);
-    if (st != DG_OK || e != cudaSuccess) {
-      if (g) cudaGraphDestroy(g);
-      cudaGetLastError();
-      return st != DG_OK ? st : fail(c, DG_ERR_CUDA, "step capture: %s", cudaGetErrorString(e));
+    } else {
+      EntropyCall e{};
+      e.args.temperature = 1.f;
+      e.canvas_out = c->io_canvas_out;
+      st = lm_head_and_entropy_sample(c, c->B, e);
     }
-    c->step_graph = g;
-    DG_CUDA(c, cudaGraphInstantiate(&c->step_exec, g, 0));
-    size_t n = 0;
-    DG_CUDA(c, cudaGraphGetNodes(g, nullptr, &n));
-    std::vector<cudaGraphNode_t> nodes(n);
-    DG_CUDA(c, cudaGraphGetNodes(g, nodes.data(), &n));
-    c->embed_node = c->sample_node = nullptr;
-    for (cudaGraphNode_t nd : nodes) {
-      cudaGraphNodeType ty;
-      if (cudaGraphNodeGetType(nd, &ty) != cudaSuccess || ty != cudaGraphNodeTypeKernel) continue;
-      cudaKernelNodeParams kp;
-      if (cudaGraphKernelNodeGetParams(nd, &kp) != cudaSuccess) continue;
-      if (kp.func == reinterpret_cast<void*>(embed_norm_kernel)) {
-        c->embed_node = nd;
-        c->embed_kp = kp;
-      } else if (kp.func == reinterpret_cast<void*>(lmhead_merge_sample_kernel)) {
-        c->sample_node = nd;
-        c->sample_kp = kp;
-      }
-    }
-    if (!c->embed_node || !c->sample_node) {
-      drop_step_graph(c);
-      return fail(c, DG_ERR_CUDA, "step graph: entry/exit kernels not found");
-    }
-    // argument pointer arrays: point at the graph's stored values except the rebound ones
-    c->embed_args.assign(c->embed_kp.kernelParams, c->embed_kp.kernelParams + 14);
-    c->sample_args.assign(c->sample_kp.kernelParams, c->sample_kp.kernelParams + 2);
-    c->graph_launches = c->launches - l0;
-    c->launches = l0;
-    c->graph_B = c->B;
-    c->graph_P = c->P;
   }
+  cudaGraph_t g = nullptr;
+  const cudaError_t ce = cudaStreamEndCapture(c->stream, &g);
+  if (st != DG_OK || ce != cudaSuccess) {
+    if (g) cudaGraphDestroy(g);
+    cudaGetLastError();
+    return st != DG_OK ? st : fail(c, DG_ERR_CUDA, "step capture: %s", cudaGetErrorString(ce));
+  }
+  sg.graph = g;
+  DG_CUDA(c, cudaGraphInstantiate(&sg.exec, g, 0));
+  size_t n = 0;
+  DG_CUDA(c, cudaGraphGetNodes(g, nullptr, &n));
+  std::vector<cudaGraphNode_t> nodes(n);
+  DG_CUDA(c, cudaGraphGetNodes(g, nodes.data(), &n));
+  const void* sampler_fn = mode == SAMPLER_TAU ? reinterpret_cast<const void*>(lmhead_merge_sample_kernel)
+                                               : reinterpret_cast<const void*>(entropy_sample_kernel);
+  for (cudaGraphNode_t nd : nodes) {
+    cudaGraphNodeType ty;
+    if (cudaGraphNodeGetType(nd, &ty) != cudaSuccess || ty != cudaGraphNodeTypeKernel) continue;
+    cudaKernelNodeParams kp;
+    if (cudaGraphKernelNodeGetParams(nd, &kp) != cudaSuccess) continue;
+    if (kp.func == reinterpret_cast<void*>(embed_norm_kernel)) {
+      sg.embed_node = nd;
+      sg.embed_kp = kp;
+    } else if (kp.func == reinterpret_cast<void*>(gemm_kernel<GEMM_LMHEAD>)) {
+      sg.lm_node = nd;
+      sg.lm_kp = kp;
+    } else if (kp.func == sampler_fn) {
+      sg.sample_node = nd;
+      sg.sample_kp = kp;
+    }
+  }
+  if (!sg.embed_node || !sg.lm_node || !sg.sample_node) {
+    drop_step_graph(sg);
+    return fail(c, DG_ERR_CUDA, "step graph: entry/exit kernels not found");
+  }
+  // argument pointer arrays: point at the graph's stored values except the rebound ones
+  sg.embed_args.assign(sg.embed_kp.kernelParams, sg.embed_kp.kernelParams + 14);
+  sg.sample_args.assign(sg.sample_kp.kernelParams, sg.sample_kp.kernelParams + (mode == SAMPLER_TAU ? 2 : 1));
+  sg.launches = c->launches - l0;
+  c->launches = l0;
+  sg.B = c->B;
+  sg.P = c->P;
+  return DG_OK;
+}
+
+// rebind the embedding node: canvas and settled flags
+dg_status rebind_embed(dg_ctx* c, StepGraph& sg, const int32_t* canvas_in, int32_t* settled) {
   // embed_norm_kernel(tokens, tok_stride, tok_off, n, embed, gain, eps, d, h, u, capture, settled, n_settled, vocab)
   const int32_t* tok = canvas_in;
   int32_t* set0 = settled;
-  std::vector<void*> ea = c->embed_args;
+  std::vector<void*> ea = sg.embed_args;
   ea[0] = &tok;
   ea[11] = &set0;
-  cudaKernelNodeParams ekp = c->embed_kp;
+  cudaKernelNodeParams ekp = sg.embed_kp;
   ekp.kernelParams = ea.data();
-  DG_CUDA(c, cudaGraphExecKernelNodeSetParams(c->step_exec, c->embed_node, &ekp));
+  DG_CUDA(c, cudaGraphExecKernelNodeSetParams(sg.exec, sg.embed_node, &ekp));
+  return DG_OK;
+}
+
+dg_status launch_graph(dg_ctx* c, StepGraph& sg) {
+  DG_CUDA(c, cudaGraphLaunch(sg.exec, c->stream));
+  c->launches += sg.launches;
+  return DG_OK;
+}
+
+// threshold sampler step as a graph: rebinds the first kernel (canvas,
+// settled flags) and the last one (step, seed, tau, outputs)
+dg_status step_via_graph(dg_ctx* c, const int32_t* canvas_in, int32_t step, uint64_t seed, float tau,
+                         int32_t* canvas_out, float* conf, int32_t* settled) {
+  StepGraph& sg = c->graphs[SAMPLER_TAU];
+  if (!sg.exec || sg.B != c->B || sg.P != c->P) {
+    dg_status st = capture_step(c, SAMPLER_TAU);
+    if (st != DG_OK) return st;
+  }
+  dg_status st = rebind_embed(c, sg, canvas_in, settled);
+  if (st != DG_OK) return st;
   // lmhead_merge_sample_kernel(part, SampleArgs)
-  SampleArgs a = *static_cast<SampleArgs*>(c->sample_args[1]);
+  SampleArgs a = *static_cast<SampleArgs*>(sg.sample_args[1]);
   a.step = step;
   a.seed_lo = static_cast<uint32_t>(seed & 0xFFFFFFFFull);
   a.seed_hi = static_cast<uint32_t>(seed >> 32);
@@ -644,18 +777,40 @@ dg_status step_via_graph(dg_ctx* c, const int32_t* canvas_in, int32_t step, uint
   a.canvas_out = canvas_out;
   a.conf_out = conf;
   a.settled = settled;
-  std::vector<void*> sa = c->sample_args;
+  std::vector<void*> sa = sg.sample_args;
   sa[1] = &a;
-  cudaKernelNodeParams skp = c->sample_kp;
+  cudaKernelNodeParams skp = sg.sample_kp;
   skp.kernelParams = sa.data();
-  DG_CUDA(c, cudaGraphExecKernelNodeSetParams(c->step_exec, c->sample_node, &skp));
-  DG_CUDA(c, cudaGraphLaunch(c->step_exec, c->stream));
-  c->launches += c->graph_launches;
-  return DG_OK;
+  DG_CUDA(c, cudaGraphExecKernelNodeSetParams(sg.exec, sg.sample_node, &skp));
+  return launch_graph(c, sg);
+}
+
+// entropy sampler step as a graph: rebinds the embedding (canvas), the LM
+// head (temperature) and the entropy sampler (its arguments)
+dg_status entropy_step_via_graph(dg_ctx* c, const int32_t* canvas_in, const EntropyCall& e) {
+  StepGraph& sg = c->graphs[SAMPLER_ENTROPY];
+  if (!sg.exec || sg.B != c->B || sg.P != c->P) {
+    dg_status st = capture_step(c, SAMPLER_ENTROPY);
+    if (st != DG_OK) return st;
+  }
+  dg_status st = rebind_embed(c, sg, canvas_in, nullptr);
+  if (st != DG_OK) return st;
+  GemmParams lp = *static_cast<GemmParams*>(sg.lm_kp.kernelParams[0]);
+  lp.logit_scale_log2 = static_cast<float>(1.4426950408889634 / static_cast<double>(e.args.temperature));
+  void* la[1] = {&lp};
+  cudaKernelNodeParams lkp = sg.lm_kp;
+  lkp.kernelParams = la;
+  DG_CUDA(c, cudaGraphExecKernelNodeSetParams(sg.exec, sg.lm_node, &lkp));
+  EntropyArgs ea = entropy_args(c, e);
+  void* sa[1] = {&ea};
+  cudaKernelNodeParams skp = sg.sample_kp;
+  skp.kernelParams = sa;
+  DG_CUDA(c, cudaGraphExecKernelNodeSetParams(sg.exec, sg.sample_node, &skp));
+  return launch_graph(c, sg);
 }
 
 void free_all(dg_ctx* c) {
-  drop_step_graph(c);
+  drop_step_graphs(c);
   for (cudaEvent_t e : c->ev_pool) cudaEventDestroy(e);
   c->ev_pool.clear();
   if (c->ws) cudaFree(c->ws);
@@ -745,7 +900,9 @@ dg_status dg_create(const dg_config* cfg, const dg_weights* w, void* cuda_stream
   c->HD = c->Hq * c->D;
   c->R_step = g.max_batch * g.canvas;
   c->R = std::max(c->R_step, g.prefill_rows);
+  if (c->R > kMaxRows) return reject(DG_ERR_UNSUPPORTED, "max_batch * canvas and prefill_rows must be <= 32768");
   if (const char* s = getenv("DG_WAIT_LIMIT_NS")) c->wait_limit_ns = strtoull(s, nullptr, 10);
+  if (const char* s = getenv("DG_TRACE")) c->trace = atoi(s) != 0;
 
   cudaError_t e = cudaGetDevice(&c->dev);
   if (e != cudaSuccess) {
@@ -765,6 +922,11 @@ dg_status dg_create(const dg_config* cfg, const dg_weights* w, void* cuda_stream
     discard(c);
     return DG_ERR_CUDA;
   }
+  if (c->trace) {
+    fprintf(stderr, "[dg] resident attention clusters by size:");
+    for (int nc = 1; nc <= ATC_MAX_CHUNKS; ++nc) fprintf(stderr, " %d:%d", nc, c->attn_max_clusters[nc]);
+    fprintf(stderr, "\n");
+  }
 
   // ---- workspace plan ----
   const size_t R = c->R, d = c->d, k = c->k;
@@ -773,9 +935,10 @@ dg_status dg_create(const dg_config* cfg, const dg_weights* w, void* cuda_stream
   const size_t CH = MOE_CHUNK_ROWS;
   const size_t chunks_max = (R * k + CH - 1) / CH + c->E;  // routed token chunks
   const size_t chunks_shared = (R + CH - 1) / CH;
-  c->max_gu_tiles = chunks_max * (c->F / 64) + chunks_shared * (c->Fs / 64);
-  c->max_dn_tiles = (chunks_max + chunks_shared) * (d / 128);
   c->max_chunks = chunks_max + chunks_shared;
+  // routed rows: expert e owns rows [e * T, e * T + rows_e) of xp, hbuf and yp
+  // for a forward of T <= R rows (shared-expert outputs follow at E * T)
+  const size_t ER = static_cast<size_t>(c->E) * R;
   size_t bytes = 0;
   auto add = [&](size_t n, size_t sz) { bytes += (n * sz + 255) / 256 * 256; };
   add(R * d, 4);                                  // h
@@ -785,24 +948,24 @@ dg_status dg_create(const dg_config* cfg, const dg_weights* w, void* cuda_stream
   add(R * c->HD, 2);                              // o
   add(R * k, 4);                                  // idx
   add(R * k, 4);                                  // gates
-  add(R * k, 4);                                  // perm_tok
   add(R * k, 4);                                  // inv_slot
-  add(c->max_gu_tiles + c->max_dn_tiles, 16);    // tiles
   add(c->max_chunks, 4);                          // chunk_done
-  add(2 * PERM_MAXE + 1, 4);                     // route
+  add(PERM_MAXE, 4);                              // expert_rows
+  add(2, 4);                                      // moe_work
   add(2, 4);                                      // dense_work
-  add(16, 4);                                     // counters
-  add(R * k * d, 2);                              // xp
-  add(R * k * c->F, 2);                           // hbuf
+  add(ER * d, 2);                                 // xp
+  add(ER * c->F, 2);                              // hbuf
   add(R * c->Fs, 2);                              // hsbuf
-  add((R * k + R) * d, 4);                        // yp
+  add((ER + R) * d, 4);                           // yp
   add(static_cast<size_t>(c->V / GEMM_BN) * c->R_step, 16);  // lm_part
+  add(static_cast<size_t>(c->V / GEMM_BN) * c->R_step, 4);   // lm_s1
   add(static_cast<size_t>(g.max_seq) * (c->D / 2), 8);        // rope
   add(4, 4);                                      // err word
   add(c->R_step, 4);                              // dbg_argmax
   add(c->R_step, 4);
   add(c->R_step, 4);
   add(c->R_step, 4);
+  add(c->R_step, 4);                              // dbg_entropy
   add(c->R_step, 4);                              // io canvas in
   add(c->R_step, 4);                              // io canvas out
   add(c->R_step, 4);                              // io conf
@@ -821,24 +984,24 @@ dg_status dg_create(const dg_config* cfg, const dg_weights* w, void* cuda_stream
   c->o = carve<uint16_t>(cur, R * c->HD);
   c->idx = carve<int32_t>(cur, R * k);
   c->gates = carve<float>(cur, R * k);
-  c->perm_tok = carve<int32_t>(cur, R * k);
   c->inv_slot = carve<int32_t>(cur, R * k);
-  c->tiles = carve<int4>(cur, c->max_gu_tiles + c->max_dn_tiles);
   c->chunk_done = carve<int32_t>(cur, c->max_chunks);
-  c->route = carve<int32_t>(cur, 2 * PERM_MAXE + 1);
+  c->expert_rows = carve<int32_t>(cur, PERM_MAXE);
+  c->moe_work = carve<int32_t>(cur, 2);
   c->dense_work = carve<int32_t>(cur, 2);
-  c->counters = carve<int32_t>(cur, 16);
-  c->xp = carve<uint16_t>(cur, R * k * d);
-  c->hbuf = carve<uint16_t>(cur, R * k * c->F);
+  c->xp = carve<uint16_t>(cur, ER * d);
+  c->hbuf = carve<uint16_t>(cur, ER * c->F);
   c->hsbuf = carve<uint16_t>(cur, R * c->Fs);
-  c->yp = carve<float>(cur, (R * k + R) * d);
+  c->yp = carve<float>(cur, (ER + R) * d);
   c->lm_part = carve<float4>(cur, static_cast<size_t>(c->V / GEMM_BN) * c->R_step);
+  c->lm_s1 = carve<float>(cur, static_cast<size_t>(c->V / GEMM_BN) * c->R_step);
   c->rope = carve<float2>(cur, static_cast<size_t>(g.max_seq) * (c->D / 2));
   c->err_word = carve<int>(cur, 4);
   c->dbg_argmax = carve<int32_t>(cur, c->R_step);
   c->dbg_lse = carve<float>(cur, c->R_step);
   c->dbg_conf = carve<float>(cur, c->R_step);
   c->dbg_margin = carve<float>(cur, c->R_step);
+  c->dbg_entropy = carve<float>(cur, c->R_step);
   c->io_canvas_in = carve<int32_t>(cur, c->R_step);
   c->io_canvas_out = carve<int32_t>(cur, c->R_step);
   c->io_conf = carve<float>(cur, c->R_step);
@@ -904,11 +1067,11 @@ dg_status dg_create(const dg_config* cfg, const dg_weights* w, void* cuda_stream
   ok &= make_map(&c->m_u64, c->u, R, d, 64);
   ok &= make_map(&c->m_u128, c->u, R, d, 128);
   ok &= make_map(&c->m_o64, c->o, R, c->HD, 64);
-  ok &= make_map(&c->m_xp16, c->xp, R * k, d, 16);
-  ok &= make_map(&c->m_xp64, c->xp, R * k, d, 64);
-  ok &= make_map(&c->m_h64, c->hbuf, R * k, c->F, 64);
+  ok &= make_map(&c->m_xp16, c->xp, ER, d, 16);
+  ok &= make_map(&c->m_xp64, c->xp, ER, d, 64);
+  ok &= make_map(&c->m_h64, c->hbuf, ER, c->F, 64);
   ok &= make_map(&c->m_hs64, c->hsbuf, R, c->Fs, 64);
-  ok &= make_map(&c->m_h16, c->hbuf, R * k, c->F, 16);
+  ok &= make_map(&c->m_h16, c->hbuf, ER, c->F, 16);
   ok &= make_map(&c->m_hs16, c->hsbuf, R, c->Fs, 16);
   ok &= make_map(&c->m_embed, c->embed, c->V, d, 128);
   if (!ok) {
@@ -960,6 +1123,23 @@ dg_status dg_denoise_step(dg_ctx* c, const int32_t* canvas_in, int32_t step, uin
   dg_status st = forward(c, canvas_in, c->cfg.canvas, 0, c->B, c->cfg.canvas, c->P, false, settled);
   if (st != DG_OK) return st;
   return lm_head_and_sample(c, c->B, step, seed, tau, canvas_out, conf, settled);
+}
+
+dg_status dg_denoise_step_entropy(dg_ctx* c, const int32_t* canvas_in, int32_t step, uint64_t seed,
+                                  const dg_entropy_args* args, const int32_t* prev_argmax, int32_t* argmax_out,
+                                  int32_t* canvas_out, float* entropy, int32_t* stopped) {
+  if (!c) return DG_ERR_INVALID_ARG;
+  if (!canvas_in || !canvas_out || !args) return fail(c, DG_ERR_INVALID_ARG, "step_entropy: null argument");
+  if (!(args->temperature > 0.f) || !(args->gamma >= 0.f) || args->stop_entropy != args->stop_entropy)
+    return fail(c, DG_ERR_INVALID_ARG, "step_entropy: temperature must be > 0, gamma >= 0");
+  if (!c->prefilled) return fail(c, DG_ERR_STATE, "step before prefill");
+  if (c->P + c->cfg.canvas > c->cfg.max_seq) return fail(c, DG_ERR_CAPACITY, "step: cache full");
+  EntropyCall e{step, seed, *args, prev_argmax, argmax_out, canvas_out, entropy, stopped};
+  if (c->use_graphs && !c->capture && c->prof_mask == 0 && c->stream != nullptr)
+    return entropy_step_via_graph(c, canvas_in, e);
+  dg_status st = forward(c, canvas_in, c->cfg.canvas, 0, c->B, c->cfg.canvas, c->P, false, nullptr);
+  if (st != DG_OK) return st;
+  return lm_head_and_entropy_sample(c, c->B, e);
 }
 
 dg_status dg_denoise_step_host(dg_ctx* c, const int32_t* canvas_in_host, int32_t step, uint64_t seed, float tau,
@@ -1067,8 +1247,7 @@ dg_status dg_debug_lmhead(dg_ctx* c, int32_t* argmax, float* lse, float* conf, f
 
 dg_status dg_debug_router(dg_ctx* c, const float* logits, int32_t n_rows, int32_t* idx, float* gates) {
   if (!c || !logits || !idx || !gates || n_rows <= 0) return fail(c, DG_ERR_INVALID_ARG, "debug_router");
-  router_topk_kernel<<<(n_rows + 7) / 8, 256, 0, c->stream>>>(logits, 1, n_rows, c->E, c->k, nullptr, idx, gates,
-                                                               nullptr, 8, nullptr);
+  router_topk_kernel<<<(n_rows + 7) / 8, 256, 0, c->stream>>>(logits, 1, n_rows, c->E, c->k, nullptr, idx, gates);
   DG_LAUNCHED(c);
   return DG_OK;
 }
@@ -1081,6 +1260,38 @@ dg_status dg_debug_sample(dg_ctx* c, const int32_t* argmax, const float* conf, i
                                                               static_cast<uint32_t>(seed & 0xFFFFFFFFull),
                                                               static_cast<uint32_t>(seed >> 32), tau, c->V, out);
   DG_LAUNCHED(c);
+  return DG_OK;
+}
+
+dg_status dg_debug_entropy_sample(dg_ctx* c, const int32_t* argmax, const float* entropy, const int32_t* prev,
+                                  int32_t B, int32_t step, uint64_t seed, float gamma, float stop_entropy,
+                                  int32_t* out, int32_t* stopped) {
+  if (!c || !argmax || !entropy || !out || B <= 0 || B > c->cfg.max_batch)
+    return fail(c, DG_ERR_INVALID_ARG, "debug_entropy_sample");
+  EntropyArgs a;
+  memset(&a, 0, sizeof(a));
+  a.C = c->cfg.canvas;
+  a.P = c->P;
+  a.step = step;
+  a.vocab = c->V;
+  a.seed_lo = static_cast<uint32_t>(seed & 0xFFFFFFFFull);
+  a.seed_hi = static_cast<uint32_t>(seed >> 32);
+  a.gamma = gamma;
+  a.stop_entropy = stop_entropy;
+  a.argmax = argmax;
+  a.entropy = entropy;
+  a.prev_argmax = prev;
+  a.canvas_out = out;
+  a.stopped = stopped;
+  entropy_sample_kernel<<<B, 256, 0, c->stream>>>(a);
+  DG_LAUNCHED(c);
+  return DG_OK;
+}
+
+dg_status dg_debug_entropy(dg_ctx* c, float* out) {
+  if (!c || !out) return fail(c, DG_ERR_INVALID_ARG, "debug_entropy");
+  DG_CUDA(c, cudaMemcpyAsync(out, c->dbg_entropy, static_cast<size_t>(c->B) * c->cfg.canvas * 4,
+                             cudaMemcpyDeviceToDevice, c->stream));
   return DG_OK;
 }
 
@@ -1180,25 +1391,9 @@ std::mutex g_static_setup_mutex;  // the first calls on a device may come from s
 __global__ void lmhead_static_merge_kernel(const float4* __restrict__ part, int n_vtiles, int T,
                                            const int* __restrict__ err, int32_t* __restrict__ argmax,
                                            float* __restrict__ lse, float* __restrict__ conf) {
-  __shared__ Top2 sh[32];
   const int t = blockIdx.x;
-  Top2 acc{-INFINITY, 0x7fffffff, -INFINITY, 0.f};
-  for (int v = threadIdx.x; v < n_vtiles; v += blockDim.x) {
-    const float4 p = part[static_cast<size_t>(v) * T + t];
-    acc = top2_merge(acc, Top2{p.x, __float_as_int(p.y), p.z, p.w});
-  }
-  for (int o = 16; o > 0; o >>= 1) {
-    Top2 other;
-    other.m1 = __shfl_xor_sync(0xffffffffu, acc.m1, o);
-    other.idx = __shfl_xor_sync(0xffffffffu, acc.idx, o);
-    other.m2 = __shfl_xor_sync(0xffffffffu, acc.m2, o);
-    other.s = __shfl_xor_sync(0xffffffffu, acc.s, o);
-    acc = top2_merge(acc, other);
-  }
-  if ((threadIdx.x & 31) == 0) sh[threadIdx.x >> 5] = acc;
-  __syncthreads();
+  const Top2 acc = merge_token_partials(part, nullptr, n_vtiles, T, t);
   if (threadIdx.x == 0) {
-    for (int w = 1; w < (blockDim.x >> 5); ++w) acc = top2_merge(acc, sh[w]);
     const bool bad = err[0] != 0;
     if (argmax) argmax[t] = bad ? -1 : acc.idx;
     if (lse) lse[t] = bad ? NAN : (acc.m1 + log2f(acc.s)) * 0.69314718055994531f;

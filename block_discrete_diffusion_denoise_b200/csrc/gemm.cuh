@@ -16,16 +16,18 @@
 //           gate/up tiles (A = 64 gate rows stacked on the same 64 up rows, B =
 //           the expert's tokens; the epilogue forms SiLU(gate) * up and stores
 //           bf16 hidden rows), then the down tiles (A = 128 rows of the down
-//           projection, B = hidden rows; fp32 output rows in permuted order).
-//           Tiles are claimed from an atomic counter in list order; a down tile
-//           waits until every gate/up tile of its token chunk has published its
-//           hidden rows.  Every claimed tile's dependencies were claimed
-//           earlier by running CTAs and depend on nothing, so the wait always
-//           ends.
+//           projection, B = hidden rows; fp32 output rows in the expert's
+//           region).  Every CTA derives the tile list from the per-expert row
+//           counts in shared memory; tiles are claimed from an atomic counter
+//           in list order; a down tile waits until every gate/up tile of its
+//           token chunk has published its hidden rows.  Every claimed tile's
+//           dependencies were claimed earlier by running CTAs and depend on
+//           nothing, so the wait always ends.
 //   LMHEAD  A = 128 tokens, B = 128 vocabulary rows of the tied embedding; the
-//           epilogue keeps, per token, the running top-2 logits, the argmax
-//           and the sum of exp, and writes one 16-byte partial per
-//           (vocabulary tile, token) — the logits never reach memory.
+//           epilogue keeps, per token, the running top-2 logits, the argmax,
+//           the sum of 2^x and the sum of 2^x * x (for the entropy), and
+//           writes one 16-byte partial (+ 4 bytes) per (vocabulary tile,
+//           token) — the logits never reach memory.
 #pragma once
 
 #include "common.cuh"
@@ -46,6 +48,9 @@ constexpr int MOE_CHUNK_ROWS = 128;                  // tokens per expert tile
 enum GemmMode : int { GEMM_DENSE = 0, GEMM_MOE = 1, GEMM_LMHEAD = 3 };
 
 constexpr int DENSE_BN = 256;                        // tokens per dense tile: each weight tile streamed once
+constexpr int MOE_MAX_EXPERTS = 256;                 // routed experts (+1 shared group) the tile tables hold
+// MOE tile tables in shared memory: chunk offsets [E + 2] and group rows [E + 1], 16-bit
+constexpr int MOE_TABLE_BYTES = ((MOE_MAX_EXPERTS + 2) + (MOE_MAX_EXPERTS + 1)) * 2 + 32;
 
 // Stage ring depth (16 KB of A plus the B rows per stage).
 template <int MODE>
@@ -68,7 +73,8 @@ constexpr int gemm_acc_cols() {
 }
 template <int MODE>
 constexpr int gemm_smem_bytes() {
-  return 1024 + gemm_stages<MODE>() * (GEMM_A_BYTES + gemm_b_bytes<MODE>()) + GEMM_XCHG_FLOATS * 4 + 512;
+  return 1024 + gemm_stages<MODE>() * (GEMM_A_BYTES + gemm_b_bytes<MODE>()) + GEMM_XCHG_FLOATS * 4 + 512 +
+         (MODE == GEMM_MOE ? MOE_TABLE_BYTES : 0);
 }
 
 enum TileKind : int { KIND_DENSE = 0, KIND_GATEUP = 1, KIND_DOWN = 2, KIND_LMHEAD = 3 };
@@ -99,17 +105,18 @@ struct GemmParams {
   // DENSE, MOE: claimed tiles
   int* work;              // [0] claim counter, [1] exit counter; zero at launch, reset by the last CTA
   // MOE
-  const int* counts;      // [0] gate/up tiles, [1] down tiles
-  const int4* tiles;      // gate/up tiles, then down tiles: {group | blk << 16, chunk, first row, rows}
-  int* chunk_done;        // finished gate/up tiles per token chunk, zero at launch
-  int n_groups_routed;    // group == n_groups_routed is the shared expert
+  int* expert_rows;       // [E] rows routed to each expert (zeroed by the last CTA out)
+  int region;             // rows per expert region of the routed buffers
+  int* chunk_done;        // finished gate/up tiles per token chunk, zero at launch (zeroed by the last CTA)
+  int n_groups_routed;    // E; group == n_groups_routed is the shared expert (its T rows are the tokens)
   int F, Fs, d;
   float* out_f32;         // DENSE partials [splits][T][M]; MOE down output rows [.][out_ld]
   int out_ld;
   int shared_row_base;    // MOE down: output row of shared-expert token 0
   uint16_t* h_out;        // MOE routed hidden [rows][F]
   uint16_t* hs_out;       // MOE shared hidden [tokens][Fs]
-  float4* lm_part;        // LMHEAD partials [vocab tiles][M]
+  float4* lm_part;        // LMHEAD partials [vocab tiles][M]: {max, argmax, second max, sum 2^(x - max)}
+  float* lm_s1;           // LMHEAD [vocab tiles][M]: sum 2^(x - max) * x (entropy), or NULL
   float logit_scale_log2; // LMHEAD: log2(e) / temperature
   DevErr err;
 };
@@ -207,9 +214,83 @@ __device__ __forceinline__ void decode_tile(const GemmParams& p, int tile, int4 
   }
 }
 
+// MOE tile list, derived from the row counts.  Groups g = 0 (shared expert,
+// T rows) and g = 1 + e (routed expert e); group g has nch_g = ceil(rows_g /
+// MOE_CHUNK_ROWS) token chunks; ch_off[g] = sum of nch over the groups before
+// g (ch_off[G] = all chunks).  Gate/up tiles first: the shared group's Fs/64
+// blocks x nch_0 chunks, then each routed group's F/64 blocks x nch_g chunks;
+// then the down tiles: each group's d/128 blocks x nch_g chunks.  Within a
+// group the order is block-major, so re-reads of a weight block by its chunks
+// hit L2.  Record: {group (E = shared) | block << 16, chunk id, first row,
+// rows}.
+struct MoeTables {
+  const uint16_t* ch_off;  // [G + 1]
+  const uint16_t* rows;    // [G]
+  int G;                   // E + 1 groups
+  int n_gu, n_dn;
+};
+
+__device__ __forceinline__ int moe_upper(const uint16_t* a, int n, int q) {  // first i in [0, n) with a[i] > q
+  int lo = 0, hi = n;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (static_cast<int>(a[mid]) > q) hi = mid;
+    else lo = mid + 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ int4 moe_record(const GemmParams& p, const MoeTables& tb, int t) {
+  const int mb_s = p.Fs / 64, mb_r = p.F / 64, mb_dn = p.d / GEMM_BM;
+  const int nch_s = tb.ch_off[1];
+  int g, local;
+  if (t < tb.n_gu) {
+    if (t < nch_s * mb_s) {
+      g = 0;
+      local = t;
+    } else {
+      const int tp = t - nch_s * mb_s;
+      g = moe_upper(tb.ch_off, tb.G + 1, tp / mb_r + nch_s) - 1;
+      local = tp - (static_cast<int>(tb.ch_off[g]) - nch_s) * mb_r;
+    }
+  } else {
+    const int tp = t - tb.n_gu;
+    g = moe_upper(tb.ch_off, tb.G + 1, tp / mb_dn) - 1;
+    local = tp - static_cast<int>(tb.ch_off[g]) * mb_dn;
+  }
+  const int nch = tb.ch_off[g + 1] - tb.ch_off[g];
+  const int blk = local / nch, ch = local % nch;
+  const int first = (g == 0 ? 0 : (g - 1) * p.region) + ch * MOE_CHUNK_ROWS;
+  return make_int4((g == 0 ? p.n_groups_routed : g - 1) | (blk << 16), tb.ch_off[g] + ch, first,
+                   min(MOE_CHUNK_ROWS, static_cast<int>(tb.rows[g]) - ch * MOE_CHUNK_ROWS));
+}
+
+// exclusive scan of one value per thread over the whole block (blockDim.x a
+// multiple of 32); tmp >= 32 ints; every thread receives the total
+__device__ __forceinline__ int block_excl_scan(int v, int* tmp, int& total) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) tmp[warp] = x;
+  __syncthreads();
+  int base = 0;
+  total = 0;
+  for (int w = 0; w < nw; ++w) {
+    const int t = tmp[w];
+    if (w < warp) base += t;
+    total += t;
+  }
+  __syncthreads();
+  return base + x - v;
+}
+
 template <int MODE>
-__device__ __forceinline__ int tile_total(const GemmParams& p) {
-  if constexpr (MODE == GEMM_MOE) return p.counts[0] + p.counts[1];
+__device__ __forceinline__ int tile_total(const GemmParams& p, const MoeTables& tb) {
+  if constexpr (MODE == GEMM_MOE) return tb.n_gu + tb.n_dn;
   return p.tiles_static;
 }
 
@@ -328,9 +409,41 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
   int* sched = reinterpret_cast<int*>(sched_rec + GEMM_SCHED);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sched + GEMM_SCHED);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  int* scan_tmp = reinterpret_cast<int*>(tmem_holder + 4);           // 8 ints
+  uint16_t* tb_ch_off = reinterpret_cast<uint16_t*>(xchg + GEMM_XCHG_FLOATS) + 256;  // after the 512-byte tail
+  uint16_t* tb_rows = tb_ch_off + MOE_MAX_EXPERTS + 2;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+
+  MoeTables tb{tb_ch_off, tb_rows, 0, 0, 0};
+  if constexpr (MODE == GEMM_MOE) {
+    // tile tables from the row counts (two groups per thread, G <= 2 * 192)
+    const int G = p.n_groups_routed + 1;
+    int nch2[2], rows2[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int g = 2 * threadIdx.x + h;
+      rows2[h] = g == 0 ? p.T : (g < G ? p.expert_rows[g - 1] : 0);
+      nch2[h] = (rows2[h] + MOE_CHUNK_ROWS - 1) / MOE_CHUNK_ROWS;
+    }
+    int total;
+    const int base = block_excl_scan(nch2[0] + nch2[1], scan_tmp, total);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int g = 2 * threadIdx.x + h;
+      if (g < G) {
+        tb_rows[g] = static_cast<uint16_t>(rows2[h]);
+        tb_ch_off[g] = static_cast<uint16_t>(base + (h ? nch2[0] : 0));
+      }
+    }
+    if (threadIdx.x == 0) tb_ch_off[G] = static_cast<uint16_t>(total);
+    __syncthreads();
+    const int nch_s = tb_ch_off[1];
+    tb.G = G;
+    tb.n_gu = nch_s * (p.Fs / 64) + (total - nch_s) * (p.F / 64);
+    tb.n_dn = total * (p.d / GEMM_BM);
+  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -357,8 +470,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
-  const int n_tiles = tile_total<MODE>(p);
-  const int n_gu = (MODE == GEMM_MOE) ? p.counts[0] : 0;
+  const int n_tiles = tile_total<MODE>(p, tb);
+  const int n_gu = tb.n_gu;
 
   if (warp == 0) {
     // ------------------------------ TMA producer ------------------------------
@@ -376,7 +489,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
       int4 cur_rec = make_int4(0, 0, 0, 0);
       if constexpr (claims_tiles<MODE>()) {
         cur = atomicAdd(p.work, 1);
-        if (cur < n_tiles) cur_rec = p.tiles[cur];
+        if (cur < n_tiles) cur_rec = moe_record(p, tb, cur);
         claim = atomicAdd(p.work, 1);
       }
       for (int it = 0;; ++it) {
@@ -388,7 +501,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
           if (cur >= n_tiles || *abort_flag) cur = -1;
           if (cur >= 0 && claim < n_tiles) {
             nxt = claim;
-            nxt_rec = p.tiles[nxt];          // consumed in the next iteration
+            nxt_rec = moe_record(p, tb, nxt);  // consumed in the next iteration
             claim = atomicAdd(p.work, 1);
           }
           tile = cur;
@@ -636,7 +749,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
         }
       } else {  // GEMM_LMHEAD
         const int tok = t.a_row + row;
-        float m1 = -INFINITY, m2 = -INFINITY, s = 0.f;
+        float m1 = -INFINITY, m2 = -INFINITY, s = 0.f, s1 = 0.f;
         int idx = 0x7fffffff;
         for (int c0 = 0; c0 < GEMM_BN; c0 += 32) {
           float v[32];
@@ -646,17 +759,23 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
             const float x = v[i] * p.logit_scale_log2;
             if (x > m1) {
               m2 = m1;
-              s = s * exp2f(m1 - x) + 1.f;
+              const float sc = exp2f(m1 - x);
+              s = s * sc + 1.f;
+              s1 = s1 * sc + x;
               m1 = x;
               idx = t.b_row + c0 + i;
             } else {
               m2 = fmaxf(m2, x);
-              s += exp2f(x - m1);
+              const float e = exp2f(x - m1);
+              s += e;
+              s1 = fmaf(e, x, s1);
             }
           }
         }
-        if (tok < p.M)
+        if (tok < p.M) {
           p.lm_part[static_cast<size_t>(t.group) * p.M + tok] = make_float4(m1, __int_as_float(idx), m2, s);
+          if (p.lm_s1) p.lm_s1[static_cast<size_t>(t.group) * p.M + tok] = s1;
+        }
       }
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
@@ -671,11 +790,20 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
     tmem_dealloc(tmem_base, 2 * ACC_COLS);
   }
   if constexpr (claims_tiles<MODE>()) {
-    // the last CTA out resets the claim counter for the next launch (all
-    // claims of this launch were made before their CTA reached this point)
+    // the last CTA out resets, for the next launch, the claim counter, the
+    // per-expert row counts and the chunk flags (every CTA read the counts
+    // and made its claims, and every flag wait ended, before its CTA counted
+    // itself out)
     if (threadIdx.x == 0) {
       __threadfence();
-      if (atomicAdd(p.work + 1, 1) == static_cast<int>(gridDim.x) - 1) {
+      scan_tmp[0] = atomicAdd(p.work + 1, 1) == static_cast<int>(gridDim.x) - 1;
+    }
+    __syncthreads();
+    if (scan_tmp[0]) {
+      __threadfence();
+      for (int e = threadIdx.x; e < p.n_groups_routed; e += blockDim.x) p.expert_rows[e] = 0;
+      for (int c = threadIdx.x; c < tb_ch_off[tb.G]; c += blockDim.x) p.chunk_done[c] = 0;
+      if (threadIdx.x == 0) {
         atomicExch(p.work, 0);
         atomicExch(p.work + 1, 0);
       }

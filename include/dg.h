@@ -146,6 +146,41 @@ dg_status dg_denoise_step(dg_ctx* ctx, const int32_t* canvas_in_dev, int32_t ste
                           float tau, int32_t* canvas_out_dev, float* conf_dev,
                           int32_t* all_settled_dev);
 
+/* Entropy-constrained sampler of one step (codemajin.net "DiffusionGemma
+ * architecture", section 3.3).
+ *   temperature   this step's temperature (the page anneals it linearly from
+ *                 0.8 to 0.4 over at most 48 steps; the caller picks it)
+ *   gamma         entropy budget (nats): positions are accepted in ascending
+ *                 (entropy, position) order while the float32 running sum of
+ *                 their entropies stays <= gamma; the first is always accepted
+ *   stop_entropy  adaptive stop (nats): when a previous argmax is given, the
+ *                 canvas's mean entropy (float32 sum in position order / C)
+ *                 is < stop_entropy and every argmax equals the previous
+ *                 one, every position takes its argmax and the sequence is
+ *                 reported stopped */
+typedef struct dg_entropy_args {
+  float temperature;
+  float gamma;
+  float stop_entropy;
+} dg_entropy_args;
+
+/* One denoising step like dg_denoise_step, ended by the entropy-constrained
+ * sampler instead of the confidence threshold.  Accepted positions take
+ * their argmax, the others the same Philox uniform draw as dg_denoise_step.
+ *   prev_argmax_dev [batch, canvas] int32: the previous step's argmax, or
+ *                   NULL at the first step of a block (no stop possible)
+ *   argmax_out_dev  [batch, canvas] int32 or NULL: this step's argmax (may
+ *                   equal prev_argmax_dev, for the next call)
+ *   canvas_out_dev  [batch, canvas] int32 (may equal canvas_in_dev)
+ *   entropy_dev     [batch, canvas] fp32 or NULL: softmax entropy (nats)
+ *   stopped_dev     [batch] int32 or NULL: 1 where the adaptive stop fired
+ * The committed cache is not modified.  The logits never leave the chip: the
+ * entropy comes from one more running sum in the LM-head reduction. */
+dg_status dg_denoise_step_entropy(dg_ctx* ctx, const int32_t* canvas_in_dev, int32_t step, uint64_t seed,
+                                  const dg_entropy_args* args, const int32_t* prev_argmax_dev,
+                                  int32_t* argmax_out_dev, int32_t* canvas_out_dev, float* entropy_dev,
+                                  int32_t* stopped_dev);
+
 /* Same step with HOST buffers: copies canvas_in_host to the device, runs the
  * step, copies canvas_out/conf/all_settled back and synchronises.  Any of
  * conf_host and all_settled_host may be NULL. */
@@ -210,6 +245,16 @@ dg_status dg_debug_router(dg_ctx* ctx, const float* logits_dev, int32_t n_rows, 
  * P + i of the current cache length). */
 dg_status dg_debug_sample(dg_ctx* ctx, const int32_t* argmax_dev, const float* conf_dev,
                           int32_t batch, int32_t step, uint64_t seed, float tau, int32_t* out_dev);
+
+/* Entropy sampler decision alone on given argmax / entropy [batch*canvas]
+ * (positions P + i of the current cache length), prev_argmax or NULL:
+ * out_dev [batch*canvas] int32, stopped_dev [batch] int32 or NULL. */
+dg_status dg_debug_entropy_sample(dg_ctx* ctx, const int32_t* argmax_dev, const float* entropy_dev,
+                                  const int32_t* prev_argmax_dev, int32_t batch, int32_t step, uint64_t seed,
+                                  float gamma, float stop_entropy, int32_t* out_dev, int32_t* stopped_dev);
+
+/* Softmax entropy (nats) per position of the last step [batch*canvas]. */
+dg_status dg_debug_entropy(dg_ctx* ctx, float* out_dev);
 
 /* Launch a kernel that waits on a barrier nothing ever signals, with a wait
  * limit of limit_ns nanoseconds; the following dg_sync must report

@@ -186,7 +186,7 @@ def teacher_forced_checks(g: dict, r, temperature: float, out: dict, fails: list
 
 
 def compare_step(g: dict, r: "oracle.StepResult", tau: float, orc=None, check_hidden=True, report=None,
-                 temperature: float = 1.0):
+                 temperature: float = 1.0, drift_tol: float | None = None):
     """Apply the criteria; returns a dict of measured errors (asserts at the end).
 
     Router near-ties.  The GPU feeds the router bf16 operands derived from its
@@ -199,6 +199,13 @@ def compare_step(g: dict, r: "oracle.StepResult", tau: float, orc=None, check_hi
     failure; a token within it is counted and, from that layer on, left out of
     the hidden-state and log-probability comparisons (its residual stream has
     legitimately left the oracle's).
+
+    The 1e-2 per-layer criterion is the error one layer adds: it is checked
+    teacher-forced (teacher_forced_checks).  The free-running residual stream
+    carries the rounding of every layer before it; it is held to the same 1e-2
+    unless drift_tol is given (the 30-layer test gives 2e-2: a bf16-operand
+    emulation of the first layer already reaches 0.7%, and the drift
+    accumulates over depth).
     """
     out = {}
     B, C = r.canvas_out.shape
@@ -238,8 +245,9 @@ def compare_step(g: dict, r: "oracle.StepResult", tau: float, orc=None, check_hi
         out["hidden_rel_l2"] = errs
         out["hidden_rel_l2_all_tokens"] = errs_all
         out["expert_flips"] = flips
-        if out["hidden_rel_l2_max"] > HIDDEN_REL_L2:
-            fails.append(f"hidden rel-L2 {out['hidden_rel_l2_max']:.4g} > {HIDDEN_REL_L2}")
+        tol = HIDDEN_REL_L2 if drift_tol is None else drift_tol
+        if out["hidden_rel_l2_max"] > tol:
+            fails.append(f"free-running hidden rel-L2 {out['hidden_rel_l2_max']:.4g} > {tol}")
     if check_hidden and "hidden" in g and r.forced_hidden:
         teacher_forced_checks(g, r, temperature, out, fails)
     keep = ~diverged
