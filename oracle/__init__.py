@@ -11,7 +11,7 @@ Parity status of each function is recorded beside its pin in tests/.
 """
 from .model import (Oracle, Shape, StepResult, anneal_temperature, apply_rope, attention, entropy_accept,
                     entropy_sample, lm_head_stats, mean_entropy, moe,
-                    renoise_tokens, rms_norm, rope_angles, route_top_k, sample, selected_gates, silu,
+                    renoise_tokens, rms_norm, rope_angles, route_top_k, sample, selected_gates, self_condition, silu,
                     swiglu_ffn, tokens_per_forward, tokens_per_second)
 from .philox import philox4x32_10, uniform_token
 

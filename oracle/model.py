@@ -166,6 +166,30 @@ def lm_head_stats(z: np.ndarray, embed, temperature: float, row_chunk: int = 64,
     return res
 
 
+def self_condition(z: np.ndarray, embed, temperature: float, sc_gate, sc_up, sc_down,
+                   row_chunk: int = 64, vocab_chunk: int = 32768) -> np.ndarray:
+    """Self-conditioning signal of rows z [n, d] (codemajin.net "DiffusionGemma
+    architecture", section 3.2): the predicted clean-token distribution
+    p = softmax(z E^T / T) is passed through the embedding matrix, e = p E, and
+    then through a small feed-forward layer, here SwiGLU:
+    (SiLU(e Wg^T) * (e Wu^T)) Wd^T.  Returns [n, d]; the next step adds it to
+    its input embeddings."""
+    n, d = z.shape
+    V = embed.shape[0]
+    e = np.zeros((n, d))
+    for r0 in range(0, n, row_chunk):
+        zr = z[r0:r0 + row_chunk]
+        s = np.empty((zr.shape[0], V))
+        for v0 in range(0, V, vocab_chunk):
+            s[:, v0:v0 + vocab_chunk] = zr @ _f64(embed[v0:v0 + vocab_chunk]).T
+        s /= temperature
+        p = np.exp(s - s.max(axis=1, keepdims=True))
+        p /= p.sum(axis=1, keepdims=True)
+        for v0 in range(0, V, vocab_chunk):
+            e[r0:r0 + zr.shape[0]] += p[:, v0:v0 + vocab_chunk] @ _f64(embed[v0:v0 + vocab_chunk])
+    return swiglu_ffn(e, _f64(sc_gate), _f64(sc_up), _f64(sc_down))
+
+
 def renoise_tokens(positions, step: int, seq_ids, seed: int, vocab: int) -> np.ndarray:
     """Uniform replacement tokens: Philox4x32-10 with counter (absolute
     position, step, sequence, 0) and key (seed low word, seed high word)."""
@@ -331,6 +355,7 @@ class StepResult:
     gap: np.ndarray | None = None                    # top-1 minus top-2 logit (after /T)
     entropy: np.ndarray | None = None                # softmax entropy per position (nats)
     stopped: np.ndarray | None = None                # entropy sampler: adaptive stop per sequence
+    self_cond: np.ndarray | None = None              # [B, C, d] signal for the next step (if enabled)
     forced_hidden: list = field(default_factory=list)  # teacher-forced layer outputs, [B, C, d]
     forced_experts: list = field(default_factory=list)  # top-k of given router rows, [B, C, k]
     forced_router_margin: list = field(default_factory=list)  # their k-th minus (k+1)-th logit
@@ -465,7 +490,8 @@ class Oracle:
     # -- bidirectional decoder + sampler --
     def denoise_step(self, canvas: np.ndarray, step: int, seed: int, tau: float,
                      temperature: float = 1.0, record: bool = True,
-                     teacher: dict | None = None) -> StepResult:
+                     teacher: dict | None = None, self_cond_in=None,
+                     sc_weights: dict | None = None) -> StepResult:
         """One denoising step of the canvas [B, C] (cache unchanged).
 
         teacher = {"hidden": [L+1 of [B, C, d]], "experts": [L of [B, C, k]]},
@@ -477,7 +503,13 @@ class Oracle:
         layer's router consumed) give forced_experts / forced_router_margin,
         the top-k of those rows' logits; teacher["lm_rows"] ([B, C, d], the
         normalised rows the LM head consumed) give forced_lm, the LM-head
-        statistics of those rows."""
+        statistics of those rows.
+
+        Self-conditioning (codemajin.net section 3.2): self_cond_in [B, C, d]
+        (the previous step's signal, or None at the first step of a block) is
+        added to the input embeddings; with sc_weights (sc_gate, sc_up,
+        sc_down) the step also returns self_cond, its own signal for the next
+        step."""
         canvas = np.asarray(canvas)
         B, C = canvas.shape
         s = self.s
@@ -495,6 +527,8 @@ class Oracle:
                 f_mar = [np.empty((B, C)) for _ in range(s.n_layers)]
         for b in range(B):
             h = _f64(self.embed[_index(canvas[b])])
+            if self_cond_in is not None:
+                h = h + np.asarray(self_cond_in[b], dtype=np.float64)
             if record:
                 hidden[0][b] = h
             for l in range(s.n_layers):
@@ -522,6 +556,10 @@ class Oracle:
                     rmar[l][b] = dbg["margin"]
             z[b] = rms_norm(h, self.final_norm, s.rms_eps)
         st = lm_head_stats(z.reshape(B * C, s.d_model), self.embed, temperature)
+        sc_next = None
+        if sc_weights is not None:
+            sc_next = self_condition(z.reshape(B * C, s.d_model), self.embed, temperature, sc_weights["sc_gate"],
+                                     sc_weights["sc_up"], sc_weights["sc_down"]).reshape(B, C, s.d_model)
         if teacher is not None and teacher.get("lm_rows") is not None:
             zf = np.asarray(teacher["lm_rows"], dtype=np.float64).reshape(B * C, s.d_model)
             f_lm = {k: v.reshape(B, C) for k, v in lm_head_stats(zf, self.embed, temperature).items()}
@@ -535,7 +573,8 @@ class Oracle:
                           hidden=hidden, experts=experts, router_logits=rlog,
                           router_margin=rmar, gap=rs(st["gap"]), entropy=rs(st["entropy"]),
                           forced_hidden=forced,
-                          forced_experts=f_exp, forced_router_margin=f_mar, forced_lm=f_lm)
+                          forced_experts=f_exp, forced_router_margin=f_mar, forced_lm=f_lm,
+                          self_cond=sc_next)
 
 
 def _entropy_step(self, canvas, step: int, seed: int, temperature: float, gamma: float, stop_entropy: float,

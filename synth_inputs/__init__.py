@@ -27,7 +27,7 @@ import torch
 __all__ = [
     "ModelShape", "Workload", "WORKLOADS", "workload", "tensor_id",
     "hash_u32", "weight", "layer_weights", "global_weights", "uniform_tokens",
-    "router_bias", "tau_schedule", "norm_weight",
+    "router_bias", "tau_schedule", "norm_weight", "self_cond_weights",
 ]
 
 MASK32 = 0xFFFFFFFF
@@ -189,7 +189,9 @@ def _normalish(seed: int, tid: int, start: int, n: int, std: float, device) -> t
 _LAYER_NAMES = ["attn_norm", "wqkv", "wo", "ffn_norm", "w_router", "w_gate", "w_up",
                 "w_down", "ws_gate", "ws_up", "ws_down"]
 _GLOBAL_IDS = {"embed": 1_000_001, "final_norm": 1_000_002, "prefix": 2_000_001,
-               "canvas": 2_000_002}
+               "canvas": 2_000_002, "sc_gate": 1_000_003, "sc_up": 1_000_004, "sc_down": 1_000_005}
+# the self-conditioning feed-forward layer: SwiGLU of the routed-expert width
+_SELF_COND = ("sc_gate", "sc_up", "sc_down")
 
 
 def tensor_id(name: str, layer: int | None = None) -> int:
@@ -223,6 +225,9 @@ def weight(w: Workload, name: str, layer: int | None = None, device="cpu",
         return norm_weight(s, device)
     if name == "embed":
         shape = (s.vocab, s.d_model)
+    elif name in _SELF_COND:
+        F = s.expert_hidden
+        shape = (s.d_model, F) if name == "sc_down" else (F, s.d_model)
     else:
         shape = layer_shapes(s)[name]
     std = s.std * (s.out_scale if name in _OUT_PROJ else 1.0)
@@ -250,6 +255,12 @@ def global_weights(w: Workload, device="cpu") -> dict:
     return {"embed": weight(w, "embed", None, device),
             "final_norm": norm_weight(w.shape, device),
             "router_bias": router_bias(w, device)}
+
+
+def self_cond_weights(w: Workload, device="cpu") -> dict:
+    """Weights of the self-conditioning feed-forward layer (bf16): sc_gate,
+    sc_up [F, d] and sc_down [d, F], F the routed-expert width."""
+    return {name: weight(w, name, None, device) for name in _SELF_COND}
 
 
 def router_bias(w: Workload, device="cpu") -> torch.Tensor | None:

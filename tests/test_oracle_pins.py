@@ -412,3 +412,46 @@ def test_entropy_step_reuses_forward_and_noise():
     np.testing.assert_array_equal(r2.canvas_out[0][acc], r2.argmax[0][acc])
     np.testing.assert_array_equal(r2.canvas_out[0][~acc], r1.canvas_out[0][~acc])
     assert not r2.stopped[0]
+
+
+# --- self-conditioning (codemajin.net section 3.2) ----------------------------
+def test_self_condition_matches_torch_restatement():
+    z = rng.standard_normal((7, 12))
+    E = rng.standard_normal((53, 12)) * 0.5
+    wg, wu, wd = (rng.standard_normal(s) * 0.3 for s in ((9, 12), (9, 12), (12, 9)))
+    got = om.self_condition(z, E, 0.7, wg, wu, wd, row_chunk=3, vocab_chunk=16)
+    t = lambda a: torch.tensor(a, dtype=torch.float64)
+    e = torch.softmax(t(z) @ t(E).T / 0.7, dim=1) @ t(E)
+    ref = (torch.nn.functional.silu(e @ t(wg).T) * (e @ t(wu).T)) @ t(wd).T
+    np.testing.assert_allclose(got, ref.numpy(), rtol=1e-12, atol=1e-14)
+
+
+def test_self_condition_closed_forms():
+    E = rng.standard_normal((40, 8))
+    wg, wu, wd = (rng.standard_normal(s) for s in ((5, 8), (5, 8), (8, 5)))
+    ffn = lambda e: om.swiglu_ffn(e, wg, wu, wd)
+    # a flat distribution (z = 0): the mean embedding
+    got = om.self_condition(np.zeros((2, 8)), E, 1.0, wg, wu, wd)
+    np.testing.assert_allclose(got, ffn(np.tile(E.mean(axis=0), (2, 1))), rtol=1e-12, atol=1e-12)
+    # a one-hot distribution (a very sharp temperature): that token's embedding
+    z = E[[3, 17]]
+    got = om.self_condition(z, E, 1e-6, wg, wu, wd)
+    top = np.argmax(z @ E.T, axis=1)
+    np.testing.assert_allclose(got, ffn(E[top]), rtol=1e-9, atol=1e-9)
+
+
+def test_self_conditioned_step_adds_the_signal_to_the_input():
+    w = _tiny(prefix=16)
+    o = oracle.for_workload(w)
+    o.prefill(si.uniform_tokens(w, "prefix", 1, 16).numpy())
+    cv = si.uniform_tokens(w, "canvas", 1, 256).numpy()
+    scw = si.self_cond_weights(w)
+    r0 = o.denoise_step(cv, 0, 1, 0.9, sc_weights=scw)
+    assert r0.self_cond.shape == (1, 256, w.shape.d_model)
+    r1 = o.denoise_step(cv, 1, 1, 0.9, self_cond_in=r0.self_cond, sc_weights=scw)
+    emb = si.weight(w, "embed").to(torch.float64).numpy()
+    np.testing.assert_allclose(r1.hidden[0][0], emb[cv[0]] + r0.self_cond[0], rtol=1e-15, atol=0)
+    # the signal is the oracle's own function of the step's final normalised rows
+    z = om.rms_norm(r0.hidden[-1][0], o.final_norm, w.shape.rms_eps)
+    np.testing.assert_allclose(r0.self_cond[0], om.self_condition(z, o.embed, 1.0, scw["sc_gate"], scw["sc_up"],
+                                                                  scw["sc_down"]), rtol=1e-12, atol=1e-14)
