@@ -51,6 +51,11 @@ def parse():
     return ap.parse_args()
 
 
+PEAK_NOTE = {"measured": "of measured (MEASURED_PEAKS.json hbm_gbs, STREAM-style copy)",
+             "fallback": "of fallback (MEASURED_PEAKS.json absent: 6.65 TB/s copy, 1.59/1.4 PF/s bf16 "
+                         "burst/sustained measured earlier on this GPU type)"}
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -392,10 +397,10 @@ def run_native(args, w):
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": f"{w.name}: {w.description}", "global_batch": world * B,
                        "canvas": C, "prefix": w.prefix, "parallelism": f"replicas x{world}",
-                       "l2": "inputs larger than L2 (~50 GB of weights streamed per step)"},
+                       "l2": "inputs larger than L2 (~32 GB of weights streamed per step)"},
             "roofline": {"bound": "hbm", "kernel": "fused expert GEMM gate/up + down (tcgen05, SwiGLU epilogue)",
                          "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                         "traffic": traffic, "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)",
+                         "traffic": traffic, "peak_source": PEAK_NOTE[src],
                          "bytes_per_launch": gu_bytes, "launch_ms": gu_avg_ms, "launches": gu_n,
                          "launch_timing": "CUDA event pair around every launch of the kernel over a "
                                           "second K-step timed region with launches issued one by one"},

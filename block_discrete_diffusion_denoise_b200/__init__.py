@@ -19,6 +19,7 @@ STATUS = {0: "DG_OK", 1: "DG_ERR_INVALID_ARG", 2: "DG_ERR_OOM", 3: "DG_ERR_CAPAC
 
 # every function declared in include/dg.h
 EXPORTS = ["dg_create", "dg_destroy", "dg_prefill", "dg_denoise_step", "dg_denoise_step_entropy",
+           "dg_set_self_conditioning", "dg_debug_self_cond",
            "dg_denoise_step_host",
            "dg_commit_block", "dg_sync", "dg_cached_len", "dg_last_error", "dg_debug_capture",
            "dg_debug_hidden", "dg_debug_experts", "dg_debug_norm_rows", "dg_debug_lmhead", "dg_debug_router",
@@ -52,7 +53,8 @@ class dg_layer_weights(ctypes.Structure):
 
 class dg_weights(ctypes.Structure):
     _fields_ = [("embed", ctypes.c_void_p), ("final_norm", ctypes.c_void_p),
-                ("router_bias", ctypes.c_void_p), ("layers", ctypes.POINTER(dg_layer_weights))]
+                ("router_bias", ctypes.c_void_p), ("layers", ctypes.POINTER(dg_layer_weights)),
+                ("sc_gate", ctypes.c_void_p), ("sc_up", ctypes.c_void_p), ("sc_down", ctypes.c_void_p)]
 
 
 class dg_entropy_args(ctypes.Structure):
@@ -86,6 +88,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "dg_denoise_step_entropy": ([P, P, I32, U64, ctypes.POINTER(dg_entropy_args), P, P, P, P, P], I32),
         "dg_debug_entropy_sample": ([P, P, P, P, I32, I32, U64, F32, F32, P, P], I32),
         "dg_debug_entropy": ([P, P], I32),
+        "dg_set_self_conditioning": ([P, I32], I32),
+        "dg_debug_self_cond": ([P, P], I32),
         "dg_commit_block": ([P, P], I32),
         "dg_sync": ([P], I32),
         "dg_cached_len": ([P], I32),
@@ -137,7 +141,9 @@ class Context:
                 setattr(layers[i], f, _ptr(lw[f]))
         w = dg_weights(embed=_ptr(weights["embed"]), final_norm=_ptr(weights["final_norm"]),
                        router_bias=_ptr(weights.get("router_bias")),
-                       layers=ctypes.cast(layers, ctypes.POINTER(dg_layer_weights)))
+                       layers=ctypes.cast(layers, ctypes.POINTER(dg_layer_weights)),
+                       sc_gate=_ptr(weights.get("sc_gate")), sc_up=_ptr(weights.get("sc_up")),
+                       sc_down=_ptr(weights.get("sc_down")))
         self._layers_c = layers
         handle = ctypes.c_void_p()
         st = self.lib.dg_create(ctypes.byref(c), ctypes.byref(w), stream, ctypes.byref(handle))
@@ -223,6 +229,12 @@ class Context:
         self._check(self.lib.dg_debug_entropy_sample(self.ctx, _ptr(argmax), _ptr(entropy), _ptr(prev_argmax), batch,
                                                      int(step), int(seed), float(gamma), float(stop_entropy),
                                                      _ptr(out), _ptr(stopped)))
+
+    def set_self_conditioning(self, enable: bool):
+        self._check(self.lib.dg_set_self_conditioning(self.ctx, 1 if enable else 0))
+
+    def debug_self_cond(self, out):
+        self._check(self.lib.dg_debug_self_cond(self.ctx, _ptr(out)))
 
     def debug_entropy(self, out):
         self._check(self.lib.dg_debug_entropy(self.ctx, _ptr(out)))

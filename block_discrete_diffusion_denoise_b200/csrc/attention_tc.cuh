@@ -10,11 +10,13 @@
 // so each K/V block feeds all of them; the 256 rows are two 128-row query
 // tiles, each pulled by one 4-D TMA box out of the [token][head][D] query
 // layout, and every K/V block is read once for both.  The key chunks of one
-// query block form a thread-block cluster and are merged through distributed
-// shared memory.
+// query block form a thread-block cluster: each writes its raw rows and row
+// statistics to an L2-resident buffer, and after one cluster barrier each
+// reduces a slice of the rows over the chunks; a single chunk writes its rows
+// directly.
 //
-// Warp 0 issues TMA loads (both Q tiles once; 64-key K and V blocks into
-// 2-deep rings).  Warp 1 issues tcgen05.mma: S_q = Q_q K^T into tile q's TMEM
+// Warp 0 issues TMA loads (lane 0: both Q tiles once, then 64-key K blocks;
+// lane 1: V blocks; 2-deep rings).  Warp 1 issues tcgen05.mma: S_q = Q_q K^T into tile q's TMEM
 // buffer (128 x 64 fp32) and O_q += P_q V into tile q's TMEM accumulator
 // (128 x D fp32; V used as an MN-major operand).  Warps 2..5 and 6..9 are the
 // softmax warpgroups of tiles 0 and 1, one query row per thread, so every row
@@ -47,6 +49,8 @@ struct AttnTcParams {
   CUtensorMap k_map;   // 2-D (D, B*Hkv*S_max) over this layer's K cache; box (64, 64)
   CUtensorMap v_map;   // same over V
   uint16_t* o;         // [token][Hq][D]
+  float* part;         // several key chunks: [cluster][chunk][D/4][256 rows] float4 raw rows (L2-resident)
+  float2* part_ml;     // [cluster][chunk][256 rows] (max, sum) of those rows
   int n, B, Hq, Hkv, S_max, pos0, causal, chunk_len, n_chunks;
   float scale_log2;    // log2(e) / sqrt(D)
   DevErr err;
@@ -62,11 +66,8 @@ struct AtcCfg {
   static constexpr int S_COL = 0;                      // TMEM: S_q at q * 64, O_q at 128 + q * D
   static constexpr int O_COL = ATC_NQ * ATC_BK;
   static constexpr int TMEM_COLS = O_COL + ATC_NQ * D <= 256 ? 256 : 512;
-  static constexpr int OS_LD = D + 4;                  // fp32 row stride of the merged-O staging tile
-  static constexpr int ML_BYTES = ATC_ROWS * 8;        // per-row (max, sum), at the end of the region
   static constexpr int TAIL = 512;                     // barriers, flags
   static constexpr int SMEM = 1024 + REGION + TAIL;
-  static_assert(ATC_ROWS * OS_LD * 4 <= REGION - ML_BYTES, "merged-O staging must fit below the row statistics");
   static_assert(O_COL + ATC_NQ * D <= 512, "S and O accumulators must fit TMEM");
   static_assert(D % 16 == 0 && D <= 256, "head_dim must be a multiple of 16, at most 256");
 };
@@ -93,8 +94,6 @@ __global__ void __launch_bounds__(ATC_THREADS, 1) attn_tc_kernel(const __grid_co
   uint64_t* drain = o_done + ATC_NQ;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tail + 256);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tail + 260);
-  float2* ml_s = reinterpret_cast<float2*>(sQ + C::REGION - C::ML_BYTES);  // [256] (max, sum), after the mainloop
-  float* osm = reinterpret_cast<float*>(sQ);                             // [256][OS_LD] scaled O, after the mainloop
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.Hq / p.Hkv;
@@ -154,103 +153,108 @@ __global__ void __launch_bounds__(ATC_THREADS, 1) attn_tc_kernel(const __grid_co
   bool ok = true;
 
   if (warp == 0) {
-    // ------------------------------ TMA producer ------------------------------
-    if (lane == 0 && nb > 0) {
-      tma_prefetch_desc(&p.q_map);
-      tma_prefetch_desc(&p.k_map);
-      tma_prefetch_desc(&p.v_map);
+    // ------------------------ TMA producers: lane 0 K, lane 1 V ------------------------
+    // Separate lanes, so a K block is requested as soon as its ring slot is
+    // free, whatever the V ring is waiting for (and the other way round).
+    if (lane < 2 && nb > 0) {
+      const bool kl = lane == 0;
+      const CUtensorMap* map = kl ? &p.k_map : &p.v_map;
+      uint64_t* full = kl ? k_full : v_full;
+      uint64_t* empty = kl ? k_empty : v_empty;
+      uint8_t* ring = kl ? sK : sV;
+      constexpr int NS = ATC_KSTAGES;  // both rings have the same depth
+      static_assert(ATC_KSTAGES == ATC_VSTAGES, "K and V rings are walked by the same loop");
+      tma_prefetch_desc(map);
       const uint64_t pol = policy_evict_last();  // K/V blocks are shared by the head's query blocks
-      uint32_t k_issued = 0, k_par = 0, v_issued = 0, v_par = 0;
-      mbar_arrive_expect_tx(q_full, nq * C::Q_BYTES);
-      for (int q = 0; q < nq; ++q)
-        for (int db = 0; db < C::DK; ++db)
-          tma_load_4d(sQ + q * C::Q_BYTES + db * ATC_BQ * 128, &p.q_map, q_full, db * 64, 0, kvh,
-                      b * p.n + (row_base + q * ATC_BQ) / G, pol);
+      uint32_t issued = 0, par = 0;
+      if (kl) {
+        tma_prefetch_desc(&p.q_map);
+        mbar_arrive_expect_tx(q_full, nq * C::Q_BYTES);
+        for (int q = 0; q < nq; ++q)
+          for (int db = 0; db < C::DK; ++db)
+            tma_load_4d(sQ + q * C::Q_BYTES + db * ATC_BQ * 128, &p.q_map, q_full, db * 64, 0, kvh,
+                        b * p.n + (row_base + q * ATC_BQ) / G, pol);
+      }
       for (int j = 0; j < nb && !*abort_flag; ++j) {
-        const int s = j % ATC_KSTAGES;
-        const uint32_t ph = (j / ATC_KSTAGES) & 1;
-        if (!mbar_wait(&k_empty[s], ph ^ 1, p.err)) {
+        const int s = j % NS;
+        const uint32_t ph = (j / NS) & 1;
+        if (!mbar_wait(&empty[s], ph ^ 1, p.err)) {
           *abort_flag = 1;
           break;
         }
-        mbar_arrive_expect_tx(&k_full[s], C::KV_BYTES);
+        mbar_arrive_expect_tx(&full[s], C::KV_BYTES);
         for (int db = 0; db < C::DK; ++db)
-          tma_load_2d(sK + s * C::KV_BYTES + db * ATC_BK * 128, &p.k_map, &k_full[s], db * 64, kv_row0 + j * ATC_BK,
+          tma_load_2d(ring + s * C::KV_BYTES + db * ATC_BK * 128, map, &full[s], db * 64, kv_row0 + j * ATC_BK,
                       pol);
-        k_issued |= 1u << s;
-        k_par = (k_par & ~(1u << s)) | (ph << s);
-        const int sv = j % ATC_VSTAGES;
-        const uint32_t phv = (j / ATC_VSTAGES) & 1;
-        if (!mbar_wait(&v_empty[sv], phv ^ 1, p.err)) {
-          *abort_flag = 1;
-          break;
-        }
-        mbar_arrive_expect_tx(&v_full[sv], C::KV_BYTES);
-        for (int db = 0; db < C::DK; ++db)
-          tma_load_2d(sV + sv * C::KV_BYTES + db * ATC_BK * 128, &p.v_map, &v_full[sv], db * 64,
-                      kv_row0 + j * ATC_BK, pol);
-        v_issued |= 1u << sv;
-        v_par = (v_par & ~(1u << sv)) | (phv << sv);
+        issued |= 1u << s;
+        par = (par & ~(1u << s)) | (ph << s);
       }
       // every copy issued here has landed before its buffer is reused or the CTA exits
-      mbar_wait(q_full, 0, p.err);
-      for (int s = 0; s < ATC_KSTAGES; ++s)
-        if ((k_issued >> s) & 1) mbar_wait(&k_full[s], (k_par >> s) & 1, p.err);
-      for (int s = 0; s < ATC_VSTAGES; ++s)
-        if ((v_issued >> s) & 1) mbar_wait(&v_full[s], (v_par >> s) & 1, p.err);
+      if (kl) mbar_wait(q_full, 0, p.err);
+      for (int s = 0; s < NS; ++s)
+        if ((issued >> s) & 1) mbar_wait(&full[s], (par >> s) & 1, p.err);
     }
   } else if (warp == 1) {
     // ------------------------------ MMA issuer ------------------------------
+    // An event loop: each pass issues every S = Q K^T and every O += P V
+    // whose inputs are ready (non-blocking tests), scores first.  A score
+    // tile waits only for its K block and for its warpgroup to have read the
+    // previous scores; a P V product only for its V block and its P.
     if (lane == 0 && nb > 0) {
       constexpr uint32_t IDESC_S = umma_idesc_bf16(ATC_BQ, ATC_BK);             // Q, K both K-major
       constexpr uint32_t IDESC_PV = umma_idesc_bf16(ATC_BQ, D) | (1u << 16);    // V is MN-major
       const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK);
       const uint32_t v_addr = smem_u32(sV), p_addr = smem_u32(sP);
-      // S_q(j) = Q_q K_j^T into tile q's S buffer (freed by the warpgroup for j > 0)
-      auto issue_s = [&](int q, int j) -> bool {
-        if (j > 0 && !mbar_wait(&s_free[q], (j - 1) & 1, p.err)) return false;
-        tc_fence_after();
-        const uint32_t kb = k_addr + (j % ATC_KSTAGES) * C::KV_BYTES, qb = q_addr + q * C::Q_BYTES;
+      bool mok = mbar_wait(q_full, 0, p.err);
+      tc_fence_after();
+      int ns[ATC_NQ] = {0, 0}, np[ATC_NQ] = {0, 0};
+      uint64_t t_idle = globaltimer_ns();
+      while (mok && (np[0] < nb || (nq == 2 && np[1] < nb))) {
+        bool prog = false;
+        for (int q = 0; q < nq; ++q) {
+          const int j = ns[q];
+          if (j < nb && (j == 0 || mbar_try_wait(&s_free[q], (j - 1) & 1)) &&
+              mbar_try_wait(&k_full[j % ATC_KSTAGES], (j / ATC_KSTAGES) & 1)) {
+            tc_fence_after();
+            const uint32_t kb = k_addr + (j % ATC_KSTAGES) * C::KV_BYTES, qb = q_addr + q * C::Q_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t a_at = qb + (kk >> 2) * (ATC_BQ * 128) + (kk & 3) * 32;
-          const uint32_t b_at = kb + (kk >> 2) * (ATC_BK * 128) + (kk & 3) * 32;
-          umma_bf16(tmem_base + C::S_COL + q * ATC_BK, umma_desc_sw128(a_at), umma_desc_sw128(b_at), IDESC_S,
-                    kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t a_at = qb + (kk >> 2) * (ATC_BQ * 128) + (kk & 3) * 32;
+              const uint32_t b_at = kb + (kk >> 2) * (ATC_BK * 128) + (kk & 3) * 32;
+              umma_bf16(tmem_base + C::S_COL + q * ATC_BK, umma_desc_sw128(a_at), umma_desc_sw128(b_at), IDESC_S,
+                        kk > 0 ? 1u : 0u);
+            }
+            umma_commit(&s_full[q]);
+            ns[q] = j + 1;
+            // the K slot is released once every live tile has read block j
+            if (ns[0] > j && (nq < 2 || ns[1] > j)) umma_commit(&k_empty[j % ATC_KSTAGES]);
+            prog = true;
+          }
         }
-        umma_commit(&s_full[q]);
-        return true;
-      };
-      // O_q += P_q(j) V_j
-      auto issue_pv = [&](int q, int j) -> bool {
-        if (!mbar_wait(&p_full[q], j & 1, p.err)) return false;
-        tc_fence_after();
-        const uint32_t vb = v_addr + (j % ATC_VSTAGES) * C::KV_BYTES, pb = p_addr + q * C::P_BYTES;
+        for (int q = 0; q < nq; ++q) {
+          const int j = np[q];
+          if (j < ns[q] && mbar_try_wait(&v_full[j % ATC_VSTAGES], (j / ATC_VSTAGES) & 1) &&
+              mbar_try_wait(&p_full[q], j & 1)) {
+            tc_fence_after();
+            const uint32_t vb = v_addr + (j % ATC_VSTAGES) * C::KV_BYTES, pb = p_addr + q * C::P_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < ATC_BK / 16; ++kk)
-          umma_bf16(tmem_base + C::O_COL + q * D, umma_desc_sw128(pb + kk * 32),
-                    umma_desc_sw128_mn(vb + kk * 2048, ATC_BK * 128), IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(&o_done[q]);
-        return true;
-      };
-      bool mok = mbar_wait(q_full, 0, p.err) && mbar_wait(&k_full[0], 0, p.err);
-      for (int q = 0; q < nq && mok; ++q) mok = issue_s(q, 0);
-      if (mok) umma_commit(&k_empty[0]);
-      // block j + 1's scores are issued before block j's P V products, so the
-      // tensor core works on one tile while the other tile's warpgroup turns
-      // its scores into probabilities
-      for (int j = 0; j < nb && mok; ++j) {
-        if (j + 1 < nb) {
-          const int ks = (j + 1) % ATC_KSTAGES;
-          mok = mbar_wait(&k_full[ks], ((j + 1) / ATC_KSTAGES) & 1, p.err);
-          for (int q = 0; q < nq && mok; ++q) mok = issue_s(q, j + 1);
-          if (mok) umma_commit(&k_empty[ks]);
+            for (int kk = 0; kk < ATC_BK / 16; ++kk)
+              umma_bf16(tmem_base + C::O_COL + q * D, umma_desc_sw128(pb + kk * 32),
+                        umma_desc_sw128_mn(vb + kk * 2048, ATC_BK * 128), IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
+            umma_commit(&o_done[q]);
+            np[q] = j + 1;
+            if (np[0] > j && (nq < 2 || np[1] > j)) umma_commit(&v_empty[j % ATC_VSTAGES]);
+            prog = true;
+          }
         }
-        const int vs = j % ATC_VSTAGES;
-        mok = mok && mbar_wait(&v_full[vs], (j / ATC_VSTAGES) & 1, p.err);
-        for (int q = 0; q < nq && mok; ++q) mok = issue_pv(q, j);
-        if (mok) umma_commit(&v_empty[vs]);
-        if (*abort_flag) mok = false;
+        if (prog) {
+          t_idle = globaltimer_ns();
+        } else if (*abort_flag) {
+          mok = false;
+        } else if (globaltimer_ns() - t_idle > p.err.limit_ns) {
+          raise_error(p.err, ERR_TIMEOUT);
+          mok = false;
+        }
       }
       if (!mok) *abort_flag = 1;
       // every MMA issued has completed before TMEM or its operands are reused
@@ -338,82 +342,141 @@ __global__ void __launch_bounds__(ATC_THREADS, 1) attn_tc_kernel(const __grid_co
   }
 
   // ---------- merge the key chunks of this query block (one cluster) ----------
-  // o = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c, M = max_c m_c: each chunk
-  // scales its own rows into shared memory, then every chunk sums a slice of
-  // the rows over all chunks' tiles (distributed shared memory) and stores it.
+  // o = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c, M = max_c m_c.
   const int nc = p.n_chunks;
   if (warp >= 2) {
-    named_bar_sync(1, 256);  // both tiles' MMAs are complete: the operand region may be reused
+    named_bar_sync(1, 256);  // both tiles' MMAs are complete
     const bool have = wg < nq && nb > 0 && ok;
     if (!have) {
       mref = -INFINITY;
       lsum = 0.f;
     }
-    ml_s[wg * ATC_BQ + rloc] = make_float2(mref, lsum);
   }
-  cluster_sync_all();  // every chunk's (max, sum) is visible
-  if (warp >= 2) {
-    const int row = wg * ATC_BQ + rloc;
-    const uint32_t ml_at = smem_u32(&ml_s[row]);
-    float M = -INFINITY;
-    for (int q = 0; q < nc; ++q) M = fmaxf(M, ld_dsmem_f2(mapa_shared(ml_at, q)).x);
-    const float Mref = M == -INFINITY ? 0.f : M;
-    float den = 0.f;
-    for (int q = 0; q < nc; ++q) {
-      const float2 v = ld_dsmem_f2(mapa_shared(ml_at, q));
-      den += v.y * ex2_approx(v.x - Mref);
-    }
-    const float w = (den > 0.f && mref != -INFINITY) ? ex2_approx(mref - Mref) / den : 0.f;
-    const bool have_o = wg < nq && nb > 0 && __all_sync(0xffffffffu, ok);  // warp-uniform
-#pragma unroll 1
-    for (int c0 = 0; c0 < D; c0 += 16) {
-      float v[16];
-      if (have_o) {
-        tmem_ld16(t_row + C::O_COL + wg * D + c0, v);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 16; ++e) v[e] = 0.f;
-      }
-      float4* dst = reinterpret_cast<float4*>(osm + row * C::OS_LD + c0);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) dst[e] = make_float4(v[4 * e] * w, v[4 * e + 1] * w, v[4 * e + 2] * w, v[4 * e + 3] * w);
-    }
-  }
-  cluster_sync_all();  // every chunk's scaled tile is complete
-  if (warp >= 2) {
-    const int rank = static_cast<int>(cluster_ctarank());
-    const int rpr = (ATC_ROWS + nc - 1) / nc;
-    const int r_lo = rank * rpr, r_hi = min(ATC_ROWS, r_lo + rpr);
-    constexpr int D4 = D / 4;
-    const uint32_t os_at = smem_u32(osm);
-    const int n_items = max(0, r_hi - r_lo) * D4;
-    for (int it = threadIdx.x - 64; it < n_items; it += 256) {
-      const int rr = r_lo + it / D4, c4 = (it % D4) * 4;
-      const uint32_t off = static_cast<uint32_t>((rr * C::OS_LD + c4) * 4);
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      // peers in groups of eight, all loads of a group issued before any is used
-      for (int q0 = 0; q0 < nc; q0 += 8) {
-        float4 v[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u)
-          if (q0 + u < nc) v[u] = ld_dsmem_f4(mapa_shared(os_at + off, q0 + u));
-#pragma unroll
-        for (int u = 0; u < 8; ++u)
-          if (q0 + u < nc) {
-            acc.x += v[u].x;
-            acc.y += v[u].y;
-            acc.z += v[u].z;
-            acc.w += v[u].w;
-          }
-      }
-      const int rg = row_base + rr;
-      if (rg >= rows_total) continue;
+  const bool have_o = warp >= 2 && wg < nq && nb > 0 && __all_sync(0xffffffffu, ok);  // warp-uniform
+  const int row = (warp >= 2) ? wg * ATC_BQ + rloc : 0;
+  if (nc == 1) {
+    // one chunk: normalise and store this thread's row directly
+    if (warp >= 2) {
+      const int rg = row_base + row;
+      const float w = lsum > 0.f ? 1.f / lsum : 0.f;
       const size_t rid = (static_cast<size_t>(b) * p.n + rg / G) * p.Hq + kvh * G + rg % G;
-      *reinterpret_cast<uint2*>(p.o + rid * D + c4) =
-          make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += 16) {
+        float v[16];
+        if (have_o) {
+          tmem_ld16(t_row + C::O_COL + wg * D + c0, v);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) v[e] = 0.f;
+        }
+        if (rg < rows_total) {
+          uint4* dst = reinterpret_cast<uint4*>(p.o + rid * D + c0);
+          dst[0] = make_uint4(pack_bf16x2(v[0] * w, v[1] * w), pack_bf16x2(v[2] * w, v[3] * w),
+                              pack_bf16x2(v[4] * w, v[5] * w), pack_bf16x2(v[6] * w, v[7] * w));
+          dst[1] = make_uint4(pack_bf16x2(v[8] * w, v[9] * w), pack_bf16x2(v[10] * w, v[11] * w),
+                              pack_bf16x2(v[12] * w, v[13] * w), pack_bf16x2(v[14] * w, v[15] * w));
+        }
+      }
+    }
+  } else {
+    // Each chunk writes its raw rows and their (max, sum) to its slot of the
+    // cluster's L2-resident buffer: layout [chunk][D/4][256 rows] float4, so a
+    // warp's store covers 32 consecutive rows (512 contiguous bytes).
+    const int rank = static_cast<int>(cluster_ctarank());
+    const size_t cl = static_cast<size_t>(blockIdx.y) * gridDim.x + blockIdx.x;
+    constexpr int D4 = D / 4;
+    float4* part_cl = reinterpret_cast<float4*>(p.part) + cl * nc * D4 * ATC_ROWS;
+    float2* ml_cl = p.part_ml + cl * nc * ATC_ROWS;
+    if (warp >= 2) {
+      ml_cl[rank * ATC_ROWS + row] = make_float2(have_o ? mref : -INFINITY, have_o ? lsum : 0.f);
+      float4* dst = part_cl + static_cast<size_t>(rank) * D4 * ATC_ROWS + row;
+      auto put16 = [&](int c0, const float* v) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          dst[static_cast<size_t>(c0 / 4 + e) * ATC_ROWS] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2],
+                                                                         v[4 * e + 3]);
+      };
+      int c0 = 0;
+#pragma unroll 1
+      for (; c0 + 32 <= D; c0 += 32) {
+        float v[32];
+        if (have_o) {
+          tmem_ld32(t_row + C::O_COL + wg * D + c0, v);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = 0.f;
+        }
+        put16(c0, v);
+        put16(c0 + 16, v + 16);
+      }
+      if (c0 < D) {  // D is a multiple of 16
+        float v[16];
+        if (have_o) {
+          tmem_ld16(t_row + C::O_COL + wg * D + c0, v);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) v[e] = 0.f;
+        }
+        put16(c0, v);
+      }
+    }
+    // every chunk's rows and statistics are written
+    cluster_sync_all();
+    if (warp >= 2) {
+      // each chunk reduces one slice of the rows over the chunks, in chunk order:
+      // o = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c
+      const int t = threadIdx.x - 64;
+      const int rpr = (ATC_ROWS + nc - 1) / nc;
+      const int r_lo = rank * rpr, n_rows = max(0, min(ATC_ROWS, r_lo + rpr) - r_lo);
+      float* wts = reinterpret_cast<float*>(sQ);  // [row of the slice][chunk]; smem is free after the mainloop
+      if (t < n_rows) {
+        float2 ml[ATC_MAX_CHUNKS];
+#pragma unroll
+        for (int q = 0; q < ATC_MAX_CHUNKS; ++q)
+          if (q < nc) ml[q] = __ldcg(ml_cl + q * ATC_ROWS + r_lo + t);
+        float M = -INFINITY;
+#pragma unroll
+        for (int q = 0; q < ATC_MAX_CHUNKS; ++q)
+          if (q < nc) M = fmaxf(M, ml[q].x);
+        const float Mref = M == -INFINITY ? 0.f : M;
+        float den = 0.f;
+#pragma unroll
+        for (int q = 0; q < ATC_MAX_CHUNKS; ++q)
+          if (q < nc && ml[q].x != -INFINITY) den += ml[q].y * ex2_approx(ml[q].x - Mref);
+#pragma unroll
+        for (int q = 0; q < ATC_MAX_CHUNKS; ++q)
+          if (q < nc)
+            wts[t * ATC_MAX_CHUNKS + q] = (den > 0.f && ml[q].x != -INFINITY) ? ex2_approx(ml[q].x - Mref) / den : 0.f;
+      }
+      named_bar_sync(1, 256);
+      const int n_items = n_rows * D4;
+      for (int it = t; it < n_items; it += 256) {
+        const int rl = it % n_rows, c4 = it / n_rows, rr = r_lo + rl;
+        const float4* src = part_cl + static_cast<size_t>(c4) * ATC_ROWS + rr;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int q0 = 0; q0 < nc; q0 += 8) {
+          float4 v[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            if (q0 + u < nc) v[u] = __ldcg(src + static_cast<size_t>(q0 + u) * D4 * ATC_ROWS);
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            if (q0 + u < nc) {
+              const float wq = wts[rl * ATC_MAX_CHUNKS + q0 + u];
+              acc.x = fmaf(v[u].x, wq, acc.x);
+              acc.y = fmaf(v[u].y, wq, acc.y);
+              acc.z = fmaf(v[u].z, wq, acc.z);
+              acc.w = fmaf(v[u].w, wq, acc.w);
+            }
+        }
+        const int rg = row_base + rr;
+        if (rg >= rows_total) continue;
+        const size_t rid = (static_cast<size_t>(b) * p.n + rg / G) * p.Hq + kvh * G + rg % G;
+        *reinterpret_cast<uint2*>(p.o + rid * D + 4 * c4) =
+            make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+      }
     }
   }
-  cluster_sync_all();  // no CTA leaves while a peer may still read its shared memory
 
   tc_fence_before();
   __syncthreads();

@@ -39,10 +39,13 @@ struct StepGraph {
   cudaGraph_t graph = nullptr;
   cudaGraphExec_t exec = nullptr;
   int B = -1, P = -1;
-  cudaGraphNode_t embed_node = nullptr, lm_node = nullptr, sample_node = nullptr;
-  cudaKernelNodeParams embed_kp{}, lm_kp{}, sample_kp{};
+  cudaGraphNode_t embed_node = nullptr, sample_node = nullptr;
+  std::vector<cudaGraphNode_t> lm_nodes;       // LM-head passes (statistics, then probabilities)
+  cudaKernelNodeParams embed_kp{}, sample_kp{};
+  std::vector<cudaKernelNodeParams> lm_kps;
   std::vector<void*> embed_args, sample_args;
   int64_t launches = 0;
+  bool sc = false;                             // captured with self-conditioning
 };
 
 }  // namespace
@@ -76,6 +79,8 @@ struct dg_ctx {
   int32_t* chunk_done = nullptr;   // finished gate/up tiles per expert token chunk
   int32_t* expert_rows = nullptr;  // [E] rows routed to each expert (dispatch cursors)
   int32_t* moe_work = nullptr;     // claim / exit counters of the expert GEMM
+  float* attn_part = nullptr;      // attention chunk partials (clusters of several chunks): sms x 256 rows x D
+  float2* attn_part_ml = nullptr;  // their row statistics: sms x 256 rows
   int32_t* dense_work = nullptr;   // claim / exit counters of the dense GEMM
   int attn_max_clusters[ATC_MAX_CHUNKS + 1] = {};  // co-resident attention clusters per cluster size
   // CUDA graphs of the denoising step, one per sampler (per batch and cached length)
@@ -94,6 +99,21 @@ struct dg_ctx {
   float* dbg_margin = nullptr;
   float* dbg_entropy = nullptr;
   float* lm_s1 = nullptr;          // LM-head entropy partials [V/128][R_step]
+  // self-conditioning (weights optional): signal of the last step, added to
+  // the next step's embeddings while sc_valid
+  const uint16_t* sc_gate = nullptr;
+  const uint16_t* sc_up = nullptr;
+  const uint16_t* sc_down = nullptr;
+  bool sc_enabled = false, sc_valid = false;
+  bool capturing_graph = false;
+  void* sc_ws = nullptr;
+  uint16_t* sc_P = nullptr;        // [R_step][V] bf16 probabilities of the step
+  float* sc_lse2 = nullptr;        // [R_step] log-sum-exp, log2 units
+  uint16_t* sc_e = nullptr;        // [R_step][d] bf16 p . E
+  float* sc_tmp = nullptr;         // [R_step][F] gate sums
+  uint16_t* sc_h = nullptr;        // [R_step][F] bf16 SwiGLU hidden
+  float* sc_sig = nullptr;         // [R_step][d] the signal
+  CUtensorMap m_embed_mn{}, m_scP64{}, m_scP_store{}, m_sc_e64{}, m_sc_h64{}, m_sc_gate{}, m_sc_up{}, m_sc_down{};
   int32_t* io_canvas_in = nullptr;
   int32_t* io_canvas_out = nullptr;
   float* io_conf = nullptr;
@@ -177,6 +197,20 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// fp32 split-K partials [splits][T][M] as 3-D (M, T, splits), box 128 x 64 x 1,
+// no swizzle: the TMA-store epilogue of the dense GEMM (M a multiple of 4)
+bool make_map_partials(CUtensorMap* m, void* base, int splits, int T, int M) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc || base == nullptr || M % 4) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(M), static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(splits)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(M) * 4, static_cast<cuuint64_t>(T) * M * 4};
+  cuuint32_t box[3] = {128, 64, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Queries [token][Hq][D] seen as 4-D (D, G, Hkv, token): a box of 64 columns x
 // G heads x 1 kv head x 128/G tokens is the 128 packed rows (row = token * G +
 // head) of one GQA group, 128-byte swizzled.  Requires 128 % G == 0.
@@ -243,10 +277,11 @@ struct ProfScope {
 // out[s][t][m] = partial sums over split s of W[m, :] . X[t, :]
 // x: token rows with 64-row TMA boxes
 dg_status gemm_dense(dg_ctx* c, const CUtensorMap& w, const CUtensorMap& x, int M, int T, int K, int* splits_out,
-                     int max_splits = 11) {
+                     int max_splits = 11, bool a_mn_major = false) {
   GemmParams p;
   memset(&p, 0, sizeof(p));
   p.a_map[0] = w;
+  p.a_mn_major = a_mn_major ? 1 : 0;
   p.b_map = x;
   p.b_box_rows = 64;
   p.M = M;
@@ -286,6 +321,7 @@ dg_status gemm_dense(dg_ctx* c, const CUtensorMap& w, const CUtensorMap& x, int 
   p.splits = best_s;
   p.tiles_static = m_tiles * p.n_tiles_n * p.splits;
   p.out_f32 = c->part;
+  p.use_tma_store = make_map_partials(&p.out_map, c->part, p.splits, T, M) ? 1 : 0;
   p.work = c->dense_work;
   p.err = dev_err(c);
   ProfScope ps0(c, DG_PROF_DENSE);
@@ -345,6 +381,8 @@ dg_status attention(dg_ctx* c, int l, int B, int n, int pos0, bool causal) {
   p.k_map = c->lmaps[l].kc;
   p.v_map = c->lmaps[l].vc;
   p.o = c->o;
+  p.part = c->attn_part;
+  p.part_ml = c->attn_part_ml;
   p.n = n;
   p.B = B;
   p.Hq = c->Hq;
@@ -363,7 +401,8 @@ dg_status attention(dg_ctx* c, int l, int B, int n, int pos0, bool causal) {
   // ties: each chunk adds a merge share); one chunk when nothing fits.
   int n_chunks = 1, best_blocks = (keys + ATC_BK - 1) / ATC_BK;
   for (int nc = 2; nc <= ATC_MAX_CHUNKS; ++nc) {
-    if (units > c->attn_max_clusters[nc] || keys < nc * ATC_BK) continue;
+    // the partial buffer holds sms x 256 rows: one slot per CTA of the launch
+    if (units > c->attn_max_clusters[nc] || keys < nc * ATC_BK || units * nc > c->sms) continue;
     const int blocks = ((keys + nc - 1) / nc + ATC_BK - 1) / ATC_BK;
     if (blocks < best_blocks) {
       best_blocks = blocks;
@@ -411,7 +450,8 @@ dg_status moe(dg_ctx* c, int l, int T, bool record) {
   // the experts' regions and the copy of its activations (one warp per token)
   ProfScope ps3(c, DG_PROF_ROUTING);
   // expert e's rows: [e * T, e * T + rows_e) (a region per expert, T rows each)
-  DG_LAUNCH(c, route_dispatch_kernel, (T + 7) / 8, 256, 0, static_cast<const float*>(c->part), s3, T, c->E, c->k,
+  // two tokens (warps) per CTA: the k copies of every token's row spread over many SMs
+  DG_LAUNCH(c, route_dispatch_kernel, (T + 1) / 2, 64, 0, static_cast<const float*>(c->part), s3, T, c->E, c->k,
             c->router_bias, c->idx, c->gates, cap, c->expert_rows, T, c->d, static_cast<const uint16_t*>(c->u),
             c->xp, c->inv_slot);
   ps3.end();
@@ -467,8 +507,10 @@ dg_status forward(dg_ctx* c, const int32_t* tokens, int tok_stride, int tok_off,
   const float eps = c->cfg.rms_eps;
   float* cap0 = (c->capture && !causal) ? c->cap_h : nullptr;
   ProfScope ps8(c, DG_PROF_OTHER);
+  const float* sc_add = (!causal && c->sc_enabled && (c->sc_valid || c->capturing_graph)) ? c->sc_sig : nullptr;
   DG_LAUNCH(c, embed_norm_kernel, T, row_threads(c->d), 0, tokens, tok_stride, tok_off, n, c->embed,
-            static_cast<const uint16_t*>(c->layers[0].attn_norm), eps, c->d, c->h, c->u, cap0, settled, B, c->V);
+            static_cast<const uint16_t*>(c->layers[0].attn_norm), eps, c->d, c->h, c->u, cap0, settled, B, c->V,
+            sc_add);
   ps8.end();
   for (int l = 0; l < c->L; ++l) {
     const LayerMaps& lm = c->lmaps[l];
@@ -505,7 +547,7 @@ dg_status forward(dg_ctx* c, const int32_t* tokens, int tok_stride, int tok_off,
                                              : c->final_norm;
     float* cap = (c->capture && !causal) ? c->cap_h + static_cast<size_t>(l + 1) * c->R_step * c->d : nullptr;
     ProfScope ps11(c, DG_PROF_OTHER);
-    DG_LAUNCH(c, combine_norm_kernel, T, row_threads(c->d), 0, c->h, static_cast<const float*>(c->yp),
+    DG_LAUNCH(c, combine_norm_kernel, T, combine_threads(c->d), 0, c->h, static_cast<const float*>(c->yp),
               static_cast<const int32_t*>(c->inv_slot), static_cast<const float*>(c->gates), c->k, c->E * T,
               c->d, next_gain, eps, c->u, cap);
     ps11.end();
@@ -554,7 +596,61 @@ SampleArgs merge_args(const dg_ctx* c, int T, bool stats_only) {
   a.dbg_margin = c->dbg_margin;
   a.dbg_entropy = c->dbg_entropy;
   a.s1 = c->lm_s1;
+  a.lse2 = c->sc_enabled ? c->sc_lse2 : nullptr;
   return a;
+}
+
+// Self-conditioning signal of this step (codemajin.net "DiffusionGemma
+// architecture", section 3.2): p = softmax(z E^T / T) written as bf16 by a
+// second LM-head pass (the statistics pass gave the log-sum-exp), e = p E by
+// a split-K GEMM with E as an MN-major A operand, then the SwiGLU feed-forward
+// layer; the next step adds the result to its embeddings.
+dg_status self_condition(dg_ctx* c, int T, float temperature) {
+  {
+    GemmParams p;
+    memset(&p, 0, sizeof(p));
+    p.a_map[0] = c->m_u128;
+    p.b_map = c->m_embed;
+    p.b_box_rows = 128;
+    p.M = T;
+    p.k_steps = c->d / 64;
+    p.n_mtiles = (T + GEMM_BM - 1) / GEMM_BM;
+    p.tiles_static = (c->V / GEMM_BN) * p.n_mtiles;
+    p.lse2 = c->sc_lse2;
+    p.p_map = c->m_scP_store;
+    p.logit_scale_log2 = static_cast<float>(1.4426950408889634 / static_cast<double>(temperature));
+    p.err = dev_err(c);
+    ProfScope ps(c, DG_PROF_LMHEAD);
+    DG_LAUNCH(c, gemm_kernel<GEMM_LMHEAD>, std::min(c->sms, p.tiles_static), GEMM_THREADS,
+              gemm_smem_bytes<GEMM_LMHEAD>(), p);
+    ps.end();
+  }
+  int s = 1;
+  dg_status st = gemm_dense(c, c->m_embed_mn, c->m_scP64, c->d, T, c->V, &s, 8, true);
+  if (st != DG_OK) return st;
+  ProfScope ps(c, DG_PROF_OTHER);
+  DG_LAUNCH(c, reduce_splits_kernel, T, row_threads(c->d), 0, static_cast<const float*>(c->part), s, T, c->d,
+            static_cast<float*>(nullptr), c->sc_e);
+  ps.end();
+  st = gemm_dense(c, c->m_sc_gate, c->m_sc_e64, c->F, T, c->d, &s);
+  if (st != DG_OK) return st;
+  ProfScope ps2(c, DG_PROF_OTHER);
+  DG_LAUNCH(c, reduce_splits_kernel, T, row_threads(c->F), 0, static_cast<const float*>(c->part), s, T, c->F,
+            c->sc_tmp, static_cast<uint16_t*>(nullptr));
+  ps2.end();
+  st = gemm_dense(c, c->m_sc_up, c->m_sc_e64, c->F, T, c->d, &s);
+  if (st != DG_OK) return st;
+  ProfScope ps3(c, DG_PROF_OTHER);
+  DG_LAUNCH(c, swiglu_splits_kernel, T, row_threads(c->F), 0, static_cast<const float*>(c->sc_tmp),
+            static_cast<const float*>(c->part), s, T, c->F, c->sc_h);
+  ps3.end();
+  st = gemm_dense(c, c->m_sc_down, c->m_sc_h64, c->d, T, c->F, &s);
+  if (st != DG_OK) return st;
+  ProfScope ps4(c, DG_PROF_OTHER);
+  DG_LAUNCH(c, reduce_splits_kernel, T, row_threads(c->d), 0, static_cast<const float*>(c->part), s, T, c->d,
+            c->sc_sig, static_cast<uint16_t*>(nullptr));
+  ps4.end();
+  return DG_OK;
 }
 
 // threshold sampler: merge of the LM-head statistics + Philox re-noising
@@ -574,6 +670,7 @@ dg_status lm_head_and_sample(dg_ctx* c, int B, int step, uint64_t seed, float ta
   ProfScope ps13(c, DG_PROF_OTHER);
   DG_LAUNCH(c, lmhead_merge_sample_kernel, T, 256, 0, static_cast<const float4*>(c->lm_part), a);
   ps13.end();
+  if (c->sc_enabled) return self_condition(c, T, c->cfg.temperature);
   return DG_OK;
 }
 
@@ -620,6 +717,7 @@ dg_status lm_head_and_entropy_sample(dg_ctx* c, int B, const EntropyCall& e) {
   DG_LAUNCH(c, lmhead_merge_sample_kernel, T, 256, 0, static_cast<const float4*>(c->lm_part), a);
   DG_LAUNCH(c, entropy_sample_kernel, B, 256, 0, entropy_args(c, e));
   ps13.end();
+  if (c->sc_enabled) return self_condition(c, T, e.args.temperature);
   return DG_OK;
 }
 
@@ -680,6 +778,7 @@ dg_status capture_step(dg_ctx* c, int mode) {
   drop_step_graph(sg);
   const int64_t l0 = c->launches;
   DG_CUDA(c, cudaStreamBeginCapture(c->stream, cudaStreamCaptureModeThreadLocal));
+  c->capturing_graph = true;
   dg_status st = forward(c, c->io_canvas_in, c->cfg.canvas, 0, c->B, c->cfg.canvas, c->P, false,
                          mode == SAMPLER_TAU ? c->io_settled : nullptr);
   if (st == DG_OK) {
@@ -692,6 +791,7 @@ dg_status capture_step(dg_ctx* c, int mode) {
       st = lm_head_and_entropy_sample(c, c->B, e);
     }
   }
+  c->capturing_graph = false;
   cudaGraph_t g = nullptr;
   const cudaError_t ce = cudaStreamEndCapture(c->stream, &g);
   if (st != DG_OK || ce != cudaSuccess) {
@@ -716,24 +816,25 @@ dg_status capture_step(dg_ctx* c, int mode) {
       sg.embed_node = nd;
       sg.embed_kp = kp;
     } else if (kp.func == reinterpret_cast<void*>(gemm_kernel<GEMM_LMHEAD>)) {
-      sg.lm_node = nd;
-      sg.lm_kp = kp;
+      sg.lm_nodes.push_back(nd);
+      sg.lm_kps.push_back(kp);
     } else if (kp.func == sampler_fn) {
       sg.sample_node = nd;
       sg.sample_kp = kp;
     }
   }
-  if (!sg.embed_node || !sg.lm_node || !sg.sample_node) {
+  if (!sg.embed_node || sg.lm_nodes.empty() || !sg.sample_node) {
     drop_step_graph(sg);
     return fail(c, DG_ERR_CUDA, "step graph: entry/exit kernels not found");
   }
   // argument pointer arrays: point at the graph's stored values except the rebound ones
-  sg.embed_args.assign(sg.embed_kp.kernelParams, sg.embed_kp.kernelParams + 14);
+  sg.embed_args.assign(sg.embed_kp.kernelParams, sg.embed_kp.kernelParams + 15);
   sg.sample_args.assign(sg.sample_kp.kernelParams, sg.sample_kp.kernelParams + (mode == SAMPLER_TAU ? 2 : 1));
   sg.launches = c->launches - l0;
   c->launches = l0;
   sg.B = c->B;
   sg.P = c->P;
+  sg.sc = c->sc_enabled;
   return DG_OK;
 }
 
@@ -742,9 +843,11 @@ dg_status rebind_embed(dg_ctx* c, StepGraph& sg, const int32_t* canvas_in, int32
   // embed_norm_kernel(tokens, tok_stride, tok_off, n, embed, gain, eps, d, h, u, capture, settled, n_settled, vocab)
   const int32_t* tok = canvas_in;
   int32_t* set0 = settled;
+  const float* add = (c->sc_enabled && c->sc_valid) ? c->sc_sig : nullptr;
   std::vector<void*> ea = sg.embed_args;
   ea[0] = &tok;
   ea[11] = &set0;
+  ea[14] = &add;
   cudaKernelNodeParams ekp = sg.embed_kp;
   ekp.kernelParams = ea.data();
   DG_CUDA(c, cudaGraphExecKernelNodeSetParams(sg.exec, sg.embed_node, &ekp));
@@ -762,7 +865,7 @@ dg_status launch_graph(dg_ctx* c, StepGraph& sg) {
 dg_status step_via_graph(dg_ctx* c, const int32_t* canvas_in, int32_t step, uint64_t seed, float tau,
                          int32_t* canvas_out, float* conf, int32_t* settled) {
   StepGraph& sg = c->graphs[SAMPLER_TAU];
-  if (!sg.exec || sg.B != c->B || sg.P != c->P) {
+  if (!sg.exec || sg.B != c->B || sg.P != c->P || sg.sc != c->sc_enabled) {
     dg_status st = capture_step(c, SAMPLER_TAU);
     if (st != DG_OK) return st;
   }
@@ -789,18 +892,20 @@ dg_status step_via_graph(dg_ctx* c, const int32_t* canvas_in, int32_t step, uint
 // head (temperature) and the entropy sampler (its arguments)
 dg_status entropy_step_via_graph(dg_ctx* c, const int32_t* canvas_in, const EntropyCall& e) {
   StepGraph& sg = c->graphs[SAMPLER_ENTROPY];
-  if (!sg.exec || sg.B != c->B || sg.P != c->P) {
+  if (!sg.exec || sg.B != c->B || sg.P != c->P || sg.sc != c->sc_enabled) {
     dg_status st = capture_step(c, SAMPLER_ENTROPY);
     if (st != DG_OK) return st;
   }
   dg_status st = rebind_embed(c, sg, canvas_in, nullptr);
   if (st != DG_OK) return st;
-  GemmParams lp = *static_cast<GemmParams*>(sg.lm_kp.kernelParams[0]);
-  lp.logit_scale_log2 = static_cast<float>(1.4426950408889634 / static_cast<double>(e.args.temperature));
-  void* la[1] = {&lp};
-  cudaKernelNodeParams lkp = sg.lm_kp;
-  lkp.kernelParams = la;
-  DG_CUDA(c, cudaGraphExecKernelNodeSetParams(sg.exec, sg.lm_node, &lkp));
+  for (size_t i = 0; i < sg.lm_nodes.size(); ++i) {
+    GemmParams lp = *static_cast<GemmParams*>(sg.lm_kps[i].kernelParams[0]);
+    lp.logit_scale_log2 = static_cast<float>(1.4426950408889634 / static_cast<double>(e.args.temperature));
+    void* la[1] = {&lp};
+    cudaKernelNodeParams lkp = sg.lm_kps[i];
+    lkp.kernelParams = la;
+    DG_CUDA(c, cudaGraphExecKernelNodeSetParams(sg.exec, sg.lm_nodes[i], &lkp));
+  }
   EntropyArgs ea = entropy_args(c, e);
   void* sa[1] = {&ea};
   cudaKernelNodeParams skp = sg.sample_kp;
@@ -819,6 +924,8 @@ void free_all(dg_ctx* c) {
   if (c->cap_h) cudaFree(c->cap_h);
   if (c->cap_idx) cudaFree(c->cap_idx);
   if (c->cap_u) cudaFree(c->cap_u);
+  if (c->sc_ws) cudaFree(c->sc_ws);
+  c->sc_ws = nullptr;
   c->ws = nullptr;
   c->kcache = c->vcache = nullptr;
   c->cap_h = nullptr;
@@ -884,6 +991,14 @@ dg_status dg_create(const dg_config* cfg, const dg_weights* w, void* cuda_stream
   if (!aligned16(w->embed)) return reject(DG_ERR_INVALID_ARG, "embed not 16-byte aligned");
   c->embed = static_cast<const uint16_t*>(w->embed);
   c->final_norm = static_cast<const uint16_t*>(w->final_norm);
+  if (w->sc_gate || w->sc_up || w->sc_down) {
+    if (!w->sc_gate || !w->sc_up || !w->sc_down || !aligned16(w->sc_gate) || !aligned16(w->sc_up) ||
+        !aligned16(w->sc_down))
+      return reject(DG_ERR_INVALID_ARG, "self-conditioning weights: all three, 16-byte aligned");
+    c->sc_gate = static_cast<const uint16_t*>(w->sc_gate);
+    c->sc_up = static_cast<const uint16_t*>(w->sc_up);
+    c->sc_down = static_cast<const uint16_t*>(w->sc_down);
+  }
   c->router_bias = w->router_bias;
   c->stream = static_cast<cudaStream_t>(cuda_stream);
   c->d = g.d_model;
@@ -952,6 +1067,8 @@ dg_status dg_create(const dg_config* cfg, const dg_weights* w, void* cuda_stream
   add(c->max_chunks, 4);                          // chunk_done
   add(PERM_MAXE, 4);                              // expert_rows
   add(2, 4);                                      // moe_work
+  add(static_cast<size_t>(c->sms) * ATC_ROWS * c->D, 4);  // attn_part
+  add(static_cast<size_t>(c->sms) * ATC_ROWS, 8);         // attn_part_ml
   add(2, 4);                                      // dense_work
   add(ER * d, 2);                                 // xp
   add(ER * c->F, 2);                              // hbuf
@@ -988,6 +1105,8 @@ dg_status dg_create(const dg_config* cfg, const dg_weights* w, void* cuda_stream
   c->chunk_done = carve<int32_t>(cur, c->max_chunks);
   c->expert_rows = carve<int32_t>(cur, PERM_MAXE);
   c->moe_work = carve<int32_t>(cur, 2);
+  c->attn_part = carve<float>(cur, static_cast<size_t>(c->sms) * ATC_ROWS * c->D);
+  c->attn_part_ml = carve<float2>(cur, static_cast<size_t>(c->sms) * ATC_ROWS);
   c->dense_work = carve<int32_t>(cur, 2);
   c->xp = carve<uint16_t>(cur, ER * d);
   c->hbuf = carve<uint16_t>(cur, ER * c->F);
@@ -1074,6 +1193,33 @@ dg_status dg_create(const dg_config* cfg, const dg_weights* w, void* cuda_stream
   ok &= make_map(&c->m_h16, c->hbuf, ER, c->F, 16);
   ok &= make_map(&c->m_hs16, c->hsbuf, R, c->Fs, 16);
   ok &= make_map(&c->m_embed, c->embed, c->V, d, 128);
+  if (ok && c->sc_gate) {
+    const size_t RS = c->R_step, V = c->V, F = c->F;
+    const size_t sc_bytes = ((RS * V * 2 + 255) / 256 + (RS * 4 + 255) / 256 + (RS * d * 2 + 255) / 256 +
+                             (RS * F * 4 + 255) / 256 + (RS * F * 2 + 255) / 256 + (RS * d * 4 + 255) / 256) * 256;
+    if (cudaMalloc(&c->sc_ws, sc_bytes) != cudaSuccess) {
+      dg_status st = fail(c, DG_ERR_OOM, "self-conditioning buffers %zu bytes", sc_bytes);
+      free_all(c);
+      discard(c);
+      return st;
+    }
+    cudaMemsetAsync(c->sc_ws, 0, sc_bytes, c->stream);
+    char* sc = static_cast<char*>(c->sc_ws);
+    c->sc_P = carve<uint16_t>(sc, RS * V);
+    c->sc_lse2 = carve<float>(sc, RS);
+    c->sc_e = carve<uint16_t>(sc, RS * d);
+    c->sc_tmp = carve<float>(sc, RS * F);
+    c->sc_h = carve<uint16_t>(sc, RS * F);
+    c->sc_sig = carve<float>(sc, RS * d);
+    ok &= make_map(&c->m_embed_mn, c->embed, c->V, d, 64);      // E as [V][d]: A of p . E, MN-major
+    ok &= make_map(&c->m_scP64, c->sc_P, RS, V, 64);             // p as the B operand
+    ok &= make_map(&c->m_scP_store, c->sc_P, RS, V, 128);        // p stored by the LM-head pass
+    ok &= make_map(&c->m_sc_e64, c->sc_e, RS, d, 64);
+    ok &= make_map(&c->m_sc_h64, c->sc_h, RS, F, 64);
+    ok &= make_map(&c->m_sc_gate, c->sc_gate, F, d, 128);
+    ok &= make_map(&c->m_sc_up, c->sc_up, F, d, 128);
+    ok &= make_map(&c->m_sc_down, c->sc_down, d, F, 128);
+  }
   if (!ok) {
     dg_status st = fail(c, DG_ERR_CUDA, "cuTensorMapEncodeTiled failed");
     free_all(c);
@@ -1100,6 +1246,7 @@ dg_status dg_prefill(dg_ctx* c, const int32_t* tokens, int32_t B, int32_t P) {
   c->B = B;
   c->P = 0;
   c->prefilled = false;
+  c->sc_valid = false;  // a new canvas starts without a self-conditioning signal
   const int chunk = std::max(1, c->R / B);
   for (int p0 = 0; p0 < P; p0 += chunk) {
     const int n = std::min(chunk, P - p0);
@@ -1117,12 +1264,16 @@ dg_status dg_denoise_step(dg_ctx* c, const int32_t* canvas_in, int32_t step, uin
   if (!canvas_in || !canvas_out || !conf) return fail(c, DG_ERR_INVALID_ARG, "step: null buffer");
   if (!c->prefilled) return fail(c, DG_ERR_STATE, "step before prefill");
   if (c->P + c->cfg.canvas > c->cfg.max_seq) return fail(c, DG_ERR_CAPACITY, "step: cache full");
+  dg_status st;
   // test hooks (capture, profiling) need the eager launches
-  if (c->use_graphs && !c->capture && c->prof_mask == 0 && c->stream != nullptr)
-    return step_via_graph(c, canvas_in, step, seed, tau, canvas_out, conf, settled);
-  dg_status st = forward(c, canvas_in, c->cfg.canvas, 0, c->B, c->cfg.canvas, c->P, false, settled);
-  if (st != DG_OK) return st;
-  return lm_head_and_sample(c, c->B, step, seed, tau, canvas_out, conf, settled);
+  if (c->use_graphs && !c->capture && c->prof_mask == 0 && c->stream != nullptr) {
+    st = step_via_graph(c, canvas_in, step, seed, tau, canvas_out, conf, settled);
+  } else {
+    st = forward(c, canvas_in, c->cfg.canvas, 0, c->B, c->cfg.canvas, c->P, false, settled);
+    if (st == DG_OK) st = lm_head_and_sample(c, c->B, step, seed, tau, canvas_out, conf, settled);
+  }
+  if (st == DG_OK && c->sc_enabled) c->sc_valid = true;
+  return st;
 }
 
 dg_status dg_denoise_step_entropy(dg_ctx* c, const int32_t* canvas_in, int32_t step, uint64_t seed,
@@ -1135,11 +1286,15 @@ dg_status dg_denoise_step_entropy(dg_ctx* c, const int32_t* canvas_in, int32_t s
   if (!c->prefilled) return fail(c, DG_ERR_STATE, "step before prefill");
   if (c->P + c->cfg.canvas > c->cfg.max_seq) return fail(c, DG_ERR_CAPACITY, "step: cache full");
   EntropyCall e{step, seed, *args, prev_argmax, argmax_out, canvas_out, entropy, stopped};
-  if (c->use_graphs && !c->capture && c->prof_mask == 0 && c->stream != nullptr)
-    return entropy_step_via_graph(c, canvas_in, e);
-  dg_status st = forward(c, canvas_in, c->cfg.canvas, 0, c->B, c->cfg.canvas, c->P, false, nullptr);
-  if (st != DG_OK) return st;
-  return lm_head_and_entropy_sample(c, c->B, e);
+  dg_status st;
+  if (c->use_graphs && !c->capture && c->prof_mask == 0 && c->stream != nullptr) {
+    st = entropy_step_via_graph(c, canvas_in, e);
+  } else {
+    st = forward(c, canvas_in, c->cfg.canvas, 0, c->B, c->cfg.canvas, c->P, false, nullptr);
+    if (st == DG_OK) st = lm_head_and_entropy_sample(c, c->B, e);
+  }
+  if (st == DG_OK && c->sc_enabled) c->sc_valid = true;
+  return st;
 }
 
 dg_status dg_denoise_step_host(dg_ctx* c, const int32_t* canvas_in_host, int32_t step, uint64_t seed, float tau,
@@ -1168,6 +1323,7 @@ dg_status dg_commit_block(dg_ctx* c, const int32_t* block) {
   dg_status st = forward(c, block, c->cfg.canvas, 0, c->B, c->cfg.canvas, c->P, true, nullptr);
   if (st != DG_OK) return st;
   c->P += c->cfg.canvas;
+  c->sc_valid = false;  // the next block starts without a self-conditioning signal
   return DG_OK;
 }
 
@@ -1288,6 +1444,21 @@ dg_status dg_debug_entropy_sample(dg_ctx* c, const int32_t* argmax, const float*
   return DG_OK;
 }
 
+dg_status dg_set_self_conditioning(dg_ctx* c, int32_t enable) {
+  if (!c) return DG_ERR_INVALID_ARG;
+  if (enable && !c->sc_ws) return fail(c, DG_ERR_UNSUPPORTED, "self-conditioning needs sc_gate/sc_up/sc_down");
+  c->sc_enabled = enable != 0;
+  c->sc_valid = false;
+  return DG_OK;
+}
+
+dg_status dg_debug_self_cond(dg_ctx* c, float* out) {
+  if (!c || !out || !c->sc_ws) return fail(c, DG_ERR_INVALID_ARG, "debug_self_cond");
+  DG_CUDA(c, cudaMemcpyAsync(out, c->sc_sig, static_cast<size_t>(c->B) * c->cfg.canvas * c->d * 4,
+                             cudaMemcpyDeviceToDevice, c->stream));
+  return DG_OK;
+}
+
 dg_status dg_debug_entropy(dg_ctx* c, float* out) {
   if (!c || !out) return fail(c, DG_ERR_INVALID_ARG, "debug_entropy");
   DG_CUDA(c, cudaMemcpyAsync(out, c->dbg_entropy, static_cast<size_t>(c->B) * c->cfg.canvas * 4,
@@ -1321,6 +1492,7 @@ dg_status dg_debug_gemm(dg_ctx* c, const void* w, int32_t M, int32_t K, const vo
   p.tiles_static = ((M + GEMM_BM - 1) / GEMM_BM) * p.n_tiles_n * splits;
   if (M % 4) return fail(c, DG_ERR_INVALID_ARG, "debug_gemm: M must be a multiple of 4");
   p.out_f32 = out;
+  p.use_tma_store = make_map_partials(&p.out_map, out, splits, T, M) ? 1 : 0;
   p.work = c->dense_work;
   p.err = dev_err(c);
   gemm_kernel<GEMM_DENSE><<<std::min(c->sms, p.tiles_static), GEMM_THREADS, gemm_smem_bytes<GEMM_DENSE>(),

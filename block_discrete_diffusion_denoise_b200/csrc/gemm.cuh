@@ -92,6 +92,7 @@ struct GemmParams {
   // copy each, the rest in b_box_rows boxes (fewer copies measured faster;
   // 128-row boxes measured slower than two 64-row ones)
   CUtensorMap b_mid_map, bs_mid_map, h_mid_map, hs_mid_map;
+  CUtensorMap out_map;    // DENSE: fp32 partials as 3-D (M, T, splits), box (128, 64, 1); see use_tma_store
   int b_box_rows;         // rows per B box (16 MOE, 64 DENSE, 128 LM head)
   int b_mid_rows;         // 0 = none (64 MOE)
   int M;                  // DENSE: output features; LMHEAD: tokens
@@ -102,6 +103,12 @@ struct GemmParams {
   int bn;                 // DENSE token tile
   int n_mtiles;           // LMHEAD token tiles
   int tiles_static;       // DENSE / LMHEAD tile count
+  int use_tma_store;      // DENSE: a CTA's last tile is staged in the operand ring and stored by TMA
+  int a_mn_major;         // DENSE: A stored [K][M] (M contiguous), read as two [64 k][64 m] boxes per stage
+  // LMHEAD, probability mode: write p = 2^(x - lse2[token]) as bf16 [T][V]
+  // (via p_map, box 64 x 128, 128-byte swizzle) instead of the statistics
+  const float* lse2;      // per-token log-sum-exp in log2 units, or NULL (statistics mode)
+  CUtensorMap p_map;
   // DENSE, MOE: claimed tiles
   int* work;              // [0] claim counter, [1] exit counter; zero at launch, reset by the last CTA
   // MOE
@@ -488,9 +495,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
       int cur = -1, claim = 0, dep_hint = 0;
       int4 cur_rec = make_int4(0, 0, 0, 0);
       if constexpr (claims_tiles<MODE>()) {
-        cur = atomicAdd(p.work, 1);
+        // the first tile of every CTA is its own index; later tiles are
+        // claimed from the counter, which numbers the tiles after those
+        cur = blockIdx.x;
         if (cur < n_tiles) cur_rec = moe_record(p, tb, cur);
-        claim = atomicAdd(p.work, 1);
+        claim = static_cast<int>(gridDim.x) + atomicAdd(p.work, 1);
       }
       for (int it = 0;; ++it) {
         int tile;
@@ -502,7 +511,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
           if (cur >= 0 && claim < n_tiles) {
             nxt = claim;
             nxt_rec = moe_record(p, tb, nxt);  // consumed in the next iteration
-            claim = atomicAdd(p.work, 1);
+            claim = static_cast<int>(gridDim.x) + atomicAdd(p.work, 1);
           }
           tile = cur;
           rec = cur_rec;
@@ -549,8 +558,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
           uint8_t* a = sA + stage * GEMM_A_BYTES;
           uint8_t* b = sB + stage * B_BYTES;
           const int kx = (t.k0 + k) * GEMM_BK;
-          tma_load_2d(a, t.a0, &full[stage], kx, t.a_row, pol_a);
-          if (t.a1 != nullptr) tma_load_2d(a + GEMM_A_BYTES / 2, t.a1, &full[stage], kx, t.a_row, pol_a);
+          if (MODE == GEMM_DENSE && p.a_mn_major) {
+            // A stored [K][M]: two boxes of 64 k-rows x 64 m-columns
+            tma_load_2d(a, t.a0, &full[stage], t.a_row, kx, pol_a);
+            tma_load_2d(a + GEMM_A_BYTES / 2, t.a0, &full[stage], t.a_row + 64, kx, pol_a);
+          } else {
+            tma_load_2d(a, t.a0, &full[stage], kx, t.a_row, pol_a);
+            if (t.a1 != nullptr) tma_load_2d(a + GEMM_A_BYTES / 2, t.a1, &full[stage], kx, t.a_row, pol_a);
+          }
           int r = 0;
           if (p.b_mid_rows > 0)
             for (; r + p.b_mid_rows <= t.nmma; r += p.b_mid_rows)
@@ -615,18 +630,28 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
-        const uint32_t idesc = umma_idesc_bf16(GEMM_BM, t.nmma);
+        const bool a_mn = MODE == GEMM_DENSE && p.a_mn_major;
+        const uint32_t idesc = umma_idesc_bf16(GEMM_BM, t.nmma) | (a_mn ? (1u << 15) : 0u);
         for (int k = 0; k < t.nk; ++k) {
           if (!mbar_wait(&full[stage], phase, p.err)) {
             aborted = true;
             break;
           }
           tc_fence_after();
-          const uint64_t ad = umma_desc_sw128(smem_u32(sA + stage * GEMM_A_BYTES));
+          const uint32_t a_at = smem_u32(sA + stage * GEMM_A_BYTES);
           const uint64_t bd = umma_desc_sw128(smem_u32(sB + stage * B_BYTES));
+          if (a_mn) {
+            // MN-major A: 16 k-rows are 2048 bytes; the two 64-wide m blocks are GEMM_A_BYTES / 2 apart
 #pragma unroll
-          for (int kk = 0; kk < GEMM_BK / 16; ++kk)
-            umma_bf16(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (k | kk) != 0);
+            for (int kk = 0; kk < GEMM_BK / 16; ++kk)
+              umma_bf16(d_tmem, umma_desc_sw128_mn(a_at + kk * 2048, GEMM_A_BYTES / 2), bd + 2 * kk, idesc,
+                        (k | kk) != 0);
+          } else {
+            const uint64_t ad = umma_desc_sw128(a_at);
+#pragma unroll
+            for (int kk = 0; kk < GEMM_BK / 16; ++kk)
+              umma_bf16(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (k | kk) != 0);
+          }
           umma_commit(&empty[stage]);
           if (++stage == STAGES) {
             stage = 0;
@@ -690,6 +715,27 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
       if constexpr (MODE == GEMM_DENSE) {
         float* out = p.out_f32 + static_cast<size_t>(t.split) * p.T * p.M +
                      static_cast<size_t>(t.b_row) * p.M + t.a_row;
+        if (p.use_tma_store && tile + static_cast<int>(gridDim.x) >= n_tiles) {
+          // this CTA's last tile: every operand load has been consumed by the
+          // MMAs this accumulator waited for, so the ring is free.  Stage the
+          // tile as [token][128 features] fp32 (a warp writes 128 contiguous
+          // bytes per token) and store it with TMA, 64 tokens per box.
+          float* stage = reinterpret_cast<float*>(sA);
+          for (int c0 = 0; c0 < t.n; c0 += 64) {
+            float v[64];
+            tmem_ld64(tbase + c0, v);
+#pragma unroll
+            for (int i = 0; i < 64; ++i) stage[(c0 + i) * GEMM_BM + row] = v[i];
+          }
+          fence_proxy_async_smem();
+          named_bar_sync(1, 128);
+          if (etid == 0) {
+            for (int c0 = 0; c0 < t.n; c0 += 64)
+              tma_store_3d(&p.out_map, stage + c0 * GEMM_BM, t.a_row, t.b_row + c0, t.split);
+            bulk_commit_group();
+            bulk_wait_all();
+          }
+        } else
         for (int c0 = 0; c0 < t.n; c0 += 64) {
           float v[64];
           tmem_ld64(tbase + c0, v);
@@ -747,6 +793,38 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
                                     min(32, t.n - c0 - 32 * h), GEMM_BM);
           }
         }
+      } else if (p.lse2 != nullptr) {  // GEMM_LMHEAD, probability mode
+        // the previous tile's store must have read the staging area
+        if (etid == 0) bulk_wait_read_all();
+        named_bar_sync(1, 128);
+        const int tok = t.a_row + row;
+        const float ref = tok < p.M ? p.lse2[tok] : 0.f;
+        uint8_t* stg = reinterpret_cast<uint8_t*>(xchg);
+        for (int c0 = 0; c0 < GEMM_BN; c0 += 32) {
+          float v[32];
+          tmem_ld32(tbase + c0, v);
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            pk[i] = pack_bf16x2(exp2f(fmaf(v[2 * i], p.logit_scale_log2, -ref)),
+                                exp2f(fmaf(v[2 * i + 1], p.logit_scale_log2, -ref)));
+          // two [128 rows][64 cols] boxes, 128-byte swizzle: 16-byte chunk ch of
+          // row r sits at chunk (ch ^ (r & 7)) of the row
+          const int box = c0 >> 6;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int ch = ((c0 & 63) >> 3) + q;
+            *reinterpret_cast<uint4*>(stg + box * (GEMM_BM * 128) + row * 128 + ((ch ^ (row & 7)) << 4)) =
+                make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+          }
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        if (etid == 0) {
+          tma_store_2d(&p.p_map, stg, t.b_row, t.a_row);
+          tma_store_2d(&p.p_map, stg + GEMM_BM * 128, t.b_row + 64, t.a_row);
+          bulk_commit_group();
+        }
       } else {  // GEMM_LMHEAD
         const int tok = t.a_row + row;
         float m1 = -INFINITY, m2 = -INFINITY, s = 0.f, s1 = 0.f;
@@ -782,6 +860,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
     }
   }
 
+  if (MODE == GEMM_LMHEAD && p.lse2 != nullptr && threadIdx.x == 64) bulk_wait_all();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

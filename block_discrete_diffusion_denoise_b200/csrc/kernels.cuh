@@ -223,53 +223,82 @@ __device__ __forceinline__ void norm_store_row(float4 x, float4 g, bool valid, i
 }
 
 // h[t] += y_shared[t] + sum_j gate[t][j] * y[inv_slot[t][j]] (in that order);
-// u = RMSNorm(h) * gain
-__global__ void __launch_bounds__(1024) combine_norm_kernel(
+// u = RMSNorm(h) * gain.  blockDim = combine_threads(d): two float4 of the row
+// per thread (so several CTAs share an SM and one wave covers the rows), the
+// slots' loads issued four slots at a time.
+__host__ __device__ constexpr int combine_threads(int d) { return ((d / 8 + 31) / 32) * 32; }
+
+__global__ void __launch_bounds__(512) combine_norm_kernel(
     float* __restrict__ h, const float* __restrict__ yp, const int32_t* __restrict__ inv_slot,
     const float* __restrict__ gates, int k, int shared_base, int d, const uint16_t* __restrict__ gain, float eps,
     uint16_t* __restrict__ u, float* __restrict__ capture) {
   __shared__ float red[32];
   __shared__ int slot[ROW_MAX_K];
   __shared__ float gw[ROW_MAX_K];
-  const int row = blockIdx.x, c = threadIdx.x;
-  const bool valid = c < d / 4;
+  const int row = blockIdx.x, nv = d / 4;
+  const int c0 = threadIdx.x, c1 = threadIdx.x + blockDim.x;
+  const bool v0 = c0 < nv, v1 = c1 < nv;
   float4* hrow = reinterpret_cast<float4*>(h + static_cast<size_t>(row) * d);
-  float4 x = make_float4(0.f, 0.f, 0.f, 0.f), ys = x, g = x;
-  if (valid) {
-    x = hrow[c];
-    ys = reinterpret_cast<const float4*>(yp + static_cast<size_t>(shared_base + row) * d)[c];
-    g = load_bf16x4(gain + 4 * c);
+  const float4* ys = reinterpret_cast<const float4*>(yp + static_cast<size_t>(shared_base + row) * d);
+  const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+  float4 x0 = z, x1 = z, s0 = z, s1 = z;
+  if (v0) {
+    x0 = hrow[c0];
+    s0 = ys[c0];
+  }
+  if (v1) {
+    x1 = hrow[c1];
+    s1 = ys[c1];
   }
   if (threadIdx.x < k) {
     slot[threadIdx.x] = inv_slot[static_cast<size_t>(row) * k + threadIdx.x];
     gw[threadIdx.x] = gates[static_cast<size_t>(row) * k + threadIdx.x];
   }
   __syncthreads();
-  if (valid) {
-    x = f4_add(x, ys);
-    // slots in batches of eight, the batch's loads issued before its sums
-    for (int s0 = 0; s0 < k; s0 += 8) {
-      float4 y[8];
+  x0 = f4_add(x0, s0);
+  x1 = f4_add(x1, s1);
+  for (int q0 = 0; q0 < k; q0 += 4) {
+    float4 y0[4], y1[4];
 #pragma unroll
-      for (int s = 0; s < 8; ++s)
-        if (s0 + s < k) y[s] = reinterpret_cast<const float4*>(yp + static_cast<size_t>(slot[s0 + s]) * d)[c];
+    for (int q = 0; q < 4; ++q)
+      if (q0 + q < k) {
+        const float4* yr = reinterpret_cast<const float4*>(yp + static_cast<size_t>(slot[q0 + q]) * d);
+        if (v0) y0[q] = yr[c0];
+        if (v1) y1[q] = yr[c1];
+      }
 #pragma unroll
-      for (int s = 0; s < 8; ++s)
-        if (s0 + s < k) x = f4_fma(gw[s0 + s], y[s], x);
-    }
-    hrow[c] = x;
-    if (capture) reinterpret_cast<float4*>(capture + static_cast<size_t>(row) * d)[c] = x;
+    for (int q = 0; q < 4; ++q)
+      if (q0 + q < k) {
+        if (v0) x0 = f4_fma(gw[q0 + q], y0[q], x0);
+        if (v1) x1 = f4_fma(gw[q0 + q], y1[q], x1);
+      }
   }
-  norm_store_row(x, g, valid, d, eps, u + static_cast<size_t>(row) * d, red);
+  float4 g0 = z, g1 = z;
+  if (v0) {
+    hrow[c0] = x0;
+    if (capture) reinterpret_cast<float4*>(capture + static_cast<size_t>(row) * d)[c0] = x0;
+    g0 = load_bf16x4(gain + 4 * c0);
+  }
+  if (v1) {
+    hrow[c1] = x1;
+    if (capture) reinterpret_cast<float4*>(capture + static_cast<size_t>(row) * d)[c1] = x1;
+    g1 = load_bf16x4(gain + 4 * c1);
+  }
+  const float ss = block_sum((v0 ? f4_sumsq(x0) : 0.f) + (v1 ? f4_sumsq(x1) : 0.f), red);
+  const float r = rsqrtf(ss / d + eps);
+  uint16_t* urow = u + static_cast<size_t>(row) * d;
+  if (v0) store_bf16x4(urow + 4 * c0, make_float4(x0.x * r * g0.x, x0.y * r * g0.y, x0.z * r * g0.z, x0.w * r * g0.w));
+  if (v1) store_bf16x4(urow + 4 * c1, make_float4(x1.x * r * g1.x, x1.y * r * g1.y, x1.z * r * g1.z, x1.w * r * g1.w));
 }
 
 // Embedding gather (bf16 -> fp32 residual) + RMSNorm -> bf16.
 // Token of row b*n+i: tokens[b * tok_stride + tok_off + i]; ids outside the
-// vocabulary are clamped into it rather than read out of bounds.
+// vocabulary are clamped into it rather than read out of bounds.  add [rows, d]
+// fp32 or NULL is added to the embedding (the self-conditioning signal).
 __global__ void __launch_bounds__(1024) embed_norm_kernel(
     const int32_t* __restrict__ tokens, int tok_stride, int tok_off, int n, const uint16_t* __restrict__ embed,
     const uint16_t* __restrict__ gain, float eps, int d, float* __restrict__ h, uint16_t* __restrict__ u,
-    float* __restrict__ capture, int32_t* settled, int n_settled, int vocab) {
+    float* __restrict__ capture, int32_t* settled, int n_settled, int vocab, const float* __restrict__ add) {
   __shared__ float red[32];
   const int row = blockIdx.x, c = threadIdx.x;
   const int b = row / n, i = row % n;
@@ -280,6 +309,7 @@ __global__ void __launch_bounds__(1024) embed_norm_kernel(
   if (valid) {
     g = load_bf16x4(gain + 4 * c);
     x = load_bf16x4(embed + static_cast<size_t>(tok) * d + 4 * c);
+    if (add) x = f4_add(x, reinterpret_cast<const float4*>(add + static_cast<size_t>(row) * d)[c]);
     reinterpret_cast<float4*>(h + static_cast<size_t>(row) * d)[c] = x;
     if (capture) reinterpret_cast<float4*>(capture + static_cast<size_t>(row) * d)[c] = x;
   }
@@ -308,6 +338,49 @@ __global__ void __launch_bounds__(1024) residual_norm_kernel(
     hrow[c] = x;
   }
   norm_store_row(x, g, valid, d, eps, u + static_cast<size_t>(row) * d, red);
+}
+
+// Self-conditioning helpers (one CTA per row, one float4 per thread):
+//   reduce_splits: out = sum_s part[s][row] (splits in order) as fp32 and / or bf16
+//   swiglu_splits: out = SiLU(a[row]) * sum_s part[s][row], bf16 (a: the gate sums)
+__global__ void __launch_bounds__(1024) reduce_splits_kernel(const float* __restrict__ part, int splits, int T,
+                                                             int width, float* __restrict__ out_f32,
+                                                             uint16_t* __restrict__ out_bf16) {
+  const int row = blockIdx.x, c = threadIdx.x;
+  if (c >= width / 4) return;
+  float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s0 = 0; s0 < splits; s0 += 4) {
+    float4 a[4];
+#pragma unroll
+    for (int s = 0; s < 4; ++s)
+      if (s0 + s < splits) a[s] = reinterpret_cast<const float4*>(part + (static_cast<size_t>(s0 + s) * T + row) * width)[c];
+#pragma unroll
+    for (int s = 0; s < 4; ++s)
+      if (s0 + s < splits) x = f4_add(x, a[s]);
+  }
+  if (out_f32) reinterpret_cast<float4*>(out_f32 + static_cast<size_t>(row) * width)[c] = x;
+  if (out_bf16) store_bf16x4(out_bf16 + static_cast<size_t>(row) * width + 4 * c, x);
+}
+
+__global__ void __launch_bounds__(1024) swiglu_splits_kernel(const float* __restrict__ gate, const float* __restrict__ part,
+                                                             int splits, int T, int width,
+                                                             uint16_t* __restrict__ out_bf16) {
+  const int row = blockIdx.x, c = threadIdx.x;
+  if (c >= width / 4) return;
+  const float4 g = reinterpret_cast<const float4*>(gate + static_cast<size_t>(row) * width)[c];
+  float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s0 = 0; s0 < splits; s0 += 4) {
+    float4 a[4];
+#pragma unroll
+    for (int s = 0; s < 4; ++s)
+      if (s0 + s < splits) a[s] = reinterpret_cast<const float4*>(part + (static_cast<size_t>(s0 + s) * T + row) * width)[c];
+#pragma unroll
+    for (int s = 0; s < 4; ++s)
+      if (s0 + s < splits) x = f4_add(x, a[s]);
+  }
+  const auto silu = [](float v) { return v / (1.f + __expf(-v)); };
+  store_bf16x4(out_bf16 + static_cast<size_t>(row) * width + 4 * c,
+               make_float4(silu(g.x) * x.x, silu(g.y) * x.y, silu(g.z) * x.z, silu(g.w) * x.w));
 }
 
 // Reduce the QKV split-K partials (splits in order), rotate q and k pairs
@@ -456,6 +529,7 @@ struct SampleArgs {
   float* dbg_margin;
   float* dbg_entropy;
   const float* s1;         // entropy partials [vocab tiles][T] or NULL
+  float* lse2;             // log-sum-exp in log2 units [T] or NULL (self-conditioning)
 };
 
 __device__ __forceinline__ int sample_decision(int argmax, float conf, float tau, int pos, int step, int seq,
@@ -486,6 +560,7 @@ __global__ void lmhead_merge_sample_kernel(const float4* __restrict__ part, Samp
     if (a.dbg_conf) a.dbg_conf[t] = conf;
     if (a.dbg_margin) a.dbg_margin[t] = margin;
     if (a.dbg_entropy && a.s1) a.dbg_entropy[t] = merged_entropy(acc);
+    if (a.lse2) a.lse2[t] = acc.m1 + log2f(acc.s);
   }
 }
 

@@ -103,12 +103,17 @@ typedef struct dg_layer_weights {
 /* Model weights.  embed [V, d] bf16 is also the (tied) LM head.  router_bias
  * [E] fp32 device pointer or NULL is added to every layer's router logits
  * before top-k.  layers points to a HOST array of n_layers entries that is
- * read during dg_create only. */
+ * read during dg_create only.  sc_gate, sc_up [F, d] and sc_down [d, F] bf16
+ * (F = expert_hidden) are the feed-forward layer of the self-conditioning
+ * signal (dg_set_self_conditioning), or all NULL. */
 typedef struct dg_weights {
   const void* embed;
   const void* final_norm;
   const float* router_bias;
   const dg_layer_weights* layers;
+  const void* sc_gate;
+  const void* sc_up;
+  const void* sc_down;
 } dg_weights;
 
 /* Create a context: validates cfg, allocates the KV cache
@@ -188,6 +193,17 @@ dg_status dg_denoise_step_host(dg_ctx* ctx, const int32_t* canvas_in_host, int32
                                uint64_t seed, float tau, int32_t* canvas_out_host,
                                float* conf_host, int32_t* all_settled_host);
 
+/* Self-conditioning (codemajin.net "DiffusionGemma architecture", section
+ * 3.2): with enable = 1 every denoising step (either sampler) also computes,
+ * from its LM head, the predicted clean-token distribution p = softmax(z E^T
+ * / T), passes it through the embedding matrix (p E) and the SwiGLU layer of
+ * sc_gate / sc_up / sc_down, and the next step adds the result to its input
+ * embeddings.  The first step after dg_prefill, dg_commit_block or this call
+ * has no signal to add.  The step then also writes p as bf16 to a context
+ * buffer ([batch*canvas, vocab]; the one place probabilities reach memory).
+ * DG_ERR_UNSUPPORTED when the context was created without those weights. */
+dg_status dg_set_self_conditioning(dg_ctx* ctx, int32_t enable);
+
 /* Block commit (codemajin.net section 3.2 block-AR; section 5.1 counts it as
  * one extra forward per block): one causal forward of block_dev
  * [batch, canvas] int32 at positions [P, P+canvas), appending its keys/values
@@ -252,6 +268,9 @@ dg_status dg_debug_sample(dg_ctx* ctx, const int32_t* argmax_dev, const float* c
 dg_status dg_debug_entropy_sample(dg_ctx* ctx, const int32_t* argmax_dev, const float* entropy_dev,
                                   const int32_t* prev_argmax_dev, int32_t batch, int32_t step, uint64_t seed,
                                   float gamma, float stop_entropy, int32_t* out_dev, int32_t* stopped_dev);
+
+/* Self-conditioning signal computed by the last step, [batch*canvas, d] fp32. */
+dg_status dg_debug_self_cond(dg_ctx* ctx, float* out_dev);
 
 /* Softmax entropy (nats) per position of the last step [batch*canvas]. */
 dg_status dg_debug_entropy(dg_ctx* ctx, float* out_dev);
