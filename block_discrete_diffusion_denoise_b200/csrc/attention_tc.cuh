@@ -10,10 +10,10 @@
 // so each K/V block feeds all of them; the 256 rows are two 128-row query
 // tiles, each pulled by one 4-D TMA box out of the [token][head][D] query
 // layout, and every K/V block is read once for both.  The key chunks of one
-// query block form a thread-block cluster: each writes its raw rows and row
-// statistics to an L2-resident buffer, and after one cluster barrier each
-// reduces a slice of the rows over the chunks; a single chunk writes its rows
-// directly.
+// query block form a thread-block cluster: each stores its raw rows (one
+// bulk copy) and row statistics to an L2-resident buffer, and after one
+// cluster barrier each bulk-loads its slice of the rows from every chunk and
+// reduces it; a single chunk writes its rows directly.
 //
 // Warp 0 issues TMA loads (lane 0: both Q tiles once, then 64-key K blocks;
 // lane 1: V blocks; 2-deep rings).  Warp 1 issues tcgen05.mma: S_q = Q_q K^T into tile q's TMEM
@@ -49,7 +49,7 @@ struct AttnTcParams {
   CUtensorMap k_map;   // 2-D (D, B*Hkv*S_max) over this layer's K cache; box (64, 64)
   CUtensorMap v_map;   // same over V
   uint16_t* o;         // [token][Hq][D]
-  float* part;         // several key chunks: [cluster][chunk][D/4][256 rows] float4 raw rows (L2-resident)
+  float* part;         // several key chunks: [cluster][chunk][slice][D/4][rows of the slice] float4 raw rows
   float2* part_ml;     // [cluster][chunk][256 rows] (max, sum) of those rows
   int n, B, Hq, Hkv, S_max, pos0, causal, chunk_len, n_chunks;
   float scale_log2;    // log2(e) / sqrt(D)
@@ -70,6 +70,9 @@ struct AtcCfg {
   static constexpr int SMEM = 1024 + REGION + TAIL;
   static_assert(O_COL + ATC_NQ * D <= 512, "S and O accumulators must fit TMEM");
   static_assert(D % 16 == 0 && D <= 256, "head_dim must be a multiple of 16, at most 256");
+  // chunk merge: a chunk's rows (at most 256 + 15 with the slice rounding) and the weight table
+  static_assert((ATC_ROWS + ATC_MAX_CHUNKS) * D * 4 + ATC_ROWS * ATC_MAX_CHUNKS * 4 <= REGION,
+                "the chunk merge must fit in the mainloop's shared memory");
 };
 
 template <int D>
@@ -92,6 +95,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1) attn_tc_kernel(const __grid_co
   uint64_t* p_full = s_free + ATC_NQ;         // [NQ] warpgroup q -> MMA: P_q written
   uint64_t* o_done = p_full + ATC_NQ;         // [NQ] MMA -> warpgroup q: O_q += P_q V complete
   uint64_t* drain = o_done + ATC_NQ;
+  uint64_t* mrg = drain + 1;                  // chunk merge: this chunk's slices of every chunk have landed
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tail + 256);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tail + 260);
 
@@ -130,6 +134,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1) attn_tc_kernel(const __grid_co
       mbar_init(&o_done[q], 1);
     }
     mbar_init(drain, 1);
+    mbar_init(mrg, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -379,22 +384,26 @@ __global__ void __launch_bounds__(ATC_THREADS, 1) attn_tc_kernel(const __grid_co
       }
     }
   } else {
-    // Each chunk writes its raw rows and their (max, sum) to its slot of the
-    // cluster's L2-resident buffer: layout [chunk][D/4][256 rows] float4, so a
-    // warp's store covers 32 consecutive rows (512 contiguous bytes).
+    // Each chunk stages its raw rows in shared memory in the layout of its
+    // slot of the cluster's L2-resident buffer and stores them with one bulk
+    // copy; the slot is [slice][D/4][rows of the slice] float4, so the rows
+    // one chunk later reduces (its slice) are one contiguous run in every
+    // chunk's slot.  The row statistics (max, sum) go out with plain stores.
     const int rank = static_cast<int>(cluster_ctarank());
     const size_t cl = static_cast<size_t>(blockIdx.y) * gridDim.x + blockIdx.x;
     constexpr int D4 = D / 4;
-    float4* part_cl = reinterpret_cast<float4*>(p.part) + cl * nc * D4 * ATC_ROWS;
+    const int rpr = (ATC_ROWS + nc - 1) / nc;                  // rows per slice
+    const uint32_t slice_f4 = static_cast<uint32_t>(D4 * rpr);  // one slice of one chunk
+    const uint32_t chunk_f4 = static_cast<uint32_t>(nc) * slice_f4;
+    float4* part_cl = reinterpret_cast<float4*>(p.part) + cl * nc * chunk_f4;
     float2* ml_cl = p.part_ml + cl * nc * ATC_ROWS;
+    float4* stg = reinterpret_cast<float4*>(sQ);  // the mainloop's buffers are free: every MMA has completed
     if (warp >= 2) {
       ml_cl[rank * ATC_ROWS + row] = make_float2(have_o ? mref : -INFINITY, have_o ? lsum : 0.f);
-      float4* dst = part_cl + static_cast<size_t>(rank) * D4 * ATC_ROWS + row;
+      float4* dst = stg + (row / rpr) * slice_f4 + (row % rpr);
       auto put16 = [&](int c0, const float* v) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-          dst[static_cast<size_t>(c0 / 4 + e) * ATC_ROWS] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2],
-                                                                         v[4 * e + 3]);
+        for (int e = 0; e < 4; ++e) dst[(c0 / 4 + e) * rpr] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
       };
       int c0 = 0;
 #pragma unroll 1
@@ -419,16 +428,32 @@ __global__ void __launch_bounds__(ATC_THREADS, 1) attn_tc_kernel(const __grid_co
         }
         put16(c0, v);
       }
+      fence_proxy_async_smem();
+      named_bar_sync(1, 256);
+      if (threadIdx.x == 64) {
+        // (rows past 256 in the last slice are never read)
+        bulk_store_1d(part_cl + static_cast<size_t>(rank) * chunk_f4, stg, chunk_f4 * 16u);
+        bulk_commit_group();
+        bulk_wait_all();
+        fence_proxy_async_global();
+      }
     }
     // every chunk's rows and statistics are written
     cluster_sync_all();
     if (warp >= 2) {
-      // each chunk reduces one slice of the rows over the chunks, in chunk order:
+      // each chunk reduces its slice of the rows over the chunks, in chunk order:
       // o = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c
       const int t = threadIdx.x - 64;
-      const int rpr = (ATC_ROWS + nc - 1) / nc;
       const int r_lo = rank * rpr, n_rows = max(0, min(ATC_ROWS, r_lo + rpr) - r_lo);
-      float* wts = reinterpret_cast<float*>(sQ);  // [row of the slice][chunk]; smem is free after the mainloop
+      float4* rcv = stg;                                           // [chunk][D/4][rpr]
+      float* wts = reinterpret_cast<float*>(stg + chunk_f4);       // [row of the slice][chunk]
+      if (t == 0 && n_rows > 0) {
+        fence_proxy_async_global();
+        mbar_arrive_expect_tx(mrg, chunk_f4 * 16u);
+        for (int q = 0; q < nc; ++q)
+          bulk_load_1d(rcv + q * slice_f4, part_cl + static_cast<size_t>(q) * chunk_f4 + rank * slice_f4,
+                       slice_f4 * 16u, mrg);
+      }
       if (t < n_rows) {
         float2 ml[ATC_MAX_CHUNKS];
 #pragma unroll
@@ -449,31 +474,27 @@ __global__ void __launch_bounds__(ATC_THREADS, 1) attn_tc_kernel(const __grid_co
             wts[t * ATC_MAX_CHUNKS + q] = (den > 0.f && ml[q].x != -INFINITY) ? ex2_approx(ml[q].x - Mref) / den : 0.f;
       }
       named_bar_sync(1, 256);
-      const int n_items = n_rows * D4;
-      for (int it = t; it < n_items; it += 256) {
-        const int rl = it % n_rows, c4 = it / n_rows, rr = r_lo + rl;
-        const float4* src = part_cl + static_cast<size_t>(c4) * ATC_ROWS + rr;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int q0 = 0; q0 < nc; q0 += 8) {
-          float4 v[8];
-#pragma unroll
-          for (int u = 0; u < 8; ++u)
-            if (q0 + u < nc) v[u] = __ldcg(src + static_cast<size_t>(q0 + u) * D4 * ATC_ROWS);
-#pragma unroll
-          for (int u = 0; u < 8; ++u)
-            if (q0 + u < nc) {
-              const float wq = wts[rl * ATC_MAX_CHUNKS + q0 + u];
-              acc.x = fmaf(v[u].x, wq, acc.x);
-              acc.y = fmaf(v[u].y, wq, acc.y);
-              acc.z = fmaf(v[u].z, wq, acc.z);
-              acc.w = fmaf(v[u].w, wq, acc.w);
-            }
+      if (n_rows > 0 && mbar_wait(mrg, 0, p.err)) {
+        const int n_items = n_rows * D4;
+        for (int it = t; it < n_items; it += 256) {
+          const int rl = it / D4, c4 = it % D4;   // a warp covers consecutive columns of a row
+          const float4* src = rcv + c4 * rpr + rl;
+          const float* wr = wts + rl * ATC_MAX_CHUNKS;
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int q = 0; q < nc; ++q) {
+            const float4 v = src[q * slice_f4];
+            const float wq = wr[q];
+            acc.x = fmaf(v.x, wq, acc.x);
+            acc.y = fmaf(v.y, wq, acc.y);
+            acc.z = fmaf(v.z, wq, acc.z);
+            acc.w = fmaf(v.w, wq, acc.w);
+          }
+          const int rg = row_base + r_lo + rl;
+          if (rg >= rows_total) continue;
+          const size_t rid = (static_cast<size_t>(b) * p.n + rg / G) * p.Hq + kvh * G + rg % G;
+          *reinterpret_cast<uint2*>(p.o + rid * D + 4 * c4) =
+              make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
         }
-        const int rg = row_base + rr;
-        if (rg >= rows_total) continue;
-        const size_t rid = (static_cast<size_t>(b) * p.n + rg / G) * p.Hq + kvh * G + rg % G;
-        *reinterpret_cast<uint2*>(p.o + rid * D + 4 * c4) =
-            make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
       }
     }
   }

@@ -79,7 +79,7 @@ struct dg_ctx {
   int32_t* chunk_done = nullptr;   // finished gate/up tiles per expert token chunk
   int32_t* expert_rows = nullptr;  // [E] rows routed to each expert (dispatch cursors)
   int32_t* moe_work = nullptr;     // claim / exit counters of the expert GEMM
-  float* attn_part = nullptr;      // attention chunk partials (clusters of several chunks): sms x 256 rows x D
+  float* attn_part = nullptr;      // attention chunk partials (clusters of several chunks): sms x 272 rows x D
   float2* attn_part_ml = nullptr;  // their row statistics: sms x 256 rows
   int32_t* dense_work = nullptr;   // claim / exit counters of the dense GEMM
   int attn_max_clusters[ATC_MAX_CHUNKS + 1] = {};  // co-resident attention clusters per cluster size
@@ -401,7 +401,7 @@ dg_status attention(dg_ctx* c, int l, int B, int n, int pos0, bool causal) {
   // ties: each chunk adds a merge share); one chunk when nothing fits.
   int n_chunks = 1, best_blocks = (keys + ATC_BK - 1) / ATC_BK;
   for (int nc = 2; nc <= ATC_MAX_CHUNKS; ++nc) {
-    // the partial buffer holds sms x 256 rows: one slot per CTA of the launch
+    // the partial buffer holds sms x (256 + 16) rows: one slot per CTA of the launch
     if (units > c->attn_max_clusters[nc] || keys < nc * ATC_BK || units * nc > c->sms) continue;
     const int blocks = ((keys + nc - 1) / nc + ATC_BK - 1) / ATC_BK;
     if (blocks < best_blocks) {
@@ -1067,7 +1067,7 @@ dg_status dg_create(const dg_config* cfg, const dg_weights* w, void* cuda_stream
   add(c->max_chunks, 4);                          // chunk_done
   add(PERM_MAXE, 4);                              // expert_rows
   add(2, 4);                                      // moe_work
-  add(static_cast<size_t>(c->sms) * ATC_ROWS * c->D, 4);  // attn_part
+  add(static_cast<size_t>(c->sms) * (ATC_ROWS + ATC_MAX_CHUNKS) * c->D, 4);  // attn_part
   add(static_cast<size_t>(c->sms) * ATC_ROWS, 8);         // attn_part_ml
   add(2, 4);                                      // dense_work
   add(ER * d, 2);                                 // xp
@@ -1105,7 +1105,7 @@ dg_status dg_create(const dg_config* cfg, const dg_weights* w, void* cuda_stream
   c->chunk_done = carve<int32_t>(cur, c->max_chunks);
   c->expert_rows = carve<int32_t>(cur, PERM_MAXE);
   c->moe_work = carve<int32_t>(cur, 2);
-  c->attn_part = carve<float>(cur, static_cast<size_t>(c->sms) * ATC_ROWS * c->D);
+  c->attn_part = carve<float>(cur, static_cast<size_t>(c->sms) * (ATC_ROWS + ATC_MAX_CHUNKS) * c->D);
   c->attn_part_ml = carve<float2>(cur, static_cast<size_t>(c->sms) * ATC_ROWS);
   c->dense_work = carve<int32_t>(cur, 2);
   c->xp = carve<uint16_t>(cur, ER * d);

@@ -311,12 +311,6 @@ __device__ __forceinline__ void red_release_gpu_add(int* ptr, int v) {
   asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(ptr), "r"(v) : "memory");
 }
 
-// order this thread's earlier generic-proxy accesses with its later
-// async-proxy (TMA) accesses of global memory
-__device__ __forceinline__ void fence_proxy_async_global() {
-  asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-
 // Wait (bounded) until every gate/up tile of `chunk` has published its rows.
 __device__ __forceinline__ bool wait_chunk_ready(const GemmParams& p, const GemmTile& t) {
   const int need = (t.shared ? p.Fs : p.F) / 64;
