@@ -2,14 +2,17 @@
 """Throughput of the block discrete-diffusion denoising step on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+    python bench.py --timeline        (per-kernel spans inside the step's graph)
+    python bench.py --batch-sweep 1,2,4,8,16,32
 
 One step = one dg_denoise_step call: embedding, 30 MoE transformer layers over
 the 256-token canvas with bidirectional attention against the prefix KV cache,
 the tied 262144-vocabulary LM head fused with the argmax / log-sum-exp
 reduction, and the Philox re-noising sampler.  Workload: the 26B-A4B-shaped
 model, batch 1, 2048-token uniform-random prefix (seeded synthetic weights
-and tokens).  Each step streams ~50 GB of weights, far more than the 126 MB
-L2, so no flush is needed between steps.
+and tokens).  Each step streams ~32 GB of weights (the experts the step
+actually routes to), far more than the 126 MB L2, so no flush is needed
+between steps.
 
 Multi-GPU: independent replicas (one per rank, no collective on the data
 path); value = canvas tokens of all ranks / max-over-ranks time.
@@ -35,6 +38,46 @@ METRIC = "canvas tokens denoised/s (batch 1, 256-tok block) and % of step roofli
 UNIT = "canvas tokens/s"
 
 
+def run_timeline(args, w):
+    """Per-kernel device time inside the step's CUDA graph.  The timeline build
+    of the library records every CTA's start and end (%globaltimer); one
+    graph-replayed step after the warm-up is rebuilt into its launch sequence:
+    per kernel the launches, summed and mean spans, share of the step, and the
+    idle gaps between launches.  The records add one atomic and two timer
+    reads per CTA, so the step is not a bench number."""
+    import torch
+
+    import block_discrete_diffusion_denoise_b200 as dgp
+    import synth_inputs as si
+
+    stream = torch.cuda.Stream()
+    torch.cuda.set_stream(stream)
+    weights = si.model_weights(w, "cuda")
+    cfg = dgp.config_from_shape(w.shape, max_batch=w.batch, max_seq=w.prefix + 2 * w.canvas, canvas=w.canvas)
+    ctx = dgp.Context(cfg, weights, stream=stream.cuda_stream)
+    ctx.prefill(si.uniform_tokens(w, "prefix", w.batch, w.prefix, device="cuda"))
+    cur = si.uniform_tokens(w, "canvas", w.batch, w.canvas, device="cuda")
+    nxt = torch.empty_like(cur)
+    conf = torch.empty(w.batch, w.canvas, dtype=torch.float32, device="cuda")
+    for s in range(args.warmup):
+        ctx.denoise_step(cur, s, w.sample_seed, si.tau_schedule(w, s), nxt, conf)
+        cur, nxt = nxt, cur
+    steps = []
+    for s in range(args.steps):
+        ctx.debug_timeline_reset()
+        ctx.denoise_step(cur, s, w.sample_seed, si.tau_schedule(w, s % w.steps), nxt, conf)
+        cur, nxt = nxt, cur
+        rec, n = ctx.debug_timeline()
+        steps.append(dgp.timeline_summary(dgp.timeline_launches(rec)))
+    ctx.close()
+    # the step with the median wall time
+    med = sorted(steps, key=lambda x: x["wall_us"])[len(steps) // 2]
+    print(json.dumps({"timeline": f"{w.name}: {w.description}", "library": os.path.basename(dgp.LIB_PATH),
+                      "steps": args.steps, "warmup": args.warmup,
+                      "wall_us_per_step": [round(x["wall_us"], 1) for x in steps], "median_step": med}),
+          flush=True)
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -47,6 +90,9 @@ def parse():
                     help="reduced depth (profiling captures only; not a bench number)")
     ap.add_argument("--batch-sweep", default="",
                     help="comma-separated batch sizes: step throughput and roofline bound per batch "
+                         "(one JSON line of its own, not the bench line)")
+    ap.add_argument("--timeline", action="store_true",
+                    help="per-kernel spans and launch gaps of graph-replayed steps from libdg_timeline.so "
                          "(one JSON line of its own, not the bench line)")
     return ap.parse_args()
 
@@ -490,11 +536,16 @@ def run_batch_sweep(args, w):
 
 def main():
     args = parse()
+    if args.timeline:
+        # the timeline build of the library; chosen before the package is imported
+        os.environ["DG_LIBRARY"] = os.path.join(ROOT, "block_discrete_diffusion_denoise_b200", "libdg_timeline.so")
     import synth_inputs as si
     w = si.workload(args.workload)
     if args.layers:
         w = w.with_layers(args.layers)
-    if args.batch_sweep:
+    if args.timeline:
+        run_timeline(args, w)
+    elif args.batch_sweep:
         run_batch_sweep(args, w)
     elif args.impl == "reference":
         run_reference(args, w)

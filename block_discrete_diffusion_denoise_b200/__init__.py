@@ -12,6 +12,8 @@ import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.environ.get("DG_LIBRARY", os.path.join(HERE, "libdg.so"))
+# the same library with per-CTA timeline records (select it with DG_LIBRARY)
+TIMELINE_LIB_PATH = os.path.join(HERE, "libdg_timeline.so")
 
 DG_OK = 0
 STATUS = {0: "DG_OK", 1: "DG_ERR_INVALID_ARG", 2: "DG_ERR_OOM", 3: "DG_ERR_CAPACITY", 4: "DG_ERR_CUDA",
@@ -25,7 +27,14 @@ EXPORTS = ["dg_create", "dg_destroy", "dg_prefill", "dg_denoise_step", "dg_denoi
            "dg_debug_hidden", "dg_debug_experts", "dg_debug_norm_rows", "dg_debug_lmhead", "dg_debug_router",
            "dg_debug_sample", "dg_debug_entropy_sample", "dg_debug_entropy", "dg_debug_wait_timeout",
            "dg_debug_gemm", "dg_debug_profile",
-           "dg_debug_profile_read", "dg_debug_launch_count", "dg_lmhead_argmax_static"]
+           "dg_debug_profile_read", "dg_debug_launch_count", "dg_debug_timeline_reset", "dg_debug_timeline",
+           "dg_lmhead_argmax_static"]
+
+# kernel ids of the timeline records (DG_K_* in dg.h)
+TIMELINE_KERNELS = {10: "gemm_dense", 11: "gemm_moe", 13: "gemm_lmhead", 20: "attention", 30: "route_dispatch",
+                    31: "combine_norm", 32: "embed_norm", 33: "residual_norm", 34: "reduce_splits",
+                    35: "swiglu_splits", 36: "rope_qkv", 37: "lmhead_merge_sample", 38: "entropy_sample",
+                    39: "router_topk", 40: "sample_only", 50: "other"}
 
 # kernel classes of dg_debug_profile (DG_PROF_* in dg.h)
 PROF_CLASSES = ["experts", "routing", "lm_head", "attention", "dense_proj", "other"]
@@ -55,6 +64,11 @@ class dg_weights(ctypes.Structure):
     _fields_ = [("embed", ctypes.c_void_p), ("final_norm", ctypes.c_void_p),
                 ("router_bias", ctypes.c_void_p), ("layers", ctypes.POINTER(dg_layer_weights)),
                 ("sc_gate", ctypes.c_void_p), ("sc_up", ctypes.c_void_p), ("sc_down", ctypes.c_void_p)]
+
+
+class dg_timeline_record(ctypes.Structure):
+    _fields_ = [("t0_ns", ctypes.c_uint64), ("t1_ns", ctypes.c_uint64), ("kernel", ctypes.c_int32),
+                ("cta", ctypes.c_int32)]
 
 
 class dg_entropy_args(ctypes.Structure):
@@ -106,6 +120,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "dg_debug_profile": ([P, I32], I32),
         "dg_debug_profile_read": ([P, I32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(I64)], I32),
         "dg_debug_launch_count": ([P], I64),
+        "dg_debug_timeline_reset": ([P], I32),
+        "dg_debug_timeline": ([P, P, I32, ctypes.POINTER(I64)], I32),
         "dg_lmhead_argmax_static": ([P, I32, I32, P, I32, F32, P, P, P, P], I32),
     }
     for name, (args, res) in sig.items():
@@ -264,6 +280,21 @@ class Context:
     def launch_count(self) -> int:
         return self.lib.dg_debug_launch_count(self.ctx)
 
+    def debug_timeline_reset(self):
+        """Empty the timeline buffer (libdg_timeline.so only)."""
+        self._check(self.lib.dg_debug_timeline_reset(self.ctx))
+
+    def debug_timeline(self, capacity: int = 1 << 18):
+        """Records appended since the last reset as a numpy structured array
+        (t0_ns, t1_ns, kernel, cta), and how many were appended in all."""
+        import numpy as np
+        buf = (dg_timeline_record * capacity)()
+        n = ctypes.c_int64()
+        self._check(self.lib.dg_debug_timeline(self.ctx, buf, capacity, ctypes.byref(n)))
+        dt = np.dtype([("t0_ns", "<u8"), ("t1_ns", "<u8"), ("kernel", "<i4"), ("cta", "<i4")])
+        arr = np.frombuffer(buf, dtype=dt, count=min(n.value, capacity)).copy()
+        return arr, n.value
+
 
 def config_from_shape(shape, max_batch=1, max_seq=4096, canvas=256, temperature=1.0, prefill_rows=0) -> dict:
     """dg_config fields for a model shape (anything with the dg_config names)."""
@@ -371,3 +402,46 @@ def generate_blocks(ctx: Context, prefix, init_canvas, n_blocks: int, max_steps:
         if k + 1 < n_blocks or commit_last:
             ctx.commit_block(cur)
     return out
+
+
+def timeline_launches(records):
+    """Rebuild the launch sequence from timeline records: launches on one
+    stream run one after another, so after sorting by start time a new launch
+    begins wherever the kernel id changes or a CTA starts after every CTA so
+    far has ended.  Returns a list of dicts {kernel, name, t0_ns, t1_ns, ctas}."""
+    import numpy as np
+    if len(records) == 0:
+        return []
+    r = records[np.argsort(records["t0_ns"], kind="stable")]
+    out = []
+    cur = None
+    for t0, t1, k in zip(r["t0_ns"].tolist(), r["t1_ns"].tolist(), r["kernel"].tolist()):
+        if cur is None or k != cur["kernel"] or t0 > cur["t1_ns"]:
+            cur = {"kernel": k, "name": TIMELINE_KERNELS.get(k, str(k)), "t0_ns": t0, "t1_ns": t1, "ctas": 0}
+            out.append(cur)
+        cur["t1_ns"] = max(cur["t1_ns"], t1)
+        cur["ctas"] += 1
+    return out
+
+
+def timeline_summary(launches) -> dict:
+    """Per-kernel totals of a launch sequence: launches, summed span (us),
+    mean span, share of the wall time, and the idle gaps before each kernel's
+    launches; plus the wall time and the summed gaps."""
+    if not launches:
+        return {"wall_us": 0.0, "gaps_us": 0.0, "launches": 0, "kernels": {}}
+    wall = (max(l["t1_ns"] for l in launches) - launches[0]["t0_ns"]) / 1e3
+    kernels, gaps, prev_end = {}, 0.0, launches[0]["t0_ns"]
+    for l in launches:
+        gap = max(0.0, (l["t0_ns"] - prev_end) / 1e3)
+        span = (l["t1_ns"] - l["t0_ns"]) / 1e3
+        k = kernels.setdefault(l["name"], {"launches": 0, "total_us": 0.0, "gaps_before_us": 0.0})
+        k["launches"] += 1
+        k["total_us"] += span
+        k["gaps_before_us"] += gap
+        gaps += gap
+        prev_end = max(prev_end, l["t1_ns"])
+    for k in kernels.values():
+        k["avg_us"] = k["total_us"] / k["launches"]
+        k["share"] = k["total_us"] / wall if wall > 0 else 0.0
+    return {"wall_us": wall, "gaps_us": gaps, "launches": len(launches), "kernels": kernels}

@@ -77,6 +77,7 @@ struct AtcCfg {
 
 template <int D>
 __global__ void __launch_bounds__(ATC_THREADS, 1) attn_tc_kernel(const __grid_constant__ AttnTcParams p) {
+  DG_TIMELINE_SCOPE(TLK_ATTENTION);
   using C = AtcCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sQ = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));

@@ -30,6 +30,63 @@ __device__ __forceinline__ void raise_error(const DevErr& e, int code) {
 }
 
 // ----------------------------------------------------------------------------
+// Optional timeline (libdg_timeline.so, compiled with -DDG_TIMELINE; absent
+// from libdg.so): thread 0 of every CTA records the kernel's id and its own
+// start and end times (%globaltimer), so the host can rebuild the launch
+// sequence of a graph replay, each launch's span and the gaps between
+// launches without a profiler.  The record is taken when thread 0 leaves the
+// kernel.
+// ----------------------------------------------------------------------------
+enum TimelineKernel : int {
+  TLK_GEMM = 10,  // + the GEMM mode (10 dense, 11 expert, 13 LM head)
+  TLK_ATTENTION = 20,
+  TLK_ROUTE_DISPATCH = 30,
+  TLK_COMBINE_NORM = 31,
+  TLK_EMBED_NORM = 32,
+  TLK_RESIDUAL_NORM = 33,
+  TLK_REDUCE_SPLITS = 34,
+  TLK_SWIGLU_SPLITS = 35,
+  TLK_ROPE_QKV = 36,
+  TLK_LMHEAD_MERGE_SAMPLE = 37,
+  TLK_ENTROPY_SAMPLE = 38,
+  TLK_ROUTER_TOPK = 39,
+  TLK_SAMPLE_ONLY = 40,
+  TLK_OTHER = 50,
+};
+
+#ifdef DG_TIMELINE
+constexpr unsigned int TIMELINE_CAP = 1u << 18;
+struct TimelineRecord {
+  unsigned long long t0, t1;
+  int kernel, cta;
+};
+__device__ TimelineRecord g_timeline[TIMELINE_CAP];
+__device__ unsigned int g_timeline_n;
+
+struct TimelineScope {
+  unsigned long long t0;
+  int id;
+  __device__ __forceinline__ explicit TimelineScope(int k) : t0(0), id(k) {
+    if (threadIdx.x == 0) t0 = globaltimer_ns();
+  }
+  __device__ __forceinline__ ~TimelineScope() {
+    if (threadIdx.x == 0) {
+      const unsigned int i = atomicAdd(&g_timeline_n, 1u);
+      if (i < TIMELINE_CAP) {
+        g_timeline[i].t0 = t0;
+        g_timeline[i].t1 = globaltimer_ns();
+        g_timeline[i].kernel = id;
+        g_timeline[i].cta = static_cast<int>(blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z));
+      }
+    }
+  }
+};
+#define DG_TIMELINE_SCOPE(k) ::dg::TimelineScope dg_timeline_scope_(k)
+#else
+#define DG_TIMELINE_SCOPE(k)
+#endif
+
+// ----------------------------------------------------------------------------
 // bf16 helpers
 // ----------------------------------------------------------------------------
 __device__ __forceinline__ float bf16_to_f32(uint16_t b) {

@@ -1501,6 +1501,53 @@ dg_status dg_debug_gemm(dg_ctx* c, const void* w, int32_t M, int32_t K, const vo
   return DG_OK;
 }
 
+constexpr bool timeline_ids_match() {
+  using namespace dg;
+  const int ours[16] = {TLK_GEMM + GEMM_DENSE, TLK_GEMM + GEMM_MOE, TLK_GEMM + GEMM_LMHEAD, TLK_ATTENTION,
+                        TLK_ROUTE_DISPATCH, TLK_COMBINE_NORM, TLK_EMBED_NORM, TLK_RESIDUAL_NORM, TLK_REDUCE_SPLITS,
+                        TLK_SWIGLU_SPLITS, TLK_ROPE_QKV, TLK_LMHEAD_MERGE_SAMPLE, TLK_ENTROPY_SAMPLE, TLK_ROUTER_TOPK,
+                        TLK_SAMPLE_ONLY, TLK_OTHER};
+  const int abi[16] = {DG_K_GEMM_DENSE, DG_K_GEMM_MOE, DG_K_GEMM_LMHEAD, DG_K_ATTENTION, DG_K_ROUTE_DISPATCH,
+                       DG_K_COMBINE_NORM, DG_K_EMBED_NORM, DG_K_RESIDUAL_NORM, DG_K_REDUCE_SPLITS, DG_K_SWIGLU_SPLITS,
+                       DG_K_ROPE_QKV, DG_K_LMHEAD_MERGE_SAMPLE, DG_K_ENTROPY_SAMPLE, DG_K_ROUTER_TOPK,
+                       DG_K_SAMPLE_ONLY, DG_K_OTHER};
+  for (int i = 0; i < 16; ++i)
+    if (ours[i] != abi[i]) return false;
+  return true;
+}
+static_assert(timeline_ids_match(), "timeline kernel ids match the ABI");
+
+dg_status dg_debug_timeline_reset(dg_ctx* c) {
+  if (!c) return DG_ERR_INVALID_ARG;
+#ifdef DG_TIMELINE
+  DG_CUDA(c, cudaStreamSynchronize(c->stream));
+  const unsigned int zero = 0;
+  DG_CUDA(c, cudaMemcpyToSymbol(dg::g_timeline_n, &zero, sizeof(zero)));
+  return DG_OK;
+#else
+  return fail(c, DG_ERR_UNSUPPORTED, "this library was built without the timeline (see libdg_timeline.so)");
+#endif
+}
+
+dg_status dg_debug_timeline(dg_ctx* c, dg_timeline_record* host, int32_t capacity, int64_t* n_records) {
+  if (!c || !n_records || capacity < 0 || (capacity > 0 && !host)) return DG_ERR_INVALID_ARG;
+#ifdef DG_TIMELINE
+  static_assert(sizeof(dg_timeline_record) == sizeof(dg::TimelineRecord), "record layout");
+  DG_CUDA(c, cudaStreamSynchronize(c->stream));
+  unsigned int n = 0;
+  DG_CUDA(c, cudaMemcpyFromSymbol(&n, dg::g_timeline_n, sizeof(n)));
+  *n_records = n;
+  const size_t m = std::min<size_t>({static_cast<size_t>(n), static_cast<size_t>(capacity),
+                                     static_cast<size_t>(dg::TIMELINE_CAP)});
+  if (m > 0) DG_CUDA(c, cudaMemcpyFromSymbol(host, dg::g_timeline, m * sizeof(dg_timeline_record)));
+  return DG_OK;
+#else
+  (void)host;
+  *n_records = 0;
+  return fail(c, DG_ERR_UNSUPPORTED, "this library was built without the timeline (see libdg_timeline.so)");
+#endif
+}
+
 dg_status dg_debug_profile(dg_ctx* c, int32_t mask) {
   if (!c) return DG_ERR_INVALID_ARG;
   DG_CUDA(c, cudaStreamSynchronize(c->stream));
@@ -1563,6 +1610,7 @@ std::mutex g_static_setup_mutex;  // the first calls on a device may come from s
 __global__ void lmhead_static_merge_kernel(const float4* __restrict__ part, int n_vtiles, int T,
                                            const int* __restrict__ err, int32_t* __restrict__ argmax,
                                            float* __restrict__ lse, float* __restrict__ conf) {
+  DG_TIMELINE_SCOPE(dg::TLK_OTHER);
   const int t = blockIdx.x;
   const Top2 acc = merge_token_partials(part, nullptr, n_vtiles, T, t);
   if (threadIdx.x == 0) {

@@ -38,7 +38,9 @@ constexpr int GEMM_BM = 128;
 constexpr int GEMM_BK = 64;
 constexpr int GEMM_BN = 128;                         // accumulator columns; dense / LM-head tile width
 constexpr int GEMM_A_BYTES = GEMM_BM * GEMM_BK * 2;  // 16 KB
-constexpr int GEMM_THREADS = 192;
+// warp 0: A producer, warp 1: MMA issuer, warps 2-5: epilogue, warp 6: B producer
+constexpr int GEMM_THREADS = 224;
+constexpr int GEMM_B_WARP = 6;
 // epilogue staging: gate values of one 32-column chunk (64 x 33) or one
 // 32 x 128 fp32 block on its way to global memory
 constexpr int GEMM_XCHG_FLOATS = 2 * 32 * GEMM_BM;
@@ -52,10 +54,17 @@ constexpr int MOE_MAX_EXPERTS = 256;                 // routed experts (+1 share
 // MOE tile tables in shared memory: chunk offsets [E + 2] and group rows [E + 1], 16-bit
 constexpr int MOE_TABLE_BYTES = ((MOE_MAX_EXPERTS + 2) + (MOE_MAX_EXPERTS + 1)) * 2 + 32;
 
-// Stage ring depth (16 KB of A plus the B rows per stage).
+// Ring depths.  A (16 KB per stage) and B (the B rows of one k-step per
+// stage) have rings of their own, filled by two producer lanes, so the
+// operand streamed from HBM can run further ahead than the one read from L2:
+// in MOE the expert weights (A) run 8 k-steps ahead, the gathered rows (B) 4.
 template <int MODE>
-constexpr int gemm_stages() {
-  return MODE == GEMM_DENSE ? 4 : 6;
+constexpr int gemm_stages_a() {
+  return MODE == GEMM_DENSE ? 4 : (MODE == GEMM_MOE ? 8 : 6);
+}
+template <int MODE>
+constexpr int gemm_stages_b() {
+  return MODE == GEMM_DENSE ? 4 : (MODE == GEMM_MOE ? 4 : 6);
 }
 // rows of B one stage holds
 template <int MODE>
@@ -73,8 +82,8 @@ constexpr int gemm_acc_cols() {
 }
 template <int MODE>
 constexpr int gemm_smem_bytes() {
-  return 1024 + gemm_stages<MODE>() * (GEMM_A_BYTES + gemm_b_bytes<MODE>()) + GEMM_XCHG_FLOATS * 4 + 512 +
-         (MODE == GEMM_MOE ? MOE_TABLE_BYTES : 0);
+  return 1024 + gemm_stages_a<MODE>() * GEMM_A_BYTES + gemm_stages_b<MODE>() * gemm_b_bytes<MODE>() +
+         GEMM_XCHG_FLOATS * 4 + 512 + (MODE == GEMM_MOE ? MOE_TABLE_BYTES : 0);
 }
 
 enum TileKind : int { KIND_DENSE = 0, KIND_GATEUP = 1, KIND_DOWN = 2, KIND_LMHEAD = 3 };
@@ -380,27 +389,29 @@ constexpr bool claims_tiles() {
   return MODE == GEMM_MOE;
 }
 
-__device__ __forceinline__ int ld_relaxed_gpu(const int* ptr) {
-  int v;
-  asm volatile("ld.relaxed.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
-  return v;
-}
-
-__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
-
 template <int MODE>
 __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_constant__ GemmParams p) {
-  constexpr int STAGES = gemm_stages<MODE>();
+  DG_TIMELINE_SCOPE(TLK_GEMM + MODE);
+  constexpr int SA = gemm_stages_a<MODE>();
+  constexpr int SB = gemm_stages_b<MODE>();
   constexpr int B_BYTES = gemm_b_bytes<MODE>();
+  static_assert(gemm_smem_bytes<MODE>() <= 232448, "shared memory per CTA");
+  static_assert((2 * (SA + SB) + 5 + 2 * GEMM_SCHED) * 8 + GEMM_SCHED * 20 + 64 <= 512, "barrier area");
   constexpr int ACC_COLS = gemm_acc_cols<MODE>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
-  uint8_t* sB = sA + STAGES * GEMM_A_BYTES;
-  float* xchg = reinterpret_cast<float*>(sB + STAGES * B_BYTES);
-  uint64_t* full = reinterpret_cast<uint64_t*>(xchg + GEMM_XCHG_FLOATS);
-  uint64_t* empty = full + STAGES;
-  uint64_t* tfull = empty + STAGES;
+  uint8_t* sB = sA + SA * GEMM_A_BYTES;
+  float* xchg = reinterpret_cast<float*>(sB + SB * B_BYTES);
+  // Equal depths (DENSE, LMHEAD): one ring whose stages both producers fill
+  // (full barrier of two arrivals), so the MMA issuer waits and commits once
+  // per k-step.  Otherwise (MOE) two rings.
+  constexpr bool JOINT = SA == SB;
+  uint64_t* a_full = reinterpret_cast<uint64_t*>(xchg + GEMM_XCHG_FLOATS);
+  uint64_t* a_empty = a_full + SA;
+  uint64_t* b_full = JOINT ? a_full : a_empty + SA;
+  uint64_t* b_empty = JOINT ? a_empty : b_full + SB;
+  uint64_t* tfull = JOINT ? a_empty + SA : b_empty + SB;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint64_t* sched_full = drain + 1;
@@ -419,7 +430,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
 
   MoeTables tb{tb_ch_off, tb_rows, 0, 0, 0};
   if constexpr (MODE == GEMM_MOE) {
-    // tile tables from the row counts (two groups per thread, G <= 2 * 192)
+    // tile tables from the row counts (two groups per thread, G <= 2 * GEMM_THREADS)
     const int G = p.n_groups_routed + 1;
     int nch2[2], rows2[2];
 #pragma unroll
@@ -447,17 +458,22 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
   }
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+    for (int s = 0; s < SA; ++s) {
+      mbar_init(&a_full[s], JOINT ? 2 : 1);
+      mbar_init(&a_empty[s], 1);
     }
+    if (!JOINT)
+      for (int s = 0; s < SB; ++s) {
+        mbar_init(&b_full[s], 1);
+        mbar_init(&b_empty[s], 1);
+      }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], 128);
     }
     for (int s = 0; s < GEMM_SCHED; ++s) {
       mbar_init(&sched_full[s], 1);
-      mbar_init(&sched_empty[s], 2);  // MMA issuer + epilogue leader
+      mbar_init(&sched_empty[s], 3);  // B producer + MMA issuer + epilogue leader
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -475,18 +491,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
   const int n_gu = tb.n_gu;
 
   if (warp == 0) {
-    // ------------------------------ TMA producer ------------------------------
     if (lane == 0) {
+      // --------------------------- TMA producer of A ---------------------------
+      // Claims the tiles (MOE), publishes them to the other roles, and streams
+      // A.  It waits on nothing but free A slots, so the weight stream keeps
+      // SA k-steps in flight whatever B is waiting for.
       tma_prefetch_desc(&p.a_map[0]);
-      tma_prefetch_desc(&p.b_map);
       const uint64_t pol_first = policy_evict_first();
       const uint64_t pol_last = policy_evict_last();
       int stage = 0;
       uint32_t phase = 0, issued = 0, issued_par = 0;
-      // MOE: the claim of the next tile, its record and its dependency flag
-      // are fetched while the current tile's loads are being issued, so no
-      // global-memory round trip sits between two tiles.
-      int cur = -1, claim = 0, dep_hint = 0;
+      int cur = -1, claim = 0;
       int4 cur_rec = make_int4(0, 0, 0, 0);
       if constexpr (claims_tiles<MODE>()) {
         // the first tile of every CTA is its own index; later tiles are
@@ -501,10 +516,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
         int nxt = -1;
         int4 nxt_rec = make_int4(0, 0, 0, 0);
         if constexpr (claims_tiles<MODE>()) {
+          // the next claim and its record are fetched while this tile's
+          // loads are issued, so no global round trip sits between tiles
           if (cur >= n_tiles || *abort_flag) cur = -1;
           if (cur >= 0 && claim < n_tiles) {
             nxt = claim;
-            nxt_rec = moe_record(p, tb, nxt);  // consumed in the next iteration
+            nxt_rec = moe_record(p, tb, nxt);
             claim = static_cast<int>(gridDim.x) + atomicAdd(p.work, 1);
           }
           tile = cur;
@@ -524,55 +541,26 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
         }
         GemmTile t;
         decode_tile<MODE>(p, tile, rec, n_gu, t);
-        const int cur_hint = dep_hint;
-        dep_hint = 0;
-        if constexpr (MODE == GEMM_MOE) {
-          if (t.kind == KIND_DOWN) {
-            const int need = (t.shared ? p.Fs : p.F) / 64;
-            if (cur_hint >= need) {
-              fence_acq_rel_gpu();          // the early relaxed read saw the release
-              fence_proxy_async_global();
-            } else if (!wait_chunk_ready(p, t)) {
-              *abort_flag = 1;
-              break;
-            }
-          }
-        }
-        // B arrives in whole boxes (rows past nmma are loaded, zero-filled
-        // past the tensor's end, and ignored by the MMA)
-        const int b_rows = (t.nmma + p.b_box_rows - 1) / p.b_box_rows * p.b_box_rows;
-        const uint32_t bytes = GEMM_A_BYTES + b_rows * GEMM_BK * 2;
         const uint64_t pol_a = t.a_stream ? pol_first : pol_last;
         for (int k = 0; k < t.nk; ++k) {
-          if (!mbar_wait(&empty[stage], phase ^ 1, p.err)) {
+          if (!mbar_wait(&a_empty[stage], phase ^ 1, p.err)) {
             *abort_flag = 1;
             break;
           }
-          mbar_arrive_expect_tx(&full[stage], bytes);
+          mbar_arrive_expect_tx(&a_full[stage], GEMM_A_BYTES);
           uint8_t* a = sA + stage * GEMM_A_BYTES;
-          uint8_t* b = sB + stage * B_BYTES;
           const int kx = (t.k0 + k) * GEMM_BK;
           if (MODE == GEMM_DENSE && p.a_mn_major) {
             // A stored [K][M]: two boxes of 64 k-rows x 64 m-columns
-            tma_load_2d(a, t.a0, &full[stage], t.a_row, kx, pol_a);
-            tma_load_2d(a + GEMM_A_BYTES / 2, t.a0, &full[stage], t.a_row + 64, kx, pol_a);
+            tma_load_2d(a, t.a0, &a_full[stage], t.a_row, kx, pol_a);
+            tma_load_2d(a + GEMM_A_BYTES / 2, t.a0, &a_full[stage], t.a_row + 64, kx, pol_a);
           } else {
-            tma_load_2d(a, t.a0, &full[stage], kx, t.a_row, pol_a);
-            if (t.a1 != nullptr) tma_load_2d(a + GEMM_A_BYTES / 2, t.a1, &full[stage], kx, t.a_row, pol_a);
-          }
-          int r = 0;
-          if (p.b_mid_rows > 0)
-            for (; r + p.b_mid_rows <= t.nmma; r += p.b_mid_rows)
-              tma_load_2d(b + r * (GEMM_BK * 2), t.b_mid, &full[stage], kx, t.b_row + r, pol_last);
-          for (; r < t.nmma; r += p.b_box_rows)
-            tma_load_2d(b + r * (GEMM_BK * 2), t.b, &full[stage], kx, t.b_row + r, pol_last);
-          if constexpr (claims_tiles<MODE>()) {
-            // halfway through this tile, read the next tile's dependency flag
-            if (k == (t.nk >> 1) && nxt >= n_gu) dep_hint = ld_relaxed_gpu(p.chunk_done + nxt_rec.y);
+            tma_load_2d(a, t.a0, &a_full[stage], kx, t.a_row, pol_a);
+            if (t.a1 != nullptr) tma_load_2d(a + GEMM_A_BYTES / 2, t.a1, &a_full[stage], kx, t.a_row, pol_a);
           }
           issued |= 1u << stage;
           issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
-          if (++stage == STAGES) {
+          if (++stage == SA) {
             stage = 0;
             phase ^= 1;
           }
@@ -584,14 +572,81 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
         }
       }
       // every copy this thread issued has landed before the CTA may exit
-      for (int s = 0; s < STAGES; ++s)
-        if ((issued >> s) & 1) mbar_wait(&full[s], (issued_par >> s) & 1, p.err);
+      for (int s = 0; s < SA; ++s)
+        if ((issued >> s) & 1) mbar_wait(&a_full[s], (issued_par >> s) & 1, p.err);
+    }
+  } else if (warp == GEMM_B_WARP) {
+    if (lane == 0) {
+      // --------------------------- TMA producer of B ---------------------------
+      // Follows the same tiles.  A down tile's rows are the hidden rows its
+      // chunk's gate/up tiles publish, so before its first B load this lane
+      // waits (bounded) for the chunk's counter with acquire and orders the
+      // TMA reads after it with a proxy fence; that wait holds back only B.
+      tma_prefetch_desc(&p.b_map);
+      const uint64_t pol_last = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0, issued = 0, issued_par = 0;
+      for (int it = 0;; ++it) {
+        int tile;
+        int4 rec = make_int4(0, 0, 0, 0);
+        if constexpr (claims_tiles<MODE>()) {
+          const int slot = it % GEMM_SCHED;
+          if (!mbar_wait(&sched_full[slot], (it / GEMM_SCHED) & 1, p.err)) {
+            *abort_flag = 1;
+            break;
+          }
+          tile = sched[slot];
+          rec = sched_rec[slot];
+          mbar_arrive(&sched_empty[slot]);
+          if (tile < 0) break;
+        } else {
+          tile = blockIdx.x + it * gridDim.x;
+          if (tile >= n_tiles) break;
+        }
+        if (*abort_flag) break;
+        GemmTile t;
+        decode_tile<MODE>(p, tile, rec, n_gu, t);
+        if constexpr (MODE == GEMM_MOE) {
+          if (t.kind == KIND_DOWN && !wait_chunk_ready(p, t)) {
+            *abort_flag = 1;
+            break;
+          }
+        }
+        // B arrives in whole boxes (rows past nmma are loaded, zero-filled
+        // past the tensor's end, and ignored by the MMA)
+        const int b_rows = (t.nmma + p.b_box_rows - 1) / p.b_box_rows * p.b_box_rows;
+        const uint32_t bytes = b_rows * GEMM_BK * 2;
+        for (int k = 0; k < t.nk; ++k) {
+          if (!mbar_wait(&b_empty[stage], phase ^ 1, p.err)) {
+            *abort_flag = 1;
+            break;
+          }
+          mbar_arrive_expect_tx(&b_full[stage], bytes);
+          uint8_t* b = sB + stage * B_BYTES;
+          const int kx = (t.k0 + k) * GEMM_BK;
+          int r = 0;
+          if (p.b_mid_rows > 0)
+            for (; r + p.b_mid_rows <= t.nmma; r += p.b_mid_rows)
+              tma_load_2d(b + r * (GEMM_BK * 2), t.b_mid, &b_full[stage], kx, t.b_row + r, pol_last);
+          for (; r < t.nmma; r += p.b_box_rows)
+            tma_load_2d(b + r * (GEMM_BK * 2), t.b, &b_full[stage], kx, t.b_row + r, pol_last);
+          issued |= 1u << stage;
+          issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == SB) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (*abort_flag) break;
+      }
+      for (int s = 0; s < SB; ++s)
+        if ((issued >> s) & 1) mbar_wait(&b_full[s], (issued_par >> s) & 1, p.err);
     }
   } else if (warp == 1) {
     // ------------------------------ MMA issuer --------------------------------
     if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
+      int sa = 0, sb = 0;
+      uint32_t pa = 0, pb = 0;
       bool aborted = false;
       for (int it = 0;; ++it) {
         int tile;
@@ -627,13 +682,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
         const bool a_mn = MODE == GEMM_DENSE && p.a_mn_major;
         const uint32_t idesc = umma_idesc_bf16(GEMM_BM, t.nmma) | (a_mn ? (1u << 15) : 0u);
         for (int k = 0; k < t.nk; ++k) {
-          if (!mbar_wait(&full[stage], phase, p.err)) {
+          if (!mbar_wait(&a_full[sa], pa, p.err) || (!JOINT && !mbar_wait(&b_full[sb], pb, p.err))) {
             aborted = true;
             break;
           }
           tc_fence_after();
-          const uint32_t a_at = smem_u32(sA + stage * GEMM_A_BYTES);
-          const uint64_t bd = umma_desc_sw128(smem_u32(sB + stage * B_BYTES));
+          const uint32_t a_at = smem_u32(sA + sa * GEMM_A_BYTES);
+          const uint64_t bd = umma_desc_sw128(smem_u32(sB + sb * B_BYTES));
           if (a_mn) {
             // MN-major A: 16 k-rows are 2048 bytes; the two 64-wide m blocks are GEMM_A_BYTES / 2 apart
 #pragma unroll
@@ -646,10 +701,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
             for (int kk = 0; kk < GEMM_BK / 16; ++kk)
               umma_bf16(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (k | kk) != 0);
           }
-          umma_commit(&empty[stage]);
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1;
+          umma_commit(&a_empty[sa]);
+          if (!JOINT) umma_commit(&b_empty[sb]);
+          if (++sa == SA) {
+            sa = 0;
+            pa ^= 1;
+          }
+          if (++sb == SB) {
+            sb = 0;
+            pb ^= 1;
           }
         }
         if (aborted) break;
@@ -662,7 +722,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
       }
     }
   } else {
-    // ------------------------------ epilogue ----------------------------------
+    // ------------------------------ epilogue (warps 2-5) -----------------------
     const int q = warp & 3;              // TMEM lane quarter this warp may access
     const int row = q * 32 + lane;       // tile row owned by this thread
     const int etid = threadIdx.x - 64;   // 0..127

@@ -112,6 +112,7 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
                                                           int k, const float* __restrict__ bias,
                                                           int32_t* __restrict__ idx_out,
                                                           float* __restrict__ gates_out) {
+  DG_TIMELINE_SCOPE(TLK_ROUTER_TOPK);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * (blockDim.x >> 5) + warp;
   if (row >= T) return;
@@ -145,6 +146,7 @@ __global__ void __launch_bounds__(256) route_dispatch_kernel(
     int32_t* __restrict__ idx_out, float* __restrict__ gates_out, int32_t* __restrict__ capture,
     int32_t* __restrict__ cursor, int region, int d, const uint16_t* __restrict__ u, uint16_t* __restrict__ xp,
     int32_t* __restrict__ inv_slot) {
+  DG_TIMELINE_SCOPE(TLK_ROUTE_DISPATCH);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * (blockDim.x >> 5) + warp;
   if (row >= T) return;
@@ -232,6 +234,7 @@ __global__ void __launch_bounds__(512) combine_norm_kernel(
     float* __restrict__ h, const float* __restrict__ yp, const int32_t* __restrict__ inv_slot,
     const float* __restrict__ gates, int k, int shared_base, int d, const uint16_t* __restrict__ gain, float eps,
     uint16_t* __restrict__ u, float* __restrict__ capture) {
+  DG_TIMELINE_SCOPE(TLK_COMBINE_NORM);
   __shared__ float red[32];
   __shared__ int slot[ROW_MAX_K];
   __shared__ float gw[ROW_MAX_K];
@@ -299,6 +302,7 @@ __global__ void __launch_bounds__(1024) embed_norm_kernel(
     const int32_t* __restrict__ tokens, int tok_stride, int tok_off, int n, const uint16_t* __restrict__ embed,
     const uint16_t* __restrict__ gain, float eps, int d, float* __restrict__ h, uint16_t* __restrict__ u,
     float* __restrict__ capture, int32_t* settled, int n_settled, int vocab, const float* __restrict__ add) {
+  DG_TIMELINE_SCOPE(TLK_EMBED_NORM);
   __shared__ float red[32];
   const int row = blockIdx.x, c = threadIdx.x;
   const int b = row / n, i = row % n;
@@ -320,6 +324,7 @@ __global__ void __launch_bounds__(1024) embed_norm_kernel(
 __global__ void __launch_bounds__(1024) residual_norm_kernel(
     float* __restrict__ h, const float* __restrict__ part, int splits, int T, int d,
     const uint16_t* __restrict__ gain, float eps, uint16_t* __restrict__ u) {
+  DG_TIMELINE_SCOPE(TLK_RESIDUAL_NORM);
   __shared__ float red[32];
   const int row = blockIdx.x, c = threadIdx.x;
   const bool valid = c < d / 4;
@@ -346,6 +351,7 @@ __global__ void __launch_bounds__(1024) residual_norm_kernel(
 __global__ void __launch_bounds__(1024) reduce_splits_kernel(const float* __restrict__ part, int splits, int T,
                                                              int width, float* __restrict__ out_f32,
                                                              uint16_t* __restrict__ out_bf16) {
+  DG_TIMELINE_SCOPE(TLK_REDUCE_SPLITS);
   const int row = blockIdx.x, c = threadIdx.x;
   if (c >= width / 4) return;
   float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -365,6 +371,7 @@ __global__ void __launch_bounds__(1024) reduce_splits_kernel(const float* __rest
 __global__ void __launch_bounds__(1024) swiglu_splits_kernel(const float* __restrict__ gate, const float* __restrict__ part,
                                                              int splits, int T, int width,
                                                              uint16_t* __restrict__ out_bf16) {
+  DG_TIMELINE_SCOPE(TLK_SWIGLU_SPLITS);
   const int row = blockIdx.x, c = threadIdx.x;
   if (c >= width / 4) return;
   const float4 g = reinterpret_cast<const float4*>(gate + static_cast<size_t>(row) * width)[c];
@@ -396,6 +403,7 @@ __global__ void __launch_bounds__(ROPE_MAX_THREADS) rope_qkv_kernel(
     const float* __restrict__ part, int splits, int T, int n, int pos0, int Hq, int Hkv, int D,
     const float2* __restrict__ rope_tab, uint16_t* __restrict__ q, uint16_t* __restrict__ kc,
     uint16_t* __restrict__ vc, int S_max) {
+  DG_TIMELINE_SCOPE(TLK_ROPE_QKV);
   const int row = blockIdx.x;
   const int b = row / n, i = row % n;
   const int pos = pos0 + i;
@@ -542,6 +550,7 @@ __device__ __forceinline__ int sample_decision(int argmax, float conf, float tau
 }
 
 __global__ void lmhead_merge_sample_kernel(const float4* __restrict__ part, SampleArgs a) {
+  DG_TIMELINE_SCOPE(TLK_LMHEAD_MERGE_SAMPLE);
   const int t = blockIdx.x;
   const Top2 acc = merge_token_partials(part, a.s1, a.n_vtiles, a.T, t);
   if (threadIdx.x == 0) {
@@ -590,6 +599,7 @@ struct EntropyArgs {
 };
 
 __global__ void __launch_bounds__(256) entropy_sample_kernel(EntropyArgs a) {
+  DG_TIMELINE_SCOPE(TLK_ENTROPY_SAMPLE);
   __shared__ float se[256];
   __shared__ int order[256];
   __shared__ int s_count;
@@ -644,6 +654,7 @@ __global__ void __launch_bounds__(256) entropy_sample_kernel(EntropyArgs a) {
 __global__ void sample_only_kernel(const int32_t* __restrict__ argmax, const float* __restrict__ conf, int T,
                                    int C, int P, int step, uint32_t seed_lo, uint32_t seed_hi, float tau,
                                    int vocab, int32_t* __restrict__ out) {
+  DG_TIMELINE_SCOPE(TLK_SAMPLE_ONLY);
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
   if (t >= T) return;
   out[t] = sample_decision(argmax[t], conf[t], tau, P + t % C, step, t / C, seed_lo, seed_hi, vocab);
@@ -651,6 +662,7 @@ __global__ void sample_only_kernel(const int32_t* __restrict__ argmax, const flo
 
 // waits on a barrier that is never signalled; the bounded wait must give up
 __global__ void wait_timeout_kernel(DevErr err) {
+  DG_TIMELINE_SCOPE(TLK_OTHER);
   __shared__ uint64_t bar;
   if (threadIdx.x == 0) {
     mbar_init(&bar, 1);

@@ -313,6 +313,48 @@ dg_status dg_debug_profile_read(dg_ctx* ctx, int32_t cls, double* total_ms, int6
 int64_t dg_debug_launch_count(const dg_ctx* ctx);
 
 /* ---------------------------------------------------------------------------
+ * Timeline (tracing).  libdg_timeline.so is this library compiled with
+ * -DDG_TIMELINE: thread 0 of every CTA of every kernel appends one record
+ * {start ns, end ns (%globaltimer, taken when thread 0 leaves the kernel),
+ * kernel id, CTA index} to a device buffer of 262144 records shared by all
+ * contexts of the process (records past its end are dropped).  Launches run one after another on the context's
+ * stream, so sorting the records by start time and grouping consecutive
+ * records of one kernel id recovers the launch sequence of a graph replay
+ * with every launch's span and the gaps between launches.  In libdg.so both
+ * calls return DG_ERR_UNSUPPORTED.
+ *
+ * Kernel ids: DG_K_GEMM_DENSE 10, DG_K_GEMM_MOE 11, DG_K_GEMM_LMHEAD 13,
+ * DG_K_ATTENTION 20, DG_K_ROUTE_DISPATCH 30, DG_K_COMBINE_NORM 31,
+ * DG_K_EMBED_NORM 32, DG_K_RESIDUAL_NORM 33, DG_K_REDUCE_SPLITS 34,
+ * DG_K_SWIGLU_SPLITS 35, DG_K_ROPE_QKV 36, DG_K_LMHEAD_MERGE_SAMPLE 37,
+ * DG_K_ENTROPY_SAMPLE 38, DG_K_ROUTER_TOPK 39, DG_K_SAMPLE_ONLY 40,
+ * DG_K_OTHER 50.
+ * ------------------------------------------------------------------------- */
+enum {
+  DG_K_GEMM_DENSE = 10, DG_K_GEMM_MOE = 11, DG_K_GEMM_LMHEAD = 13, DG_K_ATTENTION = 20,
+  DG_K_ROUTE_DISPATCH = 30, DG_K_COMBINE_NORM = 31, DG_K_EMBED_NORM = 32, DG_K_RESIDUAL_NORM = 33,
+  DG_K_REDUCE_SPLITS = 34, DG_K_SWIGLU_SPLITS = 35, DG_K_ROPE_QKV = 36, DG_K_LMHEAD_MERGE_SAMPLE = 37,
+  DG_K_ENTROPY_SAMPLE = 38, DG_K_ROUTER_TOPK = 39, DG_K_SAMPLE_ONLY = 40, DG_K_OTHER = 50
+};
+
+typedef struct {
+  uint64_t t0_ns;  /* CTA start */
+  uint64_t t1_ns;  /* CTA end (thread 0) */
+  int32_t kernel;  /* DG_K_* */
+  int32_t cta;     /* linear CTA index in its grid */
+} dg_timeline_record;
+
+/* Synchronise ctx's stream and empty the record buffer. */
+dg_status dg_debug_timeline_reset(dg_ctx* ctx);
+
+/* Synchronise ctx's stream and copy up to `capacity` records (in the order
+ * they were appended) to host_records (caller-owned host memory); *n_records
+ * receives the number appended since the last reset, which may exceed
+ * capacity (and 262144, when records were dropped). */
+dg_status dg_debug_timeline(dg_ctx* ctx, dg_timeline_record* host_records, int32_t capacity,
+                            int64_t* n_records);
+
+/* ---------------------------------------------------------------------------
  * LM-head reduction without any device allocation.
  *
  * The pages describe nothing like this; it is a deployment convenience.  It
