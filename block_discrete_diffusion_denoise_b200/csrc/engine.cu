@@ -569,7 +569,7 @@ dg_status lm_head(dg_ctx* c, int T, float temperature) {
   p.M = T;
   p.k_steps = c->d / 64;
   p.n_mtiles = (T + GEMM_BM - 1) / GEMM_BM;
-  p.tiles_static = (c->V / GEMM_BN) * p.n_mtiles;
+  p.tiles_static = (c->V / GEMM_BN) * lmhead_mpairs(p.n_mtiles);
   p.lm_part = c->lm_part;
   p.lm_s1 = c->lm_s1;
   p.logit_scale_log2 = static_cast<float>(1.4426950408889634 / static_cast<double>(temperature));
@@ -615,7 +615,7 @@ dg_status self_condition(dg_ctx* c, int T, float temperature) {
     p.M = T;
     p.k_steps = c->d / 64;
     p.n_mtiles = (T + GEMM_BM - 1) / GEMM_BM;
-    p.tiles_static = (c->V / GEMM_BN) * p.n_mtiles;
+    p.tiles_static = (c->V / GEMM_BN) * lmhead_mpairs(p.n_mtiles);
     p.lse2 = c->sc_lse2;
     p.p_map = c->m_scP_store;
     p.logit_scale_log2 = static_cast<float>(1.4426950408889634 / static_cast<double>(temperature));
@@ -1661,7 +1661,7 @@ extern "C" dg_status dg_lmhead_argmax_static(const void* z, int32_t n_rows, int3
   p.M = n_rows;
   p.k_steps = d_model / 64;
   p.n_mtiles = (n_rows + GEMM_BM - 1) / GEMM_BM;
-  p.tiles_static = n_vtiles * p.n_mtiles;
+  p.tiles_static = n_vtiles * lmhead_mpairs(p.n_mtiles);
   p.lm_part = su.partials;
   p.logit_scale_log2 = static_cast<float>(1.4426950408889634 / static_cast<double>(temperature));
   p.err = DevErr{su.err, 1000000000ull};

@@ -54,18 +54,27 @@ constexpr int MOE_MAX_EXPERTS = 256;                 // routed experts (+1 share
 // MOE tile tables in shared memory: chunk offsets [E + 2] and group rows [E + 1], 16-bit
 constexpr int MOE_TABLE_BYTES = ((MOE_MAX_EXPERTS + 2) + (MOE_MAX_EXPERTS + 1)) * 2 + 32;
 
-// Ring depths.  A (16 KB per stage) and B (the B rows of one k-step per
-// stage) have rings of their own, filled by two producer lanes, so the
-// operand streamed from HBM can run further ahead than the one read from L2:
-// in MOE the expert weights (A) run 8 k-steps ahead, the gathered rows (B) 4.
+// Stage ring depth (16 KB of A plus the B rows of one k-step per stage).
+// Two producers fill each stage: warp 0 its A half, warp 6 its B half (the
+// stage's full barrier takes two arrivals), so a wait that holds back one
+// operand (a down tile's dependency) does not stop the other's loads.
 template <int MODE>
-constexpr int gemm_stages_a() {
-  return MODE == GEMM_DENSE ? 4 : (MODE == GEMM_MOE ? 8 : 6);
+constexpr int gemm_stages() {
+  return MODE == GEMM_MOE ? 6 : 4;
+}
+// 128-row A tiles per CTA tile: the LM head takes two token tiles (256
+// tokens) per vocabulary block, so each 128-row block of the embedding is
+// loaded once for both and L2 carries a third less operand traffic
+template <int MODE>
+constexpr int gemm_halves() {
+  return MODE == GEMM_LMHEAD ? 2 : 1;
 }
 template <int MODE>
-constexpr int gemm_stages_b() {
-  return MODE == GEMM_DENSE ? 4 : (MODE == GEMM_MOE ? 4 : 6);
+constexpr int gemm_a_bytes() {
+  return GEMM_A_BYTES * gemm_halves<MODE>();
 }
+// LM-head tiles per vocabulary block: pairs of 128-token tiles
+__host__ __device__ constexpr int lmhead_mpairs(int n_mtiles) { return (n_mtiles + 1) / 2; }
 // rows of B one stage holds
 template <int MODE>
 constexpr int gemm_b_rows() {
@@ -82,8 +91,8 @@ constexpr int gemm_acc_cols() {
 }
 template <int MODE>
 constexpr int gemm_smem_bytes() {
-  return 1024 + gemm_stages_a<MODE>() * GEMM_A_BYTES + gemm_stages_b<MODE>() * gemm_b_bytes<MODE>() +
-         GEMM_XCHG_FLOATS * 4 + 512 + (MODE == GEMM_MOE ? MOE_TABLE_BYTES : 0);
+  return 1024 + gemm_stages<MODE>() * (gemm_a_bytes<MODE>() + gemm_b_bytes<MODE>()) + GEMM_XCHG_FLOATS * 4 + 512 +
+         (MODE == GEMM_MOE ? MOE_TABLE_BYTES : 0);
 }
 
 enum TileKind : int { KIND_DENSE = 0, KIND_GATEUP = 1, KIND_DOWN = 2, KIND_LMHEAD = 3 };
@@ -149,6 +158,7 @@ struct GemmTile {
   int k0, nk;
   int split, group, blk, chunk;
   int kind;
+  int halves;     // 128-row A tiles (LMHEAD: 1 or 2 token tiles)
   bool shared;
   bool a_stream;  // A is read once (evict-first)
 };
@@ -160,6 +170,7 @@ template <int MODE>
 __device__ __forceinline__ void decode_tile(const GemmParams& p, int tile, int4 rec, int n_gu, GemmTile& t) {
   t.chunk = 0;
   t.shared = false;
+  t.halves = 1;
   if constexpr (MODE == GEMM_DENSE) {
     const int nt = tile % p.n_tiles_n;
     const int rest = tile / p.n_tiles_n;
@@ -180,12 +191,14 @@ __device__ __forceinline__ void decode_tile(const GemmParams& p, int tile, int4 
     t.blk = mt;
     t.a_stream = p.n_tiles_n == 1;
   } else if constexpr (MODE == GEMM_LMHEAD) {
-    const int vt = tile / p.n_mtiles;
-    const int mt = tile % p.n_mtiles;
+    const int np = lmhead_mpairs(p.n_mtiles);
+    const int vt = tile / np;
+    const int mp = tile % np;
     t.kind = KIND_LMHEAD;
     t.a0 = &p.a_map[0];
     t.a1 = nullptr;
-    t.a_row = mt * GEMM_BM;
+    t.a_row = mp * 2 * GEMM_BM;
+    t.halves = min(2, p.n_mtiles - 2 * mp);
     t.b = &p.b_map;
     t.b_mid = &p.b_mid_map;
     t.b_row = vt * GEMM_BN;
@@ -195,7 +208,7 @@ __device__ __forceinline__ void decode_tile(const GemmParams& p, int tile, int4 
     t.nk = p.k_steps;
     t.split = 0;
     t.group = vt;
-    t.blk = mt;
+    t.blk = mp;
     t.a_stream = false;
   } else {
     const int4 e = rec;
@@ -392,26 +405,21 @@ constexpr bool claims_tiles() {
 template <int MODE>
 __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_constant__ GemmParams p) {
   DG_TIMELINE_SCOPE(TLK_GEMM + MODE);
-  constexpr int SA = gemm_stages_a<MODE>();
-  constexpr int SB = gemm_stages_b<MODE>();
+  constexpr int STAGES = gemm_stages<MODE>();
+  constexpr int A_BYTES = gemm_a_bytes<MODE>();
+  constexpr int HALVES = gemm_halves<MODE>();
   constexpr int B_BYTES = gemm_b_bytes<MODE>();
   static_assert(gemm_smem_bytes<MODE>() <= 232448, "shared memory per CTA");
-  static_assert((2 * (SA + SB) + 5 + 2 * GEMM_SCHED) * 8 + GEMM_SCHED * 20 + 64 <= 512, "barrier area");
+  static_assert((2 * STAGES + 5 + 2 * GEMM_SCHED) * 8 + GEMM_SCHED * 20 + 64 <= 512, "barrier area");
   constexpr int ACC_COLS = gemm_acc_cols<MODE>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
-  uint8_t* sB = sA + SA * GEMM_A_BYTES;
-  float* xchg = reinterpret_cast<float*>(sB + SB * B_BYTES);
-  // Equal depths (DENSE, LMHEAD): one ring whose stages both producers fill
-  // (full barrier of two arrivals), so the MMA issuer waits and commits once
-  // per k-step.  Otherwise (MOE) two rings.
-  constexpr bool JOINT = SA == SB;
-  uint64_t* a_full = reinterpret_cast<uint64_t*>(xchg + GEMM_XCHG_FLOATS);
-  uint64_t* a_empty = a_full + SA;
-  uint64_t* b_full = JOINT ? a_full : a_empty + SA;
-  uint64_t* b_empty = JOINT ? a_empty : b_full + SB;
-  uint64_t* tfull = JOINT ? a_empty + SA : b_empty + SB;
+  uint8_t* sB = sA + STAGES * A_BYTES;
+  float* xchg = reinterpret_cast<float*>(sB + STAGES * B_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(xchg + GEMM_XCHG_FLOATS);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint64_t* sched_full = drain + 1;
@@ -458,15 +466,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
   }
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < SA; ++s) {
-      mbar_init(&a_full[s], JOINT ? 2 : 1);
-      mbar_init(&a_empty[s], 1);
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 2);  // the A and the B producer
+      mbar_init(&empty[s], 1);
     }
-    if (!JOINT)
-      for (int s = 0; s < SB; ++s) {
-        mbar_init(&b_full[s], 1);
-        mbar_init(&b_empty[s], 1);
-      }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], 128);
@@ -480,7 +483,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_holder, 2 * ACC_COLS);
+    tmem_alloc(tmem_holder, 2 * ACC_COLS * HALVES);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -493,9 +496,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
   if (warp == 0) {
     if (lane == 0) {
       // --------------------------- TMA producer of A ---------------------------
-      // Claims the tiles (MOE), publishes them to the other roles, and streams
-      // A.  It waits on nothing but free A slots, so the weight stream keeps
-      // SA k-steps in flight whatever B is waiting for.
+      // Claims the tiles (MOE), publishes them to the other roles, and fills
+      // the A half of each stage.
       tma_prefetch_desc(&p.a_map[0]);
       const uint64_t pol_first = policy_evict_first();
       const uint64_t pol_last = policy_evict_last();
@@ -543,24 +545,26 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
         decode_tile<MODE>(p, tile, rec, n_gu, t);
         const uint64_t pol_a = t.a_stream ? pol_first : pol_last;
         for (int k = 0; k < t.nk; ++k) {
-          if (!mbar_wait(&a_empty[stage], phase ^ 1, p.err)) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, p.err)) {
             *abort_flag = 1;
             break;
           }
-          mbar_arrive_expect_tx(&a_full[stage], GEMM_A_BYTES);
-          uint8_t* a = sA + stage * GEMM_A_BYTES;
+          mbar_arrive_expect_tx(&full[stage], GEMM_A_BYTES * t.halves);
+          uint8_t* a = sA + stage * A_BYTES;
           const int kx = (t.k0 + k) * GEMM_BK;
           if (MODE == GEMM_DENSE && p.a_mn_major) {
             // A stored [K][M]: two boxes of 64 k-rows x 64 m-columns
-            tma_load_2d(a, t.a0, &a_full[stage], t.a_row, kx, pol_a);
-            tma_load_2d(a + GEMM_A_BYTES / 2, t.a0, &a_full[stage], t.a_row + 64, kx, pol_a);
+            tma_load_2d(a, t.a0, &full[stage], t.a_row, kx, pol_a);
+            tma_load_2d(a + GEMM_A_BYTES / 2, t.a0, &full[stage], t.a_row + 64, kx, pol_a);
           } else {
-            tma_load_2d(a, t.a0, &a_full[stage], kx, t.a_row, pol_a);
-            if (t.a1 != nullptr) tma_load_2d(a + GEMM_A_BYTES / 2, t.a1, &a_full[stage], kx, t.a_row, pol_a);
+            tma_load_2d(a, t.a0, &full[stage], kx, t.a_row, pol_a);
+            if (t.a1 != nullptr) tma_load_2d(a + GEMM_A_BYTES / 2, t.a1, &full[stage], kx, t.a_row, pol_a);
+            if (HALVES > 1 && t.halves > 1)
+              tma_load_2d(a + GEMM_A_BYTES, t.a0, &full[stage], kx, t.a_row + GEMM_BM, pol_a);
           }
           issued |= 1u << stage;
           issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
-          if (++stage == SA) {
+          if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
@@ -572,16 +576,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
         }
       }
       // every copy this thread issued has landed before the CTA may exit
-      for (int s = 0; s < SA; ++s)
-        if ((issued >> s) & 1) mbar_wait(&a_full[s], (issued_par >> s) & 1, p.err);
+      for (int s = 0; s < STAGES; ++s)
+        if ((issued >> s) & 1) mbar_wait(&full[s], (issued_par >> s) & 1, p.err);
     }
   } else if (warp == GEMM_B_WARP) {
     if (lane == 0) {
       // --------------------------- TMA producer of B ---------------------------
-      // Follows the same tiles.  A down tile's rows are the hidden rows its
-      // chunk's gate/up tiles publish, so before its first B load this lane
-      // waits (bounded) for the chunk's counter with acquire and orders the
-      // TMA reads after it with a proxy fence; that wait holds back only B.
+      // Follows the same tiles and fills the B half of each stage.  A down
+      // tile's rows are the hidden rows its chunk's gate/up tiles publish, so
+      // before its first B load this warp waits (bounded) for the chunk's
+      // counter with acquire and orders the TMA reads after it with a proxy
+      // fence; meanwhile the A producer keeps loading weights.
       tma_prefetch_desc(&p.b_map);
       const uint64_t pol_last = policy_evict_last();
       int stage = 0;
@@ -617,36 +622,36 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
         const int b_rows = (t.nmma + p.b_box_rows - 1) / p.b_box_rows * p.b_box_rows;
         const uint32_t bytes = b_rows * GEMM_BK * 2;
         for (int k = 0; k < t.nk; ++k) {
-          if (!mbar_wait(&b_empty[stage], phase ^ 1, p.err)) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, p.err)) {
             *abort_flag = 1;
             break;
           }
-          mbar_arrive_expect_tx(&b_full[stage], bytes);
+          mbar_arrive_expect_tx(&full[stage], bytes);
           uint8_t* b = sB + stage * B_BYTES;
           const int kx = (t.k0 + k) * GEMM_BK;
           int r = 0;
           if (p.b_mid_rows > 0)
             for (; r + p.b_mid_rows <= t.nmma; r += p.b_mid_rows)
-              tma_load_2d(b + r * (GEMM_BK * 2), t.b_mid, &b_full[stage], kx, t.b_row + r, pol_last);
+              tma_load_2d(b + r * (GEMM_BK * 2), t.b_mid, &full[stage], kx, t.b_row + r, pol_last);
           for (; r < t.nmma; r += p.b_box_rows)
-            tma_load_2d(b + r * (GEMM_BK * 2), t.b, &b_full[stage], kx, t.b_row + r, pol_last);
+            tma_load_2d(b + r * (GEMM_BK * 2), t.b, &full[stage], kx, t.b_row + r, pol_last);
           issued |= 1u << stage;
           issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
-          if (++stage == SB) {
+          if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
         if (*abort_flag) break;
       }
-      for (int s = 0; s < SB; ++s)
-        if ((issued >> s) & 1) mbar_wait(&b_full[s], (issued_par >> s) & 1, p.err);
+      for (int s = 0; s < STAGES; ++s)
+        if ((issued >> s) & 1) mbar_wait(&full[s], (issued_par >> s) & 1, p.err);
     }
   } else if (warp == 1) {
     // ------------------------------ MMA issuer --------------------------------
     if (lane == 0) {
-      int sa = 0, sb = 0;
-      uint32_t pa = 0, pb = 0;
+      int stage = 0;
+      uint32_t phase = 0;
       bool aborted = false;
       for (int it = 0;; ++it) {
         int tile;
@@ -678,17 +683,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
+        const uint32_t d_tmem = tmem_base + acc * ACC_COLS * HALVES;
         const bool a_mn = MODE == GEMM_DENSE && p.a_mn_major;
         const uint32_t idesc = umma_idesc_bf16(GEMM_BM, t.nmma) | (a_mn ? (1u << 15) : 0u);
         for (int k = 0; k < t.nk; ++k) {
-          if (!mbar_wait(&a_full[sa], pa, p.err) || (!JOINT && !mbar_wait(&b_full[sb], pb, p.err))) {
+          if (!mbar_wait(&full[stage], phase, p.err)) {
             aborted = true;
             break;
           }
           tc_fence_after();
-          const uint32_t a_at = smem_u32(sA + sa * GEMM_A_BYTES);
-          const uint64_t bd = umma_desc_sw128(smem_u32(sB + sb * B_BYTES));
+          const uint32_t a_at = smem_u32(sA + stage * A_BYTES);
+          const uint64_t bd = umma_desc_sw128(smem_u32(sB + stage * B_BYTES));
           if (a_mn) {
             // MN-major A: 16 k-rows are 2048 bytes; the two 64-wide m blocks are GEMM_A_BYTES / 2 apart
 #pragma unroll
@@ -700,16 +705,18 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
 #pragma unroll
             for (int kk = 0; kk < GEMM_BK / 16; ++kk)
               umma_bf16(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (k | kk) != 0);
+            if (HALVES > 1 && t.halves > 1) {
+              // the second token tile against the same B (vocabulary) tile
+              const uint64_t ad1 = umma_desc_sw128(a_at + GEMM_A_BYTES);
+#pragma unroll
+              for (int kk = 0; kk < GEMM_BK / 16; ++kk)
+                umma_bf16(d_tmem + ACC_COLS, ad1 + 2 * kk, bd + 2 * kk, idesc, (k | kk) != 0);
+            }
           }
-          umma_commit(&a_empty[sa]);
-          if (!JOINT) umma_commit(&b_empty[sb]);
-          if (++sa == SA) {
-            sa = 0;
-            pa ^= 1;
-          }
-          if (++sb == SB) {
-            sb = 0;
-            pb ^= 1;
+          umma_commit(&empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
           }
         }
         if (aborted) break;
@@ -764,7 +771,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
         break;
       }
       tc_fence_after();
-      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * ACC_COLS;
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * ACC_COLS * HALVES;
 
       if constexpr (MODE == GEMM_DENSE) {
         float* out = p.out_f32 + static_cast<size_t>(t.split) * p.T * p.M +
@@ -848,15 +855,18 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
           }
         }
       } else if (p.lse2 != nullptr) {  // GEMM_LMHEAD, probability mode
-        // the previous tile's store must have read the staging area
+        for (int h = 0; h < t.halves; ++h) {
+        const uint32_t th = tbase + h * ACC_COLS;
+        const int y0 = t.a_row + h * GEMM_BM;
+        // the previous store must have read the staging area
         if (etid == 0) bulk_wait_read_all();
         named_bar_sync(1, 128);
-        const int tok = t.a_row + row;
+        const int tok = y0 + row;
         const float ref = tok < p.M ? p.lse2[tok] : 0.f;
         uint8_t* stg = reinterpret_cast<uint8_t*>(xchg);
         for (int c0 = 0; c0 < GEMM_BN; c0 += 32) {
           float v[32];
-          tmem_ld32(tbase + c0, v);
+          tmem_ld32(th + c0, v);
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i)
@@ -875,17 +885,20 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
         fence_proxy_async_smem();
         named_bar_sync(1, 128);
         if (etid == 0) {
-          tma_store_2d(&p.p_map, stg, t.b_row, t.a_row);
-          tma_store_2d(&p.p_map, stg + GEMM_BM * 128, t.b_row + 64, t.a_row);
+          tma_store_2d(&p.p_map, stg, t.b_row, y0);
+          tma_store_2d(&p.p_map, stg + GEMM_BM * 128, t.b_row + 64, y0);
           bulk_commit_group();
         }
+        }
       } else {  // GEMM_LMHEAD
-        const int tok = t.a_row + row;
+        for (int h = 0; h < t.halves; ++h) {
+        const uint32_t th = tbase + h * ACC_COLS;
+        const int tok = t.a_row + h * GEMM_BM + row;
         float m1 = -INFINITY, m2 = -INFINITY, s = 0.f, s1 = 0.f;
         int idx = 0x7fffffff;
         for (int c0 = 0; c0 < GEMM_BN; c0 += 32) {
           float v[32];
-          tmem_ld32(tbase + c0, v);
+          tmem_ld32(th + c0, v);
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const float x = v[i] * p.logit_scale_log2;
@@ -908,6 +921,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
           p.lm_part[static_cast<size_t>(t.group) * p.M + tok] = make_float4(m1, __int_as_float(idx), m2, s);
           if (p.lm_s1) p.lm_s1[static_cast<size_t>(t.group) * p.M + tok] = s1;
         }
+        }
       }
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
@@ -920,7 +934,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, 2 * ACC_COLS);
+    tmem_dealloc(tmem_base, 2 * ACC_COLS * HALVES);
   }
   if constexpr (claims_tiles<MODE>()) {
     // the last CTA out resets, for the next launch, the claim counter, the
