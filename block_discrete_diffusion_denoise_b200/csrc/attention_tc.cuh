@@ -119,6 +119,10 @@ __global__ void __launch_bounds__(ATC_THREADS, 1) attn_tc_kernel(const __grid_co
   const int kv_row0 = (b * p.Hkv + kvh) * p.S_max + kbeg;
 
   if (threadIdx.x == 0) {
+    // the descriptors are fetched while the CTA sets up
+    tma_prefetch_desc(&p.q_map);
+    tma_prefetch_desc(&p.k_map);
+    tma_prefetch_desc(&p.v_map);
     mbar_init(q_full, 1);
     for (int s = 0; s < ATC_KSTAGES; ++s) {
       mbar_init(&k_full[s], 1);

@@ -451,7 +451,10 @@ dg_status moe(dg_ctx* c, int l, int T, bool record) {
   ProfScope ps3(c, DG_PROF_ROUTING);
   // expert e's rows: [e * T, e * T + rows_e) (a region per expert, T rows each)
   // two tokens (warps) per CTA: the k copies of every token's row spread over many SMs
-  DG_LAUNCH(c, route_dispatch_kernel, (T + 1) / 2, 64, 0, static_cast<const float*>(c->part), s3, T, c->E, c->k,
+  auto* dispatch = c->E <= 32 ? route_dispatch_kernel<1>
+                   : c->E <= 64 ? route_dispatch_kernel<2>
+                   : c->E <= 128 ? route_dispatch_kernel<4> : route_dispatch_kernel<ROUTE_PER>;
+  DG_LAUNCH(c, dispatch, T, 32 * c->k, 0, static_cast<const float*>(c->part), s3, T, c->E, c->k,
             c->router_bias, c->idx, c->gates, cap, c->expert_rows, T, c->d, static_cast<const uint16_t*>(c->u),
             c->xp, c->inv_slot);
   ps3.end();

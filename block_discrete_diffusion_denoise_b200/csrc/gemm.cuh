@@ -436,6 +436,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
+  // the operand descriptors are fetched while the CTA sets up
+  if (threadIdx.x == 0) {
+    tma_prefetch_desc(&p.a_map[0]);
+    tma_prefetch_desc(&p.b_map);
+  }
   MoeTables tb{tb_ch_off, tb_rows, 0, 0, 0};
   if constexpr (MODE == GEMM_MOE) {
     // tile tables from the row counts (two groups per thread, G <= 2 * GEMM_THREADS)
@@ -781,21 +786,24 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
           // MMAs this accumulator waited for, so the ring is free.  Stage the
           // tile as [token][128 features] fp32 (a warp writes 128 contiguous
           // bytes per token) and store it with TMA, 64 tokens per box.
+          // Each 64-token box is stored as soon as it is staged, so the
+          // stores overlap the staging of the next box.  Before the CTA exits
+          // the stores must have read shared memory; kernel completion makes
+          // their writes visible to the next launch.
           float* stage = reinterpret_cast<float*>(sA);
           for (int c0 = 0; c0 < t.n; c0 += 64) {
             float v[64];
             tmem_ld64(tbase + c0, v);
 #pragma unroll
             for (int i = 0; i < 64; ++i) stage[(c0 + i) * GEMM_BM + row] = v[i];
-          }
-          fence_proxy_async_smem();
-          named_bar_sync(1, 128);
-          if (etid == 0) {
-            for (int c0 = 0; c0 < t.n; c0 += 64)
+            fence_proxy_async_smem();
+            named_bar_sync(1, 128);
+            if (etid == 0) {
               tma_store_3d(&p.out_map, stage + c0 * GEMM_BM, t.a_row, t.b_row + c0, t.split);
-            bulk_commit_group();
-            bulk_wait_all();
+              bulk_commit_group();
+            }
           }
+          if (etid == 0) bulk_wait_read_all();
         } else
         for (int c0 = 0; c0 < t.n; c0 += 64) {
           float v[64];
@@ -928,7 +936,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
     }
   }
 
-  if (MODE == GEMM_LMHEAD && p.lse2 != nullptr && threadIdx.x == 64) bulk_wait_all();
+  // bulk stores have read shared memory before it is released (kernel
+  // completion makes their writes visible to the next launch)
+  if (MODE == GEMM_LMHEAD && p.lse2 != nullptr && threadIdx.x == 64) bulk_wait_read_all();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

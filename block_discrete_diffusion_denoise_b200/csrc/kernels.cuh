@@ -33,14 +33,15 @@ __device__ __forceinline__ int uniform_token(uint32_t w, int vocab) {
 }
 
 // Router decision of one row, held by one warp: v[c] is the logit of expert
-// c * 32 + lane (-inf past E).  Top-k by (logit desc, index asc); lane r < k
-// receives the r-th selection (my_v, my_i); every lane receives the largest
-// logit (top_v).  k <= 16 < 32.
+// c * 32 + lane (-inf past E), PER >= E / 32 logits per lane.  Top-k by
+// (logit desc, index asc); lane r < k receives the r-th selection (my_v,
+// my_i); every lane receives the largest logit (top_v).  k <= 16 < 32.
 constexpr int PERM_MAXE = 256;
 constexpr int ROUTE_PER = PERM_MAXE / 32;
 
-__device__ __forceinline__ void warp_topk(const float (&v)[ROUTE_PER], int E, int k, int lane, float& my_v,
-                                          int& my_i, float& top_v) {
+template <int PER>
+__device__ __forceinline__ void warp_topk(const float (&v)[PER], int E, int k, int lane, float& my_v, int& my_i,
+                                          float& top_v) {
   uint32_t taken = 0;
   my_v = -INFINITY;
   top_v = -INFINITY;
@@ -49,7 +50,7 @@ __device__ __forceinline__ void warp_topk(const float (&v)[ROUTE_PER], int E, in
     float bv = -INFINITY;
     int bi = 0x7fffffff;
 #pragma unroll
-    for (int c = 0; c < ROUTE_PER; ++c) {
+    for (int c = 0; c < PER; ++c) {
       const int e = c * 32 + lane;
       if (e < E && !((taken >> c) & 1) && (v[c] > bv || (v[c] == bv && e < bi) || bi == 0x7fffffff)) {
         bv = v[c];
@@ -75,25 +76,26 @@ __device__ __forceinline__ void warp_topk(const float (&v)[ROUTE_PER], int E, in
 
 // logits of one row from split-K partials part[s][row][e] summed in split
 // order, plus the per-expert bias
+template <int PER>
 __device__ __forceinline__ void router_logits_row(const float* __restrict__ part, int splits, int T, int row, int E,
-                                                  const float* __restrict__ bias, int lane, float (&v)[ROUTE_PER]) {
+                                                  const float* __restrict__ bias, int lane, float (&v)[PER]) {
   constexpr int MAXS = 8;  // split-K partials (the dense GEMM uses at most 8)
 #pragma unroll
-  for (int c = 0; c < ROUTE_PER; ++c) v[c] = (c * 32 + lane < E) ? 0.f : -INFINITY;
+  for (int c = 0; c < PER; ++c) v[c] = (c * 32 + lane < E) ? 0.f : -INFINITY;
 #pragma unroll
   for (int s = 0; s < MAXS; ++s)
     if (s < splits) {
-      float t[ROUTE_PER];
+      float t[PER];
 #pragma unroll
-      for (int c = 0; c < ROUTE_PER; ++c)
+      for (int c = 0; c < PER; ++c)
         if (c * 32 + lane < E) t[c] = part[(static_cast<size_t>(s) * T + row) * E + c * 32 + lane];
 #pragma unroll
-      for (int c = 0; c < ROUTE_PER; ++c)
+      for (int c = 0; c < PER; ++c)
         if (c * 32 + lane < E) v[c] += t[c];
     }
   if (bias) {
 #pragma unroll
-    for (int c = 0; c < ROUTE_PER; ++c)
+    for (int c = 0; c < PER; ++c)
       if (c * 32 + lane < E) v[c] += bias[c * 32 + lane];
   }
 }
@@ -117,10 +119,10 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
   const int row = blockIdx.x * (blockDim.x >> 5) + warp;
   if (row >= T) return;
   float v[ROUTE_PER];
-  router_logits_row(part, splits, T, row, E, bias, lane, v);
+  router_logits_row<ROUTE_PER>(part, splits, T, row, E, bias, lane, v);
   float my_v, top_v;
   int my_i;
-  warp_topk(v, E, k, lane, my_v, my_i, top_v);
+  warp_topk<ROUTE_PER>(v, E, k, lane, my_v, my_i, top_v);
   const float g = selected_gate(my_v, top_v, k, lane);
   if (lane < k) {
     idx_out[static_cast<size_t>(row) * k + lane] = my_i;
@@ -128,53 +130,57 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
   }
 }
 
-// Router decision and dispatch of one layer, one warp per token row (the same
-// decision as router_topk_kernel).  Expert e owns rows [e * region, e * region
-// + rows_e) of the routed buffers (gathered activations xp, hidden rows, down
-// outputs); each (row, slot) pair claims the next of them from cursor[e], so
-// cursor[e] ends as rows_e (zero before the launch; the expert GEMM's last CTA
-// zeroes it again).  The order of rows inside a region is free: every row of
-// an expert tile is an independent dot product, and the combine sums a token's
-// slots in slot order through inv_slot.  The warp then copies the token's
-// normalised row u[row] to its k claimed rows of xp.
+// Router decision and dispatch of one layer, one CTA of k warps per token row
+// (the same decision as router_topk_kernel).  Expert e owns rows [e * region,
+// e * region + rows_e) of the routed buffers (gathered activations xp, hidden
+// rows, down outputs); each (row, slot) pair claims the next of them from
+// cursor[e], so cursor[e] ends as rows_e (zero before the launch; the expert
+// GEMM's last CTA zeroes it again).  The order of rows inside a region is
+// free: every row of an expert tile is an independent dot product, and the
+// combine sums a token's slots in slot order through inv_slot.  Warp 0 takes
+// the decision and the claims; then warp j copies the token's normalised row
+// u[row] (which every warp loaded at the start, overlapping the decision) to
+// the row slot j claimed.
 //   idx, gates [T, k]; inv_slot[row * k + j] = claimed row of slot j;
-//   capture [T, k] or NULL (test hook)
+//   capture [T, k] or NULL (test hook).  blockDim = 32 * k, PER >= E / 32.
 constexpr int DISPATCH_MAXV = 16;  // 16-byte chunks per lane: d <= 32 * 16 * 8 = 4096
 
-__global__ void __launch_bounds__(256) route_dispatch_kernel(
+template <int PER>
+__global__ void __launch_bounds__(512) route_dispatch_kernel(
     const float* __restrict__ part, int splits, int T, int E, int k, const float* __restrict__ bias,
     int32_t* __restrict__ idx_out, float* __restrict__ gates_out, int32_t* __restrict__ capture,
     int32_t* __restrict__ cursor, int region, int d, const uint16_t* __restrict__ u, uint16_t* __restrict__ xp,
     int32_t* __restrict__ inv_slot) {
   DG_TIMELINE_SCOPE(TLK_ROUTE_DISPATCH);
+  __shared__ int dest[32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row = blockIdx.x * (blockDim.x >> 5) + warp;
-  if (row >= T) return;
-  // the row's activations are loaded first, so their latency overlaps the decision
+  const int row = blockIdx.x;
   const int vec = d / 8;
   const uint4* src = reinterpret_cast<const uint4*>(u) + static_cast<size_t>(row) * vec;
   uint4 x[DISPATCH_MAXV];
 #pragma unroll
   for (int i = 0; i < DISPATCH_MAXV; ++i)
     if (lane + 32 * i < vec) x[i] = src[lane + 32 * i];
-  float v[ROUTE_PER];
-  router_logits_row(part, splits, T, row, E, bias, lane, v);
-  float my_v, top_v;
-  int my_i;
-  warp_topk(v, E, k, lane, my_v, my_i, top_v);
-  const float g = selected_gate(my_v, top_v, k, lane);
-  int dest = 0;
-  if (lane < k) {
-    const size_t pr = static_cast<size_t>(row) * k + lane;
-    idx_out[pr] = my_i;
-    gates_out[pr] = g;
-    if (capture) capture[pr] = my_i;
-    dest = my_i * region + atomicAdd(&cursor[my_i], 1);
-    inv_slot[pr] = dest;
+  if (warp == 0) {
+    float v[PER];
+    router_logits_row<PER>(part, splits, T, row, E, bias, lane, v);
+    float my_v, top_v;
+    int my_i;
+    warp_topk<PER>(v, E, k, lane, my_v, my_i, top_v);
+    const float g = selected_gate(my_v, top_v, k, lane);
+    if (lane < k) {
+      const size_t pr = static_cast<size_t>(row) * k + lane;
+      idx_out[pr] = my_i;
+      gates_out[pr] = g;
+      if (capture) capture[pr] = my_i;
+      const int dr = my_i * region + atomicAdd(&cursor[my_i], 1);
+      inv_slot[pr] = dr;
+      dest[lane] = dr;
+    }
   }
-  for (int r = 0; r < k; ++r) {
-    const int dr = __shfl_sync(0xffffffffu, dest, r);
-    uint4* dst = reinterpret_cast<uint4*>(xp) + static_cast<size_t>(dr) * vec;
+  __syncthreads();
+  if (warp < k) {
+    uint4* dst = reinterpret_cast<uint4*>(xp) + static_cast<size_t>(dest[warp]) * vec;
 #pragma unroll
     for (int i = 0; i < DISPATCH_MAXV; ++i)
       if (lane + 32 * i < vec) dst[lane + 32 * i] = x[i];
@@ -398,8 +404,9 @@ __global__ void __launch_bounds__(1024) swiglu_splits_kernel(const float* __rest
 __host__ __device__ constexpr int rope_items(int Hq, int Hkv, int D) { return (Hq + Hkv) * (D / 8) + Hkv * (D / 4); }
 constexpr int ROPE_CTAS_PER_ROW = 2;
 constexpr int ROPE_MAX_THREADS = 512;
+constexpr int ROPE_BATCH = 3;  // split partials loaded per round trip (two CTAs of 512 threads per SM)
 
-__global__ void __launch_bounds__(ROPE_MAX_THREADS) rope_qkv_kernel(
+__global__ void __launch_bounds__(ROPE_MAX_THREADS, 2) rope_qkv_kernel(
     const float* __restrict__ part, int splits, int T, int n, int pos0, int Hq, int Hkv, int D,
     const float2* __restrict__ rope_tab, uint16_t* __restrict__ q, uint16_t* __restrict__ kc,
     uint16_t* __restrict__ vc, int S_max) {
@@ -419,17 +426,17 @@ __global__ void __launch_bounds__(ROPE_MAX_THREADS) rope_qkv_kernel(
       const float2* cs = rope_tab + static_cast<size_t>(pos) * half + j;
       const float2 c0 = cs[0], c1 = cs[1], c2 = cs[2], c3 = cs[3];
       float4 x1 = make_float4(0.f, 0.f, 0.f, 0.f), x2 = x1;
-      // splits in batches of four, the batch's loads issued before its sums
-      for (int s0 = 0; s0 < splits; s0 += 4) {
-        float4 a[4], bq[4];
+      // splits in batches of ROPE_BATCH, the batch's loads issued before its sums
+      for (int s0 = 0; s0 < splits; s0 += ROPE_BATCH) {
+        float4 a[ROPE_BATCH], bq[ROPE_BATCH];
 #pragma unroll
-        for (int s = 0; s < 4; ++s)
+        for (int s = 0; s < ROPE_BATCH; ++s)
           if (s0 + s < splits) {
             a[s] = *reinterpret_cast<const float4*>(base + (s0 + s) * sstride + c);
             bq[s] = *reinterpret_cast<const float4*>(base + (s0 + s) * sstride + c + half);
           }
 #pragma unroll
-        for (int s = 0; s < 4; ++s)
+        for (int s = 0; s < ROPE_BATCH; ++s)
           if (s0 + s < splits) {
             x1 = f4_add(x1, a[s]);
             x2 = f4_add(x2, bq[s]);
@@ -448,13 +455,13 @@ __global__ void __launch_bounds__(ROPE_MAX_THREADS) rope_qkv_kernel(
       const int g = r / d4, j = (r % d4) * 4;
       const int c = (Hq + Hkv) * D + g * D + j;
       float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int s0 = 0; s0 < splits; s0 += 4) {
-        float4 a[4];
+      for (int s0 = 0; s0 < splits; s0 += ROPE_BATCH) {
+        float4 a[ROPE_BATCH];
 #pragma unroll
-        for (int s = 0; s < 4; ++s)
+        for (int s = 0; s < ROPE_BATCH; ++s)
           if (s0 + s < splits) a[s] = *reinterpret_cast<const float4*>(base + (s0 + s) * sstride + c);
 #pragma unroll
-        for (int s = 0; s < 4; ++s)
+        for (int s = 0; s < ROPE_BATCH; ++s)
           if (s0 + s < splits) x = f4_add(x, a[s]);
       }
       store_bf16x4(vc + ((static_cast<size_t>(b) * Hkv + g) * S_max + pos) * D + j, x);
