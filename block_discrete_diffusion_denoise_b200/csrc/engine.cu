@@ -1406,7 +1406,7 @@ dg_status dg_debug_lmhead(dg_ctx* c, int32_t* argmax, float* lse, float* conf, f
 
 dg_status dg_debug_router(dg_ctx* c, const float* logits, int32_t n_rows, int32_t* idx, float* gates) {
   if (!c || !logits || !idx || !gates || n_rows <= 0) return fail(c, DG_ERR_INVALID_ARG, "debug_router");
-  router_topk_kernel<<<(n_rows + 7) / 8, 256, 0, c->stream>>>(logits, 1, n_rows, c->E, c->k, nullptr, idx, gates);
+  router_topk_kernel<<<n_rows, 256, 0, c->stream>>>(logits, 1, n_rows, c->E, c->k, nullptr, idx, gates);
   DG_LAUNCHED(c);
   return DG_OK;
 }

@@ -32,50 +32,35 @@ __device__ __forceinline__ int uniform_token(uint32_t w, int vocab) {
   return static_cast<int>((static_cast<uint64_t>(w) * static_cast<uint64_t>(vocab)) >> 32);
 }
 
-// Router decision of one row, held by one warp: v[c] is the logit of expert
-// c * 32 + lane (-inf past E), PER >= E / 32 logits per lane.  Top-k by
-// (logit desc, index asc); lane r < k receives the r-th selection (my_v,
-// my_i); every lane receives the largest logit (top_v).  k <= 16 < 32.
 constexpr int PERM_MAXE = 256;
 constexpr int ROUTE_PER = PERM_MAXE / 32;
 
-template <int PER>
-__device__ __forceinline__ void warp_topk(const float (&v)[PER], int E, int k, int lane, float& my_v, int& my_i,
-                                          float& top_v) {
-  uint32_t taken = 0;
-  my_v = -INFINITY;
-  top_v = -INFINITY;
-  my_i = 0;
-  for (int r = 0; r < k; ++r) {
-    float bv = -INFINITY;
-    int bi = 0x7fffffff;
-#pragma unroll
-    for (int c = 0; c < PER; ++c) {
-      const int e = c * 32 + lane;
-      if (e < E && !((taken >> c) & 1) && (v[c] > bv || (v[c] == bv && e < bi) || bi == 0x7fffffff)) {
-        bv = v[c];
-        bi = e;
-      }
+// Top-k of one row by ranking, over the CTA: lg[0, E) holds the row's logits
+// in shared memory (16-byte aligned, E a multiple of 4).  Each thread takes
+// experts e = threadIdx.x, threadIdx.x + blockDim.x, ... and counts the
+// experts before e in (logit desc, index asc) order; an expert of rank r < k
+// is written to sel_v[r], sel_i[r].  The ranks of distinct (logit, index)
+// pairs are distinct, so sel holds exactly the k first in that order.
+// Callers synchronise the CTA before (lg written) and after (sel read).
+__device__ __forceinline__ void cta_rank_topk(const float* lg, int E, int k, float* sel_v, int* sel_i) {
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const float v = lg[e];
+    int rank = 0;
+    for (int j = 0; j < E; j += 4) {
+      const float4 w = *reinterpret_cast<const float4*>(lg + j);
+      rank += (w.x > v || (w.x == v && j < e)) + (w.y > v || (w.y == v && j + 1 < e)) +
+              (w.z > v || (w.z == v && j + 2 < e)) + (w.w > v || (w.w == v && j + 3 < e));
     }
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (oi != 0x7fffffff && (bi == 0x7fffffff || ov > bv || (ov == bv && oi < bi))) {
-        bv = ov;
-        bi = oi;
-      }
+    if (rank < k) {
+      sel_v[rank] = v;
+      sel_i[rank] = e;
     }
-    if (r == 0) top_v = bv;
-    if (lane == r) {
-      my_v = bv;
-      my_i = bi;
-    }
-    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
   }
 }
 
 // logits of one row from split-K partials part[s][row][e] summed in split
-// order, plus the per-expert bias
+// order, plus the per-expert bias: v[c] is the logit of expert c * 32 + lane
+// (-inf past E), PER >= E / 32 per lane
 template <int PER>
 __device__ __forceinline__ void router_logits_row(const float* __restrict__ part, int splits, int T, int row, int E,
                                                   const float* __restrict__ bias, int lane, float (&v)[PER]) {
@@ -109,24 +94,52 @@ __device__ __forceinline__ float selected_gate(float my_v, float top_v, int k, i
   return w / sum;
 }
 
-// Router decision alone (test hook): one warp per row.
+// The routing decision of one row (one CTA, blockDim >= 32): warp 0 sums the
+// split-K partials into shared memory, the CTA ranks them, and lane r < k of
+// warp 0 receives the r-th selection (my_v, my_i) and its gate (softmax over
+// the k selected logits, summed in slot order).
+template <int PER>
+__device__ __forceinline__ void cta_route_row(const float* __restrict__ part, int splits, int T, int row, int E, int k,
+                                              const float* __restrict__ bias, float& my_v, int& my_i, float& g) {
+  __shared__ __align__(16) float lg[PERM_MAXE];
+  __shared__ float sel_v[32];
+  __shared__ int sel_i[32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp == 0) {
+    float v[PER];
+    router_logits_row<PER>(part, splits, T, row, E, bias, lane, v);
+#pragma unroll
+    for (int c = 0; c < PER; ++c)
+      if (c * 32 + lane < E) lg[c * 32 + lane] = v[c];
+  }
+  __syncthreads();
+  cta_rank_topk(lg, E, k, sel_v, sel_i);
+  __syncthreads();
+  my_v = -INFINITY;
+  my_i = 0;
+  g = 0.f;
+  if (warp == 0) {
+    if (lane < k) {
+      my_v = sel_v[lane];
+      my_i = sel_i[lane];
+    }
+    g = selected_gate(my_v, sel_v[0], k, lane);
+  }
+}
+
+// Router decision alone (test hook): one CTA per row.
 __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restrict__ part, int splits, int T, int E,
                                                           int k, const float* __restrict__ bias,
                                                           int32_t* __restrict__ idx_out,
                                                           float* __restrict__ gates_out) {
   DG_TIMELINE_SCOPE(TLK_ROUTER_TOPK);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row = blockIdx.x * (blockDim.x >> 5) + warp;
-  if (row >= T) return;
-  float v[ROUTE_PER];
-  router_logits_row<ROUTE_PER>(part, splits, T, row, E, bias, lane, v);
-  float my_v, top_v;
+  const int row = blockIdx.x;
+  float my_v, g;
   int my_i;
-  warp_topk<ROUTE_PER>(v, E, k, lane, my_v, my_i, top_v);
-  const float g = selected_gate(my_v, top_v, k, lane);
-  if (lane < k) {
-    idx_out[static_cast<size_t>(row) * k + lane] = my_i;
-    gates_out[static_cast<size_t>(row) * k + lane] = g;
+  cta_route_row<ROUTE_PER>(part, splits, T, row, E, k, bias, my_v, my_i, g);
+  if (threadIdx.x < k) {
+    idx_out[static_cast<size_t>(row) * k + threadIdx.x] = my_i;
+    gates_out[static_cast<size_t>(row) * k + threadIdx.x] = g;
   }
 }
 
@@ -137,10 +150,10 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
 // cursor[e], so cursor[e] ends as rows_e (zero before the launch; the expert
 // GEMM's last CTA zeroes it again).  The order of rows inside a region is
 // free: every row of an expert tile is an independent dot product, and the
-// combine sums a token's slots in slot order through inv_slot.  Warp 0 takes
-// the decision and the claims; then warp j copies the token's normalised row
-// u[row] (which every warp loaded at the start, overlapping the decision) to
-// the row slot j claimed.
+// combine sums a token's slots in slot order through inv_slot.  The CTA takes
+// the decision (cta_route_row) and lane j of warp 0 claims slot j's row; then
+// warp j copies the token's normalised row u[row] (which every warp loaded at
+// the start, overlapping the decision) to that row.
 //   idx, gates [T, k]; inv_slot[row * k + j] = claimed row of slot j;
 //   capture [T, k] or NULL (test hook).  blockDim = 32 * k, PER >= E / 32.
 constexpr int DISPATCH_MAXV = 16;  // 16-byte chunks per lane: d <= 32 * 16 * 8 = 4096
@@ -161,22 +174,17 @@ __global__ void __launch_bounds__(512) route_dispatch_kernel(
 #pragma unroll
   for (int i = 0; i < DISPATCH_MAXV; ++i)
     if (lane + 32 * i < vec) x[i] = src[lane + 32 * i];
-  if (warp == 0) {
-    float v[PER];
-    router_logits_row<PER>(part, splits, T, row, E, bias, lane, v);
-    float my_v, top_v;
-    int my_i;
-    warp_topk<PER>(v, E, k, lane, my_v, my_i, top_v);
-    const float g = selected_gate(my_v, top_v, k, lane);
-    if (lane < k) {
-      const size_t pr = static_cast<size_t>(row) * k + lane;
-      idx_out[pr] = my_i;
-      gates_out[pr] = g;
-      if (capture) capture[pr] = my_i;
-      const int dr = my_i * region + atomicAdd(&cursor[my_i], 1);
-      inv_slot[pr] = dr;
-      dest[lane] = dr;
-    }
+  float my_v, g;
+  int my_i;
+  cta_route_row<PER>(part, splits, T, row, E, k, bias, my_v, my_i, g);
+  if (threadIdx.x < k) {
+    const size_t pr = static_cast<size_t>(row) * k + lane;
+    idx_out[pr] = my_i;
+    gates_out[pr] = g;
+    if (capture) capture[pr] = my_i;
+    const int dr = my_i * region + atomicAdd(&cursor[my_i], 1);
+    inv_slot[pr] = dr;
+    dest[lane] = dr;
   }
   __syncthreads();
   if (warp < k) {

@@ -154,8 +154,15 @@ def test_commit_then_step_matches_oracle_and_prefill_of_concatenation():
     ctx2, _ = make_context(w, temperature=0.05, weights=weights)
     ctx2.prefill(torch.cat([prefix, block], 1).cuda())
     g2 = gpu_step(ctx2, w, canvas, 0, 3, 0.9, capture=True)
+    # the two caches differ only by rounding (other chunkings); a token whose
+    # expert choice flips on that difference is left out from that layer on
+    diverged = np.zeros(g1["hidden"][0].shape[:2], dtype=bool)
     for l in range(len(g1["hidden"])):
-        assert rel_l2(g1["hidden"][l], g2["hidden"][l]) < 2e-3
+        keep = ~diverged
+        assert rel_l2(g1["hidden"][l][keep], g2["hidden"][l][keep]) < 2e-3
+        if l < len(g1["experts"]):
+            diverged |= (np.sort(g1["experts"][l], -1) != np.sort(g2["experts"][l], -1)).any(-1)
+    assert diverged.sum() <= 3
     ctx.close()
     ctx2.close()
 
