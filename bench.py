@@ -78,6 +78,63 @@ def run_timeline(args, w):
           flush=True)
 
 
+def run_variants(args, w):
+    """Cost of the step's variants on one context: the threshold sampler (the
+    bench step), the entropy-constrained sampler with the 0.8 -> 0.4
+    temperature schedule and the adaptive-stop test (codemajin.net section
+    3.3), and self-conditioning on (section 3.2: the probability pass, p E and
+    the SwiGLU layer).  CUDA events around `steps` graph-replayed steps each."""
+    import torch
+
+    import block_discrete_diffusion_denoise_b200 as dgp
+    import synth_inputs as si
+
+    stream = torch.cuda.Stream()
+    torch.cuda.set_stream(stream)
+    weights = si.model_weights(w, "cuda")
+    weights.update(si.self_cond_weights(w, "cuda"))
+    cfg = dgp.config_from_shape(w.shape, max_batch=w.batch, max_seq=w.prefix + 2 * w.canvas, canvas=w.canvas)
+    ctx = dgp.Context(cfg, weights, stream=stream.cuda_stream)
+    ctx.prefill(si.uniform_tokens(w, "prefix", w.batch, w.prefix, device="cuda"))
+    B, C = w.batch, w.canvas
+    cur = si.uniform_tokens(w, "canvas", B, C, device="cuda")
+    nxt = torch.empty_like(cur)
+    conf = torch.empty(B, C, dtype=torch.float32, device="cuda")
+    am = [torch.empty(B, C, dtype=torch.int32, device="cuda") for _ in range(2)]
+    ent = torch.empty(B, C, dtype=torch.float32, device="cuda")
+    stopped = torch.empty(B, dtype=torch.int32, device="cuda")
+
+    def threshold(s):
+        ctx.denoise_step(cur, s, w.sample_seed, w.tau0, nxt, conf)
+
+    def entropy(s):
+        temp = 0.8 - 0.4 * min(s, 47) / 47.0
+        ctx.denoise_step_entropy(cur, s, w.sample_seed, temp, 8.0, 0.5, nxt,
+                                 prev_argmax=None if s == 0 else am[(s + 1) % 2], argmax_out=am[s % 2],
+                                 entropy=ent, stopped=stopped)
+
+    def timed(fn):
+        nonlocal cur, nxt
+        for s in range(args.warmup):
+            fn(s)
+            cur, nxt = nxt, cur
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for s in range(args.steps):
+            fn(args.warmup + s)
+            cur, nxt = nxt, cur
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / args.steps
+
+    rows = {"threshold_sampler_ms": timed(threshold), "entropy_sampler_ms": timed(entropy)}
+    ctx.set_self_conditioning(True)
+    rows["self_conditioning_ms"] = timed(threshold)
+    ctx.close()
+    print(json.dumps({"variants": f"{w.name}: {w.description}", "steps": args.steps, "warmup": args.warmup,
+                      **{k: round(v, 4) for k, v in rows.items()}}), flush=True)
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -91,6 +148,9 @@ def parse():
     ap.add_argument("--batch-sweep", default="",
                     help="comma-separated batch sizes: step throughput and roofline bound per batch "
                          "(one JSON line of its own, not the bench line)")
+    ap.add_argument("--variants", action="store_true",
+                    help="step time with the threshold sampler, the entropy-constrained sampler and "
+                         "self-conditioning (one JSON line of its own, not the bench line)")
     ap.add_argument("--timeline", action="store_true",
                     help="per-kernel spans and launch gaps of graph-replayed steps from libdg_timeline.so "
                          "(one JSON line of its own, not the bench line)")
@@ -545,6 +605,8 @@ def main():
         w = w.with_layers(args.layers)
     if args.timeline:
         run_timeline(args, w)
+    elif args.variants:
+        run_variants(args, w)
     elif args.batch_sweep:
         run_batch_sweep(args, w)
     elif args.impl == "reference":
