@@ -436,8 +436,12 @@ __global__ void __launch_bounds__(ATC_THREADS, 1) attn_tc_kernel(const __grid_co
       fence_proxy_async_smem();
       named_bar_sync(1, 256);
       if (threadIdx.x == 64) {
-        // (rows past 256 in the last slice are never read)
-        bulk_store_1d(part_cl + static_cast<size_t>(rank) * chunk_f4, stg, chunk_f4 * 16u);
+        // every slice but this chunk's own, which stays in place in shared
+        // memory for its reduction (rows past 256 in the last slice are never read)
+        float4* slot = part_cl + static_cast<size_t>(rank) * chunk_f4;
+        const uint32_t own0 = static_cast<uint32_t>(rank) * slice_f4, own1 = own0 + slice_f4;
+        if (own0 > 0) bulk_store_1d(slot, stg, own0 * 16u);
+        if (own1 < chunk_f4) bulk_store_1d(slot + own1, stg + own1, (chunk_f4 - own1) * 16u);
         bulk_commit_group();
         bulk_wait_all();
         fence_proxy_async_global();
@@ -450,14 +454,16 @@ __global__ void __launch_bounds__(ATC_THREADS, 1) attn_tc_kernel(const __grid_co
       // o = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c
       const int t = threadIdx.x - 64;
       const int r_lo = rank * rpr, n_rows = max(0, min(ATC_ROWS, r_lo + rpr) - r_lo);
-      float4* rcv = stg;                                           // [chunk][D/4][rpr]
+      float4* rcv = stg;                                           // [chunk][D/4][rpr]: the staging layout
       float* wts = reinterpret_cast<float*>(stg + chunk_f4);       // [row of the slice][chunk]
       if (t == 0 && n_rows > 0) {
         fence_proxy_async_global();
-        mbar_arrive_expect_tx(mrg, chunk_f4 * 16u);
+        // the other chunks' rows of this slice; its own are already at rcv + rank * slice_f4
+        mbar_arrive_expect_tx(mrg, (chunk_f4 - slice_f4) * 16u);
         for (int q = 0; q < nc; ++q)
-          bulk_load_1d(rcv + q * slice_f4, part_cl + static_cast<size_t>(q) * chunk_f4 + rank * slice_f4,
-                       slice_f4 * 16u, mrg);
+          if (q != rank)
+            bulk_load_1d(rcv + q * slice_f4, part_cl + static_cast<size_t>(q) * chunk_f4 + rank * slice_f4,
+                         slice_f4 * 16u, mrg);
       }
       if (t < n_rows) {
         float2 ml[ATC_MAX_CHUNKS];
