@@ -31,7 +31,7 @@ EXPORTS = ["dg_create", "dg_destroy", "dg_prefill", "dg_denoise_step", "dg_denoi
            "dg_lmhead_argmax_static"]
 
 # kernel ids of the timeline records (DG_K_* in dg.h)
-TIMELINE_KERNELS = {10: "gemm_dense", 11: "gemm_moe", 13: "gemm_lmhead", 20: "attention", 30: "route_dispatch",
+TIMELINE_KERNELS = {10: "gemm_dense", 11: "gemm_moe", 13: "gemm_lmhead", 20: "attention", 21: "attn_merge", 30: "route_dispatch",
                     31: "combine_norm", 32: "embed_norm", 33: "residual_norm", 34: "reduce_splits",
                     35: "swiglu_splits", 36: "rope_qkv", 37: "lmhead_merge_sample", 38: "entropy_sample",
                     39: "router_topk", 40: "sample_only", 50: "other"}

@@ -9,11 +9,10 @@
 // query heads of a GQA group are packed as consecutive rows (row = i*G + h)
 // so each K/V block feeds all of them; the 256 rows are two 128-row query
 // tiles, each pulled by one 4-D TMA box out of the [token][head][D] query
-// layout, and every K/V block is read once for both.  The key chunks of one
-// query block form a thread-block cluster: each stores its raw rows (one
-// bulk copy) and row statistics to an L2-resident buffer, and after one
-// cluster barrier each bulk-loads its slice of the rows from every chunk and
-// reduces it; a single chunk writes its rows directly.
+// layout, and every K/V block is read once for both.  The keys are split
+// into chunks so the grid fills the SMs; with one chunk a CTA writes its
+// normalised rows, with several it writes its raw rows and row statistics to
+// a partial buffer and attn_merge_kernel combines them.
 //
 // Warp 0 issues TMA loads (lane 0: both Q tiles once, then 64-key K blocks;
 // lane 1: V blocks; 2-deep rings).  Warp 1 issues tcgen05.mma: S_q = Q_q K^T into tile q's TMEM
@@ -41,7 +40,7 @@ constexpr int ATC_BK = 64;         // keys per block (MMA N of Q K^T, K of P V)
 constexpr int ATC_KSTAGES = 2;
 constexpr int ATC_VSTAGES = 2;
 constexpr int ATC_THREADS = 320;   // producer warp, MMA warp, two softmax warpgroups
-constexpr int ATC_MAX_CHUNKS = 16; // key chunks = cluster size (above 8 needs the non-portable opt-in)
+constexpr int ATC_MAX_CHUNKS = 16; // key chunks per query block (combined by attn_merge_kernel)
 constexpr float ATC_RESCALE_LOG2 = 8.f;
 
 struct AttnTcParams {
@@ -49,8 +48,8 @@ struct AttnTcParams {
   CUtensorMap k_map;   // 2-D (D, B*Hkv*S_max) over this layer's K cache; box (64, 64)
   CUtensorMap v_map;   // same over V
   uint16_t* o;         // [token][Hq][D]
-  float* part;         // several key chunks: [cluster][chunk][slice][D/4][rows of the slice] float4 raw rows
-  float2* part_ml;     // [cluster][chunk][256 rows] (max, sum) of those rows
+  float* part;         // several key chunks: [unit][chunk][D/4][256 rows] float4 raw rows (unit = y * qblocks + x)
+  float2* part_ml;     // [unit][chunk][256 rows] (max, sum) of those rows
   int n, B, Hq, Hkv, S_max, pos0, causal, chunk_len, n_chunks;
   float scale_log2;    // log2(e) / sqrt(D)
   DevErr err;
@@ -70,9 +69,6 @@ struct AtcCfg {
   static constexpr int SMEM = 1024 + REGION + TAIL;
   static_assert(O_COL + ATC_NQ * D <= 512, "S and O accumulators must fit TMEM");
   static_assert(D % 16 == 0 && D <= 256, "head_dim must be a multiple of 16, at most 256");
-  // chunk merge: a chunk's rows (at most 256 + 15 with the slice rounding) and the weight table
-  static_assert((ATC_ROWS + ATC_MAX_CHUNKS) * D * 4 + ATC_ROWS * ATC_MAX_CHUNKS * 4 <= REGION,
-                "the chunk merge must fit in the mainloop's shared memory");
 };
 
 template <int D>
@@ -96,7 +92,6 @@ __global__ void __launch_bounds__(ATC_THREADS, 1) attn_tc_kernel(const __grid_co
   uint64_t* p_full = s_free + ATC_NQ;         // [NQ] warpgroup q -> MMA: P_q written
   uint64_t* o_done = p_full + ATC_NQ;         // [NQ] MMA -> warpgroup q: O_q += P_q V complete
   uint64_t* drain = o_done + ATC_NQ;
-  uint64_t* mrg = drain + 1;                  // chunk merge: this chunk's slices of every chunk have landed
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tail + 256);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tail + 260);
 
@@ -139,7 +134,6 @@ __global__ void __launch_bounds__(ATC_THREADS, 1) attn_tc_kernel(const __grid_co
       mbar_init(&o_done[q], 1);
     }
     mbar_init(drain, 1);
-    mbar_init(mrg, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -351,8 +345,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1) attn_tc_kernel(const __grid_co
     if (!ok) *abort_flag = 1;
   }
 
-  // ---------- merge the key chunks of this query block (one cluster) ----------
-  // o = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c, M = max_c m_c.
+  // ---------- one chunk: the rows; several: the partials for the merge ----------
   const int nc = p.n_chunks;
   if (warp >= 2) {
     named_bar_sync(1, 256);  // both tiles' MMAs are complete
@@ -388,125 +381,42 @@ __global__ void __launch_bounds__(ATC_THREADS, 1) attn_tc_kernel(const __grid_co
         }
       }
     }
-  } else {
-    // Each chunk stages its raw rows in shared memory in the layout of its
-    // slot of the cluster's L2-resident buffer and stores them with one bulk
-    // copy; the slot is [slice][D/4][rows of the slice] float4, so the rows
-    // one chunk later reduces (its slice) are one contiguous run in every
-    // chunk's slot.  The row statistics (max, sum) go out with plain stores.
-    const int rank = static_cast<int>(cluster_ctarank());
-    const size_t cl = static_cast<size_t>(blockIdx.y) * gridDim.x + blockIdx.x;
+  } else if (warp >= 2) {
+    // several key chunks: this chunk's raw rows and their (max, sum) go to its
+    // slot of the partial buffer, [unit][chunk][D/4][256 rows] float4 (a
+    // warp's store covers 32 consecutive rows, 512 contiguous bytes);
+    // attn_merge_kernel combines the chunks
     constexpr int D4 = D / 4;
-    const int rpr = (ATC_ROWS + nc - 1) / nc;                  // rows per slice
-    const uint32_t slice_f4 = static_cast<uint32_t>(D4 * rpr);  // one slice of one chunk
-    const uint32_t chunk_f4 = static_cast<uint32_t>(nc) * slice_f4;
-    float4* part_cl = reinterpret_cast<float4*>(p.part) + cl * nc * chunk_f4;
-    float2* ml_cl = p.part_ml + cl * nc * ATC_ROWS;
-    float4* stg = reinterpret_cast<float4*>(sQ);  // the mainloop's buffers are free: every MMA has completed
-    if (warp >= 2) {
-      ml_cl[rank * ATC_ROWS + row] = make_float2(have_o ? mref : -INFINITY, have_o ? lsum : 0.f);
-      float4* dst = stg + (row / rpr) * slice_f4 + (row % rpr);
-      auto put16 = [&](int c0, const float* v) {
+    const size_t slot = (static_cast<size_t>(blockIdx.y) * gridDim.x + blockIdx.x) * nc + blockIdx.z;
+    float4* dst = reinterpret_cast<float4*>(p.part) + slot * D4 * ATC_ROWS + row;
+    p.part_ml[slot * ATC_ROWS + row] = make_float2(have_o ? mref : -INFINITY, have_o ? lsum : 0.f);
+    auto put16 = [&](int c0, const float* v) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) dst[(c0 / 4 + e) * rpr] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
-      };
-      int c0 = 0;
+      for (int e = 0; e < 4; ++e)
+        dst[static_cast<size_t>(c0 / 4 + e) * ATC_ROWS] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+    };
+    int c0 = 0;
 #pragma unroll 1
-      for (; c0 + 32 <= D; c0 += 32) {
-        float v[32];
-        if (have_o) {
-          tmem_ld32(t_row + C::O_COL + wg * D + c0, v);
-        } else {
+    for (; c0 + 32 <= D; c0 += 32) {
+      float v[32];
+      if (have_o) {
+        tmem_ld32(t_row + C::O_COL + wg * D + c0, v);
+      } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = 0.f;
-        }
-        put16(c0, v);
-        put16(c0 + 16, v + 16);
+        for (int e = 0; e < 32; ++e) v[e] = 0.f;
       }
-      if (c0 < D) {  // D is a multiple of 16
-        float v[16];
-        if (have_o) {
-          tmem_ld16(t_row + C::O_COL + wg * D + c0, v);
-        } else {
-#pragma unroll
-          for (int e = 0; e < 16; ++e) v[e] = 0.f;
-        }
-        put16(c0, v);
-      }
-      fence_proxy_async_smem();
-      named_bar_sync(1, 256);
-      if (threadIdx.x == 64) {
-        // every slice but this chunk's own, which stays in place in shared
-        // memory for its reduction (rows past 256 in the last slice are never read)
-        float4* slot = part_cl + static_cast<size_t>(rank) * chunk_f4;
-        const uint32_t own0 = static_cast<uint32_t>(rank) * slice_f4, own1 = own0 + slice_f4;
-        if (own0 > 0) bulk_store_1d(slot, stg, own0 * 16u);
-        if (own1 < chunk_f4) bulk_store_1d(slot + own1, stg + own1, (chunk_f4 - own1) * 16u);
-        bulk_commit_group();
-        bulk_wait_all();
-        fence_proxy_async_global();
-      }
+      put16(c0, v);
+      put16(c0 + 16, v + 16);
     }
-    // every chunk's rows and statistics are written
-    cluster_sync_all();
-    if (warp >= 2) {
-      // each chunk reduces its slice of the rows over the chunks, in chunk order:
-      // o = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c
-      const int t = threadIdx.x - 64;
-      const int r_lo = rank * rpr, n_rows = max(0, min(ATC_ROWS, r_lo + rpr) - r_lo);
-      float4* rcv = stg;                                           // [chunk][D/4][rpr]: the staging layout
-      float* wts = reinterpret_cast<float*>(stg + chunk_f4);       // [row of the slice][chunk]
-      if (t == 0 && n_rows > 0) {
-        fence_proxy_async_global();
-        // the other chunks' rows of this slice; its own are already at rcv + rank * slice_f4
-        mbar_arrive_expect_tx(mrg, (chunk_f4 - slice_f4) * 16u);
-        for (int q = 0; q < nc; ++q)
-          if (q != rank)
-            bulk_load_1d(rcv + q * slice_f4, part_cl + static_cast<size_t>(q) * chunk_f4 + rank * slice_f4,
-                         slice_f4 * 16u, mrg);
+    if (c0 < D) {  // D is a multiple of 16
+      float v[16];
+      if (have_o) {
+        tmem_ld16(t_row + C::O_COL + wg * D + c0, v);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) v[e] = 0.f;
       }
-      if (t < n_rows) {
-        float2 ml[ATC_MAX_CHUNKS];
-#pragma unroll
-        for (int q = 0; q < ATC_MAX_CHUNKS; ++q)
-          if (q < nc) ml[q] = __ldcg(ml_cl + q * ATC_ROWS + r_lo + t);
-        float M = -INFINITY;
-#pragma unroll
-        for (int q = 0; q < ATC_MAX_CHUNKS; ++q)
-          if (q < nc) M = fmaxf(M, ml[q].x);
-        const float Mref = M == -INFINITY ? 0.f : M;
-        float den = 0.f;
-#pragma unroll
-        for (int q = 0; q < ATC_MAX_CHUNKS; ++q)
-          if (q < nc && ml[q].x != -INFINITY) den += ml[q].y * ex2_approx(ml[q].x - Mref);
-#pragma unroll
-        for (int q = 0; q < ATC_MAX_CHUNKS; ++q)
-          if (q < nc)
-            wts[t * ATC_MAX_CHUNKS + q] = (den > 0.f && ml[q].x != -INFINITY) ? ex2_approx(ml[q].x - Mref) / den : 0.f;
-      }
-      named_bar_sync(1, 256);
-      if (n_rows > 0 && mbar_wait(mrg, 0, p.err)) {
-        const int n_items = n_rows * D4;
-        for (int it = t; it < n_items; it += 256) {
-          const int rl = it / D4, c4 = it % D4;   // a warp covers consecutive columns of a row
-          const float4* src = rcv + c4 * rpr + rl;
-          const float* wr = wts + rl * ATC_MAX_CHUNKS;
-          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-          for (int q = 0; q < nc; ++q) {
-            const float4 v = src[q * slice_f4];
-            const float wq = wr[q];
-            acc.x = fmaf(v.x, wq, acc.x);
-            acc.y = fmaf(v.y, wq, acc.y);
-            acc.z = fmaf(v.z, wq, acc.z);
-            acc.w = fmaf(v.w, wq, acc.w);
-          }
-          const int rg = row_base + r_lo + rl;
-          if (rg >= rows_total) continue;
-          const size_t rid = (static_cast<size_t>(b) * p.n + rg / G) * p.Hq + kvh * G + rg % G;
-          *reinterpret_cast<uint2*>(p.o + rid * D + 4 * c4) =
-              make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
-        }
-      }
+      put16(c0, v);
     }
   }
 
@@ -517,6 +427,61 @@ __global__ void __launch_bounds__(ATC_THREADS, 1) attn_tc_kernel(const __grid_co
     tc_fence_after();
     tmem_dealloc(tmem_base, C::TMEM_COLS);
   }
+}
+
+// Merge of the key chunks of attn_tc_kernel (several chunks):
+//   o = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c,  M = max_c m_c,
+// summed in chunk order.  One thread per (unit, row, 4-column group):
+// consecutive threads take consecutive rows of one group, so the partial and
+// row-statistic loads are coalesced, and every load a thread needs (nc
+// partials, nc statistics) is issued before the first is used: one memory
+// round trip, no shared memory.  grid = (units, 256 * D/4 / 256), 256 threads.
+template <int D>
+__global__ void __launch_bounds__(256) attn_merge_kernel(const float4* __restrict__ part,
+                                                         const float2* __restrict__ part_ml, int nc, int qblocks,
+                                                         int n, int Hq, int Hkv, uint16_t* __restrict__ o) {
+  DG_TIMELINE_SCOPE(TLK_ATTN_MERGE);
+  constexpr int D4 = D / 4;
+  const int unit = blockIdx.x;  // = blockIdx.y * qblocks + blockIdx.x of the attention launch
+  const int it = blockIdx.y * blockDim.x + threadIdx.x;
+  if (it >= ATC_ROWS * D4) return;
+  const int r = it % ATC_ROWS, c4 = it / ATC_ROWS;
+  const int qb = unit % qblocks, bk = unit / qblocks;
+  const int b = bk / Hkv, kvh = bk % Hkv;
+  const int G = Hq / Hkv, rows_total = n * G;
+  const size_t slot0 = static_cast<size_t>(unit) * nc;
+  const float4* src = part + slot0 * D4 * ATC_ROWS + static_cast<size_t>(c4) * ATC_ROWS + r;
+  float2 ml[ATC_MAX_CHUNKS];
+  float4 v[ATC_MAX_CHUNKS];
+#pragma unroll
+  for (int q = 0; q < ATC_MAX_CHUNKS; ++q)
+    if (q < nc) {
+      ml[q] = part_ml[(slot0 + q) * ATC_ROWS + r];
+      v[q] = src[static_cast<size_t>(q) * D4 * ATC_ROWS];
+    }
+  float M = -INFINITY;
+#pragma unroll
+  for (int q = 0; q < ATC_MAX_CHUNKS; ++q)
+    if (q < nc) M = fmaxf(M, ml[q].x);
+  const float Mref = M == -INFINITY ? 0.f : M;
+  float den = 0.f;
+#pragma unroll
+  for (int q = 0; q < ATC_MAX_CHUNKS; ++q)
+    if (q < nc && ml[q].x != -INFINITY) den += ml[q].y * ex2_approx(ml[q].x - Mref);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int q = 0; q < ATC_MAX_CHUNKS; ++q)
+    if (q < nc) {
+      const float wq = (den > 0.f && ml[q].x != -INFINITY) ? ex2_approx(ml[q].x - Mref) / den : 0.f;
+      acc.x = fmaf(v[q].x, wq, acc.x);
+      acc.y = fmaf(v[q].y, wq, acc.y);
+      acc.z = fmaf(v[q].z, wq, acc.z);
+      acc.w = fmaf(v[q].w, wq, acc.w);
+    }
+  const int rg = qb * ATC_ROWS + r;
+  if (rg >= rows_total) return;
+  const size_t rid = (static_cast<size_t>(b) * n + rg / G) * Hq + kvh * G + rg % G;
+  *reinterpret_cast<uint2*>(o + rid * D + 4 * c4) = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
 }
 
 }  // namespace dg

@@ -40,6 +40,7 @@ __device__ __forceinline__ void raise_error(const DevErr& e, int code) {
 enum TimelineKernel : int {
   TLK_GEMM = 10,  // + the GEMM mode (10 dense, 11 expert, 13 LM head)
   TLK_ATTENTION = 20,
+  TLK_ATTN_MERGE = 21,
   TLK_ROUTE_DISPATCH = 30,
   TLK_COMBINE_NORM = 31,
   TLK_EMBED_NORM = 32,

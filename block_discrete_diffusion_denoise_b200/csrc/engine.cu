@@ -79,10 +79,9 @@ struct dg_ctx {
   int32_t* chunk_done = nullptr;   // finished gate/up tiles per expert token chunk
   int32_t* expert_rows = nullptr;  // [E] rows routed to each expert (dispatch cursors)
   int32_t* moe_work = nullptr;     // claim / exit counters of the expert GEMM
-  float* attn_part = nullptr;      // attention chunk partials (clusters of several chunks): sms x 272 rows x D
+  float* attn_part = nullptr;      // attention key-chunk partials: one 256-row slot per SM (sms x 272 rows x D)
   float2* attn_part_ml = nullptr;  // their row statistics: sms x 256 rows
   int32_t* dense_work = nullptr;   // claim / exit counters of the dense GEMM
-  int attn_max_clusters[ATC_MAX_CHUNKS + 1] = {};  // co-resident attention clusters per cluster size
   // CUDA graphs of the denoising step, one per sampler (per batch and cached length)
   bool use_graphs = true;
   StepGraph graphs[SAMPLER_COUNT];
@@ -332,49 +331,6 @@ dg_status gemm_dense(dg_ctx* c, const CUtensorMap& w, const CUtensorMap& x, int 
   return DG_OK;
 }
 
-template <int D>
-cudaError_t launch_attention(const dg_ctx* c, const AttnTcParams& p, dim3 grid) {
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = grid;
-  cfg.blockDim = dim3(ATC_THREADS, 1, 1);
-  cfg.dynamicSmemBytes = AtcCfg<D>::SMEM;
-  cfg.stream = c->stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = grid.z;  // the key chunks of one query block
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, attn_tc_kernel<D>, p);
-}
-
-template <int D>
-cudaError_t attention_cluster_limits(dg_ctx* c) {
-  for (int nc = 1; nc <= ATC_MAX_CHUNKS; ++nc) {
-    cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(1, 1, nc);
-    cfg.blockDim = dim3(ATC_THREADS, 1, 1);
-    cfg.dynamicSmemBytes = AtcCfg<D>::SMEM;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 1;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = nc;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int num = 0;
-    cudaError_t e = cudaOccupancyMaxActiveClusters(&num, attn_tc_kernel<D>, &cfg);
-    if (e != cudaSuccess) {
-      if (nc <= 8) return e;
-      cudaGetLastError();  // a non-portable size this device does not offer: not used
-      num = 0;
-    }
-    c->attn_max_clusters[nc] = num;
-  }
-  return cudaSuccess;
-}
-
 dg_status attention(dg_ctx* c, int l, int B, int n, int pos0, bool causal) {
   AttnTcParams p;
   p.q_map = c->m_q4;
@@ -396,44 +352,42 @@ dg_status attention(dg_ctx* c, int l, int B, int n, int pos0, bool causal) {
   const int qblocks = (n * G + ATC_ROWS - 1) / ATC_ROWS;
   const int units = qblocks * B * c->Hkv;
   const int keys = pos0 + n;
-  // Split the keys into the cluster of chunks that gives each CTA the fewest
-  // 64-key blocks while every cluster is resident at once (fewer chunks on
-  // ties: each chunk adds a merge share); one chunk when nothing fits.
-  int n_chunks = 1, best_blocks = (keys + ATC_BK - 1) / ATC_BK;
-  for (int nc = 2; nc <= ATC_MAX_CHUNKS; ++nc) {
-    // the partial buffer holds sms x (256 + 16) rows: one slot per CTA of the launch
-    if (units > c->attn_max_clusters[nc] || keys < nc * ATC_BK || units * nc > c->sms) continue;
-    const int blocks = ((keys + nc - 1) / nc + ATC_BK - 1) / ATC_BK;
-    if (blocks < best_blocks) {
-      best_blocks = blocks;
-      n_chunks = nc;
-    }
-  }
-  const int chunk_len = best_blocks * ATC_BK;
+  // Split the keys into chunks so that units x chunks fills the SMs in one
+  // wave (the partial buffer holds one slot per SM), at least four 64-key
+  // blocks per chunk; several chunks are combined by attn_merge_kernel.
+  int n_chunks = std::max(1, std::min({ATC_MAX_CHUNKS, c->sms / std::max(1, units), keys / (4 * ATC_BK)}));
+  const int chunk_len = ((keys + n_chunks - 1) / n_chunks + ATC_BK - 1) / ATC_BK * ATC_BK;
   n_chunks = (keys + chunk_len - 1) / chunk_len;
   p.chunk_len = chunk_len;
   p.n_chunks = n_chunks;
   if (c->trace && l == 0)
-    fprintf(stderr, "[dg] attention: keys %d, units %d, chunks %d x %d keys (resident clusters of that size %d)\n",
-            keys, units, n_chunks, chunk_len, c->attn_max_clusters[n_chunks]);
+    fprintf(stderr, "[dg] attention: keys %d, units %d, chunks %d x %d keys\n", keys, units, n_chunks, chunk_len);
   const dim3 grid(qblocks, B * c->Hkv, n_chunks);
+  const dim3 mgrid(units, (ATC_ROWS * (c->D / 4) + 255) / 256);
+  const float4* part4 = reinterpret_cast<const float4*>(c->attn_part);
   ProfScope ps1(c, DG_PROF_ATTENTION);
-  cudaError_t e;
   switch (c->D) {
     case 64:
-      e = launch_attention<64>(c, p, grid);
+      DG_LAUNCH(c, attn_tc_kernel<64>, grid, ATC_THREADS, AtcCfg<64>::SMEM, p);
+      if (n_chunks > 1)
+        DG_LAUNCH(c, attn_merge_kernel<64>, mgrid, 256, 0, part4, static_cast<const float2*>(c->attn_part_ml),
+                  n_chunks, qblocks, n, c->Hq, c->Hkv, c->o);
       break;
     case 128:
-      e = launch_attention<128>(c, p, grid);
+      DG_LAUNCH(c, attn_tc_kernel<128>, grid, ATC_THREADS, AtcCfg<128>::SMEM, p);
+      if (n_chunks > 1)
+        DG_LAUNCH(c, attn_merge_kernel<128>, mgrid, 256, 0, part4, static_cast<const float2*>(c->attn_part_ml),
+                  n_chunks, qblocks, n, c->Hq, c->Hkv, c->o);
       break;
     case 176:
-      e = launch_attention<176>(c, p, grid);
+      DG_LAUNCH(c, attn_tc_kernel<176>, grid, ATC_THREADS, AtcCfg<176>::SMEM, p);
+      if (n_chunks > 1)
+        DG_LAUNCH(c, attn_merge_kernel<176>, mgrid, 256, 0, part4, static_cast<const float2*>(c->attn_part_ml),
+                  n_chunks, qblocks, n, c->Hq, c->Hkv, c->o);
       break;
     default:
       return fail(c, DG_ERR_UNSUPPORTED, "head_dim %d", c->D);
   }
-  if (e != cudaSuccess) return fail(c, DG_ERR_CUDA, "attention launch: %s", cudaGetErrorString(e));
-  DG_LAUNCHED(c);
   ps1.end();
   return DG_OK;
 }
@@ -757,10 +711,6 @@ dg_status set_smem_attrs(dg_ctx* c) {
   DG_CUDA(c, cudaFuncSetAttribute(attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, AtcCfg<64>::SMEM));
   DG_CUDA(c, cudaFuncSetAttribute(attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, AtcCfg<128>::SMEM));
   DG_CUDA(c, cudaFuncSetAttribute(attn_tc_kernel<176>, cudaFuncAttributeMaxDynamicSharedMemorySize, AtcCfg<176>::SMEM));
-  // clusters of up to 16 key chunks (above the portable 8)
-  DG_CUDA(c, cudaFuncSetAttribute(attn_tc_kernel<64>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
-  DG_CUDA(c, cudaFuncSetAttribute(attn_tc_kernel<128>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
-  DG_CUDA(c, cudaFuncSetAttribute(attn_tc_kernel<176>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
   return DG_OK;
 }
 
@@ -1033,18 +983,7 @@ dg_status dg_create(const dg_config* cfg, const dg_weights* w, void* cuda_stream
     discard(c);
     return DG_ERR_CUDA;
   }
-  e = c->D == 64 ? attention_cluster_limits<64>(c)
-                 : c->D == 128 ? attention_cluster_limits<128>(c) : attention_cluster_limits<176>(c);
-  if (e != cudaSuccess) {
-    fail(c, DG_ERR_CUDA, "cluster occupancy query: %s", cudaGetErrorString(e));
-    discard(c);
-    return DG_ERR_CUDA;
-  }
-  if (c->trace) {
-    fprintf(stderr, "[dg] resident attention clusters by size:");
-    for (int nc = 1; nc <= ATC_MAX_CHUNKS; ++nc) fprintf(stderr, " %d:%d", nc, c->attn_max_clusters[nc]);
-    fprintf(stderr, "\n");
-  }
+
 
   // ---- workspace plan ----
   const size_t R = c->R, d = c->d, k = c->k;
@@ -1506,15 +1445,15 @@ dg_status dg_debug_gemm(dg_ctx* c, const void* w, int32_t M, int32_t K, const vo
 
 constexpr bool timeline_ids_match() {
   using namespace dg;
-  const int ours[16] = {TLK_GEMM + GEMM_DENSE, TLK_GEMM + GEMM_MOE, TLK_GEMM + GEMM_LMHEAD, TLK_ATTENTION,
+  const int ours[17] = {TLK_GEMM + GEMM_DENSE, TLK_GEMM + GEMM_MOE, TLK_GEMM + GEMM_LMHEAD, TLK_ATTENTION, TLK_ATTN_MERGE,
                         TLK_ROUTE_DISPATCH, TLK_COMBINE_NORM, TLK_EMBED_NORM, TLK_RESIDUAL_NORM, TLK_REDUCE_SPLITS,
                         TLK_SWIGLU_SPLITS, TLK_ROPE_QKV, TLK_LMHEAD_MERGE_SAMPLE, TLK_ENTROPY_SAMPLE, TLK_ROUTER_TOPK,
                         TLK_SAMPLE_ONLY, TLK_OTHER};
-  const int abi[16] = {DG_K_GEMM_DENSE, DG_K_GEMM_MOE, DG_K_GEMM_LMHEAD, DG_K_ATTENTION, DG_K_ROUTE_DISPATCH,
+  const int abi[17] = {DG_K_GEMM_DENSE, DG_K_GEMM_MOE, DG_K_GEMM_LMHEAD, DG_K_ATTENTION, DG_K_ATTN_MERGE, DG_K_ROUTE_DISPATCH,
                        DG_K_COMBINE_NORM, DG_K_EMBED_NORM, DG_K_RESIDUAL_NORM, DG_K_REDUCE_SPLITS, DG_K_SWIGLU_SPLITS,
                        DG_K_ROPE_QKV, DG_K_LMHEAD_MERGE_SAMPLE, DG_K_ENTROPY_SAMPLE, DG_K_ROUTER_TOPK,
                        DG_K_SAMPLE_ONLY, DG_K_OTHER};
-  for (int i = 0; i < 16; ++i)
+  for (int i = 0; i < 17; ++i)
     if (ours[i] != abi[i]) return false;
   return true;
 }

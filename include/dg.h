@@ -324,14 +324,14 @@ int64_t dg_debug_launch_count(const dg_ctx* ctx);
  * calls return DG_ERR_UNSUPPORTED.
  *
  * Kernel ids: DG_K_GEMM_DENSE 10, DG_K_GEMM_MOE 11, DG_K_GEMM_LMHEAD 13,
- * DG_K_ATTENTION 20, DG_K_ROUTE_DISPATCH 30, DG_K_COMBINE_NORM 31,
+ * DG_K_ATTENTION 20, DG_K_ATTN_MERGE 21, DG_K_ROUTE_DISPATCH 30, DG_K_COMBINE_NORM 31,
  * DG_K_EMBED_NORM 32, DG_K_RESIDUAL_NORM 33, DG_K_REDUCE_SPLITS 34,
  * DG_K_SWIGLU_SPLITS 35, DG_K_ROPE_QKV 36, DG_K_LMHEAD_MERGE_SAMPLE 37,
  * DG_K_ENTROPY_SAMPLE 38, DG_K_ROUTER_TOPK 39, DG_K_SAMPLE_ONLY 40,
  * DG_K_OTHER 50.
  * ------------------------------------------------------------------------- */
 enum {
-  DG_K_GEMM_DENSE = 10, DG_K_GEMM_MOE = 11, DG_K_GEMM_LMHEAD = 13, DG_K_ATTENTION = 20,
+  DG_K_GEMM_DENSE = 10, DG_K_GEMM_MOE = 11, DG_K_GEMM_LMHEAD = 13, DG_K_ATTENTION = 20, DG_K_ATTN_MERGE = 21,
   DG_K_ROUTE_DISPATCH = 30, DG_K_COMBINE_NORM = 31, DG_K_EMBED_NORM = 32, DG_K_RESIDUAL_NORM = 33,
   DG_K_REDUCE_SPLITS = 34, DG_K_SWIGLU_SPLITS = 35, DG_K_ROPE_QKV = 36, DG_K_LMHEAD_MERGE_SAMPLE = 37,
   DG_K_ENTROPY_SAMPLE = 38, DG_K_ROUTER_TOPK = 39, DG_K_SAMPLE_ONLY = 40, DG_K_OTHER = 50
