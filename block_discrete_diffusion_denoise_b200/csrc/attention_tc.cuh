@@ -40,7 +40,7 @@ constexpr int ATC_BK = 64;         // keys per block (MMA N of Q K^T, K of P V)
 constexpr int ATC_KSTAGES = 2;
 constexpr int ATC_VSTAGES = 2;
 constexpr int ATC_THREADS = 320;   // producer warp, MMA warp, two softmax warpgroups
-constexpr int ATC_MAX_CHUNKS = 16; // key chunks per query block (combined by attn_merge_kernel)
+constexpr int ATC_MAX_CHUNKS = 10; // key chunks per query block (combined by attn_merge_kernel)
 constexpr float ATC_RESCALE_LOG2 = 8.f;
 
 struct AttnTcParams {
@@ -437,7 +437,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1) attn_tc_kernel(const __grid_co
 // partials, nc statistics) is issued before the first is used: one memory
 // round trip, no shared memory.  grid = (units, 256 * D/4 / 256), 256 threads.
 template <int D>
-__global__ void __launch_bounds__(256) attn_merge_kernel(const float4* __restrict__ part,
+__global__ void __launch_bounds__(256, 3) attn_merge_kernel(const float4* __restrict__ part,
                                                          const float2* __restrict__ part_ml, int nc, int qblocks,
                                                          int n, int Hq, int Hkv, uint16_t* __restrict__ o) {
   DG_TIMELINE_SCOPE(TLK_ATTN_MERGE);
