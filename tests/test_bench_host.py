@@ -86,3 +86,19 @@ def test_clock_reasons_inside_the_window_are_reported():
     clk = _clocks_with_rows(rows).stop(t0, t0 + 0.2)
     assert clk["reasons"] == ["sw_power_cap"]
     assert clk["sm_mhz"] == 1510.0
+
+
+def test_mode_flags_parse_and_the_timeline_mode_selects_the_tracing_build(monkeypatch):
+    """--timeline, --variants and --batch-sweep are modes with JSON lines of
+    their own; --timeline points the binding at libdg_timeline.so before the
+    package is imported (main() sets DG_LIBRARY)."""
+    import sys
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--timeline", "--steps", "2"])
+    args = bench.parse()
+    assert args.timeline and not args.variants and args.steps == 2
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--variants"])
+    assert bench.parse().variants
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--batch-sweep", "1,2"])
+    assert bench.parse().batch_sweep == "1,2"
+    src = open(bench.__file__).read()
+    assert 'os.environ["DG_LIBRARY"] = os.path.join(ROOT, "block_discrete_diffusion_denoise_b200", "libdg_timeline.so")' in src
