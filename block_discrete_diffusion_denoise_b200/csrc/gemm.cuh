@@ -441,6 +441,28 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
     tma_prefetch_desc(&p.a_map[0]);
     tma_prefetch_desc(&p.b_map);
   }
+  // barriers and TMEM first: their latency overlaps the tile-table loads
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 2);  // the A and the B producer
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+    }
+    for (int s = 0; s < GEMM_SCHED; ++s) {
+      mbar_init(&sched_full[s], 1);
+      mbar_init(&sched_empty[s], 3);  // B producer + MMA issuer + epilogue leader
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, 2 * ACC_COLS * HALVES);
+    tmem_relinquish();
+  }
   MoeTables tb{tb_ch_off, tb_rows, 0, 0, 0};
   if constexpr (MODE == GEMM_MOE) {
     // tile tables from the row counts (two groups per thread, G <= 2 * GEMM_THREADS)
@@ -470,27 +492,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
     tb.n_dn = total * (p.d / GEMM_BM);
   }
 
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 2);  // the A and the B producer
-      mbar_init(&empty[s], 1);
-    }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 128);
-    }
-    for (int s = 0; s < GEMM_SCHED; ++s) {
-      mbar_init(&sched_full[s], 1);
-      mbar_init(&sched_empty[s], 3);  // B producer + MMA issuer + epilogue leader
-    }
-    mbar_init(drain, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_holder, 2 * ACC_COLS * HALVES);
-    tmem_relinquish();
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -523,14 +524,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
         int nxt = -1;
         int4 nxt_rec = make_int4(0, 0, 0, 0);
         if constexpr (claims_tiles<MODE>()) {
-          // the next claim and its record are fetched while this tile's
-          // loads are issued, so no global round trip sits between tiles
           if (cur >= n_tiles || *abort_flag) cur = -1;
-          if (cur >= 0 && claim < n_tiles) {
-            nxt = claim;
-            nxt_rec = moe_record(p, tb, nxt);
-            claim = static_cast<int>(gridDim.x) + atomicAdd(p.work, 1);
-          }
           tile = cur;
           rec = cur_rec;
           const int slot = it % GEMM_SCHED;
@@ -550,6 +544,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_kernel(const __grid_cons
         decode_tile<MODE>(p, tile, rec, n_gu, t);
         const uint64_t pol_a = t.a_stream ? pol_first : pol_last;
         for (int k = 0; k < t.nk; ++k) {
+          if constexpr (claims_tiles<MODE>()) {
+            // the next claim and its record are taken once this tile's first
+            // loads are in flight (the claim's atomic was issued a tile
+            // earlier, or at setup), so no global round trip sits between
+            // tiles or before the first one
+            if (k == min(2, t.nk - 1) && claim < n_tiles) {
+              nxt = claim;
+              nxt_rec = moe_record(p, tb, nxt);
+              claim = static_cast<int>(gridDim.x) + atomicAdd(p.work, 1);
+            }
+          }
           if (!mbar_wait(&empty[stage], phase ^ 1, p.err)) {
             *abort_flag = 1;
             break;
