@@ -13,6 +13,7 @@ from .model import (Oracle, Shape, StepResult, anneal_temperature, apply_rope, a
                     entropy_sample, lm_head_stats, mean_entropy, moe,
                     renoise_tokens, rms_norm, rope_angles, route_top_k, sample, selected_gates, self_condition, silu,
                     swiglu_ffn, tokens_per_forward, tokens_per_second)
+from .mx import e4m3_round, moe_mx, mx_dequantize, mx_linear, mx_quantize, mx_round_trip, mx_swiglu_ffn
 from .philox import philox4x32_10, uniform_token
 
 
@@ -25,11 +26,13 @@ def shape_of(w) -> Shape:
                  vocab=s.vocab, rope_base=s.rope_base, rms_eps=s.rms_eps)
 
 
-def for_workload(w, keep_layers: bool = True, layer_override=None, seq_ids=None) -> Oracle:
+def for_workload(w, keep_layers: bool = True, layer_override=None, seq_ids=None,
+                 expert_format: str = "bf16") -> Oracle:
     """Oracle over the seeded weights of workload `w` (generated on the CPU).
 
     layer_override(l, tensors) may edit a layer's tensors (planted cases);
-    seq_ids gives the batch index of each of the oracle's sequences."""
+    seq_ids gives the batch index of each of the oracle's sequences;
+    expert_format "mxfp8" runs every expert GEMM in MXFP8 (oracle/mx.py)."""
     import synth_inputs as si
 
     def layer_fn(l):
@@ -40,4 +43,4 @@ def for_workload(w, keep_layers: bool = True, layer_override=None, seq_ids=None)
 
     g = si.global_weights(w, "cpu")
     return Oracle(shape_of(w), layer_fn, g["embed"], g["final_norm"], g["router_bias"],
-                  batch=w.batch, keep_layers=keep_layers, seq_ids=seq_ids)
+                  batch=w.batch, keep_layers=keep_layers, seq_ids=seq_ids, expert_format=expert_format)

@@ -38,6 +38,7 @@ from dataclasses import dataclass, field
 
 import numpy as np
 
+from .mx import moe_mx
 from .philox import philox4x32_10, uniform_token
 
 
@@ -370,8 +371,12 @@ class Oracle:
     """
 
     def __init__(self, shape: Shape, layer_fn, embed, final_norm, router_bias=None,
-                 batch: int = 1, keep_layers: bool = True, seq_ids=None):
+                 batch: int = 1, keep_layers: bool = True, seq_ids=None, expert_format: str = "bf16"):
         self.s = shape
+        # "bf16": experts as stored; "mxfp8": every expert GEMM with both
+        # operands in MXFP8 (oracle/mx.py, the FP8 reading of section 5.2)
+        assert expert_format in ("bf16", "mxfp8")
+        self.expert_format = expert_format
         self.layer_fn = layer_fn
         self.embed = embed            # kept in storage precision; rows converted on use
         self.final_norm = _f64(final_norm)
@@ -447,7 +452,7 @@ class Oracle:
             else:
                 idx = np.asarray(forced_idx, dtype=np.int64)
                 gates = selected_gates(r, idx)
-            h = h + moe(u2, lw, idx, gates)
+            h = h + (moe(u2, lw, idx, gates) if self.expert_format == "bf16" else moe_mx(u2, lw, idx, gates))
             if dbg is not None:
                 dbg["idx"], dbg["logits"] = idx, r
                 srt = -np.sort(-r, axis=1)
