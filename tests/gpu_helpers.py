@@ -301,5 +301,6 @@ def compare_step(g: dict, r: "oracle.StepResult", tau: float, orc=None, check_hi
         report.append(out)
     print({k: v for k, v in out.items()})
     assert not fails, fails
-    out["diverged"] = diverged   # tokens whose routing legitimately left the oracle's
-    return out
+    res = dict(out)
+    res["diverged"] = diverged   # tokens whose routing legitimately left the oracle's
+    return res

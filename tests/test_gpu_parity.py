@@ -246,7 +246,7 @@ def test_a4b_full_depth_step_prefix_2048():
     r = oracle_step(orc, canvas, 0, w.sample_seed, tau, 1.0, g)
     # per layer (teacher-forced) at 1e-2; the free-running drift over 30 layers at 2e-2
     res = compare_step(g, r, tau, orc=orc, drift_tol=2e-2)
-    print("a4b full depth:", res)
+    print("a4b full depth:", {k: v for k, v in res.items() if k != "diverged"})
     assert res["forced_hidden_rel_l2_max"] <= 1e-2
     assert res["forced_argmax_checked"] > 200
 
