@@ -2,6 +2,7 @@
 """Throughput of the block discrete-diffusion denoising step on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+    python bench.py --impl reference --reference-sample full --steps 1 --warmup 0
     python bench.py --timeline        (per-kernel spans inside the step's graph)
     python bench.py --batch-sweep 1,2,4,8,16,32
 
@@ -143,6 +144,11 @@ def parse():
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--workload", default="a4b_p2k")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--reference-sample", choices=["bounded", "full"], default="bounded",
+                    help="--impl reference: time a bounded sample of each step (default, minutes in all) "
+                         "or whole oracle steps over every layer and the full vocabulary (the a4b step "
+                         "takes minutes per step on the host cores and holds its bf16 weights, ~23 GB, "
+                         "in host memory)")
     ap.add_argument("--layers", type=int, default=0,
                     help="reduced depth (profiling captures only; not a bench number)")
     ap.add_argument("--batch-sweep", default="",
@@ -334,13 +340,49 @@ class OracleSample:
         return w.batch * w.canvas / t_step, t_step, t_layer + t_lm_sample, desc
 
 
+class OracleFullStep:
+    """The fp64 oracle timed on whole steps: every layer over the whole canvas,
+    then the LM head over the full vocabulary and the sampler.  Each layer's
+    seeded bf16 weights are generated once, during the (untimed) prefill, and
+    kept in host memory; the bf16 -> fp64 conversions the oracle makes during
+    its step are inside the timing, as in the bounded sample."""
+
+    def __init__(self, w):
+        import oracle
+        import synth_inputs as si
+        self.w = w
+        bf16 = {}
+
+        def layer_fn(l):
+            if l not in bf16:
+                bf16[l] = si.layer_weights(w, l, "cpu")
+            return bf16[l]
+
+        g = si.global_weights(w, "cpu")
+        self.orc = oracle.Oracle(oracle.shape_of(w), layer_fn, g["embed"], g["final_norm"], g["router_bias"],
+                                 batch=w.batch, keep_layers=False)
+        self.orc.prefill(si.uniform_tokens(w, "prefix", w.batch, w.prefix).numpy())
+        self.canvas = si.uniform_tokens(w, "canvas", w.batch, w.canvas).numpy()
+
+    def run(self, step=0):
+        """Returns (canvas tokens/s, step seconds, step seconds, description)."""
+        w = self.w
+        t0 = time.perf_counter()
+        self.orc.denoise_step(self.canvas, step, w.sample_seed, w.tau0)
+        t = time.perf_counter() - t0
+        desc = (f"oracle (fp64 numpy) whole step: {w.shape.n_layers} layers over the {w.batch}x{w.canvas} canvas "
+                f"with the {w.prefix}-token cache, LM head over all {w.shape.vocab} vocabulary rows, sampler")
+        return w.batch * w.canvas / t, t, t, desc
+
+
 def run_reference(args, w):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     vals, spent = [], []
     desc = ""
-    sample = OracleSample(w)
+    full = args.reference_sample == "full"
+    sample = OracleFullStep(w) if full else OracleSample(w)
     for i in range(args.warmup + args.steps):
         v, t, t_sample, desc = sample.run()
         if i >= args.warmup:
@@ -350,7 +392,8 @@ def run_reference(args, w):
     value = w.batch * w.canvas / t
     cores = _cores()
     # each timed step is one bounded sample of the step (ms_per_step: the time
-    # it took); value is the full step's throughput extrapolated from it
+    # it took; value: the full step's throughput extrapolated from it), or
+    # with --reference-sample full one whole step
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": statistics.median(spent) * 1e3,
             "extrapolated_ms_per_full_step": t * 1e3, "higher_is_better": True,
@@ -358,6 +401,9 @@ def run_reference(args, w):
             "config": {"workload": f"{w.name}: {w.description}"},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    if full:
+        line.pop("extrapolated_ms_per_full_step")
+        line["step_seconds"] = [round(x, 3) for x in vals]
     print(json.dumps(line), flush=True)
 
 

@@ -102,3 +102,25 @@ def test_mode_flags_parse_and_the_timeline_mode_selects_the_tracing_build(monkey
     assert bench.parse().batch_sweep == "1,2"
     src = open(bench.__file__).read()
     assert 'os.environ["DG_LIBRARY"] = os.path.join(ROOT, "block_discrete_diffusion_denoise_b200", "libdg_timeline.so")' in src
+
+
+@pytest.mark.parametrize("mode", ["bounded", "full"])
+def test_reference_arm_line_on_the_tiny_workload(mode, capsys):
+    """--impl reference prints one line on the oracle's own clock: the bounded
+    sample extrapolates to the full step; --reference-sample full times whole
+    steps, so its value is the canvas over the measured step time."""
+    import argparse
+    import json
+    args = argparse.Namespace(gpus=1, steps=1, warmup=0, reference_sample=mode)
+    bench.run_reference(args, si.workload("tiny"))
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["dtype"] == "f64" and line["unit"] == bench.UNIT
+    assert line["e2e"]["value"] == line["value"] == line["cpu_baseline"]["value"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+    if mode == "full":
+        assert "whole step" in line["cpu_baseline"]["sample"]
+        assert line["value"] == pytest.approx(256 / line["step_seconds"][0], rel=1e-2)
+        assert line["ms_per_step"] == pytest.approx(line["step_seconds"][0] * 1e3, rel=1e-2)
+    else:
+        assert line["extrapolated_ms_per_full_step"] > line["ms_per_step"] > 0
+        assert line["value"] == pytest.approx(256 / (line["extrapolated_ms_per_full_step"] * 1e-3))
