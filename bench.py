@@ -147,7 +147,7 @@ def parse():
     ap.add_argument("--reference-sample", choices=["bounded", "full"], default="bounded",
                     help="--impl reference: time a bounded sample of each step (default, minutes in all) "
                          "or whole oracle steps over every layer and the full vocabulary (the a4b step "
-                         "takes minutes per step on the host cores and holds its bf16 weights, ~23 GB, "
+                         "takes minutes per step on the host cores and holds its bf16 weights, ~50 GB, "
                          "in host memory)")
     ap.add_argument("--layers", type=int, default=0,
                     help="reduced depth (profiling captures only; not a bench number)")
