@@ -138,14 +138,105 @@ def _ptr(t) -> int | None:
     return t.data_ptr()
 
 
+DG_ERR_INVALID_ARG = 1
+
+
+def _invalid(msg: str):
+    raise DGError(DG_ERR_INVALID_ARG, msg)
+
+
+def _check_tensor(t, dtype, n: int, what: str, device_type: str = "cuda", exact: bool = False,
+                  optional: bool = False):
+    """The checks a bare pointer cannot carry through the C ABI: t is a
+    contiguous torch tensor of `dtype` on `device_type` holding at least (with
+    exact, exactly) n elements.  The library reads or writes n elements at the
+    address; a smaller, strided, misplaced or wrongly typed buffer would be
+    read or written out of bounds or misread, so it is refused here
+    (DG_ERR_INVALID_ARG) with nothing launched."""
+    import torch
+    if t is None:
+        if optional:
+            return
+        _invalid(f"{what}: required")
+    if not isinstance(t, torch.Tensor) or t.device.type != device_type or t.dtype != dtype \
+            or not t.is_contiguous():
+        _invalid(f"{what}: expected a contiguous {device_type} tensor of {dtype}, got "
+                 f"{getattr(t, 'dtype', type(t).__name__)} on {getattr(t, 'device', '?')}"
+                 f"{'' if getattr(t, 'is_contiguous', lambda: True)() else ' (strided)'}")
+    if (t.numel() != n) if exact else (t.numel() < n):
+        _invalid(f"{what}: {t.numel()} elements, {'expected' if exact else 'the call needs'} {n}")
+
+
+def _check_host(a, dtype, n: int, what: str, optional: bool = False):
+    """Host buffers of dg_denoise_step_host: a C-contiguous numpy array or a
+    contiguous CPU tensor of `dtype` with at least n elements."""
+    import numpy as np
+    import torch
+    if a is None:
+        if optional:
+            return
+        _invalid(f"{what}: required")
+    if isinstance(a, np.ndarray):
+        if a.dtype != np.dtype(dtype) or not a.flags["C_CONTIGUOUS"] or a.size < n:
+            _invalid(f"{what}: expected a C-contiguous {np.dtype(dtype)} array of at least {n} elements")
+        return
+    tdt = {np.int32: torch.int32, np.float32: torch.float32}[dtype]
+    _check_tensor(a, tdt, n, what, device_type="cpu")
+
+
+def weight_numels(cfg: dict) -> dict:
+    """Element count of every weight tensor the C ABI reads for a dg_config
+    (dg_weights / dg_layer_weights layouts of include/dg.h)."""
+    d, E, F, Fs = cfg["d_model"], cfg["n_experts"], cfg["expert_hidden"], cfg["shared_hidden"]
+    Hq, Hkv, D = cfg["n_q_heads"], cfg["n_kv_heads"], cfg["head_dim"]
+    return {
+        "embed": cfg["vocab"] * d, "final_norm": d, "router_bias": E,
+        "sc_gate": F * d, "sc_up": F * d, "sc_down": d * F,
+        "layer": {"attn_norm": d, "wqkv": (Hq + 2 * Hkv) * D * d, "wo": d * Hq * D, "ffn_norm": d,
+                  "w_router": E * d, "w_gate": E * F * d, "w_up": E * F * d, "w_down": E * d * F,
+                  "ws_gate": Fs * d, "ws_up": Fs * d, "ws_down": d * Fs},
+    }
+
+
+def check_weights(cfg: dict, weights: dict, device_type: str = "cuda"):
+    """Refuse (DG_ERR_INVALID_ARG) weights the library would read out of
+    bounds or misread: every tensor contiguous on the device, bf16 (the router
+    bias fp32), with the element count the configuration implies, one layer
+    dict per layer; the self-conditioning weights all three or none."""
+    import torch
+    n = weight_numels(cfg)
+    bf16 = torch.bfloat16
+    _check_tensor(weights.get("embed"), bf16, n["embed"], "embed", device_type, exact=True)
+    _check_tensor(weights.get("final_norm"), bf16, n["final_norm"], "final_norm", device_type, exact=True)
+    _check_tensor(weights.get("router_bias"), torch.float32, n["router_bias"], "router_bias", device_type,
+                  exact=True, optional=True)
+    layers = weights.get("layers")
+    if layers is None or len(layers) != cfg["n_layers"]:
+        _invalid(f"layers: expected {cfg['n_layers']} layer dicts, got {None if layers is None else len(layers)}")
+    for i, lw in enumerate(layers):
+        for f in LAYER_FIELDS:
+            _check_tensor(lw.get(f), bf16, n["layer"][f], f"layers[{i}].{f}", device_type, exact=True)
+    sc = [weights.get(k) is not None for k in ("sc_gate", "sc_up", "sc_down")]
+    if any(sc) and not all(sc):
+        _invalid("self-conditioning weights: give sc_gate, sc_up and sc_down, or none")
+    for k in ("sc_gate", "sc_up", "sc_down"):
+        _check_tensor(weights.get(k), bf16, n[k], k, device_type, exact=True, optional=True)
+
+
 class Context:
     """One dg_ctx.  `weights` holds torch CUDA tensors (bf16) named as in
     dg.h: embed, final_norm, router_bias (fp32 or None) and layers (list of
     dicts with the LAYER_FIELDS keys).  The tensors are referenced for the
     lifetime of the context."""
 
+    # where the context's buffers must live (the tests of the argument checks
+    # set "cpu" on an instance that never reaches the library)
+    _device_type = "cuda"
+
     def __init__(self, cfg: dict, weights: dict, stream=None):
         self.lib = load_library()
+        self._batch = None            # batch of the last successful prefill
+        check_weights(cfg, weights, self._device_type)
         self._weights = weights
         c = dg_config()
         for name, _ in dg_config._fields_:
@@ -183,23 +274,55 @@ class Context:
             pass
 
     # --- the path ---
+    # The library sees bare pointers; the buffers are checked here against the
+    # sizes the call reads and writes (the batch of the last prefill times the
+    # canvas), and a bad one raises DGError(DG_ERR_INVALID_ARG) with nothing
+    # launched.  Before the first prefill the library itself refuses the call.
+    def _n(self) -> int:
+        return 0 if self._batch is None else self._batch * int(self.cfg["canvas"])
+
+    def _dev(self, t, dtype, n, what, optional=False):
+        _check_tensor(t, dtype, n, what, self._device_type, optional=optional)
+        return _ptr(t)
+
     def prefill(self, tokens):
+        import torch
+        if getattr(tokens, "dim", lambda: 0)() != 2:
+            _invalid("prefill: tokens must be a [batch, prefix_len] tensor")
         B, P = tokens.shape
-        self._check(self.lib.dg_prefill(self.ctx, _ptr(tokens), B, P))
+        self._check(self.lib.dg_prefill(self.ctx, self._dev(tokens, torch.int32, B * P, "tokens"), B, P))
+        self._batch = int(B)
 
     def denoise_step(self, canvas_in, step, seed, tau, canvas_out, conf, settled=None):
-        self._check(self.lib.dg_denoise_step(self.ctx, _ptr(canvas_in), int(step), int(seed), float(tau),
-                                             _ptr(canvas_out), _ptr(conf), _ptr(settled)))
+        import torch
+        n, B = self._n(), self._batch or 0
+        self._check(self.lib.dg_denoise_step(
+            self.ctx, self._dev(canvas_in, torch.int32, n, "canvas_in"), int(step), int(seed), float(tau),
+            self._dev(canvas_out, torch.int32, n, "canvas_out"), self._dev(conf, torch.float32, n, "conf"),
+            self._dev(settled, torch.int32, B, "settled", optional=True)))
 
     def denoise_step_entropy(self, canvas_in, step, seed, temperature, gamma, stop_entropy, canvas_out,
                              prev_argmax=None, argmax_out=None, entropy=None, stopped=None):
+        import torch
+        n, B = self._n(), self._batch or 0
         a = dg_entropy_args(float(temperature), float(gamma), float(stop_entropy))
-        self._check(self.lib.dg_denoise_step_entropy(self.ctx, _ptr(canvas_in), int(step), int(seed), ctypes.byref(a),
-                                                     _ptr(prev_argmax), _ptr(argmax_out), _ptr(canvas_out),
-                                                     _ptr(entropy), _ptr(stopped)))
+        self._check(self.lib.dg_denoise_step_entropy(
+            self.ctx, self._dev(canvas_in, torch.int32, n, "canvas_in"), int(step), int(seed), ctypes.byref(a),
+            self._dev(prev_argmax, torch.int32, n, "prev_argmax", optional=True),
+            self._dev(argmax_out, torch.int32, n, "argmax_out", optional=True),
+            self._dev(canvas_out, torch.int32, n, "canvas_out"),
+            self._dev(entropy, torch.float32, n, "entropy", optional=True),
+            self._dev(stopped, torch.int32, B, "stopped", optional=True)))
 
     def denoise_step_host(self, canvas_in, step, seed, tau, canvas_out, conf=None, settled=None):
         """Host-buffer variant: numpy int32/float32 arrays (or pinned CPU tensors)."""
+        import numpy as np
+        n, B = self._n(), self._batch or 0
+        _check_host(canvas_in, np.int32, n, "canvas_in")
+        _check_host(canvas_out, np.int32, n, "canvas_out")
+        _check_host(conf, np.float32, n, "conf", optional=True)
+        _check_host(settled, np.int32, B, "settled", optional=True)
+
         def hp(a):
             if a is None:
                 return None
@@ -208,7 +331,8 @@ class Context:
                                                   hp(canvas_out), hp(conf), hp(settled)))
 
     def commit_block(self, block):
-        self._check(self.lib.dg_commit_block(self.ctx, _ptr(block)))
+        import torch
+        self._check(self.lib.dg_commit_block(self.ctx, self._dev(block, torch.int32, self._n(), "block")))
 
     def sync(self):
         self._check(self.lib.dg_sync(self.ctx))
