@@ -259,6 +259,30 @@ def test_tpf_tps_definitions():
     assert om.tokens_per_second(20.0, 0.01356) == pytest.approx(1474.9, rel=1e-4)
 
 
+def test_tps_reproduces_the_printed_worked_example():
+    """The pages' own numbers (tests/golden/codemajin_throughput_example.txt):
+    TPS = TPF / t_fwd gives the printed 1,456 tok/s from TPF 19.74 and a
+    13.56 ms step, and the printed speed-ups and sampling ratio follow from
+    the printed rates and times, each at the precision it is printed to."""
+    g = {}
+    for line in open(os.path.join(GOLD, "codemajin_throughput_example.txt")):
+        if line.strip() and not line.startswith("#"):
+            name, value, dec = line.split()
+            g[name] = (float(value), int(dec))
+
+    def printed(x, name):
+        v, dec = g[name]
+        assert round(x, dec) == v, (name, x, v)
+
+    tps = om.tokens_per_second(g["tpf"][0], g["t_fwd_ms"][0] * 1e-3)
+    printed(tps, "tps")
+    printed(g["tps"][0] / g["ar_tps"][0], "speedup_vs_ar")
+    printed(g["tps"][0] / g["ar_mtp_tps"][0], "speedup_vs_ar_mtp")
+    printed(g["sampling_diffusion_ms"][0] / g["sampling_ar_ms"][0], "sampling_ratio")
+    # t_fwd must be in seconds: in milliseconds the same formula misses it
+    assert round(om.tokens_per_second(g["tpf"][0], g["t_fwd_ms"][0])) != g["tps"][0]
+
+
 # --- whole-model invariants on a tiny seeded workload ------------------------
 def _tiny(**kw):
     w = si.workload("tiny").with_(**kw)
