@@ -292,9 +292,9 @@ dg_status dg_debug_gemm(dg_ctx* ctx, const void* w_dev, int32_t M, int32_t K, co
 /* Kernel classes timed by the profiling hooks. */
 enum {
   DG_PROF_EXPERTS = 0,       /* fused routed + shared expert GEMM: gate/up (SwiGLU) and down   */
-  DG_PROF_ROUTING = 1,       /* router top-k, token permutation and row gather                 */
+  DG_PROF_ROUTING = 1,       /* router top-k, expert row claim and row gather (one kernel)    */
   DG_PROF_LMHEAD = 2,        /* LM-head GEMM with the argmax / log-sum-exp epilogue            */
-  DG_PROF_ATTENTION = 3,     /* attention kernel (key chunks merged inside the kernel)         */
+  DG_PROF_ATTENTION = 3,     /* attention kernel and the merge of its key chunks              */
   DG_PROF_DENSE = 4,         /* QKV, output and router projections                            */
   DG_PROF_OTHER = 5,         /* norms, RoPE, combine, LM-head merge + sampler                 */
   DG_PROF_CLASSES = 6
