@@ -260,6 +260,18 @@ class Clocks:
 # ---------------------------------------------------------------------------
 # replicas: one process per GPU, no collective on the data path
 # ---------------------------------------------------------------------------
+def code_sha256(path: str) -> str:
+    """sha256 of a CUDA/C++ source with its comments removed and whitespace
+    collapsed: the identity of the code a set of ncu counters was taken on,
+    unchanged by edits to comments or layout, changed by any edit to code."""
+    import hashlib
+    import re
+    src = open(path).read()
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", " ", src)
+    return hashlib.sha256(" ".join(src.split()).encode()).hexdigest()
+
+
 def max_over_ranks(value: float, world: int, device) -> float:
     """The slowest rank's value; every rank must call it (a no-op on one rank)."""
     if world <= 1:
@@ -533,11 +545,9 @@ def run_native(args, w):
     tp = os.path.join(ROOT, "profiles", "expert_gemm_traffic.json")
     if os.path.exists(tp):
         try:
-            import hashlib
             rec = json.load(open(tp))
-            src_hash = hashlib.sha256(open(os.path.join(ROOT, "block_discrete_diffusion_denoise_b200", "csrc",
-                                                        "gemm.cuh"), "rb").read()).hexdigest()
-            if rec.get("gemm_cuh_sha256") == src_hash and rec.get("workload") == w.name:
+            src_hash = code_sha256(os.path.join(ROOT, "block_discrete_diffusion_denoise_b200", "csrc", "gemm.cuh"))
+            if rec.get("gemm_cuh_code_sha256") == src_hash and rec.get("workload") == w.name:
                 traffic = rec["bytes_per_launch"]
         except Exception:
             traffic = None

@@ -2,11 +2,12 @@
 //
 //   D[m, n] = sum_k A[m, k] * B[n, k]        (A, B bf16 K-major; D fp32 in TMEM)
 //
-// One CTA per SM.  Warp 0 (one lane) issues TMA loads into a ring of
-// shared-memory stages (4 for DENSE, 6 otherwise), warp 1 (one lane) issues
-// tcgen05.mma into one of two TMEM accumulators (128 lanes x 128 or 256 fp32
-// columns each), warps 2..5 drain the other accumulator through the epilogue.
-// All waits are bounded.
+// One CTA per SM.  Warp 0 (one lane) loads the A operand and warp 6 (one
+// lane) the B operand of every stage of one ring of shared-memory stages (6
+// for MOE, 4 otherwise) with TMA, warp 1 (one lane) issues tcgen05.mma into
+// one of two TMEM accumulators (128 lanes x 128 or 256 fp32 columns each),
+// warps 2..5 drain the other accumulator through the epilogue.  All waits are
+// bounded.
 //
 // Three launch modes share the pipeline:
 //   DENSE   A = weight rows (output features), B = up to 256 tokens; split-K
@@ -23,7 +24,8 @@
 //           token chunk has published its hidden rows.  Every claimed tile's
 //           dependencies were claimed earlier by running CTAs and depend on
 //           nothing, so the wait always ends.
-//   LMHEAD  A = 128 tokens, B = 128 vocabulary rows of the tied embedding; the
+//   LMHEAD  A = two 128-token tiles (each vocabulary block is loaded once for
+//           256 tokens), B = 128 vocabulary rows of the tied embedding; the
 //           epilogue keeps, per token, the running top-2 logits, the argmax,
 //           the sum of 2^x and the sum of 2^x * x (for the entropy), and
 //           writes one 16-byte partial (+ 4 bytes) per (vocabulary tile,

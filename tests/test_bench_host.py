@@ -124,3 +124,24 @@ def test_reference_arm_line_on_the_tiny_workload(mode, capsys):
     else:
         assert line["extrapolated_ms_per_full_step"] > line["ms_per_step"] > 0
         assert line["value"] == pytest.approx(256 / (line["extrapolated_ms_per_full_step"] * 1e-3))
+
+
+def test_code_hash_ignores_comments_and_layout_but_not_code(tmp_path):
+    """The traffic record stays valid across comment edits of the kernel
+    source and lapses with any code edit."""
+    src = ("// header comment\n#include \"common.cuh\"\n/* block\n comment */\n"
+           "constexpr int A = 4;  // trailing\n__global__ void k(int* p) { p[0] = A; }\n")
+    variants = {
+        "same": src,
+        "comments": src.replace("header comment", "another header").replace("trailing", "changed"),
+        "layout": src.replace("constexpr int A = 4;", "constexpr   int A =\n    4;"),
+        "code": src.replace("A = 4", "A = 5"),
+        "code in body": src.replace("p[0] = A", "p[1] = A"),
+    }
+    h = {}
+    for name, text in variants.items():
+        f = tmp_path / f"{name}.cuh"
+        f.write_text(text)
+        h[name] = bench.code_sha256(str(f))
+    assert h["same"] == h["comments"] == h["layout"]
+    assert h["code"] != h["same"] and h["code in body"] != h["same"]
