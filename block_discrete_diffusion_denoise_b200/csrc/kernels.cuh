@@ -2,7 +2,8 @@
 // reduction + residual + RMSNorm, QKV reduction + RoPE + KV write, router
 // top-k with the dispatch of every token's activations to its experts' rows,
 // gate-weighted combine + residual + RMSNorm, LM-head partial merge + Philox
-// sampler.
+// sampler, the entropy-constrained sampler, and the split reductions of the
+// self-conditioning layer.
 #pragma once
 
 #include "common.cuh"
