@@ -423,7 +423,6 @@ def run_reference(args, w):
 # native
 # ---------------------------------------------------------------------------
 def run_native(args, w):
-    import numpy as np
     import torch
     import torch.distributed as dist
 
@@ -518,11 +517,14 @@ def run_native(args, w):
     breakdown = {k: round(v[0] / 2, 4) for k, v in ctx.debug_profile_read().items()}
     ctx.debug_profile([])
 
-    # ---- end to end through the host-buffer entry point ----
-    hin = np.ascontiguousarray(cur.cpu().numpy(), dtype=np.int32)
-    hout = np.empty_like(hin)
-    hconf = np.empty((B, C), np.float32)
-    hset = np.empty(B, np.int32)
+    # ---- end to end through the host-buffer entry point, from pinned host
+    # memory (each call copies the canvas in, runs the step, copies canvas,
+    # confidences and flags out and synchronises) ----
+    hin = torch.empty((B, C), dtype=torch.int32, pin_memory=True)
+    hin.copy_(cur)
+    hout = torch.empty((B, C), dtype=torch.int32, pin_memory=True)
+    hconf = torch.empty((B, C), dtype=torch.float32, pin_memory=True)
+    hset = torch.empty(B, dtype=torch.int32, pin_memory=True)
     ctx.denoise_step_host(hin, 0, seed, w.tau0, hout, hconf, hset)
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
