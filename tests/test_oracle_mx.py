@@ -16,6 +16,10 @@ def test_e4m3_round_matches_torch_inside_the_finite_range():
     x = np.concatenate([rng.standard_normal(20000) * s for s in (1e-3, 0.05, 1.0, 30.0, 150.0)])
     x = np.concatenate([x, np.ldexp(rng.uniform(1, 2, 2000), rng.integers(-12, 9, 2000))])
     x = x[np.abs(x) < 464.0]                 # torch turns |x| >= 464 into NaN; MX saturates (below)
+    # torch converts a float64 tensor to E4M3 through float32, so a value
+    # within half a float32 ulp of an E4M3 midpoint would be rounded twice
+    # there; on the float32 grid both sides round once
+    x = x.astype(np.float32).astype(np.float64)
     ref = torch.tensor(x, dtype=torch.float64).to(torch.float8_e4m3fn).to(torch.float64).numpy()
     np.testing.assert_array_equal(mx.e4m3_round(x), ref)
     codes = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
