@@ -2,7 +2,10 @@
 wrong sign, index, exponent or comparison, a transposed or swapped operand)
 is planted in the oracle on the CPU, and at least one pin of
 test_oracle_pins.py / test_oracle_mx.py must then fail with an assertion.
-The mutants are test code; the oracle itself is restored after each case."""
+Mistakes in the step's wiring (which keys a canvas row sees, where RoPE
+positions start) are planted in the oracle too and must break its agreement
+with the one-pass restatement of test_oracle_step_wiring.py.  The mutants are
+test code; the oracle itself is restored after each case."""
 import numpy as np
 import pytest
 
@@ -320,3 +323,81 @@ def test_unmutated_pins_pass():
     for module, attr, make, checks in MUTANTS.values():
         for check in checks:
             check()
+
+
+# --- wiring mistakes planted in the oracle's step, caught by the one-pass ----
+# restatement of test_oracle_step_wiring.py (computed once, unmutated)
+def _step_attention(transform):
+    """attention() wrapper applying `transform` only to step-mode calls (every
+    row sees the same number of keys: the cache plus the whole canvas)."""
+    def mutant(orig):
+        def f(q, k, v, key_limit):
+            lim = np.asarray(key_limit)
+            if lim.size > 1 and (lim == lim[0]).all():
+                q, k, v, lim = transform(q, k, v, lim)
+            return orig(q, k, v, lim)
+        return f
+    return mutant
+
+
+def _causal_canvas(q, k, v, lim):
+    n = q.shape[1]
+    return q, k, v, lim[0] - n + 1 + np.arange(n)
+
+
+def _canvas_only(q, k, v, lim):
+    n = q.shape[1]
+    return q, k[:, -n:], v[:, -n:], np.full(n, n)
+
+
+def _cache_only(q, k, v, lim):
+    n = q.shape[1]
+    S = k.shape[1]
+    return q, k[:, :S - n], v[:, :S - n], np.full(n, S - n)
+
+
+def _rope_from_zero(orig):
+    return lambda positions, head_dim, base: orig(np.asarray(positions) - np.min(positions), head_dim, base)
+
+
+WIRING_MUTANTS = {
+    "step: causal among canvas rows": (om, "attention", _step_attention(_causal_canvas)),
+    "step: canvas sees only itself": (om, "attention", _step_attention(_canvas_only)),
+    "step: canvas sees only the cache": (om, "attention", _step_attention(_cache_only)),
+    "RoPE positions restart at 0 in every call": (om, "rope_angles", _rope_from_zero),
+}
+
+
+@pytest.fixture(scope="module")
+def one_pass():
+    import synth_inputs as si
+    import test_oracle_step_wiring as wiring
+    import torch
+    w = si.workload("tiny").with_(prefix=48)
+    weights = si.model_weights(w, "cpu")
+    prompt = si.uniform_tokens(w, "prefix", 1, w.prefix)
+    canvas = si.uniform_tokens(w, "canvas", 1, w.canvas)
+    hidden, _, _ = wiring._sequence_forward(w, weights, torch.cat([prompt, canvas], 1)[0], w.prefix,
+                                            "bidirectional")
+    return w, prompt.numpy(), canvas.numpy(), [h[w.prefix:].numpy() for h in hidden]
+
+
+def _step_matches_one_pass(w, prompt, canvas, hidden):
+    import oracle
+    orc = oracle.for_workload(w)
+    orc.prefill(prompt)
+    r = orc.denoise_step(canvas, 0, 1, 0.9, temperature=0.5)
+    for l in range(w.shape.n_layers + 1):
+        np.testing.assert_allclose(r.hidden[l][0], hidden[l], rtol=1e-10, atol=1e-12)
+
+
+def test_unmutated_step_matches_one_pass(one_pass):
+    _step_matches_one_pass(*one_pass)
+
+
+@pytest.mark.parametrize("name", sorted(WIRING_MUTANTS))
+def test_planted_wiring_mistake_in_the_oracle_fails(name, one_pass, monkeypatch):
+    module, attr, make = WIRING_MUTANTS[name]
+    monkeypatch.setattr(module, attr, make(getattr(module, attr)))
+    with pytest.raises(AssertionError):
+        _step_matches_one_pass(*one_pass)
