@@ -244,6 +244,10 @@ def _e4m3_no_saturation(orig):
     return f
 
 
+def _mx_activations_unquantised(orig):
+    return lambda x, w: np.asarray(x, dtype=np.float64) @ mx.mx_round_trip(w).T
+
+
 def _mx_exponent_off_by_one(orig):
     return lambda x, block=mx.MX_BLOCK: orig(x, block) + 1
 
@@ -301,6 +305,8 @@ MUTANTS = {
     "e4m3: no saturation": (mx, "e4m3_round", _e4m3_no_saturation, [mxpins.test_e4m3_saturation_and_subnormal_ties]),
     "mx: block exponent off by one": (mx, "mx_block_exponents", _mx_exponent_off_by_one,
                                       [mxpins.test_block_exponent_closed_forms]),
+    "mx: activations left unquantised": (mx, "mx_linear", _mx_activations_unquantised,
+                                         [mxpins.test_mx_linear_worked_example_by_hand]),
 }
 
 

@@ -82,6 +82,23 @@ def test_mx_linear_is_exact_on_representable_operands():
     np.testing.assert_array_equal(mx.mx_linear(x, w), x @ w.T)
 
 
+def test_mx_linear_worked_example_by_hand():
+    """One 32-element block each, worked by hand.  x = (448, 1.06, 0...):
+    max 448 = 1.75 * 2^8 gives exponent 0, scale 1; 448 is on the grid, 1.06
+    lies in [1, 2) where the step is 1/8, nearest 1.0.  w = (1, 0.53, 0...):
+    max 1 gives exponent -8, scale 2^-8; 0.53 * 256 = 135.68 lies in
+    [128, 256) where the step is 16, nearest 128, i.e. 0.5.  So the product
+    is 448 * 1 + 1.0 * 0.5 = 448.5, where unquantised operands give 448.5618."""
+    x = np.zeros((1, 32))
+    x[0, :2] = (448.0, 1.06)
+    w = np.zeros((1, 32))
+    w[0, :2] = (1.0, 0.53)
+    assert mx.mx_block_exponents(x).tolist() == [[0]] and mx.mx_block_exponents(w).tolist() == [[-8]]
+    np.testing.assert_array_equal(mx.mx_round_trip(x)[0, :2], [448.0, 1.0])
+    np.testing.assert_array_equal(mx.mx_round_trip(w)[0, :2], [1.0, 0.5])
+    assert mx.mx_linear(x, w)[0, 0] == 448.5
+
+
 def test_moe_with_all_experts_is_the_dense_mixture_of_mxfp8_experts():
     d, F, E = 64, 32, 4
 
