@@ -26,6 +26,10 @@
  *     reported by the next dg_sync as DG_ERR_DEVICE_TIMEOUT.
  *   - dg_last_error() returns a message for the last failed call on ctx
  *     (or, for ctx == NULL, for this thread's last failed dg_create).
+ *   - A context holds host-side state (its captured step graphs, the cached
+ *     length, error text): calls on one ctx must not overlap in time (one
+ *     host thread at a time, or the caller's own lock).  Distinct contexts
+ *     are independent of each other.
  */
 #ifndef DG_H
 #define DG_H
