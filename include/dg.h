@@ -29,7 +29,9 @@
  *   - A context holds host-side state (its captured step graphs, the cached
  *     length, error text): calls on one ctx must not overlap in time (one
  *     host thread at a time, or the caller's own lock).  Distinct contexts
- *     are independent of each other.
+ *     share nothing but the two process-wide device buffers described below
+ *     (the timeline records of the tracing build, and the scratch of
+ *     dg_lmhead_argmax_static).
  */
 #ifndef DG_H
 #define DG_H
