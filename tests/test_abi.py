@@ -104,3 +104,27 @@ def test_create_rejects_bad_arguments_without_a_device():
     lib = dgp.load_library()
     assert lib.dg_create(None, ctypes.byref(w), None, None) == 1
     assert lib.dg_last_error(None) == b"dg_create: null argument"
+
+
+def test_every_call_refuses_a_null_context_without_a_device():
+    """Each entry point checks its context (and, for the no-allocation LM
+    head, its operands) before anything else: with NULL it returns
+    DG_ERR_INVALID_ARG, or -1 for the two counters, and touches no device."""
+    lib = dgp.load_library()
+    for name in dgp.EXPORTS:
+        if name == "dg_create":
+            continue                                   # its NULL arguments: test_create_rejects_bad_arguments
+        f = getattr(lib, name)
+        args = [None] * len(f.argtypes)
+        for i, t in enumerate(f.argtypes):
+            if t in (ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64):
+                args[i] = 0
+            elif t is ctypes.c_float:
+                args[i] = 0.0
+        res = f(*args)
+        if name in ("dg_cached_len", "dg_debug_launch_count"):
+            assert res == -1, name
+        elif name == "dg_last_error":
+            assert isinstance(res, bytes), name
+        else:
+            assert res == 1, (name, res)
