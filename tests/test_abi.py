@@ -128,3 +128,23 @@ def test_every_call_refuses_a_null_context_without_a_device():
             assert isinstance(res, bytes), name
         else:
             assert res == 1, (name, res)
+
+
+def test_static_lmhead_refuses_bad_arguments_without_a_device():
+    """dg_lmhead_argmax_static checks shapes, alignment, temperature, outputs
+    and its fixed scratch capacity before it asks for a device (the addresses
+    below are never dereferenced)."""
+    lib = dgp.load_library()
+    z, e, out = 0x100000, 0x200000, ctypes.cast(0x300000, ctypes.POINTER(ctypes.c_int32))
+
+    def call(n_rows=256, d=2816, vocab=262144, temp=1.0, zp=z, ep=e, am=out):
+        return lib.dg_lmhead_argmax_static(zp, n_rows, d, ep, vocab, temp, am, None, None, None)
+
+    assert call(d=100) == 1                      # d_model not a multiple of 64
+    assert call(vocab=1000) == 1                 # vocab not a multiple of 128
+    assert call(n_rows=0) == 1
+    assert call(temp=0.0) == 1 and call(temp=float("nan")) == 1
+    assert call(zp=z + 8) == 1 and call(ep=e + 4) == 1      # not 16-byte aligned
+    assert call(zp=None) == 1
+    assert call(am=None) == 1                    # no output at all
+    assert call(n_rows=257) == 3                 # 257 x 262144 / 128 partials exceed the fixed scratch
