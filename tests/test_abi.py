@@ -82,11 +82,26 @@ def test_create_rejects_unsupported_shapes_without_a_device():
         "canvas": dict(canvas=200),                         # not a multiple of 16
         "d_model": dict(d_model=320),                       # not a multiple of 128
         "max_seq": dict(max_seq=128),                       # shorter than the canvas
+        "d_model too wide": dict(d_model=4224),             # a row kernel holds at most 4096
+        "vocab": dict(vocab=8000),                          # not a multiple of 128
+        "expert width": dict(expert_hidden=500),            # not a multiple of 64
+        "shared width": dict(shared_hidden=96 + 1),
+        "experts not a multiple of 4": dict(n_experts=18),
+        "top-k beyond 16": dict(n_experts=32, top_k=17),
+        "top-k beyond the experts": dict(top_k=20),
+        "canvas beyond 256": dict(canvas=272),
     }
     for what, over in cases.items():
         st, ctx, msg = _create(_tiny_config(**over), w)
         assert st == 7 and ctx is None, (what, st)          # DG_ERR_UNSUPPORTED, no context
         assert msg == "dg_create: unsupported shape", (what, msg)
+
+
+def test_create_rejects_workspaces_beyond_the_row_limit_without_a_device():
+    w, keep = _fake_weights(2)
+    for over in (dict(max_batch=129), dict(prefill_rows=40000)):     # more than 32768 rows
+        st, ctx, msg = _create(_tiny_config(**over), w)
+        assert (st, ctx) == (7, None) and "32768" in msg, (over, st, msg)
 
 
 def test_create_rejects_bad_arguments_without_a_device():
