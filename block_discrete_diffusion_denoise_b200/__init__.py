@@ -227,7 +227,10 @@ class Context:
     """One dg_ctx.  `weights` holds torch CUDA tensors (bf16) named as in
     dg.h: embed, final_norm, router_bias (fp32 or None) and layers (list of
     dicts with the LAYER_FIELDS keys).  The tensors are referenced for the
-    lifetime of the context."""
+    lifetime of the context.  Every call runs on `stream` (a cudaStream_t
+    handle, e.g. torch.cuda.Stream().cuda_stream; None is the legacy default
+    stream, on which steps are not captured into a graph): make inputs on it
+    (torch.cuda.stream(...)) or make it wait for the stream that did."""
 
     # where the context's buffers must live (the tests of the argument checks
     # set "cpu" on an instance that never reaches the library)

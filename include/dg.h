@@ -20,7 +20,9 @@
  *     dg_destroy.  The context owns the KV cache and every workspace buffer.
  *   - Every call is asynchronous on the stream given to dg_create, except
  *     dg_create, dg_destroy, dg_sync and dg_denoise_step_host, which
- *     synchronise.  Arguments and capacities are checked on the host before
+ *     synchronise.  Device inputs must be ready in that stream's order (made
+ *     on it, or the stream made to wait for the one that made them), and
+ *     device outputs are ready in that order too.  Arguments and capacities are checked on the host before
  *     anything is launched; a rejected call returns an error and changes no
  *     state.  Errors raised on the device (a bounded wait that ran out) are
  *     reported by the next dg_sync as DG_ERR_DEVICE_TIMEOUT.
