@@ -145,3 +145,10 @@ def test_code_hash_ignores_comments_and_layout_but_not_code(tmp_path):
         h[name] = bench.code_sha256(str(f))
     assert h["same"] == h["comments"] == h["layout"]
     assert h["code"] != h["same"] and h["code in body"] != h["same"]
+
+
+def test_l2_note_follows_the_step_bytes():
+    by, _, _ = bench.step_cost(si.workload("a4b_p2k"), [77] * 30)
+    assert bench.l2_note(by).startswith("inputs larger than L2 (3") and "no flush" in bench.l2_note(by)
+    tiny, _, _ = bench.step_cost(si.workload("tiny"), [16, 16])
+    assert bench.l2_note(tiny).startswith("inputs fit in L2 (32 MB")
