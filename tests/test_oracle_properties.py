@@ -100,3 +100,18 @@ def test_sampler_picks_one_of_its_inputs(seed, tau):
     assert ((out == a) | (out == noise)).all()
     assert (out[conf >= tau] == a[conf >= tau]).all()
     assert noise.min() >= 0 and noise.max() < 1000
+
+
+@SETTINGS
+@given(seeds, st.integers(min_value=-20, max_value=20))
+def test_mx_encoding_commutes_with_powers_of_two(seed, k):
+    """Scaling a block by 2^k shifts its shared exponent by k and nothing
+    else, so the MXFP8 encoding commutes with it exactly (away from the
+    float64 range limits), and encoding twice changes nothing."""
+    from oracle import mx
+    r = np.random.default_rng(seed)
+    x = r.standard_normal((2, 96)) * np.exp(r.uniform(-6, 6, (2, 1)))
+    y = mx.mx_round_trip(x)
+    np.testing.assert_array_equal(mx.mx_round_trip(np.ldexp(x, k)), np.ldexp(y, k))
+    np.testing.assert_array_equal(mx.mx_block_exponents(np.ldexp(x, k)), mx.mx_block_exponents(x) + k)
+    np.testing.assert_array_equal(mx.mx_round_trip(y), y)
