@@ -5,7 +5,8 @@ of how the oracle computes it: scale invariance of RMSNorm, linearity of
 attention in the values and its indifference to the order of the keys it
 sees, equivariance of the router under a relabelling of the experts, the
 LM-head statistics under a constant shift of every logit, the monotonicity
-of the entropy budget, and the sampler choosing between its two inputs."""
+of the entropy budget, the sampler choosing between its two inputs, and the
+MXFP8 encoding under powers of two."""
 import numpy as np
 from hypothesis import given, settings
 from hypothesis import strategies as st
